@@ -1,0 +1,145 @@
+"""Seeded synthetic inputs for the fused W8A8 MoE layer and the standalone
+SwiGLU+MXFP8 op.
+
+This module is shared by the CUDA path's tests/benchmark and by the CPU
+oracle's tests.  It holds none of the layer's own arithmetic: it draws router
+logits, picks top-k experts and softmax weights (the router is the step
+*before* the layer; its outputs are the layer's inputs), draws bf16
+activations, and produces FP8 E4M3 weights with fp32 128x128 block scales by
+torch's own fp32 -> float8_e4m3fn cast (weights reach the layer already
+quantised, so weight quantisation is input preparation, not a layer step).
+
+Workloads (sizes from the method's pages' MoE settings):
+  tiny     T=16,   H=256,  I=128,  E=4,   top-2, logits ~N(0,1)
+  mid      T=512,  H=2048, I=768,  E=128, top-8, logits ~N(0,1)
+  decode   T=64,   H=7168, I=2048, E=256, top-8, logits ~N(0,1)
+  prefill  T=8192, H=7168, I=2048, E=256, top-8, logits ~N(0,1) plus a
+           per-expert bias -1.2*ln(rank), ranks a seeded permutation of 1..E
+           (Zipf(1.2)-shaped popularity)
+Weights: w13 [E,2I,H] ~ N(0, 1/sqrt(H)), w2 [E,H,I] ~ N(0, 1/sqrt(I)).
+Draw order for one seed: logits, (Zipf ranks), x, then w13 and w2 expert by
+expert.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import torch
+
+
+@dataclass(frozen=True)
+class MoEConfig:
+    name: str
+    T: int
+    H: int
+    I: int
+    E: int
+    k: int
+    routing: str = "normal"   # "normal" or "zipf"
+
+    @property
+    def R(self) -> int:
+        return self.T * self.k
+
+
+CONFIGS = {
+    "tiny": MoEConfig("tiny", 16, 256, 128, 4, 2),
+    "mid": MoEConfig("mid", 512, 2048, 768, 128, 8),
+    "decode": MoEConfig("decode", 64, 7168, 2048, 256, 8),
+    "prefill": MoEConfig("prefill", 8192, 7168, 2048, 256, 8, "zipf"),
+}
+
+SWIGLU_SHAPES = ((128, 128), (1024, 2048), (8192, 7168))
+ZIPF_S = 1.2
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def quantize_weight_blocks(w: torch.Tensor):
+    """[N, K] fp32 -> (float8_e4m3fn [N, K], fp32 scales [N/128, K/128]) with
+    scale = blockwise amax / 448 and torch's float8 cast of w / scale."""
+    N, K = w.shape
+    blocks = w.view(N // 128, 128, K // 128, 128)
+    amax = blocks.abs().amax(dim=(1, 3))
+    scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    q = (blocks / scale[:, None, :, None]).to(torch.float8_e4m3fn)
+    return q.view(N, K), scale.contiguous()
+
+
+def _expert_weights(E: int, N: int, K: int, sigma: float, g, device):
+    q = torch.empty(E, N, K, dtype=torch.float8_e4m3fn, device=device)
+    s = torch.empty(E, N // 128, K // 128, dtype=torch.float32, device=device)
+    for e in range(E):
+        w = torch.randn(N, K, generator=g, device=device, dtype=torch.float32) * sigma
+        q[e], s[e] = quantize_weight_blocks(w)
+    return q, s
+
+
+def make_routing(T: int, E: int, k: int, routing: str, g, device):
+    logits = torch.randn(T, E, generator=g, device=device, dtype=torch.float32)
+    if routing == "zipf":
+        ranks = torch.randperm(E, generator=g, device=device).to(torch.float32) + 1.0
+        logits = logits + (-ZIPF_S) * torch.log(ranks)[None, :]
+    elif routing != "normal":
+        raise ValueError(routing)
+    top_v, top_i = torch.topk(logits, k, dim=1, largest=True, sorted=True)
+    topk_w = torch.softmax(top_v, dim=1).to(torch.float32)
+    return top_i.to(torch.int32).contiguous(), topk_w.contiguous()
+
+
+def make_moe_inputs(cfg: MoEConfig, seed: int = 0, device="cpu", weights: bool = True):
+    """Returns a dict of tensors on `device`: x (bf16 [T,H]), topk_ids (int32
+    [T,k]), topk_w (fp32 [T,k]), w13 (fp8 [E,2I,H]), w13_scale (fp32
+    [E,2I/128,H/128]), w2 (fp8 [E,H,I]), w2_scale (fp32 [E,H/128,I/128])."""
+    g = _gen(seed, device)
+    topk_ids, topk_w = make_routing(cfg.T, cfg.E, cfg.k, cfg.routing, g, device)
+    x = torch.randn(cfg.T, cfg.H, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+    out = dict(x=x, topk_ids=topk_ids, topk_w=topk_w)
+    if weights:
+        out["w13"], out["w13_scale"] = _expert_weights(cfg.E, 2 * cfg.I, cfg.H,
+                                                       1.0 / math.sqrt(cfg.H), g, device)
+        out["w2"], out["w2_scale"] = _expert_weights(cfg.E, cfg.H, cfg.I,
+                                                     1.0 / math.sqrt(cfg.I), g, device)
+    return out
+
+
+def make_swiglu_input(M: int, K: int, variant: str = "normal", seed: int = 0, device="cpu"):
+    """bf16 [M, 2K] (gate | up halves) ~ N(0,1); variant "block_scaled"
+    multiplies each 32-column block by 2^u, u ~ U{-8..8} (integers)."""
+    g = _gen(seed, device)
+    x = torch.randn(M, 2 * K, generator=g, device=device, dtype=torch.float32)
+    if variant == "block_scaled":
+        u = torch.randint(-8, 9, (M, 2 * K // 32), generator=g, device=device).to(torch.float32)
+        x = (x.view(M, 2 * K // 32, 32) * torch.exp2(u)[:, :, None]).view(M, 2 * K)
+    elif variant != "normal":
+        raise ValueError(variant)
+    return x.to(torch.bfloat16).contiguous()
+
+
+def make_grouped_gemm_inputs(R: int, N: int, K: int, E: int, seed: int = 0, device="cpu",
+                             group_sizes=None):
+    """Inputs for the standalone grouped GEMM: activations already quantised
+    per row per 128 (drawn as bf16 N(0,1), cast the same way as weights but
+    with 1x128 blocks), B [E,N,K] fp8 with 128x128 scales, m_indptr from
+    `group_sizes` (default: a seeded multinomial split of R over E)."""
+    g = _gen(seed, device)
+    if group_sizes is None:
+        idx = torch.randint(0, E, (R,), generator=g, device=device)
+        group_sizes = torch.bincount(idx, minlength=E)
+    group_sizes = torch.as_tensor(group_sizes, device=device, dtype=torch.int64)
+    m_indptr = torch.zeros(E + 1, dtype=torch.int32, device=device)
+    m_indptr[1:] = torch.cumsum(group_sizes, 0).to(torch.int32)
+    R = int(m_indptr[-1])
+    a32 = torch.randn(R, K, generator=g, device=device, dtype=torch.float32)
+    blocks = a32.view(R, K // 128, 128)
+    amax = blocks.abs().amax(dim=2)
+    a_scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    a = (blocks / a_scale[:, :, None]).to(torch.float8_e4m3fn).view(R, K)
+    b, b_scale = _expert_weights(E, N, K, 1.0 / math.sqrt(K), g, device)
+    return dict(a=a.contiguous(), a_scale=a_scale.contiguous(), b=b, b_scale=b_scale,
+                m_indptr=m_indptr)
