@@ -1,0 +1,383 @@
+#!/usr/bin/env python
+"""Benchmark of the fused W8A8 block-scaled MoE layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill|decode|mid|tiny]
+                    [--impl ours|reference]
+
+One step = one full fused layer (routing/permutation, activation quant,
+GEMM1 gate/up + SwiGLU + FP8 requant, GEMM2 down + weighted combine, bf16
+output) through the C ABI on one batch of synthetic, seeded inputs already
+resident in HBM.  With N GPUs (torchrun) every rank runs an independent
+replica of the workload (weak scaling); time is the max over ranks.
+
+Prints one JSON line (rank 0).  `value` is the effective throughput in
+TFLOP/s of algorithmic work (6*T*k*H*I flops per layer); `ms_per_step` is the
+layer latency.  The reference arm (--impl reference) times the CPU oracle on
+a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "fused MoE layer µs & TFLOPS/GB/s as % of B200 FP8-tensor/HBM roofline"
+FP8_OVER_BF16 = 2.0        # nominal dense FP8 / BF16 tensor ratio (4.5 / 2.25 PFLOP/s)
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+KERNELS_PER_LAYER = 7      # route hist/scan/scatter, quant, GEMM1, GEMM2, bf16 conversion
+
+
+def workload_desc(cfg: synth.MoEConfig) -> str:
+    r = "zipf(1.2)-biased routing" if cfg.routing == "zipf" else "logits ~N(0,1)"
+    return (f"{cfg.name}: T={cfg.T} H={cfg.H} I={cfg.I} E={cfg.E} top-{cfg.k}, {r}, "
+            f"FP8 e4m3 weights with fp32 128x128 block scales, bf16 in/out")
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), \
+            "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def work_counts(cfg: synth.MoEConfig, topk_ids: torch.Tensor):
+    """Algorithmic flops and bytes of the layer and of GEMM1, from the actual
+    routing (only experts with at least one row are read)."""
+    ids = topk_ids.flatten()
+    valid = ids[(ids >= 0) & (ids < cfg.E)]
+    R = int(valid.numel())
+    touched = int(torch.unique(valid).numel())
+    H, I = cfg.H, cfg.I
+    w13_b = 2 * I * H + 4 * (2 * I // 128) * (H // 128)
+    w2_b = H * I + 4 * (H // 128) * (I // 128)
+    flops = 6.0 * R * H * I
+    layer_bytes = touched * (w13_b + w2_b) + 2 * cfg.T * H * 2 + cfg.T * cfg.k * 8
+    g1_flops = 4.0 * R * H * I
+    # GEMM1 reads the touched gate/up weights, the FP8 activations and their
+    # scales, and writes the FP8 intermediate with its scales
+    g1_bytes = touched * w13_b + R * H + 4 * R * (H // 128) + R * I + 4 * R * (I // 128)
+    return dict(R=R, touched=touched, flops=flops, bytes=layer_bytes, g1_flops=g1_flops,
+                g1_bytes=g1_bytes)
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle sampling while the timed region runs."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: str):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.index, f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def sample_tokens(cfg, n):
+    step = max(1, cfg.T // max(1, n))
+    return list(range(0, cfg.T, step))[:n]
+
+
+def oracle_sample_rate(inp, cfg, n_tok, repeats=1):
+    """Times the CPU oracle (per-token form) on n_tok tokens; returns
+    (flops per sample, seconds per sample, threads)."""
+    import oracle
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from tests import gpu_helpers as G
+    toks = sample_tokens(cfg, n_tok)
+    sub = G.compact_experts(inp, toks)
+    args = (sub["x"], sub["topk_ids"], sub["topk_w"], sub["w13"], sub["w13_scale"], sub["w2"],
+            sub["w2_scale"], np.arange(len(toks), dtype=np.int32))
+    valid = int(((sub["topk_ids"] >= 0)).sum())
+    flops = 6.0 * valid * cfg.H * cfg.I
+    times = []
+    for _ in range(repeats):
+        t0 = time.perf_counter()
+        oracle.moe_tokens(*args)
+        times.append(time.perf_counter() - t0)
+    return flops, times, oracle.num_threads(), len(toks)
+
+
+def run_reference(args, cfg):
+    world, rank, local = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    dev = f"cuda:{local}" if torch.cuda.is_available() else "cpu"
+    big = cfg.H * cfg.I * cfg.E > (1 << 30)
+    inp = synth.make_moe_inputs(cfg, seed=0, device=dev if big else "cpu")
+    threads = oracle.num_threads()
+    # size one step to about two seconds of oracle work
+    n = max(1, min(cfg.T, threads))
+    f, t, _, _ = oracle_sample_rate(inp, cfg, n)
+    n = int(max(1, min(cfg.T, n * max(1.0, 2.0 / max(t[0], 1e-3)))))
+    flops, times, threads, ntok = oracle_sample_rate(inp, cfg, n, repeats=args.warmup + args.steps)
+    timed = times[args.warmup:]
+    sec = sum(timed) / len(timed)
+    value = flops / sec / 1e12
+    sample = f"{ntok} of {cfg.T} tokens per step (per-token oracle form), all top-{cfg.k} slots"
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp32 (fp8 e4m3 operands)",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": workload_desc(cfg), "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, cfg):
+    import fp8_block_scaled_route_b200 as moe
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+    moe.lib()
+    inp = synth.make_moe_inputs(cfg, seed=rank, device=dev)
+    T, H, I, E, k = cfg.T, cfg.H, cfg.I, cfg.E, cfg.k
+    ws = torch.empty(moe.moe_workspace_size(T, H, I, E, k), dtype=torch.uint8, device=dev)
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    counts = work_counts(cfg, inp["topk_ids"])
+
+    def step():
+        moe.moe_fp8_fused(inp["x"], inp["topk_ids"], inp["topk_w"], inp["w13"], inp["w13_scale"],
+                          inp["w2"], inp["w2_scale"], out, ws, stream=stream)
+
+    # warm-up
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st = moe.moe_get_device_status(ws, stream=stream)
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device status after warm-up: {moe.moe_status_string(st)}")
+
+    # stage events for the dominant kernel (GEMM1) over the timed region
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    for evs in stage_ev:          # torch creates the CUDA event on its first record
+        for e in evs:
+            e.record(stream)
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    smi_index = vis.split(",")[local] if vis else str(local)
+    clocks = ClockSampler(smi_index)
+    clocks.start()
+    time.sleep(0.3)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        moe.moe_set_stage_events(stage_ev[i])
+        step()
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    moe.moe_set_stage_events(None)
+    if pg:
+        pg.barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    st = moe.moe_get_device_status(ws, stream=stream)
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device status after timing: {moe.moe_status_string(st)}")
+    stages = np.array([[ev[j].elapsed_time(ev[j + 1]) for j in range(5)] for ev in stage_ev])
+    stage_ms = stages.mean(axis=0)   # route, quant, gemm1, gemm2, finish
+
+    # end to end through the C ABI with host buffers (inputs H2D, output D2H)
+    x_h = inp["x"].cpu().pin_memory()
+    ids_h = inp["topk_ids"].cpu().pin_memory()
+    w_h = inp["topk_w"].cpu().pin_memory()
+    out_h = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
+    x_d = torch.empty_like(inp["x"])
+    ids_d = torch.empty_like(inp["topk_ids"])
+    w_d = torch.empty_like(inp["topk_w"])
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        ids_d.copy_(ids_h, non_blocking=True)
+        w_d.copy_(w_h, non_blocking=True)
+        moe.moe_fp8_fused(x_d, ids_d, w_d, inp["w13"], inp["w13_scale"], inp["w2"],
+                          inp["w2_scale"], out, ws, stream=stream)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.stop()
+    e2e_ms = e_start.elapsed_time(e_end)
+
+    # max over ranks
+    tvec = torch.tensor([elapsed_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if pg:
+        pg.all_reduce(tvec, op=pg.ReduceOp.MAX)
+    elapsed_ms, e2e_ms = float(tvec[0]), float(tvec[1])
+
+    if rank == 0:
+        ms_step = elapsed_ms / args.steps
+        value = world * counts["flops"] / (ms_step * 1e-3) / 1e12
+        e2e_value = world * counts["flops"] / (e2e_ms / args.steps * 1e-3) / 1e12
+        hbm, bf16, bf16_sus, src = load_peaks()
+        g1_ms = float(stage_ms[2])
+        g1_tflops = counts["g1_flops"] / (g1_ms * 1e-3) / 1e12
+        g1_gbs = counts["g1_bytes"] / (g1_ms * 1e-3) / 1e9
+        fp8_peak = bf16 * FP8_OVER_BF16
+        t_tensor = counts["g1_flops"] / (fp8_peak * 1e12)
+        t_hbm = counts["g1_bytes"] / (hbm * 1e9)
+        if t_tensor >= t_hbm:
+            roof = {"bound": "tensor", "achieved": g1_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
+                    "frac": g1_tflops / fp8_peak}
+        else:
+            roof = {"bound": "hbm", "achieved": g1_gbs, "peak": hbm, "unit": "GB/s",
+                    "frac": g1_gbs / hbm}
+        roof.update({"traffic": None, "kernel": "grouped GEMM1 (gate/up + SwiGLU + FP8 requant)",
+                     "peak_source": f"{src} (FP8 = bf16 burst x {FP8_OVER_BF16:g})"
+                     if roof["bound"] == "tensor" else f"{src} copy bandwidth"})
+        layer_gbs = counts["bytes"] / (ms_step * 1e-3) / 1e9
+        layer_tflops = counts["flops"] / (ms_step * 1e-3) / 1e12
+        layer_frac = max(counts["flops"] / (fp8_peak * 1e12), counts["bytes"] / (hbm * 1e9)) / \
+            (ms_step * 1e-3)
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp8_e4m3 (fp32 accumulate)", "data": "synthetic",
+            "config": {"workload": workload_desc(cfg), "l2": "inputs larger than L2 (no flush)"
+                       if counts["touched"] * 3 * H * I > 126e6 else "working set fits L2",
+                       "parallelism": f"replicas x{world}", "seed": "rank"},
+            "layer": {"us": ms_step * 1e3, "tflops": layer_tflops, "gbs": layer_gbs,
+                      "roofline_frac": layer_frac, "rows": counts["R"],
+                      "experts_touched": counts["touched"], "alg_bytes": counts["bytes"],
+                      "alg_flops": counts["flops"]},
+            "stages_us": {n: float(v) * 1e3 for n, v in
+                          zip(["route", "quant", "gemm1", "gemm2", "finish"], stage_ms)},
+            "roofline": roof,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": T * H * 2 + T * k * 8, "d2h_bytes_per_step": T * H * 2},
+            "gpu_launches": KERNELS_PER_LAYER * args.steps,
+            "clocks": clocks.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+            oracle.build()
+            threads = oracle.num_threads()
+            n = max(1, min(T, threads))
+            f, t, _, _ = oracle_sample_rate(inp, cfg, n)
+            target = 10.0
+            n2 = int(max(1, min(T, n * max(1.0, target / max(t[0], 1e-3)))))
+            if n2 > n:
+                f, t, threads, n = oracle_sample_rate(inp, cfg, n2)
+            line["cpu_baseline"] = {"value": f / t[0] / 1e12, "unit": "TFLOP/s", "cores": threads,
+                                    "kind": "oracle",
+                                    "sample": f"{n} of {T} tokens, per-token oracle form, "
+                                              f"{t[0]:.1f} s"}
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="prefill", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    cfg = synth.CONFIGS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    return run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

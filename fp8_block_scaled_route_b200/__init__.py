@@ -1,0 +1,227 @@
+"""Python binding of libmoefp8.so, the sm_100a fused W8A8 block-scaled MoE
+library (C ABI in include/moefp8.h).
+
+Argument marshalling only: every step of the computation runs in the
+library's CUDA kernels.  PyTorch supplies device memory and streams.  The
+binding raises if the compiled library is missing; there is no fallback.
+
+Functions keep the C names:
+  moe_route_permute, moe_fp8_fused, moe_fp8_fused_debug,
+  fp8_groupwise_moe_gemm, swiglu_mxfp8_quant, moe_select_tile_m,
+  moe_workspace_size, moe_route_workspace_size, moe_get_device_status,
+  moe_set_wait_timeout_ns, moe_status_string.
+Tensor arguments may be torch tensors (their data_ptr is passed) or raw
+integer device addresses.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "MoEError", "lib", "lib_path", "EXPORTS",
+    "moe_route_permute", "moe_fp8_fused", "moe_fp8_fused_debug", "fp8_groupwise_moe_gemm",
+    "swiglu_mxfp8_quant", "moe_select_tile_m", "moe_workspace_size", "moe_route_workspace_size",
+    "moe_get_device_status", "moe_set_wait_timeout_ns", "moe_status_string",
+    "moe_set_stage_events",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoefp8.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED = 2
+MOE_ERR_CUDA = 3
+MOE_ERR_NO_TILE_CONFIG = 4
+MOE_ERR_DEVICE_TIMEOUT = 5
+MOE_ERR_BAD_EXPERT_ID = 6
+
+# Every symbol declared in include/moefp8.h.
+EXPORTS = (
+    "moe_status_string", "moe_route_workspace_size", "moe_route_permute", "moe_workspace_size",
+    "moe_fp8_fused", "moe_fp8_fused_debug", "fp8_groupwise_moe_gemm", "moe_select_tile_m",
+    "swiglu_mxfp8_quant", "moe_get_device_status", "moe_set_wait_timeout_ns",
+    "moe_set_stage_events",
+)
+
+_lib = None
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, where: str = ""):
+        self.status = int(status)
+        super().__init__(f"{where}: {moe_status_string(status)} ({status})")
+
+
+def lib_path() -> str:
+    return LIB_PATH
+
+
+def lib():
+    """Loads libmoefp8.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with `python -m fp8_block_scaled_route_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, Z, U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint64
+    L.moe_status_string.restype = ctypes.c_char_p
+    L.moe_status_string.argtypes = [I]
+    L.moe_route_workspace_size.restype = Z
+    L.moe_route_workspace_size.argtypes = [I, I, I]
+    L.moe_route_permute.restype = I
+    L.moe_route_permute.argtypes = [P, I, I, I, P, P, P, P, Z, P]
+    L.moe_workspace_size.restype = Z
+    L.moe_workspace_size.argtypes = [I] * 5
+    L.moe_fp8_fused.restype = I
+    L.moe_fp8_fused.argtypes = [P] * 8 + [I] * 5 + [P, Z, P]
+    L.moe_fp8_fused_debug.restype = I
+    L.moe_fp8_fused_debug.argtypes = [P] * 8 + [I] * 5 + [P, Z, P] + [P] * 4
+    L.fp8_groupwise_moe_gemm.restype = I
+    L.fp8_groupwise_moe_gemm.argtypes = [P] * 6 + [I] * 11 + [P]
+    L.moe_select_tile_m.restype = I
+    L.moe_select_tile_m.argtypes = [I] * 6 + [ctypes.POINTER(I), ctypes.POINTER(I)]
+    L.swiglu_mxfp8_quant.restype = I
+    L.swiglu_mxfp8_quant.argtypes = [P, P, P, I, I, P]
+    L.moe_get_device_status.restype = I
+    L.moe_get_device_status.argtypes = [P, P]
+    L.moe_set_wait_timeout_ns.restype = None
+    L.moe_set_wait_timeout_ns.argtypes = [U64]
+    L.moe_set_stage_events.restype = I
+    L.moe_set_stage_events.argtypes = [ctypes.POINTER(P), I]
+    _lib = L
+    return L
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return ctypes.c_void_p(t)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(status: int, where: str, check: bool) -> int:
+    if check and status != MOE_OK:
+        raise MoEError(status, where)
+    return status
+
+
+def moe_status_string(status: int) -> str:
+    return lib().moe_status_string(int(status)).decode()
+
+
+def moe_set_wait_timeout_ns(ns: int) -> None:
+    lib().moe_set_wait_timeout_ns(int(ns))
+
+
+def moe_workspace_size(T: int, H: int, I: int, E: int, k: int) -> int:
+    return int(lib().moe_workspace_size(T, H, I, E, k))
+
+
+def moe_route_workspace_size(T: int, k: int, E: int) -> int:
+    return int(lib().moe_route_workspace_size(T, k, E))
+
+
+def moe_select_tile_m(total_rows: int, n: int, k: int, E: int, num_sms: int, is_gated: bool):
+    tm, tn = ctypes.c_int(0), ctypes.c_int(0)
+    st = lib().moe_select_tile_m(total_rows, n, k, E, num_sms, int(bool(is_gated)),
+                                 ctypes.byref(tm), ctypes.byref(tn))
+    _check(st, "moe_select_tile_m", True)
+    return tm.value, tn.value
+
+
+def moe_route_permute(topk_ids, E: int, m_indptr, perm, inv_perm, ws, ws_bytes=None, *,
+                      T=None, k=None, stream=None, check=True) -> int:
+    if T is None or k is None:
+        T, k = topk_ids.shape
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size()
+    st = lib().moe_route_permute(_ptr(topk_ids), T, k, E, _ptr(m_indptr), _ptr(perm),
+                                 _ptr(inv_perm), _ptr(ws), ws_bytes, _stream(stream))
+    return _check(st, "moe_route_permute", check)
+
+
+def _fused_dims(x, topk_ids, w13):
+    T, H = x.shape
+    k = topk_ids.shape[1]
+    E, I2, _ = w13.shape
+    return T, H, I2 // 2, E, k
+
+
+def moe_fp8_fused(x, topk_ids, topk_w, w13, w13_scale, w2, w2_scale, out, ws, ws_bytes=None, *,
+                  dims=None, stream=None, check=True) -> int:
+    """dims = (T, H, I, E, k) when raw addresses are passed."""
+    T, H, I, E, k = dims if dims is not None else _fused_dims(x, topk_ids, w13)
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size()
+    st = lib().moe_fp8_fused(_ptr(x), _ptr(topk_ids), _ptr(topk_w), _ptr(w13), _ptr(w13_scale),
+                             _ptr(w2), _ptr(w2_scale), _ptr(out), T, H, I, E, k, _ptr(ws),
+                             ws_bytes, _stream(stream))
+    return _check(st, "moe_fp8_fused", check)
+
+
+def moe_fp8_fused_debug(x, topk_ids, topk_w, w13, w13_scale, w2, w2_scale, out, ws,
+                        m_indptr=None, perm=None, h_fp8=None, h_scale=None, ws_bytes=None, *,
+                        dims=None, stream=None, check=True) -> int:
+    T, H, I, E, k = dims if dims is not None else _fused_dims(x, topk_ids, w13)
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size()
+    st = lib().moe_fp8_fused_debug(_ptr(x), _ptr(topk_ids), _ptr(topk_w), _ptr(w13),
+                                   _ptr(w13_scale), _ptr(w2), _ptr(w2_scale), _ptr(out), T, H, I,
+                                   E, k, _ptr(ws), ws_bytes, _stream(stream), _ptr(m_indptr),
+                                   _ptr(perm), _ptr(h_fp8), _ptr(h_scale))
+    return _check(st, "moe_fp8_fused_debug", check)
+
+
+def fp8_groupwise_moe_gemm(a, b, a_scale, b_scale, m_indptr, out, scale_major_mode="K",
+                           scale_granularity=(1, 128, 128), is_gated=False, tile_m=-1, tile_n=-1,
+                           *, dims=None, stream=None, check=True) -> int:
+    """scale_major_mode "K": a_scale [R, K/128]; "MN": [K/128, R].
+    dims = (R, N, K, E) when raw addresses are passed."""
+    if dims is None:
+        R, K = a.shape
+        E, N, _ = b.shape
+    else:
+        R, N, K, E = dims
+    mode = {"K": 0, "MN": 1}.get(scale_major_mode, scale_major_mode)
+    sg_m, sg_n, sg_k = scale_granularity
+    st = lib().fp8_groupwise_moe_gemm(_ptr(a), _ptr(b), _ptr(a_scale), _ptr(b_scale),
+                                      _ptr(m_indptr), _ptr(out), R, N, K, E, mode, sg_m, sg_n,
+                                      sg_k, int(bool(is_gated)), tile_m, tile_n, _stream(stream))
+    return _check(st, "fp8_groupwise_moe_gemm", check)
+
+
+def swiglu_mxfp8_quant(inp, out, scale, *, dims=None, stream=None, check=True) -> int:
+    if dims is None:
+        M, K2 = inp.shape
+        K = K2 // 2
+    else:
+        M, K = dims
+    st = lib().swiglu_mxfp8_quant(_ptr(inp), _ptr(out), _ptr(scale), M, K, _stream(stream))
+    return _check(st, "swiglu_mxfp8_quant", check)
+
+
+def moe_set_stage_events(events) -> int:
+    """events: six torch.cuda.Event (timing enabled, already created on the
+    device) or None to switch stage timing off."""
+    if events is None:
+        return _check(lib().moe_set_stage_events(None, 0), "moe_set_stage_events", True)
+    handles = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    return _check(lib().moe_set_stage_events(handles, len(events)), "moe_set_stage_events", True)
+
+
+def moe_get_device_status(ws=None, *, stream=None) -> int:
+    return int(lib().moe_get_device_status(_ptr(ws), _stream(stream)))

@@ -1,0 +1,373 @@
+// C ABI of the library (declared in include/moefp8.h): argument checks,
+// tile selection, workspace carving and the launch sequence of the fused
+// layer.  No entry point allocates device memory.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "../../include/moefp8.h"
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace moe;
+
+namespace {
+
+// Status word for the entry points that take no workspace.
+__device__ int g_lib_status[kStatusInts];
+
+std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
+
+constexpr int kStageEvents = 6;
+cudaEvent_t g_stage_events[kStageEvents];
+std::atomic<bool> g_stage_events_on{false};
+
+inline void stage_mark(int i, cudaStream_t s) {
+    if (g_stage_events_on.load(std::memory_order_relaxed)) cudaEventRecord(g_stage_events[i], s);
+}
+
+struct DevInfo {
+    int sms = 0;
+    int major = 0, minor = 0;
+    int* lib_status = nullptr;
+    bool ok = false;
+};
+
+constexpr int kMaxDevices = 64;
+DevInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+// Per-device facts, looked up once per device with that device current.
+const DevInfo* dev_info() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DevInfo& d = g_dev[dev];
+    if (!d.ok) {
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return nullptr;
+        cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev);
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_lib_status) != cudaSuccess) return nullptr;
+        d.lib_status = static_cast<int*>(p);
+        d.ok = true;
+    }
+    return &d;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Workspace of the fused layer, in carve order.
+struct FusedWs {
+    size_t status, m_indptr, chunk_hist, perm, inv_perm, xq, xs, hq, hs, out_acc, total;
+};
+
+FusedWs fused_layout(int T, int H, int I, int E, int k) {
+    const size_t R = static_cast<size_t>(T) * k;
+    const size_t nchunks = (R + kRouteChunk - 1) / kRouteChunk;
+    FusedWs w{};
+    size_t o = 0;
+    w.status = o;     o += up256(sizeof(int) * kStatusInts);
+    w.m_indptr = o;   o += up256(sizeof(int32_t) * (E + 1));
+    w.chunk_hist = o; o += up256(sizeof(int32_t) * nchunks * E);
+    w.perm = o;       o += up256(sizeof(int32_t) * R);
+    w.inv_perm = o;   o += up256(sizeof(int32_t) * R);
+    w.xq = o;         o += up256(R * H);
+    w.xs = o;         o += up256(sizeof(float) * R * (H / 128));
+    w.hq = o;         o += up256(R * I);
+    w.hs = o;         o += up256(sizeof(float) * R * (I / 128));
+    w.out_acc = o;    o += up256(sizeof(float) * static_cast<size_t>(T) * H);
+    w.total = o;
+    return w;
+}
+
+size_t route_ws_bytes(int T, int k, int E) {
+    const size_t R = static_cast<size_t>(T) * k;
+    const size_t nchunks = (R + kRouteChunk - 1) / kRouteChunk;
+    return up256(sizeof(int) * kStatusInts) + up256(sizeof(int32_t) * nchunks * E);
+}
+
+// --- tile selection (wave + residue), sm_100a tile menu -----------------
+// Token tiles of 16/32/64 rows run with the weights as the 128-row MMA
+// operand; 128-row tiles with the tokens as the MMA M operand.  Each tile
+// covers 256 weight rows: 128 output columns gated, 256 plain.
+constexpr int kTileOverheadRows = 32;
+
+long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
+
+long long balanced_tile_count(long long total_rows, long long n_out, long long E, int tile_m,
+                              int tile_n) {
+    const long long q = total_rows / E, r = total_rows % E;
+    const long long m_tiles = r * ceil_div(q + 1, tile_m) + (E - r) * ceil_div(q, tile_m);
+    return m_tiles * ceil_div(n_out, tile_n);
+}
+
+void select_tile(int total_rows, int n, int k, int E, int num_sms, int gated, int* tm, int* tn) {
+    const long long n_out = gated ? n / 2 : n;
+    const int tile_n = gated ? 128 : 256;
+    *tn = tile_n;
+    if (E <= 0 || total_rows <= 0) { *tm = 16; return; }
+    const long long max_m = ceil_div(total_rows, E);
+    auto tiles = [&](int t) { return balanced_tile_count(total_rows, n_out, E, t, tile_n); };
+    if (max_m <= 16 || (tiles(32) < num_sms / 2 && tiles(16) <= num_sms)) { *tm = 16; return; }
+    if (max_m <= 32) { *tm = 32; return; }
+    if (k <= 2048) { *tm = max_m < 192 ? 64 : 128; return; }
+    auto cost = [&](int t) { return ceil_div(tiles(t), num_sms) * (t + kTileOverheadRows); };
+    *tm = cost(64) < cost(128) ? 64 : 128;
+}
+
+// Token tiles of the swapped kernels stage K/128 x tile_m scales on chip.
+int fit_tile_to_k(int tm, int K) {
+    while (tm < 128 && K > swap_max_k(tm)) tm *= 2;
+    return tm;
+}
+
+int check_device(const DevInfo* d) {
+    if (!d) return MOE_ERR_CUDA;
+    if (d->major != 10 || d->minor != 0) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(int status) {
+    switch (status) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+        case MOE_ERR_NO_TILE_CONFIG: return "MOE_ERR_NO_TILE_CONFIG";
+        case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
+        case MOE_ERR_BAD_EXPERT_ID: return "MOE_ERR_BAD_EXPERT_ID";
+        default: return "MOE_ERR_UNKNOWN";
+    }
+}
+
+void moe_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns > 0 ? ns : 1); }
+
+int moe_set_stage_events(void* const* events, int n) {
+    if (events == nullptr) {
+        g_stage_events_on.store(false);
+        return MOE_OK;
+    }
+    if (n != kStageEvents) return MOE_ERR_INVALID_ARG;
+    for (int i = 0; i < kStageEvents; ++i) {
+        if (!events[i]) return MOE_ERR_INVALID_ARG;
+        g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
+    }
+    g_stage_events_on.store(true);
+    return MOE_OK;
+}
+
+int moe_select_tile_m(int total_rows, int n, int k, int E, int num_sms, int is_gated, int* tile_m,
+                      int* tile_n) {
+    if (!tile_m || !tile_n || num_sms <= 0 || total_rows < 0 || n <= 0 || k <= 0 || E <= 0)
+        return MOE_ERR_INVALID_ARG;
+    select_tile(total_rows, n, k, E, num_sms, is_gated ? 1 : 0, tile_m, tile_n);
+    return MOE_OK;
+}
+
+size_t moe_route_workspace_size(int T, int k, int E) {
+    if (T < 0 || k < 1 || E < 1) return 0;
+    return route_ws_bytes(T, k, E);
+}
+
+int moe_route_permute(const int32_t* topk_ids, int T, int k, int E, int32_t* m_indptr,
+                      int32_t* perm, int32_t* inv_perm, void* ws, size_t ws_bytes,
+                      moe_stream_t stream) {
+    if (T < 0 || k < 1 || E < 1 || E > MOE_MAX_EXPERTS) return MOE_ERR_INVALID_ARG;
+    if (!m_indptr || !ws || (T > 0 && (!topk_ids || !perm))) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < route_ws_bytes(T, k, E) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+    const DevInfo* d = dev_info();
+    if (int st = check_device(d)) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    char* base = static_cast<char*>(ws);
+    int* status = reinterpret_cast<int*>(base);
+    if (cudaMemsetAsync(status, 0, sizeof(int) * kStatusInts, s) != cudaSuccess) return MOE_ERR_CUDA;
+    RouteArgs ra{topk_ids, T, k, E, m_indptr, perm, inv_perm,
+                 reinterpret_cast<int32_t*>(base + up256(sizeof(int) * kStatusInts)), status};
+    return launch_route_permute(ra, s);
+}
+
+size_t moe_workspace_size(int T, int H, int I, int E, int k) {
+    if (T < 0 || H <= 0 || I <= 0 || E < 1 || k < 1) return 0;
+    return fused_layout(T, H, I, E, k).total;
+}
+
+static int fused_impl(const void* x, const int32_t* topk_ids, const float* topk_w, const void* w13,
+                      const float* w13_scale, const void* w2, const float* w2_scale, void* out, int T,
+                      int H, int I, int E, int k, void* ws, size_t ws_bytes, moe_stream_t stream,
+                      int32_t* dbg_m_indptr, int32_t* dbg_perm, uint8_t* dbg_hq, float* dbg_hs) {
+    if (T < 0 || H <= 0 || I <= 0 || H % 128 || I % 128 || k < 1) return MOE_ERR_INVALID_ARG;
+    if (E < 1) return MOE_ERR_INVALID_ARG;
+    if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+    if (k > E) return MOE_ERR_INVALID_ARG;
+    if (!ws) return MOE_ERR_INVALID_ARG;
+    const FusedWs L = fused_layout(T, H, I, E, k);
+    if (ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+    if (T > 0) {
+        if (!x || !topk_ids || !topk_w || !w13 || !w13_scale || !w2 || !w2_scale || !out)
+            return MOE_ERR_INVALID_ARG;
+        if (!aligned16(x) || !aligned16(w13) || !aligned16(w2) || !aligned16(out))
+            return MOE_ERR_INVALID_ARG;
+    }
+    const DevInfo* d = dev_info();
+    if (int st = check_device(d)) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    char* b = static_cast<char*>(ws);
+    int* status = reinterpret_cast<int*>(b + L.status);
+    int32_t* m_indptr = reinterpret_cast<int32_t*>(b + L.m_indptr);
+    int32_t* perm = reinterpret_cast<int32_t*>(b + L.perm);
+    int32_t* inv_perm = reinterpret_cast<int32_t*>(b + L.inv_perm);
+    uint8_t* xq = reinterpret_cast<uint8_t*>(b + L.xq);
+    float* xs = reinterpret_cast<float*>(b + L.xs);
+    uint8_t* hq = reinterpret_cast<uint8_t*>(b + L.hq);
+    float* hs = reinterpret_cast<float*>(b + L.hs);
+    float* out_acc = reinterpret_cast<float*>(b + L.out_acc);
+    if (cudaMemsetAsync(status, 0, sizeof(int) * kStatusInts, s) != cudaSuccess) return MOE_ERR_CUDA;
+    const int R = T * k;
+    RouteArgs ra{topk_ids, T, k, E, m_indptr, perm, inv_perm,
+                 reinterpret_cast<int32_t*>(b + L.chunk_hist), status};
+    stage_mark(0, s);
+    int st = launch_route_permute(ra, s);
+    if (st) return st;
+    stage_mark(1, s);
+    if (T > 0) {
+        st = launch_quant_scatter(x, T, H, k, R, inv_perm, xq, xs, out_acc, s);
+        if (st) return st;
+        stage_mark(2, s);
+        const unsigned long long tmo = g_timeout_ns.load();
+        int tm1, tn1, tm2, tn2;
+        select_tile(R, 2 * I, H, E, d->sms, 1, &tm1, &tn1);
+        select_tile(R, H, I, E, d->sms, 0, &tm2, &tn2);
+        tm1 = fit_tile_to_k(tm1, H);
+        tm2 = fit_tile_to_k(tm2, I);
+        GemmArgs g1{};
+        g1.a = xq; g1.b = w13; g1.R = R; g1.N = 2 * I; g1.K = H; g1.E = E;
+        g1.a_scale = xs; g1.as_row = 1; g1.as_kb = R; g1.b_scale = w13_scale;
+        g1.m_indptr = m_indptr; g1.epi = EPI_SWIGLU_QUANT; g1.tile_m = tm1;
+        g1.hq = hq; g1.hs = hs; g1.status = status; g1.timeout_ns = tmo; g1.num_sms = d->sms;
+        st = launch_grouped_gemm(g1, s);
+        if (st) return st;
+        stage_mark(3, s);
+        GemmArgs g2{};
+        g2.a = hq; g2.b = w2; g2.R = R; g2.N = H; g2.K = I; g2.E = E;
+        g2.a_scale = hs; g2.as_row = 1; g2.as_kb = R; g2.b_scale = w2_scale;
+        g2.m_indptr = m_indptr; g2.epi = EPI_COMBINE; g2.tile_m = tm2;
+        g2.perm = perm; g2.topk_w = topk_w; g2.topk = k; g2.out_acc = out_acc; g2.out_ld = H;
+        g2.status = status; g2.timeout_ns = tmo; g2.num_sms = d->sms;
+        st = launch_grouped_gemm(g2, s);
+        if (st) return st;
+        stage_mark(4, s);
+        st = launch_f32_to_bf16(out_acc, out, static_cast<long long>(T) * H, d->sms, s);
+        if (st) return st;
+        stage_mark(5, s);
+    }
+    if (dbg_m_indptr &&
+        cudaMemcpyAsync(dbg_m_indptr, m_indptr, sizeof(int32_t) * (E + 1), cudaMemcpyDeviceToDevice, s))
+        return MOE_ERR_CUDA;
+    if (R > 0) {
+        if (dbg_perm &&
+            cudaMemcpyAsync(dbg_perm, perm, sizeof(int32_t) * R, cudaMemcpyDeviceToDevice, s))
+            return MOE_ERR_CUDA;
+        if (dbg_hq &&
+            cudaMemcpyAsync(dbg_hq, hq, static_cast<size_t>(R) * I, cudaMemcpyDeviceToDevice, s))
+            return MOE_ERR_CUDA;
+        if (dbg_hs && cudaMemcpyAsync(dbg_hs, hs, sizeof(float) * static_cast<size_t>(R) * (I / 128),
+                                      cudaMemcpyDeviceToDevice, s))
+            return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+}
+
+int moe_fp8_fused(const void* x, const int32_t* topk_ids, const float* topk_w, const void* w13,
+                  const float* w13_scale, const void* w2, const float* w2_scale, void* out, int T,
+                  int H, int I, int E, int k, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    return fused_impl(x, topk_ids, topk_w, w13, w13_scale, w2, w2_scale, out, T, H, I, E, k, ws,
+                      ws_bytes, stream, nullptr, nullptr, nullptr, nullptr);
+}
+
+int moe_fp8_fused_debug(const void* x, const int32_t* topk_ids, const float* topk_w, const void* w13,
+                        const float* w13_scale, const void* w2, const float* w2_scale, void* out,
+                        int T, int H, int I, int E, int k, void* ws, size_t ws_bytes,
+                        moe_stream_t stream, int32_t* m_indptr, int32_t* perm, uint8_t* h_fp8,
+                        float* h_scale) {
+    return fused_impl(x, topk_ids, topk_w, w13, w13_scale, w2, w2_scale, out, T, H, I, E, k, ws,
+                      ws_bytes, stream, m_indptr, perm, h_fp8, h_scale);
+}
+
+int fp8_groupwise_moe_gemm(const void* a, const void* b, const float* a_scale, const float* b_scale,
+                           const int32_t* m_indptr, void* out, int R, int N, int K, int E,
+                           int scale_major_mode, int sg_m, int sg_n, int sg_k, int is_gated,
+                           int tile_m, int tile_n, moe_stream_t stream) {
+    if (R < 0 || N <= 0 || K <= 0 || E < 1 || N % 128 || K % 128) return MOE_ERR_INVALID_ARG;
+    if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+    if (scale_major_mode != 0 && scale_major_mode != 1) return MOE_ERR_INVALID_ARG;
+    if (sg_m != 1 || sg_n != 128 || sg_k != 128) return MOE_ERR_UNSUPPORTED;
+    // gated (fused SwiGLU) needs an even N: gate rows then up rows
+    if (is_gated && (N % 2 || (N / 2) % 128)) return MOE_ERR_INVALID_ARG;
+    if (!m_indptr || (R > 0 && (!a || !b || !a_scale || !b_scale || !out))) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(b) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    const int want_tn = is_gated ? 128 : 256;
+    if (tile_n != -1 && tile_n != want_tn) return MOE_ERR_NO_TILE_CONFIG;
+    if (tile_m != -1 && tile_m != 16 && tile_m != 32 && tile_m != 64 && tile_m != 128)
+        return MOE_ERR_NO_TILE_CONFIG;
+    const DevInfo* d = dev_info();
+    if (int st = check_device(d)) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(d->lib_status, 0, sizeof(int) * kStatusInts, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (R == 0) return MOE_OK;
+    int tm = tile_m, tn = want_tn;
+    if (tm == -1) select_tile(R, N, K, E, d->sms, is_gated ? 1 : 0, &tm, &tn);
+    if (tm < 128 && K > swap_max_k(tm)) {
+        if (tile_m != -1) return MOE_ERR_NO_TILE_CONFIG;
+        tm = fit_tile_to_k(tm, K);
+    }
+    GemmArgs g{};
+    g.a = a; g.b = b; g.R = R; g.N = N; g.K = K; g.E = E;
+    g.a_scale = a_scale;
+    if (scale_major_mode == 0) { g.as_row = K / 128; g.as_kb = 1; }
+    else { g.as_row = 1; g.as_kb = R; }
+    g.b_scale = b_scale; g.m_indptr = m_indptr;
+    g.epi = is_gated ? EPI_SWIGLU_BF16 : EPI_BF16;
+    g.tile_m = tm;
+    g.out_bf16 = out;
+    g.status = d->lib_status;
+    g.timeout_ns = g_timeout_ns.load();
+    g.num_sms = d->sms;
+    return launch_grouped_gemm(g, s);
+}
+
+int swiglu_mxfp8_quant(const void* in, void* out, uint8_t* scale, int M, int K, moe_stream_t stream) {
+    if (M < 0 || K <= 0 || K % 32) return MOE_ERR_INVALID_ARG;
+    if (M > 0 && (!in || !out || !scale)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(in) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    const DevInfo* d = dev_info();
+    if (int st = check_device(d)) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(d->lib_status, 0, sizeof(int) * kStatusInts, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return launch_swiglu_mxfp8(in, out, scale, M, K, d->sms, s);
+}
+
+int moe_get_device_status(const void* ws, moe_stream_t stream) {
+    const DevInfo* d = dev_info();
+    if (!d) return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    int h[kStatusInts] = {0, 0, 0, 0};
+    const void* src = ws ? ws : d->lib_status;
+    if (cudaMemcpy(h, src, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    return h[0];
+}
+
+}  // extern "C"

@@ -1,0 +1,67 @@
+// Shared device-side definitions: status codes, the device status word and
+// bounded waits.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "ptx.cuh"
+
+namespace moe {
+
+enum : int {
+    ST_OK = 0,
+    ST_INVALID_ARG = 1,
+    ST_UNSUPPORTED = 2,
+    ST_CUDA = 3,
+    ST_NO_TILE_CONFIG = 4,
+    ST_DEVICE_TIMEOUT = 5,
+    ST_BAD_EXPERT_ID = 6,
+};
+
+// Layout of a device status word (4 ints, 16 bytes):
+//   [0] first error code recorded (0 = none)
+//   [1] where a timeout happened (role id), for diagnostics
+//   [2] number of dropped pairs (bad expert ids)
+//   [3] reserved
+constexpr int kStatusInts = 4;
+
+__device__ __forceinline__ void report_error(int* status, int code, int where) {
+    if (status == nullptr) return;
+    if (atomicCAS(status, 0, code) == 0) status[1] = where;
+}
+
+// Control block for bounded waits inside one CTA.  `abort` lives in shared
+// memory: once any thread of the CTA gives up, the others stop waiting too.
+struct WaitCtl {
+    volatile int* abort;
+    int* status;
+    uint64_t timeout_ns;
+};
+
+// Bound of the waits that drain in-flight copies and MMAs before a CTA
+// exits; independent of the caller's timeout so that an early abort still
+// lets every outstanding copy land.
+constexpr uint64_t kDrainTimeoutNs = 2000000000ull;
+
+// Waits until the mbarrier phase with the given parity has completed.
+// Returns false when the CTA is aborting or the wait ran out of time (the
+// first thread to run out records ST_DEVICE_TIMEOUT).  With `drain = true`
+// the wait ignores the abort flag and is bounded by kDrainTimeoutNs.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const WaitCtl& c,
+                                         int where, bool drain = false) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    const uint64_t limit = drain ? kDrainTimeoutNs : c.timeout_ns;
+#pragma unroll 1
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (!drain && *c.abort) return false;
+        if (globaltimer() - t0 > limit) {
+            *c.abort = 1;
+            report_error(c.status, ST_DEVICE_TIMEOUT, where);
+            return false;
+        }
+    }
+}
+
+}  // namespace moe

@@ -1,0 +1,807 @@
+// Grouped FP8 GEMM with 128x128 block scales on sm_100a (tcgen05 + TMEM + TMA).
+//
+// Computes, for every expert e and grouped row r of that expert (rows
+// [m_indptr[e], m_indptr[e+1]) of A):
+//   G[r, n] = sum_kb a_scale(r, kb) * b_scale[e, n/128, kb] * sum_{k in kb} A[r, k] * B[e, n, k]
+// which is stage 1 (gate/up projection) and stage 4 (down projection) of the
+// expert pipeline on the page "FlashInfer: Blackwell W8A8 AlphaMoE Expert
+// 계산 커널 퓨전으로 성능 비약적 향상" (flashinfer PR #4287, section
+// "문제점: MoE Expert 계산의 병목"), with the grouped "nt" interface of the page
+// "FlashInfer SM120 MoE GEMM 최적화: 웨이브+잔여물 비용 모델 도입" (flashinfer
+// PR #4318, "코드 분석 1.").  The epilogue fuses the next stages: SwiGLU and
+// FP8 requantisation of the intermediate (stages 2-3), or the router-weighted
+// combine (stage 5), or a bf16 store for the standalone GEMM.
+//
+// Design (one persistent CTA per SM, warp-specialised):
+//  * warp 0 lane 0 - producer: TMA loads of a token tile [BT x 128] and a
+//    weight tile [256 x 128] (two 128-row boxes) per 128-wide K block into
+//    a multi-stage shared-memory ring (128-byte swizzle).
+//  * warp 1 - allocates TMEM; lane 0 issues tcgen05.mma kind::f8f6f4 (K=32
+//    per instruction, four per K block).  Each K block is accumulated into a
+//    fresh TMEM buffer (two buffers, ping-pong) because the fp32 block scales
+//    are not powers of two and must be applied per K block.
+//  * epilogue warps - read each K-block partial out of TMEM, multiply by
+//    a_scale * b_scale and accumulate in fp32 registers; after the last K
+//    block they run the fused epilogue.
+//  Two orientations:
+//  * BT = 128 ("direct"): tokens are the MMA M operand (M=128), the 256
+//    weight rows are N.  8 epilogue warps; each thread owns one token row and
+//    128 of the 256 columns.  Register split via setmaxnreg.
+//  * BT = 16/32/64 ("swapped", the small-M path): the weights are the MMA M
+//    operand (two M=128 MMAs, one per 128-row weight block) and the tokens
+//    are N = BT.  4 epilogue warps; each thread owns one weight row.
+//  Every wait is bounded by %globaltimer; on expiry the CTA records
+//  ST_DEVICE_TIMEOUT, drains its in-flight copies and MMAs, frees TMEM and
+//  returns.
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+constexpr int kSmemLimit = 232448;  // 227 KB of opt-in dynamic shared memory per CTA
+constexpr int kMaxE = 1024;
+constexpr int kTableBytes = ((2 * (kMaxE + 1) * 4) + 15) / 16 * 16;
+// Register split of the direct kernel (384 threads x 168 registers at launch):
+// the producer/MMA warpgroup drops to 56, the two epilogue warpgroups rise to
+// 224:  128*56 + 256*224 = 64512 = 384*168.
+constexpr int kDirectLaunchRegs = 168;
+constexpr int kDirectLowRegs = 56;
+constexpr int kDirectHighRegs = 224;
+static_assert(128 * kDirectLowRegs + 256 * kDirectHighRegs <= 384 * kDirectLaunchRegs,
+              "register split exceeds the launch allocation");
+
+template <int BT>
+struct Cfg {
+    static constexpr bool SWAP = BT < 128;
+    static constexpr int EPI_WARPS = SWAP ? 4 : 8;
+    static constexpr int EPI_THREADS = EPI_WARPS * 32;
+    static constexpr int THREADS = 128 + EPI_THREADS;
+    static constexpr int A_BYTES = BT * 128;       // token tile per stage
+    static constexpr int B_BYTES = 256 * 128;      // weight tile per stage
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int A_OFF = SWAP ? B_BYTES : 0;
+    static constexpr int B_OFF = SWAP ? 0 : A_BYTES;
+    static constexpr int AS_TILE_BYTES = SWAP ? 32768 : 0;  // a_scale staging [nkb][BT]
+    static constexpr int XCH_BYTES = SWAP ? ((4 * BT + 2 * BT) * 4 + 15) / 16 * 16 : 2 * 128 * 4;
+    static constexpr int BAR_BYTES = 256;
+    static constexpr int FIXED = 1024 + AS_TILE_BYTES + kTableBytes + XCH_BYTES + BAR_BYTES;
+    static constexpr int STAGES_FIT = (kSmemLimit - FIXED) / STAGE_BYTES;
+    static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+    static constexpr int SMEM_BYTES = FIXED + STAGES * STAGE_BYTES;
+    static constexpr uint32_t TMEM_COLS = SWAP ? 4 * BT : 512;
+    static constexpr int TBUF_COLS = SWAP ? 2 * BT : 256;
+    static constexpr int MAX_NKB = SWAP ? AS_TILE_BYTES / (4 * BT) : 1 << 20;
+    static_assert(STAGES >= 3, "pipeline too shallow");
+    static_assert(SMEM_BYTES <= kSmemLimit, "shared memory budget");
+    static_assert(STAGE_BYTES % 1024 == 0 && A_OFF % 1024 == 0 && B_OFF % 1024 == 0,
+                  "operand tiles must be 1024-byte aligned for the 128-byte swizzle");
+};
+
+struct KParams {
+    int R, N, K, E, nkb;
+    const float* a_scale;
+    long long as_row, as_kb;
+    const float* b_scale;
+    const int32_t* m_indptr;
+    uint8_t* hq;
+    float* hs;
+    const int32_t* perm;
+    const float* topk_w;
+    int topk;
+    float* out_acc;
+    int out_ld;
+    __nv_bfloat16* out_bf16;
+    int* status;
+    unsigned long long timeout_ns;
+};
+
+struct Smem {
+    uint8_t* stages;
+    float* as_tile;
+    int* tstart;  // [E+1] first tile of each expert
+    int* mind;    // [E+1] clamped m_indptr
+    float* xch;   // epilogue exchange area
+    uint64_t* full;
+    uint64_t* empty;
+    uint64_t* tfull;
+    uint64_t* tempty;
+    uint64_t* drain;
+    uint64_t* epi;
+    uint32_t* tmem;
+    volatile int* abort;
+};
+
+template <int BT>
+__device__ __forceinline__ Smem carve(uint8_t* base) {
+    using C = Cfg<BT>;
+    Smem s;
+    uint8_t* p = base;
+    s.stages = p;
+    p += C::STAGES * C::STAGE_BYTES;
+    s.as_tile = reinterpret_cast<float*>(p);
+    p += C::AS_TILE_BYTES;
+    s.tstart = reinterpret_cast<int*>(p);
+    s.mind = s.tstart + (kMaxE + 1);
+    p += kTableBytes;
+    s.xch = reinterpret_cast<float*>(p);
+    p += C::XCH_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(p);
+    s.full = bars;
+    s.empty = bars + 8;
+    s.tfull = bars + 16;
+    s.tempty = bars + 18;
+    s.drain = bars + 20;
+    s.epi = bars + 21;
+    s.tmem = reinterpret_cast<uint32_t*>(bars + 22);
+    s.abort = reinterpret_cast<volatile int*>(bars + 23);
+    return s;
+}
+
+struct Tile {
+    int e, mt, nt, row0, rows;
+};
+
+template <int BT>
+__device__ __forceinline__ Tile decode_tile(int t, const Smem& s, int E) {
+    int lo = 0, hi = E;  // tstart[lo] <= t < tstart[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s.tstart[mid] <= t) lo = mid; else hi = mid;
+    }
+    Tile r;
+    r.e = lo;
+    const int local = t - s.tstart[lo];
+    const int me = max(0, s.mind[lo + 1] - s.mind[lo]);
+    const int mtiles = (me + BT - 1) / BT;
+    r.nt = local / mtiles;
+    r.mt = local - r.nt * mtiles;
+    r.row0 = s.mind[lo] + r.mt * BT;
+    r.rows = min(BT, me - r.mt * BT);
+    return r;
+}
+
+// Weight-tile geometry of a tile: global B rows of the two 128-row boxes and
+// the scale-block indices (into b_scale viewed as [E * N/128, nkb]).
+struct WTile {
+    int wrow0, wrow1;
+    int sb0, sb1;
+    bool v1;  // second block exists (plain tiles may end on an odd block)
+};
+
+template <bool GATED>
+__device__ __forceinline__ WTile weight_tile(const Tile& t, int N) {
+    WTile w;
+    const int nblk = N >> 7;
+    if (GATED) {
+        w.wrow0 = t.e * N + t.nt * 128;
+        w.wrow1 = t.e * N + (N >> 1) + t.nt * 128;
+        w.sb0 = t.e * nblk + t.nt;
+        w.sb1 = t.e * nblk + (nblk >> 1) + t.nt;
+        w.v1 = true;
+    } else {
+        w.wrow0 = t.e * N + t.nt * 256;
+        w.wrow1 = w.wrow0 + 128;
+        w.sb0 = t.e * nblk + 2 * t.nt;
+        w.v1 = (2 * t.nt + 1) < nblk;
+        w.sb1 = w.v1 ? w.sb0 + 1 : w.sb0;
+    }
+    return w;
+}
+
+__device__ __forceinline__ float silu_f(float z) {
+    return __fdiv_rn(z, 1.0f + expf(-z));
+}
+
+// Wait of a whole epilogue warp: every lane waits, and the warp proceeds only
+// if every lane succeeded, so warp-collective tcgen05.ld never diverges.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& wc,
+                                          int where) {
+    const bool ok = wait_bar(bar, parity, wc, where);
+    return __all_sync(0xffffffffu, ok) != 0;
+}
+
+__device__ __forceinline__ bool epi_sync(const Smem& s, uint32_t& phase, const WaitCtl& wc) {
+    mbar_arrive(s.epi);
+    const bool ok = warp_wait(s.epi, phase, wc, 7);
+    phase ^= 1;
+    return ok;
+}
+
+template <int BT>
+__device__ __forceinline__ void tmem_load_cols(uint32_t taddr, float (&v)[BT]) {
+    if constexpr (BT == 16) {
+        tmem_ld16(taddr, v);
+    } else if constexpr (BT == 32) {
+        tmem_ld32(taddr, v);
+    } else {
+        float* lo = v;
+        float* hi = v + 32;
+        tmem_ld32(taddr, *reinterpret_cast<float(*)[32]>(lo));
+        tmem_ld32(taddr + 32, *reinterpret_cast<float(*)[32]>(hi));
+    }
+}
+
+// ---------------------------------------------------------------- roles
+template <int BT, bool GATED>
+__device__ void producer_role(const CUtensorMap* tmA, const CUtensorMap* tmB, const KParams& p,
+                              const Smem& s, const WaitCtl& wc) {
+    using C = Cfg<BT>;
+    uint32_t stage = 0, phase = 0, armed = 0, armed_par = 0;
+    const int total = s.tstart[p.E];
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const Tile tl = decode_tile<BT>(t, s, p.E);
+        const WTile wt = weight_tile<GATED>(tl, p.N);
+        for (int kb = 0; kb < p.nkb; ++kb) {
+            if (!wait_bar(&s.empty[stage], phase ^ 1, wc, 1)) { ok = false; break; }
+            uint8_t* st = s.stages + stage * C::STAGE_BYTES;
+            mbar_arrive_expect_tx(&s.full[stage], C::STAGE_BYTES);
+            tma_load_2d(st + C::A_OFF, tmA, &s.full[stage], kb * 128, tl.row0);
+            tma_load_2d(st + C::B_OFF, tmB, &s.full[stage], kb * 128, wt.wrow0);
+            tma_load_2d(st + C::B_OFF + 16384, tmB, &s.full[stage], kb * 128, wt.wrow1);
+            armed |= 1u << stage;
+            armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+            if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        }
+    }
+    // make sure no copy is still writing into shared memory when the CTA exits
+    for (int st = 0; st < C::STAGES; ++st)
+        if ((armed >> st) & 1u) wait_bar(&s.full[st], (armed_par >> st) & 1u, wc, 2, /*drain=*/true);
+}
+
+template <int BT>
+__device__ void mma_role(const KParams& p, const Smem& s, const WaitCtl& wc, uint32_t tmem_base) {
+    using C = Cfg<BT>;
+    constexpr uint32_t idesc = C::SWAP ? idesc_e4m3_f32(128, BT) : idesc_e4m3_f32(128, 256);
+    uint32_t stage = 0, phase = 0, buf = 0, bphase = 0;
+    const int total = s.tstart[p.E];
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        for (int kb = 0; kb < p.nkb; ++kb) {
+            if (!wait_bar(&s.tempty[buf], bphase ^ 1, wc, 3)) { ok = false; break; }
+            if (!wait_bar(&s.full[stage], phase, wc, 4)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(s.stages + stage * C::STAGE_BYTES + C::A_OFF);
+            const uint32_t sb = smem_u32(s.stages + stage * C::STAGE_BYTES + C::B_OFF);
+            const uint32_t d = tmem_base + buf * C::TBUF_COLS;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                if constexpr (C::SWAP) {
+                    umma_f8(d, smem_desc_k_sw128(sb + kk * 32), smem_desc_k_sw128(sa + kk * 32),
+                            idesc, kk);
+                    umma_f8(d + BT, smem_desc_k_sw128(sb + 16384 + kk * 32),
+                            smem_desc_k_sw128(sa + kk * 32), idesc, kk);
+                } else {
+                    umma_f8(d, smem_desc_k_sw128(sa + kk * 32), smem_desc_k_sw128(sb + kk * 32),
+                            idesc, kk);
+                }
+            }
+            umma_commit(&s.empty[stage]);
+            umma_commit(&s.tfull[buf]);
+            if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+            buf ^= 1;
+            if (buf == 0) bphase ^= 1;
+        }
+    }
+    // every MMA this thread issued must be complete before TMEM is freed
+    umma_commit(s.drain);
+    wait_bar(s.drain, 0, wc, 5, /*drain=*/true);
+}
+
+__device__ __forceinline__ float a_scale_at(const KParams& p, int row, int kb) {
+    return p.a_scale[static_cast<long long>(row) * p.as_row + static_cast<long long>(kb) * p.as_kb];
+}
+
+// Direct orientation epilogue: thread = one token row, 128 of 256 columns.
+template <int EPI>
+__device__ void epilogue_direct(const KParams& p, const Smem& s, const WaitCtl& wc,
+                                uint32_t tmem_base) {
+    constexpr bool GATED = (EPI == EPI_SWIGLU_BF16 || EPI == EPI_SWIGLU_QUANT);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = warp & 3;          // TMEM lane quarter this warp may access
+    const int g = (warp - 4) >> 2;   // column half
+    const int rl = q * 32 + lane;    // row inside the tile
+    // columns of the two 64-wide groups this thread accumulates
+    const int colA = GATED ? g * 64 : g * 128;
+    const int colB = GATED ? 128 + g * 64 : g * 128 + 64;
+    uint32_t buf = 0, bphase = 0, ephase = 0;
+    const int total = s.tstart[p.E];
+    const int nkb = p.nkb;
+    float acc[128];
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+        const Tile tl = decode_tile<128>(t, s, p.E);
+        const WTile wt = weight_tile<GATED>(tl, p.N);
+        const bool row_ok = rl < tl.rows;
+        const int row = tl.row0 + rl;
+        // scale block of each column group
+        const int sbA = GATED ? wt.sb0 : (g == 0 ? wt.sb0 : wt.sb1);
+        const int sbB = GATED ? wt.sb1 : sbA;
+        const bool cols_ok = GATED ? true : (g == 0 ? true : wt.v1);
+        const float* bsA = p.b_scale + static_cast<long long>(sbA) * nkb;
+        const float* bsB = p.b_scale + static_cast<long long>(sbB) * nkb;
+#pragma unroll
+        for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+        float sa_n = row_ok ? a_scale_at(p, row, 0) : 0.0f;
+        float ba_n = bsA[0], bb_n = bsB[0];
+        for (int kb = 0; kb < nkb; ++kb) {
+            const float fA = sa_n * ba_n;
+            const float fB = sa_n * bb_n;
+            if (kb + 1 < nkb) {
+                sa_n = row_ok ? a_scale_at(p, row, kb + 1) : 0.0f;
+                ba_n = bsA[kb + 1];
+                bb_n = bsB[kb + 1];
+            }
+            if (!warp_wait(&s.tfull[buf], bphase, wc, 6)) return;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * 256;
+            float v[32];
+            tmem_ld32(taddr + colA, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc[i] = fmaf(v[i], fA, acc[i]);
+            tmem_ld32(taddr + colA + 32, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc[32 + i] = fmaf(v[i], fA, acc[32 + i]);
+            tmem_ld32(taddr + colB, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc[64 + i] = fmaf(v[i], fB, acc[64 + i]);
+            tmem_ld32(taddr + colB + 32, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc[96 + i] = fmaf(v[i], fB, acc[96 + i]);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.tempty[buf]);
+            buf ^= 1;
+            if (buf == 0) bphase ^= 1;
+        }
+
+        if constexpr (EPI == EPI_SWIGLU_QUANT) {
+            float amax = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+                const float h = silu_f(acc[j]) * acc[64 + j];
+                acc[j] = h;
+                amax = fmaxf(amax, fabsf(h));
+            }
+            s.xch[g * 128 + rl] = amax;
+            if (!epi_sync(s, ephase, wc)) return;
+            amax = fmaxf(s.xch[rl], s.xch[128 + rl]);
+            const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+            if (row_ok) {
+                const int ldh = p.N >> 1;
+                uint4* dst = reinterpret_cast<uint4*>(p.hq + static_cast<long long>(row) * ldh +
+                                                      tl.nt * 128 + g * 64);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint4 w;
+                    w.x = cvt_e4m3x4(__fdiv_rn(acc[16 * c + 0], sc), __fdiv_rn(acc[16 * c + 1], sc),
+                                     __fdiv_rn(acc[16 * c + 2], sc), __fdiv_rn(acc[16 * c + 3], sc));
+                    w.y = cvt_e4m3x4(__fdiv_rn(acc[16 * c + 4], sc), __fdiv_rn(acc[16 * c + 5], sc),
+                                     __fdiv_rn(acc[16 * c + 6], sc), __fdiv_rn(acc[16 * c + 7], sc));
+                    w.z = cvt_e4m3x4(__fdiv_rn(acc[16 * c + 8], sc), __fdiv_rn(acc[16 * c + 9], sc),
+                                     __fdiv_rn(acc[16 * c + 10], sc), __fdiv_rn(acc[16 * c + 11], sc));
+                    w.w = cvt_e4m3x4(__fdiv_rn(acc[16 * c + 12], sc), __fdiv_rn(acc[16 * c + 13], sc),
+                                     __fdiv_rn(acc[16 * c + 14], sc), __fdiv_rn(acc[16 * c + 15], sc));
+                    dst[c] = w;
+                }
+                if (g == 0) p.hs[static_cast<long long>(tl.nt) * p.R + row] = sc;
+            }
+            if (!epi_sync(s, ephase, wc)) return;
+        } else if constexpr (EPI == EPI_COMBINE) {
+            if (row_ok && cols_ok) {
+                const int pair = p.perm[row];
+                const int tok = pair / p.topk;
+                const float w = p.topk_w[pair];
+                float* dst = p.out_acc + static_cast<long long>(tok) * p.out_ld + tl.nt * 256 + g * 128;
+#pragma unroll
+                for (int j = 0; j < 128; j += 4)
+                    red_add_v4(dst + j, w * acc[j], w * acc[j + 1], w * acc[j + 2], w * acc[j + 3]);
+            }
+        } else if constexpr (EPI == EPI_BF16) {
+            if (row_ok && cols_ok) {
+                uint4* dst = reinterpret_cast<uint4*>(p.out_bf16 + static_cast<long long>(row) * p.N +
+                                                      tl.nt * 256 + g * 128);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    uint4 w;
+                    __nv_bfloat162 b0 = __floats2bfloat162_rn(acc[8 * c + 0], acc[8 * c + 1]);
+                    __nv_bfloat162 b1 = __floats2bfloat162_rn(acc[8 * c + 2], acc[8 * c + 3]);
+                    __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[8 * c + 4], acc[8 * c + 5]);
+                    __nv_bfloat162 b3 = __floats2bfloat162_rn(acc[8 * c + 6], acc[8 * c + 7]);
+                    memcpy(&w.x, &b0, 4); memcpy(&w.y, &b1, 4);
+                    memcpy(&w.z, &b2, 4); memcpy(&w.w, &b3, 4);
+                    dst[c] = w;
+                }
+            }
+        } else {  // EPI_SWIGLU_BF16
+            if (row_ok) {
+                const int ldo = p.N >> 1;
+                uint4* dst = reinterpret_cast<uint4*>(p.out_bf16 + static_cast<long long>(row) * ldo +
+                                                      tl.nt * 128 + g * 64);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    float h[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) h[i] = silu_f(acc[8 * c + i]) * acc[64 + 8 * c + i];
+                    uint4 w;
+                    __nv_bfloat162 b0 = __floats2bfloat162_rn(h[0], h[1]);
+                    __nv_bfloat162 b1 = __floats2bfloat162_rn(h[2], h[3]);
+                    __nv_bfloat162 b2 = __floats2bfloat162_rn(h[4], h[5]);
+                    __nv_bfloat162 b3 = __floats2bfloat162_rn(h[6], h[7]);
+                    memcpy(&w.x, &b0, 4); memcpy(&w.y, &b1, 4);
+                    memcpy(&w.z, &b2, 4); memcpy(&w.w, &b3, 4);
+                    dst[c] = w;
+                }
+            }
+        }
+    }
+}
+
+// Swapped orientation epilogue: thread = one weight row of each 128-row
+// block, BT token columns per block.
+template <int BT, int EPI>
+__device__ void epilogue_swap(const KParams& p, const Smem& s, const WaitCtl& wc,
+                              uint32_t tmem_base) {
+    constexpr bool GATED = (EPI == EPI_SWIGLU_BF16 || EPI == EPI_SWIGLU_QUANT);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = warp & 3;
+    const int w = q * 32 + lane;          // weight row inside each block
+    const int et = threadIdx.x - 128;     // epilogue thread index 0..127
+    uint32_t buf = 0, bphase = 0, ephase = 0;
+    const int total = s.tstart[p.E];
+    const int nkb = p.nkb;
+    int* s_tok = reinterpret_cast<int*>(s.xch + 4 * BT);
+    float* s_wt = s.xch + 5 * BT;
+    float acc0[BT], acc1[BT];
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+        const Tile tl = decode_tile<BT>(t, s, p.E);
+        const WTile wt = weight_tile<GATED>(tl, p.N);
+        // stage this tile's activation scales (and combine metadata)
+        if (!epi_sync(s, ephase, wc)) return;
+        for (int idx = et; idx < nkb * BT; idx += 128) {
+            const int kb = idx / BT, j = idx - kb * BT;
+            s.as_tile[idx] = (j < tl.rows) ? a_scale_at(p, tl.row0 + j, kb) : 0.0f;
+        }
+        if constexpr (EPI == EPI_COMBINE) {
+            if (et < BT) {
+                int tok = 0;
+                float wgt = 0.0f;
+                if (et < tl.rows) {
+                    const int pair = p.perm[tl.row0 + et];
+                    tok = pair / p.topk;
+                    wgt = p.topk_w[pair];
+                }
+                s_tok[et] = tok;
+                s_wt[et] = wgt;
+            }
+        }
+        if (!epi_sync(s, ephase, wc)) return;
+        const float* bs0 = p.b_scale + static_cast<long long>(wt.sb0) * nkb;
+        const float* bs1 = p.b_scale + static_cast<long long>(wt.sb1) * nkb;
+#pragma unroll
+        for (int j = 0; j < BT; ++j) { acc0[j] = 0.0f; acc1[j] = 0.0f; }
+        float b0n = bs0[0], b1n = bs1[0];
+        for (int kb = 0; kb < nkb; ++kb) {
+            const float b0 = b0n, b1 = b1n;
+            if (kb + 1 < nkb) { b0n = bs0[kb + 1]; b1n = bs1[kb + 1]; }
+            if (!warp_wait(&s.tfull[buf], bphase, wc, 6)) return;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * (2 * BT);
+            const float4* asv = reinterpret_cast<const float4*>(s.as_tile + kb * BT);
+            float v[BT];
+            tmem_load_cols<BT>(taddr, v);
+#pragma unroll
+            for (int j4 = 0; j4 < BT / 4; ++j4) {
+                const float4 a4 = asv[j4];
+                acc0[4 * j4 + 0] = fmaf(v[4 * j4 + 0], a4.x * b0, acc0[4 * j4 + 0]);
+                acc0[4 * j4 + 1] = fmaf(v[4 * j4 + 1], a4.y * b0, acc0[4 * j4 + 1]);
+                acc0[4 * j4 + 2] = fmaf(v[4 * j4 + 2], a4.z * b0, acc0[4 * j4 + 2]);
+                acc0[4 * j4 + 3] = fmaf(v[4 * j4 + 3], a4.w * b0, acc0[4 * j4 + 3]);
+            }
+            tmem_load_cols<BT>(taddr + BT, v);
+#pragma unroll
+            for (int j4 = 0; j4 < BT / 4; ++j4) {
+                const float4 a4 = asv[j4];
+                acc1[4 * j4 + 0] = fmaf(v[4 * j4 + 0], a4.x * b1, acc1[4 * j4 + 0]);
+                acc1[4 * j4 + 1] = fmaf(v[4 * j4 + 1], a4.y * b1, acc1[4 * j4 + 1]);
+                acc1[4 * j4 + 2] = fmaf(v[4 * j4 + 2], a4.z * b1, acc1[4 * j4 + 2]);
+                acc1[4 * j4 + 3] = fmaf(v[4 * j4 + 3], a4.w * b1, acc1[4 * j4 + 3]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.tempty[buf]);
+            buf ^= 1;
+            if (buf == 0) bphase ^= 1;
+        }
+
+        if constexpr (EPI == EPI_SWIGLU_QUANT) {
+            float* red = s.xch;  // [4 warps][BT] per-token partial amax
+#pragma unroll
+            for (int j = 0; j < BT; ++j) {
+                const float h = silu_f(acc0[j]) * acc1[j];
+                acc0[j] = h;
+                float m = fabsf(h);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                if (lane == 0) red[q * BT + j] = m;
+            }
+            if (!epi_sync(s, ephase, wc)) return;
+            const int ldh = p.N >> 1;
+            const int col = tl.nt * 128 + w;
+#pragma unroll
+            for (int j = 0; j < BT; ++j) {
+                if (j < tl.rows) {
+                    const float amax = fmaxf(fmaxf(red[j], red[BT + j]), fmaxf(red[2 * BT + j], red[3 * BT + j]));
+                    const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+                    const float x = __fdiv_rn(acc0[j], sc);
+                    p.hq[static_cast<long long>(tl.row0 + j) * ldh + col] =
+                        static_cast<uint8_t>(cvt_e4m3x2(x, 0.0f) & 0xFF);
+                    if (w == j) p.hs[static_cast<long long>(tl.nt) * p.R + tl.row0 + j] = sc;
+                }
+            }
+        } else if constexpr (EPI == EPI_COMBINE) {
+            const int colA = tl.nt * 256 + w;
+            const int colB = colA + 128;
+#pragma unroll
+            for (int j = 0; j < BT; ++j) {
+                if (j < tl.rows) {
+                    float* rowp = p.out_acc + static_cast<long long>(s_tok[j]) * p.out_ld;
+                    const float wgt = s_wt[j];
+                    red_add(rowp + colA, wgt * acc0[j]);
+                    if (wt.v1) red_add(rowp + colB, wgt * acc1[j]);
+                }
+            }
+        } else if constexpr (EPI == EPI_BF16) {
+            const int colA = tl.nt * 256 + w;
+#pragma unroll
+            for (int j = 0; j < BT; ++j) {
+                if (j < tl.rows) {
+                    __nv_bfloat16* rowp = p.out_bf16 + static_cast<long long>(tl.row0 + j) * p.N;
+                    rowp[colA] = __float2bfloat16_rn(acc0[j]);
+                    if (wt.v1) rowp[colA + 128] = __float2bfloat16_rn(acc1[j]);
+                }
+            }
+        } else {  // EPI_SWIGLU_BF16
+            const int ldo = p.N >> 1;
+            const int col = tl.nt * 128 + w;
+#pragma unroll
+            for (int j = 0; j < BT; ++j) {
+                if (j < tl.rows)
+                    p.out_bf16[static_cast<long long>(tl.row0 + j) * ldo + col] =
+                        __float2bfloat16_rn(silu_f(acc0[j]) * acc1[j]);
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------- kernel
+template <int BT, int EPI>
+__global__ void __launch_bounds__(Cfg<BT>::THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB, const KParams p) {
+    using C = Cfg<BT>;
+    constexpr bool GATED = (EPI == EPI_SWIGLU_BF16 || EPI == EPI_SWIGLU_QUANT);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const Smem s = carve<BT>(base);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::STAGES; ++i) {
+            mbar_init(&s.full[i], 1);
+            mbar_init(&s.empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s.tfull[i], 1);
+            mbar_init(&s.tempty[i], C::EPI_WARPS);
+        }
+        mbar_init(s.drain, 1);
+        mbar_init(s.epi, C::EPI_THREADS);
+        *s.abort = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(s.tmem, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == 2) {
+        // per-expert tile table: tiles of expert e = ceil(rows_e / BT) * n_tiles
+        const int E = p.E;
+        const int ntn = GATED ? (p.N >> 8) : ((p.N + 255) >> 8);
+        const int per = (E + 31) >> 5;
+        const int lo = min(E, lane * per), hi = min(E, lo + per);
+        int sum = 0;
+        for (int e = lo; e < hi; ++e) {
+            const int m0 = min(max(p.m_indptr[e], 0), p.R);
+            const int m1 = min(max(p.m_indptr[e + 1], 0), p.R);
+            s.mind[e] = m0;
+            sum += ((max(0, m1 - m0) + BT - 1) / BT) * ntn;
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - sum;
+        for (int e = lo; e < hi; ++e) {
+            s.tstart[e] = run;
+            const int m0 = s.mind[e];
+            const int m1 = min(max(p.m_indptr[e + 1], 0), p.R);
+            run += ((max(0, m1 - m0) + BT - 1) / BT) * ntn;
+        }
+        if (lane == 31) {
+            s.tstart[E] = incl;
+            s.mind[E] = min(max(p.m_indptr[E], 0), p.R);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *s.tmem;
+    const WaitCtl wc{s.abort, p.status, p.timeout_ns};
+
+    if (warp < 4) {
+        if constexpr (!C::SWAP) setmaxnreg_dec<kDirectLowRegs>();
+        if (warp == 0 && lane == 0) producer_role<BT, GATED>(&tmA, &tmB, p, s, wc);
+        else if (warp == 1 && lane == 0) mma_role<BT>(p, s, wc, tmem_base);
+    } else {
+        if constexpr (!C::SWAP) {
+            setmaxnreg_inc<kDirectHighRegs>();
+            epilogue_direct<EPI>(p, s, wc, tmem_base);
+        } else {
+            epilogue_swap<BT, EPI>(p, s, wc, tmem_base);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+}
+
+// ---------------------------------------------------------------- host side
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// Descriptor cache keyed by (address, rows, row bytes, box rows): repeated
+// calls on the same weights reuse the encoded TMA descriptor.
+struct MapKey {
+    const void* ptr;
+    long long rows, cols;
+    int box_rows;
+    bool operator==(const MapKey& o) const {
+        return ptr == o.ptr && rows == o.rows && cols == o.cols && box_rows == o.box_rows;
+    }
+};
+struct MapEntry {
+    MapKey key;
+    CUtensorMap map;
+    bool used;
+};
+constexpr int kMapCache = 64;
+MapEntry g_maps[kMapCache];
+int g_map_next = 0;
+std::mutex g_map_mu;
+
+// 2-D map over a row-major FP8 matrix [rows, cols] with boxes of
+// [box_rows x 128] bytes and the 128-byte swizzle; rows past the end read 0.
+bool make_map(CUtensorMap* out, const void* ptr, long long rows, long long cols, int box_rows) {
+    const MapKey key{ptr, rows, cols, box_rows};
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    for (auto& e : g_maps)
+        if (e.used && e.key == key) { *out = e.map; return true; }
+    auto fn = encode_fn();
+    if (!fn) return false;
+    CUtensorMap m;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
+    cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t es[2] = {1u, 1u};
+    CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
+                    es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return false;
+    g_maps[g_map_next] = MapEntry{key, m, true};
+    g_map_next = (g_map_next + 1) % kMapCache;
+    *out = m;
+    return true;
+}
+
+template <int BT, int EPI>
+int launch_inst(const CUtensorMap& ma, const CUtensorMap& mb, const KParams& kp, int num_sms,
+                cudaStream_t stream) {
+    using C = Cfg<BT>;
+    auto kern = grouped_gemm_kernel<BT, EPI>;
+    static int configured_dev = -1;  // per-instance one-time set-up (device 0 assumed shared)
+    static int checked = 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+            cudaSuccess)
+            return ST_CUDA;
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return ST_CUDA;
+        // the direct kernel's setmaxnreg split assumes exactly this launch size
+        checked = C::SWAP ? 1 : (fa.numRegs == kDirectLaunchRegs ? 1 : 0);
+        if (!checked)
+            fprintf(stderr, "moefp8: direct GEMM kernel has %d registers, expected %d\n", fa.numRegs,
+                    kDirectLaunchRegs);
+        configured_dev = dev;
+    }
+    if (!checked) return ST_UNSUPPORTED;
+    kern<<<num_sms, C::THREADS, C::SMEM_BYTES, stream>>>(ma, mb, kp);
+    return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
+}
+
+template <int BT>
+int launch_bt(int epi, const CUtensorMap& ma, const CUtensorMap& mb, const KParams& kp, int num_sms,
+              cudaStream_t stream) {
+    switch (epi) {
+        case EPI_BF16: return launch_inst<BT, EPI_BF16>(ma, mb, kp, num_sms, stream);
+        case EPI_SWIGLU_BF16: return launch_inst<BT, EPI_SWIGLU_BF16>(ma, mb, kp, num_sms, stream);
+        case EPI_SWIGLU_QUANT: return launch_inst<BT, EPI_SWIGLU_QUANT>(ma, mb, kp, num_sms, stream);
+        case EPI_COMBINE: return launch_inst<BT, EPI_COMBINE>(ma, mb, kp, num_sms, stream);
+        default: return ST_INVALID_ARG;
+    }
+}
+
+}  // namespace
+
+int swap_max_k(int tile_m) {
+    switch (tile_m) {
+        case 16: return Cfg<16>::MAX_NKB * 128;
+        case 32: return Cfg<32>::MAX_NKB * 128;
+        case 64: return Cfg<64>::MAX_NKB * 128;
+        default: return 1 << 30;
+    }
+}
+
+int launch_grouped_gemm(const GemmArgs& g, cudaStream_t stream) {
+    if (g.R <= 0 || g.E <= 0) return ST_OK;
+    if (g.tile_m != 128 && g.K > swap_max_k(g.tile_m)) return ST_UNSUPPORTED;
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, g.a, g.R, g.K, g.tile_m)) return ST_CUDA;
+    if (!make_map(&mb, g.b, static_cast<long long>(g.E) * g.N, g.K, 128)) return ST_CUDA;
+    KParams kp;
+    kp.R = g.R; kp.N = g.N; kp.K = g.K; kp.E = g.E; kp.nkb = g.K / 128;
+    kp.a_scale = g.a_scale; kp.as_row = g.as_row; kp.as_kb = g.as_kb;
+    kp.b_scale = g.b_scale; kp.m_indptr = g.m_indptr;
+    kp.hq = g.hq; kp.hs = g.hs;
+    kp.perm = g.perm; kp.topk_w = g.topk_w; kp.topk = g.topk > 0 ? g.topk : 1;
+    kp.out_acc = g.out_acc; kp.out_ld = g.out_ld;
+    kp.out_bf16 = static_cast<__nv_bfloat16*>(g.out_bf16);
+    kp.status = g.status;
+    kp.timeout_ns = g.timeout_ns;
+    switch (g.tile_m) {
+        case 16: return launch_bt<16>(g.epi, ma, mb, kp, g.num_sms, stream);
+        case 32: return launch_bt<32>(g.epi, ma, mb, kp, g.num_sms, stream);
+        case 64: return launch_bt<64>(g.epi, ma, mb, kp, g.num_sms, stream);
+        case 128: return launch_bt<128>(g.epi, ma, mb, kp, g.num_sms, stream);
+        default: return ST_NO_TILE_CONFIG;
+    }
+}
+
+}  // namespace moe

@@ -1,0 +1,73 @@
+// Internal host-side interface between the C ABI layer and the kernels.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace moe {
+
+// Epilogue of the grouped GEMM.
+enum Epilogue : int {
+    EPI_BF16 = 0,          // plain: out[r, n] = bf16(G)
+    EPI_SWIGLU_BF16 = 1,   // gated: out[r, i] = bf16(silu(G_gate) * G_up)
+    EPI_SWIGLU_QUANT = 2,  // gated: h = silu(G_gate) * G_up, FP8 per row per 128 cols
+    EPI_COMBINE = 3,       // plain: out_acc[token, n] += topk_w * G   (fp32 reduction)
+};
+
+struct GemmArgs {
+    // A [R, K] FP8 (grouped rows), B [E, N, K] FP8
+    const void* a;
+    const void* b;
+    int R, N, K, E;
+    // a_scale(r, kb) = a_scale[r * as_row + kb * as_kb]; b_scale [E, N/128, K/128]
+    const float* a_scale;
+    long long as_row, as_kb;
+    const float* b_scale;
+    const int32_t* m_indptr;  // [E+1]
+    int epi;
+    int tile_m;  // 16, 32, 64 (weights as the MMA M operand) or 128 (tokens as M)
+    // EPI_SWIGLU_QUANT: hq [R, N/2] codes, hs [(N/2)/128, R]
+    uint8_t* hq;
+    float* hs;
+    // EPI_COMBINE: out_acc[token * out_ld + n], token = perm[r] / topk, weight topk_w[perm[r]]
+    const int32_t* perm;
+    const float* topk_w;
+    int topk;
+    float* out_acc;
+    int out_ld;
+    // EPI_BF16 / EPI_SWIGLU_BF16
+    void* out_bf16;
+    int* status;
+    uint64_t timeout_ns;
+    int num_sms;
+};
+
+// Returns a moe_status_t value.
+int launch_grouped_gemm(const GemmArgs& g, cudaStream_t stream);
+
+// Largest K the swapped (tile_m < 128) kernels accept for a token tile.
+int swap_max_k(int tile_m);
+
+struct RouteArgs {
+    const int32_t* topk_ids;
+    int T, k, E;
+    int32_t* m_indptr;
+    int32_t* perm;
+    int32_t* inv_perm;
+    int32_t* chunk_hist;  // [nchunks, E]
+    int* status;
+};
+constexpr int kRouteChunk = 1024;
+int launch_route_permute(const RouteArgs& r, cudaStream_t stream);
+
+// x [T, H] bf16 -> xq rows inv_perm[t*k + j] of [R, H], xs [H/128, R];
+// also zeroes out_acc [T, H] when not null.
+int launch_quant_scatter(const void* x, int T, int H, int k, int R, const int32_t* inv_perm,
+                         uint8_t* xq, float* xs, float* out_acc, cudaStream_t stream);
+
+// out [n] bf16 = in [n] fp32
+int launch_f32_to_bf16(const float* in, void* out, long long n, int num_sms, cudaStream_t stream);
+
+int launch_swiglu_mxfp8(const void* in, void* out, uint8_t* scale, int M, int K, int num_sms,
+                        cudaStream_t stream);
+
+}  // namespace moe

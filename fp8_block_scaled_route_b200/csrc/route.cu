@@ -1,0 +1,140 @@
+// Routing and permutation: groups the T*k (token, slot) pairs by expert.
+//
+// The grouped layout is the m_indptr prefix array of the grouped GEMM
+// interface on the page "FlashInfer SM120 MoE GEMM 최적화: 웨이브+잔여물 비용
+// 모델 도입" (flashinfer PR #4318, "코드 분석 1."): rows of A grouped by
+// expert, m_indptr[e] the first row of expert e.  Grouping is a stable
+// counting sort on the pair id p = t*k + j, so the result is unique and
+// bit-reproducible.
+//
+// Three launches, no atomics on the output order:
+//  1. route_hist:    one 1024-pair chunk per CTA -> per-chunk expert histogram
+//  2. route_scan:    one CTA: per-expert exclusive scan over chunks, then the
+//                    exclusive scan over experts -> m_indptr and the first
+//                    output row of every (chunk, expert)
+//  3. route_scatter: one warp per chunk walks its pairs in order, 32 at a
+//                    time; lanes with the same expert are ranked with
+//                    __match_any_sync, so each pair lands at
+//                    chunk_base[e] + (earlier pairs of e in the chunk).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+__global__ void __launch_bounds__(256) route_hist(const int32_t* __restrict__ ids, int R, int E,
+                                                  int32_t* __restrict__ chunk_hist, int* status) {
+    extern __shared__ int hist[];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
+    const int base = blockIdx.x * kRouteChunk;
+    const int end = min(R, base + kRouteChunk);
+    int bad = 0;
+    for (int p = base + threadIdx.x; p < end; p += blockDim.x) {
+        const int e = ids[p];
+        if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+        else ++bad;
+    }
+    if (bad) {
+        atomicAdd(&status[2], bad);
+        report_error(status, ST_BAD_EXPERT_ID, 0);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+        chunk_hist[static_cast<long long>(blockIdx.x) * E + e] = hist[e];
+}
+
+// blockDim.x = 1024 >= E
+__global__ void __launch_bounds__(1024) route_scan(int nchunks, int E, int32_t* __restrict__ chunk_hist,
+                                                   int32_t* __restrict__ m_indptr) {
+    __shared__ int warp_tot[32];
+    const int e = threadIdx.x;
+    int count = 0;
+    if (e < E) {
+        for (int c = 0; c < nchunks; ++c) {
+            const long long i = static_cast<long long>(c) * E + e;
+            const int h = chunk_hist[i];
+            chunk_hist[i] = count;  // rows of e in earlier chunks
+            count += h;
+        }
+    }
+    // exclusive scan of count over experts
+    const int lane = e & 31, w = e >> 5;
+    int incl = count;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) warp_tot[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+        int t = warp_tot[lane];
+        int ti = t;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, ti, o);
+            if (lane >= o) ti += v;
+        }
+        warp_tot[lane] = ti - t;  // exclusive prefix of warp totals
+    }
+    __syncthreads();
+    const int excl = warp_tot[w] + incl - count;
+    if (e < E) {
+        m_indptr[e] = excl;
+        for (int c = 0; c < nchunks; ++c) chunk_hist[static_cast<long long>(c) * E + e] += excl;
+    }
+    if (e == E - 1) m_indptr[E] = excl + count;
+}
+
+// blockDim.x = 32: one warp per chunk
+__global__ void __launch_bounds__(32) route_scatter(const int32_t* __restrict__ ids, int R, int E,
+                                                    const int32_t* __restrict__ chunk_base,
+                                                    int32_t* __restrict__ perm,
+                                                    int32_t* __restrict__ inv_perm) {
+    extern __shared__ int cursor[];
+    const int lane = threadIdx.x;
+    for (int e = lane; e < E; e += 32)
+        cursor[e] = chunk_base[static_cast<long long>(blockIdx.x) * E + e];
+    __syncwarp();
+    const int base = blockIdx.x * kRouteChunk;
+    const int end = min(R, base + kRouteChunk);
+    for (int p0 = base; p0 < end; p0 += 32) {
+        const int p = p0 + lane;
+        const bool live = p < end;
+        const int e = live ? ids[p] : -1;
+        const bool ok = live && e >= 0 && e < E;
+        const unsigned peers = __match_any_sync(0xffffffffu, ok ? e : -1);
+        const int rank = __popc(peers & ((1u << lane) - 1u));
+        const int first = cursor[ok ? e : 0];
+        __syncwarp();
+        if (ok) {
+            const int row = first + rank;
+            perm[row] = p;
+            if (inv_perm) inv_perm[p] = row;
+            if (rank == 0) cursor[e] = first + __popc(peers);
+        } else if (live && inv_perm) {
+            inv_perm[p] = -1;
+        }
+        __syncwarp();
+    }
+}
+
+int launch_route_permute(const RouteArgs& r, cudaStream_t stream) {
+    const int R = r.T * r.k;
+    const int nchunks = (R + kRouteChunk - 1) / kRouteChunk;
+    const size_t hist_smem = static_cast<size_t>(r.E) * sizeof(int);
+    if (nchunks > 0) {
+        route_hist<<<nchunks, 256, hist_smem, stream>>>(r.topk_ids, R, r.E, r.chunk_hist, r.status);
+        if (cudaGetLastError() != cudaSuccess) return ST_CUDA;
+    }
+    route_scan<<<1, 1024, 0, stream>>>(nchunks, r.E, r.chunk_hist, r.m_indptr);
+    if (cudaGetLastError() != cudaSuccess) return ST_CUDA;
+    if (nchunks > 0) {
+        route_scatter<<<nchunks, 32, hist_smem, stream>>>(r.topk_ids, R, r.E, r.chunk_hist, r.perm,
+                                                          r.inv_perm);
+        if (cudaGetLastError() != cudaSuccess) return ST_CUDA;
+    }
+    return ST_OK;
+}
+
+}  // namespace moe

@@ -1,0 +1,216 @@
+/*
+ * moefp8.h - C ABI of the sm_100a (B200) fused W8A8 block-scaled MoE library.
+ *
+ * The operation is the Mixture-of-Experts expert computation described on
+ * the page "FlashInfer: Blackwell W8A8 AlphaMoE Expert 계산 커널 퓨전으로 성능
+ * 비약적 향상" (flashinfer PR #4287), section "문제점: MoE Expert 계산의 병목":
+ *   (1) GEMM1 gate/up projection, (2) SwiGLU, (3) FP8 requantisation of the
+ *   intermediate, (4) GEMM2 down projection, (5) combine,
+ * preceded by grouping the (token, slot) pairs by expert.  The grouped GEMM
+ * interface (m_indptr, per-block fp32 scales with explicit granularities,
+ * scale_major_mode, is_gated, tactic tile sizes with -1 = automatic) follows
+ * the page "FlashInfer SM120 MoE GEMM 최적화: 웨이브+잔여물 비용 모델 도입"
+ * (flashinfer PR #4318), "코드 분석 1." and "2.".
+ *
+ * Conventions for every entry point:
+ *  - Pointers named as device buffers are device pointers owned by the
+ *    caller; the library never allocates, frees or keeps them.  Buffers must
+ *    be 16-byte aligned; row pitches are the dense row lengths given.
+ *  - Every call is asynchronous on `stream` (NULL = legacy default stream)
+ *    and returns a moe_status_t that reflects host-side validation and
+ *    launch errors only.  Errors detected on the device (a bounded wait that
+ *    ran out, an expert id outside [0,E)) are written to a status word and
+ *    read back with moe_get_device_status().
+ *  - FP8 means OCP E4M3 "FN" (bias 7, max 448, no infinities), one byte per
+ *    value.  bf16 is passed as 2-byte words.  Matrices are row-major.
+ *  - Block scales are fp32.  Activation scales cover 1 row x 128 columns;
+ *    weight scales cover 128 rows x 128 columns.  H, I, K and N must be
+ *    multiples of 128.
+ *  - Device requirement: compute capability 10.0 (sm_100a).
+ */
+#ifndef MOEFP8_H
+#define MOEFP8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,     /* null pointer, bad size, misaligned pointer, k > E */
+    MOE_ERR_UNSUPPORTED = 2,     /* granularity other than (1,128,128), device not sm_100, size limits */
+    MOE_ERR_CUDA = 3,            /* a CUDA runtime call or launch failed */
+    MOE_ERR_NO_TILE_CONFIG = 4,  /* requested tile sizes not in the kernel menu (mirrors the
+                                    explicit error when shape filtering leaves no candidate,
+                                    cuTile backend page, flashinfer PR #4646, review section) */
+    MOE_ERR_DEVICE_TIMEOUT = 5,  /* device: a bounded pipeline wait ran out; outputs undefined */
+    MOE_ERR_BAD_EXPERT_ID = 6    /* device: a topk id outside [0, E); that pair was dropped */
+} moe_status_t;
+
+/* Maximum number of experts. */
+#define MOE_MAX_EXPERTS 1024
+
+/* Human-readable name of a status code (static string). */
+MOE_API const char* moe_status_string(int status);
+
+/* ------------------------------------------------------------------ */
+/* Routing and permutation (stage before GEMM1)                         */
+/* ------------------------------------------------------------------ */
+
+/* Workspace bytes moe_route_permute needs for T tokens, top-k, E experts. */
+MOE_API size_t moe_route_workspace_size(int T, int k, int E);
+
+/* Groups the R = T*k (token, slot) pairs by expert with a stable counting
+ * sort (pair id p = t*k + j, ascending inside each expert).
+ *  topk_ids  device int32 [T, k]  expert of each pair
+ *  m_indptr  device int32 [E+1]   out: exclusive prefix of per-expert counts
+ *  perm      device int32 [R]     out: grouped row -> pair id
+ *  inv_perm  device int32 [R]     out: pair id -> grouped row (-1 if dropped);
+ *                                  may be NULL
+ *  ws        device, >= moe_route_workspace_size(T, k, E) bytes; its first
+ *            bytes hold the device status word
+ * Ids outside [0, E) are dropped and reported as MOE_ERR_BAD_EXPERT_ID by
+ * moe_get_device_status(ws); m_indptr[E] then counts only valid pairs.
+ * Returns MOE_ERR_INVALID_ARG for T < 0, k < 1, E < 1, E > MOE_MAX_EXPERTS,
+ * null pointers or a workspace that is too small. */
+MOE_API int moe_route_permute(const int32_t* topk_ids, int T, int k, int E,
+                      int32_t* m_indptr, int32_t* perm, int32_t* inv_perm,
+                      void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* ------------------------------------------------------------------ */
+/* The fused layer                                                      */
+/* ------------------------------------------------------------------ */
+
+/* Workspace bytes moe_fp8_fused needs (routing tables, quantised
+ * activations, FP8 intermediate, fp32 combine buffer, status word). */
+MOE_API size_t moe_workspace_size(int T, int H, int I, int E, int k);
+
+/* out[t, :] = bf16( sum_j topk_w[t,j] * Down_e( requant( SwiGLU( GateUp_e(
+ *             quant(x[t, :]) ) ) ) ) ),  e = topk_ids[t, j].
+ *  x          device bf16 [T, H]
+ *  topk_ids   device int32 [T, k], distinct experts per token expected
+ *  topk_w     device fp32  [T, k]
+ *  w13        device FP8  [E, 2I, H]   rows [0,I) gate, rows [I,2I) up
+ *  w13_scale  device fp32 [E, 2I/128, H/128]
+ *  w2         device FP8  [E, H, I]
+ *  w2_scale   device fp32 [E, H/128, I/128]
+ *  out        device bf16 [T, H]
+ *  ws         device, >= moe_workspace_size(T, H, I, E, k) bytes
+ * Activations are quantised per token per 128 columns (scale = amax/448,
+ * round-to-nearest-even, saturating); the intermediate is requantised the
+ * same way per row per 128 columns; the router weight is applied after the
+ * down projection.  T = 0 is a no-op.  Returns MOE_ERR_INVALID_ARG for
+ * sizes that are not multiples of 128, k > E, null pointers, misaligned
+ * pointers or a small workspace; MOE_ERR_UNSUPPORTED for E > 1024. */
+MOE_API int moe_fp8_fused(const void* x, const int32_t* topk_ids, const float* topk_w,
+                  const void* w13, const float* w13_scale,
+                  const void* w2, const float* w2_scale,
+                  void* out, int T, int H, int I, int E, int k,
+                  void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Same as moe_fp8_fused, and also copies the routing tables and the FP8
+ * intermediate out of the workspace (all device buffers, grouped-row order):
+ *  m_indptr [E+1], perm [T*k], h_fp8 [T*k, I] codes, h_scale fp32
+ *  [I/128, T*k] (column-block major).  Any of the four may be NULL. */
+MOE_API int moe_fp8_fused_debug(const void* x, const int32_t* topk_ids, const float* topk_w,
+                        const void* w13, const float* w13_scale,
+                        const void* w2, const float* w2_scale,
+                        void* out, int T, int H, int I, int E, int k,
+                        void* ws, size_t ws_bytes, moe_stream_t stream,
+                        int32_t* m_indptr, int32_t* perm, uint8_t* h_fp8, float* h_scale);
+
+/* ------------------------------------------------------------------ */
+/* Standalone grouped FP8 GEMM ("nt": both operands K-major)            */
+/* ------------------------------------------------------------------ */
+
+/* For every expert e and grouped row r in [m_indptr[e], m_indptr[e+1]):
+ *   G[r, n] = sum_kb a_scale(r,kb) * b_scale[e, n/128, kb] * sum_{k in kb} a[r,k] * b[e,n,k]
+ *   plain  (is_gated = 0): out[r, n] = bf16(G[r, n]),            out [R, N]
+ *   gated  (is_gated = 1): out[r, i] = bf16(silu(G[r,i]) * G[r, N/2+i]), out [R, N/2]
+ *  a        device FP8 [R, K]
+ *  b        device FP8 [E, N, K]
+ *  a_scale  device fp32; scale_major_mode 0: [R, K/128] (K-major),
+ *           1: [K/128, R] (MN-major)
+ *  b_scale  device fp32 [E, N/128, K/128]
+ *  m_indptr device int32 [E+1], m_indptr[0] = 0, non-decreasing, m_indptr[E] <= R
+ *  sg_m, sg_n, sg_k  scale granularities; only (1, 128, 128) is supported
+ *  tile_m   -1 = automatic (wave+residue model), else one of 16, 32, 64, 128
+ *  tile_n   -1 = automatic, else 128 (gated) / 256 (plain): output columns per tile
+ * Rows of out outside [0, m_indptr[E]) are not written.  Gated needs an
+ * even N with N/2 a multiple of 128.  Device-side errors go to the
+ * library's own status word: read it with moe_get_device_status(NULL, ...). */
+MOE_API int fp8_groupwise_moe_gemm(const void* a, const void* b,
+                           const float* a_scale, const float* b_scale,
+                           const int32_t* m_indptr, void* out,
+                           int R, int N, int K, int E, int scale_major_mode,
+                           int sg_m, int sg_n, int sg_k, int is_gated,
+                           int tile_m, int tile_n, moe_stream_t stream);
+
+/* Host-only tile selection used when tile_m = -1 (no device access).
+ * total_rows = rows over all experts, n = weight rows per expert (2I when
+ * gated), k = reduction size.  Writes tile_m (16, 32, 64 or 128) and tile_n
+ * (output columns per tile).  Follows the wave+residue description of the
+ * page "FlashInfer SM120 MoE GEMM 최적화: 웨이브+잔여물 비용 모델 도입", "코드
+ * 분석 2." and "리뷰 피드백 반영", on the sm_100a tile menu. */
+MOE_API int moe_select_tile_m(int total_rows, int n, int k, int E, int num_sms, int is_gated,
+                      int* tile_m, int* tile_n);
+
+/* ------------------------------------------------------------------ */
+/* Standalone SwiGLU + MXFP8 quantisation                               */
+/* ------------------------------------------------------------------ */
+
+/* Page "NVIDIA R200(SM107)을 위한 SwiGLU + MXFP8 커널 최적화" (flashinfer
+ * PR #8023): v = silu(gate) * up in fp32, then per 32 consecutive outputs an
+ * E8M0 scale X = 2^s with s the smallest integer such that amax <= 448*2^s
+ * (code s+127 clamped to [0,254]; an all-zero block gets code 0) and
+ * codes RNE_sat(v / X).  Launch shape is chosen by size band: M*K < 2^20
+ * uses small 256-thread CTAs, larger sizes a grid-stride streaming launch.
+ *  in     device bf16 [M, 2K]: columns [0,K) gate, [K,2K) up
+ *  out    device FP8  [M, K]
+ *  scale  device uint8 [M, K/32] row-major E8M0 codes (not swizzled)
+ * K must be a multiple of 32; M = 0 is a no-op. */
+MOE_API int swiglu_mxfp8_quant(const void* in, void* out, uint8_t* scale, int M, int K,
+                       moe_stream_t stream);
+
+/* ------------------------------------------------------------------ */
+/* Device status                                                        */
+/* ------------------------------------------------------------------ */
+
+/* Synchronises `stream`, then returns the device status word written by the
+ * last calls that used `ws` (a moe_fp8_fused / moe_route_permute workspace),
+ * or, with ws = NULL, the library's own word used by fp8_groupwise_moe_gemm
+ * and swiglu_mxfp8_quant.  Each entry point clears its word when it starts.
+ * Returns MOE_OK, MOE_ERR_DEVICE_TIMEOUT, MOE_ERR_BAD_EXPERT_ID or
+ * MOE_ERR_CUDA (the synchronise or the read failed). */
+MOE_API int moe_get_device_status(const void* ws, moe_stream_t stream);
+
+/* Stage timing for profiling.  When `events` is non-NULL, moe_fp8_fused and
+ * moe_fp8_fused_debug record events[i] (cudaEvent_t handles created by the
+ * caller) on the call's stream: 0 before routing, 1 after routing, 2 after
+ * activation quantisation, 3 after GEMM1 (gate/up + SwiGLU + requant), 4
+ * after GEMM2 (down + combine), 5 after the bf16 conversion.  n must be 6;
+ * events = NULL switches it off.  Process-wide setting. */
+MOE_API int moe_set_stage_events(void* const* events, int n);
+
+/* Upper bound, in nanoseconds of %globaltimer, on every spin-wait inside the
+ * kernels launched by later calls from this process (default 2e9).  A wait
+ * that runs out sets MOE_ERR_DEVICE_TIMEOUT and the kernel returns early. */
+MOE_API void moe_set_wait_timeout_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOEFP8_H */
