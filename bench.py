@@ -41,6 +41,14 @@ FALLBACK_BF16_TFLOPS = 1590.0
 KERNELS_PER_LAYER = 7      # route hist/scan/scatter, quant, GEMM1, GEMM2, bf16 conversion
 
 
+# Slices of the prefill and decode workloads (same H, I, top-k and routing,
+# 32 experts) that keep a profiler capture to a couple of GB on the device.
+PROFILE_SLICES = {
+    "prefill_slice": synth.MoEConfig("prefill_slice", 1024, 7168, 2048, 32, 8, "zipf"),
+    "decode_slice": synth.MoEConfig("decode_slice", 64, 7168, 2048, 32, 8),
+}
+
+
 def workload_desc(cfg: synth.MoEConfig) -> str:
     r = "zipf(1.2)-biased routing" if cfg.routing == "zipf" else "logits ~N(0,1)"
     return (f"{cfg.name}: T={cfg.T} H={cfg.H} I={cfg.I} E={cfg.E} top-{cfg.k}, {r}, "
@@ -367,13 +375,14 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="prefill", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--workload", default="prefill",
+                    choices=sorted(synth.CONFIGS) + sorted(PROFILE_SLICES))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    cfg = synth.CONFIGS[args.workload]
+    cfg = synth.CONFIGS.get(args.workload) or PROFILE_SLICES[args.workload]
     if args.impl == "reference":
         return run_reference(args, cfg)
     return run_ours(args, cfg)
