@@ -23,7 +23,7 @@ __all__ = [
     "moe_route_permute", "moe_fp8_fused", "moe_fp8_fused_debug", "fp8_groupwise_moe_gemm",
     "swiglu_mxfp8_quant", "moe_select_tile_m", "moe_workspace_size", "moe_route_workspace_size",
     "moe_get_device_status", "moe_set_wait_timeout_ns", "moe_status_string",
-    "moe_set_stage_events",
+    "moe_set_stage_events", "moe_route_permute_noalloc",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -42,7 +42,7 @@ EXPORTS = (
     "moe_status_string", "moe_route_workspace_size", "moe_route_permute", "moe_workspace_size",
     "moe_fp8_fused", "moe_fp8_fused_debug", "fp8_groupwise_moe_gemm", "moe_select_tile_m",
     "swiglu_mxfp8_quant", "moe_get_device_status", "moe_set_wait_timeout_ns",
-    "moe_set_stage_events",
+    "moe_set_stage_events", "moe_route_permute_noalloc",
 )
 
 _lib = None
@@ -90,6 +90,8 @@ def lib():
     L.moe_get_device_status.argtypes = [P, P]
     L.moe_set_wait_timeout_ns.restype = None
     L.moe_set_wait_timeout_ns.argtypes = [U64]
+    L.moe_route_permute_noalloc.restype = I
+    L.moe_route_permute_noalloc.argtypes = [P, I, I, I, P, P, P, P]
     L.moe_set_stage_events.restype = I
     L.moe_set_stage_events.argtypes = [ctypes.POINTER(P), I]
     _lib = L
@@ -152,6 +154,17 @@ def moe_route_permute(topk_ids, E: int, m_indptr, perm, inv_perm, ws, ws_bytes=N
     st = lib().moe_route_permute(_ptr(topk_ids), T, k, E, _ptr(m_indptr), _ptr(perm),
                                  _ptr(inv_perm), _ptr(ws), ws_bytes, _stream(stream))
     return _check(st, "moe_route_permute", check)
+
+
+def moe_route_permute_noalloc(topk_ids, E: int, m_indptr, perm, inv_perm, *, T=None, k=None,
+                              stream=None, check=True) -> int:
+    """moe_route_permute without a workspace: the scratch is a device array
+    inside the library, shared by every call (T*k <= 65536)."""
+    if T is None or k is None:
+        T, k = topk_ids.shape
+    st = lib().moe_route_permute_noalloc(_ptr(topk_ids), T, k, E, _ptr(m_indptr), _ptr(perm),
+                                         _ptr(inv_perm), _stream(stream))
+    return _check(st, "moe_route_permute_noalloc", check)
 
 
 def _fused_dims(x, topk_ids, w13):

@@ -89,6 +89,23 @@ MOE_API int moe_route_permute(const int32_t* topk_ids, int T, int k, int E,
                       int32_t* m_indptr, int32_t* perm, int32_t* inv_perm,
                       void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_route_permute for callers that cannot allocate device memory or
+ * hand the library a workspace (for example code running inside a host
+ * runtime that owns every device allocation through a fixed memory plan).
+ * The method's pages have no counterpart of this entry point.
+ * Same arguments and results as moe_route_permute without ws/ws_bytes; the
+ * scratch lives in one device array inside the library (about 256 KB per
+ * GPU, held until the process exits).  Limits: T*k <= 65536 pairs and
+ * E <= MOE_MAX_EXPERTS, else MOE_ERR_INVALID_ARG.  All calls share that
+ * array: calls whose kernels overlap on the GPU race and give undefined
+ * results.  The first call on a device looks up the array's address on that
+ * device; make it before any stream capture.  Ids outside [0, E) are
+ * dropped (m_indptr[E] then counts only valid pairs) and not reported
+ * through moe_get_device_status.  Allocates nothing. */
+MOE_API int moe_route_permute_noalloc(const int32_t* topk_ids, int T, int k, int E,
+                                      int32_t* m_indptr, int32_t* perm, int32_t* inv_perm,
+                                      moe_stream_t stream);
+
 /* ------------------------------------------------------------------ */
 /* The fused layer                                                      */
 /* ------------------------------------------------------------------ */
