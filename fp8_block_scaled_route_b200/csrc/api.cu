@@ -9,7 +9,7 @@
 #include <cstdio>
 #include <mutex>
 
-#include "../../include/moefp8.h"
+#include "moefp8.h"
 #include "common.cuh"
 #include "kernels.h"
 

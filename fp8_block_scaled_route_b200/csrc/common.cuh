@@ -47,19 +47,48 @@ constexpr uint64_t kDrainTimeoutNs = 2000000000ull;
 // Returns false when the CTA is aborting or the wait ran out of time (the
 // first thread to run out records ST_DEVICE_TIMEOUT).  With `drain = true`
 // the wait ignores the abort flag and is bounded by kDrainTimeoutNs.
+// The thread sleeps in the barrier (hardware suspend, woken by the phase
+// completing) instead of spinning, and reads the clock only every 8th round,
+// so waiting warps take almost no issue slots from working ones.
+constexpr uint32_t kWaitSuspendNs = 20000;
+
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const WaitCtl& c,
                                          int where, bool drain = false) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     const uint64_t limit = drain ? kDrainTimeoutNs : c.timeout_ns;
 #pragma unroll 1
-    while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+    for (uint32_t round = 1;; ++round) {
+        if (mbar_try_wait_sleep(bar, parity, kWaitSuspendNs)) return true;
         if (!drain && *c.abort) return false;
-        if (globaltimer() - t0 > limit) {
-            *c.abort = 1;
-            report_error(c.status, ST_DEVICE_TIMEOUT, where);
-            return false;
+        if ((round & 7) == 0 || limit < 1000000ull) {
+            if (globaltimer() - t0 > limit) {
+                *c.abort = 1;
+                report_error(c.status, ST_DEVICE_TIMEOUT, where);
+                return false;
+            }
+        }
+    }
+}
+
+// Spinning variant for the single producer and MMA threads: no hardware
+// suspend, so a completed phase is seen within a few cycles; the clock is
+// read every 256th poll.
+__device__ __forceinline__ bool wait_bar_spin(uint64_t* bar, uint32_t parity, const WaitCtl& c,
+                                              int where) {
+    if (mbar_test_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    const bool short_limit = c.timeout_ns < 1000000ull;
+#pragma unroll 1
+    for (uint32_t round = 1;; ++round) {
+        if (mbar_test_wait(bar, parity)) return true;
+        if ((round & 255) == 0 || short_limit) {
+            if (*c.abort) return false;
+            if (globaltimer() - t0 > c.timeout_ns) {
+                *c.abort = 1;
+                report_error(c.status, ST_DEVICE_TIMEOUT, where);
+                return false;
+            }
         }
     }
 }

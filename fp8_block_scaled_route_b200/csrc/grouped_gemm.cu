@@ -48,6 +48,8 @@ namespace moe {
 constexpr int kSmemLimit = 232448;  // 227 KB of opt-in dynamic shared memory per CTA
 constexpr int kMaxE = 1024;
 constexpr int kTableBytes = ((2 * (kMaxE + 1) * 4) + 15) / 16 * 16;
+constexpr int kScaleSlots = 8;        // depth of the direct kernel's scale ring
+constexpr int kScaleSlotFloats = 132;  // a_scale of 128 rows, then b_scale of the two blocks
 // Register split of the direct kernel (384 threads x 168 registers at launch):
 // the producer/MMA warpgroup drops to 56, the two epilogue warpgroups rise to
 // 224:  128*56 + 256*224 = 64512 = 384*168.
@@ -70,14 +72,27 @@ struct Cfg {
     static constexpr int B_OFF = SWAP ? 0 : A_BYTES;
     static constexpr int AS_TILE_BYTES = SWAP ? 32768 : 0;  // a_scale staging [nkb][BT]
     static constexpr int XCH_BYTES = SWAP ? ((4 * BT + 2 * BT) * 4 + 15) / 16 * 16 : 2 * 128 * 4;
-    static constexpr int BAR_BYTES = 256;
-    static constexpr int FIXED = 1024 + AS_TILE_BYTES + kTableBytes + XCH_BYTES + BAR_BYTES;
+    static constexpr int SCALE_BYTES = SWAP ? 0 : kScaleSlots * kScaleSlotFloats * 4;
+    static constexpr int BAR_BYTES = 512;
+    static constexpr int FIXED =
+        1024 + AS_TILE_BYTES + SCALE_BYTES + kTableBytes + XCH_BYTES + BAR_BYTES;
     static constexpr int STAGES_FIT = (kSmemLimit - FIXED) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
     static constexpr int SMEM_BYTES = FIXED + STAGES * STAGE_BYTES;
     static constexpr uint32_t TMEM_COLS = SWAP ? 4 * BT : 512;
+    // TMEM accumulator slots: two K blocks in flight, each slot holding both
+    // 128-row weight blocks of the tile (direct: one N = 256 MMA per K step;
+    // swapped: two N = BT MMAs).
+    static constexpr int TSLOTS = 2;
     static constexpr int TBUF_COLS = SWAP ? 2 * BT : 256;
     static constexpr int MAX_NKB = SWAP ? AS_TILE_BYTES / (4 * BT) : 1 << 20;
+    // TMA boxes per stage, one per issuing producer lane: the token tile in
+    // boxes of at most 64 rows, and the 256 weight rows in four 64-row boxes.
+    // A single thread's TMA issue rate (about 40 B/clk) cannot feed the MMA;
+    // several lanes issuing in parallel can.
+    static constexpr int A_BOX_ROWS = BT < 64 ? BT : 64;
+    static constexpr int A_BOXES = BT / A_BOX_ROWS;
+    static constexpr int NBOX = A_BOXES + 4;
     static_assert(STAGES >= 3, "pipeline too shallow");
     static_assert(SMEM_BYTES <= kSmemLimit, "shared memory budget");
     static_assert(STAGE_BYTES % 1024 == 0 && A_OFF % 1024 == 0 && B_OFF % 1024 == 0,
@@ -108,12 +123,15 @@ struct Smem {
     int* tstart;  // [E+1] first tile of each expert
     int* mind;    // [E+1] clamped m_indptr
     float* xch;   // epilogue exchange area
+    float* scales;  // direct kernel: kScaleSlots x {a_scale[128], b_scale[2], pad[2]}
     uint64_t* full;
     uint64_t* empty;
     uint64_t* tfull;
     uint64_t* tempty;
     uint64_t* drain;
     uint64_t* epi;
+    uint64_t* sfull;
+    uint64_t* sempty;
     uint32_t* tmem;
     volatile int* abort;
 };
@@ -132,15 +150,19 @@ __device__ __forceinline__ Smem carve(uint8_t* base) {
     p += kTableBytes;
     s.xch = reinterpret_cast<float*>(p);
     p += C::XCH_BYTES;
+    s.scales = reinterpret_cast<float*>(p);
+    p += C::SCALE_BYTES;
     uint64_t* bars = reinterpret_cast<uint64_t*>(p);
     s.full = bars;
     s.empty = bars + 8;
     s.tfull = bars + 16;
-    s.tempty = bars + 18;
-    s.drain = bars + 20;
-    s.epi = bars + 21;
-    s.tmem = reinterpret_cast<uint32_t*>(bars + 22);
-    s.abort = reinterpret_cast<volatile int*>(bars + 23);
+    s.tempty = bars + 20;
+    s.drain = bars + 24;
+    s.epi = bars + 25;
+    s.sfull = bars + 26;
+    s.sempty = bars + 26 + kScaleSlots;
+    s.tmem = reinterpret_cast<uint32_t*>(bars + 26 + 2 * kScaleSlots);
+    s.abort = reinterpret_cast<volatile int*>(bars + 27 + 2 * kScaleSlots);
     return s;
 }
 
@@ -199,11 +221,28 @@ __device__ __forceinline__ float silu_f(float z) {
     return __fdiv_rn(z, 1.0f + expf(-z));
 }
 
+__device__ __forceinline__ float a_scale_at(const KParams& p, int row, int kb) {
+    return p.a_scale[static_cast<long long>(row) * p.as_row + static_cast<long long>(kb) * p.as_kb];
+}
+
+// silu with the hardware exp2 and reciprocal (about 2 ulp); used where the
+// result feeds a requantisation or a bf16 rounding, whose steps are 2^19 times
+// coarser.
+__device__ __forceinline__ float silu_fast(float z) {
+    return z * __frcp_rn(1.0f + __expf(-z));
+}
+
 // Wait of a whole epilogue warp: every lane waits, and the warp proceeds only
 // if every lane succeeded, so warp-collective tcgen05.ld never diverges.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& wc,
                                           int where) {
     const bool ok = wait_bar(bar, parity, wc, where);
+    return __all_sync(0xffffffffu, ok) != 0;
+}
+
+__device__ __forceinline__ bool warp_wait_spin(uint64_t* bar, uint32_t parity, const WaitCtl& wc,
+                                               int where) {
+    const bool ok = wait_bar_spin(bar, parity, wc, where);
     return __all_sync(0xffffffffu, ok) != 0;
 }
 
@@ -229,23 +268,30 @@ __device__ __forceinline__ void tmem_load_cols(uint32_t taddr, float (&v)[BT]) {
 }
 
 // ---------------------------------------------------------------- roles
+// Producer: lane l < NBOX of warp 0 issues box l of every stage.
 template <int BT, bool GATED>
 __device__ void producer_role(const CUtensorMap* tmA, const CUtensorMap* tmB, const KParams& p,
                               const Smem& s, const WaitCtl& wc) {
     using C = Cfg<BT>;
+    const int l = threadIdx.x & 31;
+    // this lane's box: which map, smem offset inside the stage, row offset, bytes
+    const bool is_a = l < C::A_BOXES;
+    const int b = l - C::A_BOXES;  // weight box 0..3: block b/2, half b%2
+    const uint32_t off = is_a ? C::A_OFF + l * C::A_BOX_ROWS * 128 : C::B_OFF + b * 64 * 128;
+    const uint32_t bytes = is_a ? C::A_BOX_ROWS * 128 : 64 * 128;
     uint32_t stage = 0, phase = 0, armed = 0, armed_par = 0;
     const int total = s.tstart[p.E];
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const Tile tl = decode_tile<BT>(t, s, p.E);
         const WTile wt = weight_tile<GATED>(tl, p.N);
+        const int row = is_a ? tl.row0 + l * C::A_BOX_ROWS
+                             : ((b >> 1) ? wt.wrow1 : wt.wrow0) + (b & 1) * 64;
         for (int kb = 0; kb < p.nkb; ++kb) {
-            if (!wait_bar(&s.empty[stage], phase ^ 1, wc, 1)) { ok = false; break; }
+            if (!wait_bar_spin(&s.empty[stage], phase ^ 1, wc, 1)) { ok = false; break; }
             uint8_t* st = s.stages + stage * C::STAGE_BYTES;
-            mbar_arrive_expect_tx(&s.full[stage], C::STAGE_BYTES);
-            tma_load_2d(st + C::A_OFF, tmA, &s.full[stage], kb * 128, tl.row0);
-            tma_load_2d(st + C::B_OFF, tmB, &s.full[stage], kb * 128, wt.wrow0);
-            tma_load_2d(st + C::B_OFF + 16384, tmB, &s.full[stage], kb * 128, wt.wrow1);
+            mbar_arrive_expect_tx(&s.full[stage], bytes);
+            tma_load_2d(st + off, is_a ? tmA : tmB, &s.full[stage], kb * 128, row);
             armed |= 1u << stage;
             armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
             if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
@@ -256,38 +302,44 @@ __device__ void producer_role(const CUtensorMap* tmA, const CUtensorMap* tmB, co
         if ((armed >> st) & 1u) wait_bar(&s.full[st], (armed_par >> st) & 1u, wc, 2, /*drain=*/true);
 }
 
+// MMA issue (one thread).  Each K block goes into TMEM slot j (two slots
+// alternate): direct = one 128 x 256 MMA per K step (both weight blocks);
+// swapped = one 128 x BT MMA per weight block per K step.
 template <int BT>
 __device__ void mma_role(const KParams& p, const Smem& s, const WaitCtl& wc, uint32_t tmem_base) {
     using C = Cfg<BT>;
     constexpr uint32_t idesc = C::SWAP ? idesc_e4m3_f32(128, BT) : idesc_e4m3_f32(128, 256);
-    uint32_t stage = 0, phase = 0, buf = 0, bphase = 0;
+    uint32_t stage = 0, phase = 0, j = 0, jphase = 0;
     const int total = s.tstart[p.E];
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         for (int kb = 0; kb < p.nkb; ++kb) {
-            if (!wait_bar(&s.tempty[buf], bphase ^ 1, wc, 3)) { ok = false; break; }
-            if (!wait_bar(&s.full[stage], phase, wc, 4)) { ok = false; break; }
+            if (!wait_bar_spin(&s.tempty[j], jphase ^ 1, wc, 3)) { ok = false; break; }
+            if (!wait_bar_spin(&s.full[stage], phase, wc, 4)) { ok = false; break; }
             tc_fence_after();
             const uint32_t sa = smem_u32(s.stages + stage * C::STAGE_BYTES + C::A_OFF);
             const uint32_t sb = smem_u32(s.stages + stage * C::STAGE_BYTES + C::B_OFF);
-            const uint32_t d = tmem_base + buf * C::TBUF_COLS;
+            const uint32_t d = tmem_base + j * C::TBUF_COLS;
+            if constexpr (C::SWAP) {
+                // weight block 0 into columns [0, BT), block 1 into [BT, 2BT)
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                if constexpr (C::SWAP) {
+                for (int kk = 0; kk < 4; ++kk) {
                     umma_f8(d, smem_desc_k_sw128(sb + kk * 32), smem_desc_k_sw128(sa + kk * 32),
                             idesc, kk);
                     umma_f8(d + BT, smem_desc_k_sw128(sb + 16384 + kk * 32),
                             smem_desc_k_sw128(sa + kk * 32), idesc, kk);
-                } else {
+                }
+            } else {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
                     umma_f8(d, smem_desc_k_sw128(sa + kk * 32), smem_desc_k_sw128(sb + kk * 32),
                             idesc, kk);
-                }
             }
             umma_commit(&s.empty[stage]);
-            umma_commit(&s.tfull[buf]);
+            umma_commit(&s.tfull[j]);
+            j ^= 1;
+            if (j == 0) jphase ^= 1;
             if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
-            buf ^= 1;
-            if (buf == 0) bphase ^= 1;
         }
     }
     // every MMA this thread issued must be complete before TMEM is freed
@@ -295,8 +347,52 @@ __device__ void mma_role(const KParams& p, const Smem& s, const WaitCtl& wc, uin
     wait_bar(s.drain, 0, wc, 5, /*drain=*/true);
 }
 
-__device__ __forceinline__ float a_scale_at(const KParams& p, int row, int kb) {
-    return p.a_scale[static_cast<long long>(row) * p.as_row + static_cast<long long>(kb) * p.as_kb];
+// Scale stager of the direct kernel (warp 2): for every K block of every
+// tile, in the pipeline's order, copies the tile's 128 activation scales of
+// that K block and the two weight-block scales into a ring of shared-memory
+// slots with cp.async; each lane's copies complete on the slot's mbarrier, so
+// the stager never waits for global memory and runs up to kScaleSlots K
+// blocks ahead of the epilogue.
+template <bool GATED>
+__device__ void scale_role(const KParams& p, const Smem& s, const WaitCtl& wc) {
+    const int lane = threadIdx.x & 31;
+    const int total = s.tstart[p.E];
+    const int nkb = p.nkb;
+    uint32_t slot = 0, sphase = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+        const Tile tl = decode_tile<128>(t, s, p.E);
+        const WTile wt = weight_tile<GATED>(tl, p.N);
+        const float* bs0 = p.b_scale + static_cast<long long>(wt.sb0) * nkb;
+        const float* bs1 = p.b_scale + static_cast<long long>(wt.sb1) * nkb;
+        for (int kb = 0; kb < nkb; ++kb) {
+            if (!wait_bar(&s.sempty[slot], sphase ^ 1, wc, 8)) return;
+            float* f = s.scales + slot * kScaleSlotFloats;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int r = lane + 32 * i;
+                const bool ok = r < tl.rows;
+                const float* src = ok ? p.a_scale + static_cast<long long>(tl.row0 + r) * p.as_row +
+                                            static_cast<long long>(kb) * p.as_kb
+                                      : p.b_scale;
+                cp_async_4(f + r, src, ok ? 4u : 0u);
+            }
+            if (lane == 0) cp_async_4(f + 128, bs0 + kb, 4u);
+            if (lane == 1) cp_async_4(f + 129, bs1 + kb, 4u);
+            cp_async_arrive_noinc(&s.sfull[slot]);
+            if (++slot == kScaleSlots) { slot = 0; sphase ^= 1; }
+        }
+    }
+    // copies still in flight land before the CTA exits
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+__device__ __forceinline__ void ffma_chunk(float2* acc, const uint32_t (&v)[32], float f) {
+    const float2 f2 = make_float2(f, f);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float2 x = make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+        acc[i] = __ffma2_rn(x, f2, acc[i]);
+    }
 }
 
 // Direct orientation epilogue: thread = one token row, 128 of 256 columns.
@@ -308,71 +404,73 @@ __device__ void epilogue_direct(const KParams& p, const Smem& s, const WaitCtl& 
     const int q = warp & 3;          // TMEM lane quarter this warp may access
     const int g = (warp - 4) >> 2;   // column half
     const int rl = q * 32 + lane;    // row inside the tile
-    // columns of the two 64-wide groups this thread accumulates
-    const int colA = GATED ? g * 64 : g * 128;
-    const int colB = GATED ? 128 + g * 64 : g * 128 + 64;
-    uint32_t buf = 0, bphase = 0, ephase = 0;
+    // Each thread accumulates 64 columns of each of the tile's two 128-row
+    // weight blocks: acc[0..63] = block 0 columns g*64.., acc[64..127] =
+    // block 1 columns g*64.. (gated: gate and up; plain: the tile's first and
+    // second 128 output columns).
+    const int colg = g * 64;
+    uint32_t tj = 0, tjphase = 0, ephase = 0, slot = 0, sphase = 0;
     const int total = s.tstart[p.E];
     const int nkb = p.nkb;
-    float acc[128];
+    float2 acc[64];
+    uint32_t va[32], vb[32];
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
         const Tile tl = decode_tile<128>(t, s, p.E);
         const WTile wt = weight_tile<GATED>(tl, p.N);
         const bool row_ok = rl < tl.rows;
         const int row = tl.row0 + rl;
-        // scale block of each column group
-        const int sbA = GATED ? wt.sb0 : (g == 0 ? wt.sb0 : wt.sb1);
-        const int sbB = GATED ? wt.sb1 : sbA;
-        const bool cols_ok = GATED ? true : (g == 0 ? true : wt.v1);
-        const float* bsA = p.b_scale + static_cast<long long>(sbA) * nkb;
-        const float* bsB = p.b_scale + static_cast<long long>(sbB) * nkb;
+        const bool v1 = GATED ? true : wt.v1;   // plain tiles may lack the second block
 #pragma unroll
-        for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
-        float sa_n = row_ok ? a_scale_at(p, row, 0) : 0.0f;
-        float ba_n = bsA[0], bb_n = bsB[0];
+        for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
+        const uint32_t tlane = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + colg;
         for (int kb = 0; kb < nkb; ++kb) {
-            const float fA = sa_n * ba_n;
-            const float fB = sa_n * bb_n;
-            if (kb + 1 < nkb) {
-                sa_n = row_ok ? a_scale_at(p, row, kb + 1) : 0.0f;
-                ba_n = bsA[kb + 1];
-                bb_n = bsB[kb + 1];
-            }
-            if (!warp_wait(&s.tfull[buf], bphase, wc, 6)) return;
+            if (!warp_wait(&s.tfull[tj], tjphase, wc, 6)) return;
             tc_fence_after();
-            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * 256;
-            float v[32];
-            tmem_ld32(taddr + colA, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) acc[i] = fmaf(v[i], fA, acc[i]);
-            tmem_ld32(taddr + colA + 32, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) acc[32 + i] = fmaf(v[i], fA, acc[32 + i]);
-            tmem_ld32(taddr + colB, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) acc[64 + i] = fmaf(v[i], fB, acc[64 + i]);
-            tmem_ld32(taddr + colB + 32, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) acc[96 + i] = fmaf(v[i], fB, acc[96 + i]);
+            const uint32_t tb = tlane + tj * 256;
+            // weight block 0 columns: two 32-column loads, one wait
+            tmem_ld32_async(tb, va);
+            tmem_ld32_async(tb + 32, vb);
+            if (!warp_wait(&s.sfull[slot], sphase, wc, 9)) return;
+            const float* sl = s.scales + slot * kScaleSlotFloats;
+            const float a_s = sl[rl];
+            const float fA = a_s * sl[128];
+            const float fB = a_s * sl[129];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.sempty[slot]);
+            if (++slot == kScaleSlots) { slot = 0; sphase ^= 1; }
+            tmem_wait_ld(va);
+            tmem_wait_ld(vb);
+            // block 1 loads reuse each staging buffer as soon as its FMAs are issued
+            ffma_chunk(acc, va, fA);
+            tmem_ld32_async(tb + 128, va);
+            ffma_chunk(acc + 16, vb, fA);
+            tmem_ld32_async(tb + 160, vb);
+            tmem_wait_ld(va);
+            tmem_wait_ld(vb);
+            // the TMEM slot is no longer read: hand it back before the last FMAs
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&s.tempty[buf]);
-            buf ^= 1;
-            if (buf == 0) bphase ^= 1;
+            if (lane == 0) mbar_arrive(&s.tempty[tj]);
+            tj ^= 1;
+            if (tj == 0) tjphase ^= 1;
+            ffma_chunk(acc + 32, va, fB);
+            ffma_chunk(acc + 48, vb, fB);
         }
+        const float* accf = reinterpret_cast<const float*>(acc);
 
         if constexpr (EPI == EPI_SWIGLU_QUANT) {
+            float h[64];
             float amax = 0.0f;
 #pragma unroll
             for (int j = 0; j < 64; ++j) {
-                const float h = silu_f(acc[j]) * acc[64 + j];
-                acc[j] = h;
-                amax = fmaxf(amax, fabsf(h));
+                h[j] = silu_fast(accf[j]) * accf[64 + j];
+                amax = fmaxf(amax, fabsf(h[j]));
             }
             s.xch[g * 128 + rl] = amax;
             if (!epi_sync(s, ephase, wc)) return;
             amax = fmaxf(s.xch[rl], s.xch[128 + rl]);
             const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+            const float inv = __frcp_rn(sc);
             if (row_ok) {
                 const int ldh = p.N >> 1;
                 uint4* dst = reinterpret_cast<uint4*>(p.hq + static_cast<long long>(row) * ldh +
@@ -380,43 +478,50 @@ __device__ void epilogue_direct(const KParams& p, const Smem& s, const WaitCtl& 
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint4 w;
-                    w.x = cvt_e4m3x4(__fdiv_rn(acc[16 * c + 0], sc), __fdiv_rn(acc[16 * c + 1], sc),
-                                     __fdiv_rn(acc[16 * c + 2], sc), __fdiv_rn(acc[16 * c + 3], sc));
-                    w.y = cvt_e4m3x4(__fdiv_rn(acc[16 * c + 4], sc), __fdiv_rn(acc[16 * c + 5], sc),
-                                     __fdiv_rn(acc[16 * c + 6], sc), __fdiv_rn(acc[16 * c + 7], sc));
-                    w.z = cvt_e4m3x4(__fdiv_rn(acc[16 * c + 8], sc), __fdiv_rn(acc[16 * c + 9], sc),
-                                     __fdiv_rn(acc[16 * c + 10], sc), __fdiv_rn(acc[16 * c + 11], sc));
-                    w.w = cvt_e4m3x4(__fdiv_rn(acc[16 * c + 12], sc), __fdiv_rn(acc[16 * c + 13], sc),
-                                     __fdiv_rn(acc[16 * c + 14], sc), __fdiv_rn(acc[16 * c + 15], sc));
+                    w.x = cvt_e4m3x4(h[16 * c + 0] * inv, h[16 * c + 1] * inv, h[16 * c + 2] * inv,
+                                     h[16 * c + 3] * inv);
+                    w.y = cvt_e4m3x4(h[16 * c + 4] * inv, h[16 * c + 5] * inv, h[16 * c + 6] * inv,
+                                     h[16 * c + 7] * inv);
+                    w.z = cvt_e4m3x4(h[16 * c + 8] * inv, h[16 * c + 9] * inv, h[16 * c + 10] * inv,
+                                     h[16 * c + 11] * inv);
+                    w.w = cvt_e4m3x4(h[16 * c + 12] * inv, h[16 * c + 13] * inv,
+                                     h[16 * c + 14] * inv, h[16 * c + 15] * inv);
                     dst[c] = w;
                 }
                 if (g == 0) p.hs[static_cast<long long>(tl.nt) * p.R + row] = sc;
             }
             if (!epi_sync(s, ephase, wc)) return;
         } else if constexpr (EPI == EPI_COMBINE) {
-            if (row_ok && cols_ok) {
+            if (row_ok) {
                 const int pair = p.perm[row];
                 const int tok = pair / p.topk;
                 const float w = p.topk_w[pair];
-                float* dst = p.out_acc + static_cast<long long>(tok) * p.out_ld + tl.nt * 256 + g * 128;
+                float* dst = p.out_acc + static_cast<long long>(tok) * p.out_ld + tl.nt * 256 + colg;
 #pragma unroll
-                for (int j = 0; j < 128; j += 4)
-                    red_add_v4(dst + j, w * acc[j], w * acc[j + 1], w * acc[j + 2], w * acc[j + 3]);
+                for (int j = 0; j < 64; j += 4)
+                    red_add_v4(dst + j, w * accf[j], w * accf[j + 1], w * accf[j + 2], w * accf[j + 3]);
+                if (v1) {
+#pragma unroll
+                    for (int j = 0; j < 64; j += 4)
+                        red_add_v4(dst + 128 + j, w * accf[64 + j], w * accf[65 + j], w * accf[66 + j],
+                                   w * accf[67 + j]);
+                }
             }
         } else if constexpr (EPI == EPI_BF16) {
-            if (row_ok && cols_ok) {
-                uint4* dst = reinterpret_cast<uint4*>(p.out_bf16 + static_cast<long long>(row) * p.N +
-                                                      tl.nt * 256 + g * 128);
+            if (row_ok) {
+                __nv_bfloat16* rowp = p.out_bf16 + static_cast<long long>(row) * p.N + tl.nt * 256 + colg;
 #pragma unroll
                 for (int c = 0; c < 16; ++c) {
+                    if (c >= 8 && !v1) break;
+                    uint4* dst = reinterpret_cast<uint4*>(rowp + (c < 8 ? 8 * c : 128 + 8 * (c - 8)));
                     uint4 w;
-                    __nv_bfloat162 b0 = __floats2bfloat162_rn(acc[8 * c + 0], acc[8 * c + 1]);
-                    __nv_bfloat162 b1 = __floats2bfloat162_rn(acc[8 * c + 2], acc[8 * c + 3]);
-                    __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[8 * c + 4], acc[8 * c + 5]);
-                    __nv_bfloat162 b3 = __floats2bfloat162_rn(acc[8 * c + 6], acc[8 * c + 7]);
+                    __nv_bfloat162 b0 = __floats2bfloat162_rn(accf[8 * c + 0], accf[8 * c + 1]);
+                    __nv_bfloat162 b1 = __floats2bfloat162_rn(accf[8 * c + 2], accf[8 * c + 3]);
+                    __nv_bfloat162 b2 = __floats2bfloat162_rn(accf[8 * c + 4], accf[8 * c + 5]);
+                    __nv_bfloat162 b3 = __floats2bfloat162_rn(accf[8 * c + 6], accf[8 * c + 7]);
                     memcpy(&w.x, &b0, 4); memcpy(&w.y, &b1, 4);
                     memcpy(&w.z, &b2, 4); memcpy(&w.w, &b3, 4);
-                    dst[c] = w;
+                    *dst = w;
                 }
             }
         } else {  // EPI_SWIGLU_BF16
@@ -428,7 +533,7 @@ __device__ void epilogue_direct(const KParams& p, const Smem& s, const WaitCtl& 
                 for (int c = 0; c < 8; ++c) {
                     float h[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) h[i] = silu_f(acc[8 * c + i]) * acc[64 + 8 * c + i];
+                    for (int i = 0; i < 8; ++i) h[i] = silu_fast(accf[8 * c + i]) * accf[64 + 8 * c + i];
                     uint4 w;
                     __nv_bfloat162 b0 = __floats2bfloat162_rn(h[0], h[1]);
                     __nv_bfloat162 b1 = __floats2bfloat162_rn(h[2], h[3]);
@@ -595,15 +700,19 @@ __global__ void __launch_bounds__(Cfg<BT>::THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::STAGES; ++i) {
-            mbar_init(&s.full[i], 1);
+            mbar_init(&s.full[i], C::NBOX);
             mbar_init(&s.empty[i], 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < C::TSLOTS; ++i) {
             mbar_init(&s.tfull[i], 1);
             mbar_init(&s.tempty[i], C::EPI_WARPS);
         }
         mbar_init(s.drain, 1);
         mbar_init(s.epi, C::EPI_THREADS);
+        for (int i = 0; i < kScaleSlots; ++i) {
+            mbar_init(&s.sfull[i], 32);
+            mbar_init(&s.sempty[i], C::EPI_WARPS);
+        }
         *s.abort = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
@@ -652,8 +761,9 @@ __global__ void __launch_bounds__(Cfg<BT>::THREADS, 1)
 
     if (warp < 4) {
         if constexpr (!C::SWAP) setmaxnreg_dec<kDirectLowRegs>();
-        if (warp == 0 && lane == 0) producer_role<BT, GATED>(&tmA, &tmB, p, s, wc);
+        if (warp == 0 && lane < C::NBOX) producer_role<BT, GATED>(&tmA, &tmB, p, s, wc);
         else if (warp == 1 && lane == 0) mma_role<BT>(p, s, wc, tmem_base);
+        else if (warp == 2) { if constexpr (!C::SWAP) scale_role<GATED>(p, s, wc); }
     } else {
         if constexpr (!C::SWAP) {
             setmaxnreg_inc<kDirectHighRegs>();
@@ -783,8 +893,8 @@ int launch_grouped_gemm(const GemmArgs& g, cudaStream_t stream) {
     if (g.R <= 0 || g.E <= 0) return ST_OK;
     if (g.tile_m != 128 && g.K > swap_max_k(g.tile_m)) return ST_UNSUPPORTED;
     CUtensorMap ma, mb;
-    if (!make_map(&ma, g.a, g.R, g.K, g.tile_m)) return ST_CUDA;
-    if (!make_map(&mb, g.b, static_cast<long long>(g.E) * g.N, g.K, 128)) return ST_CUDA;
+    if (!make_map(&ma, g.a, g.R, g.K, g.tile_m < 64 ? g.tile_m : 64)) return ST_CUDA;
+    if (!make_map(&mb, g.b, static_cast<long long>(g.E) * g.N, g.K, 64)) return ST_CUDA;
     KParams kp;
     kp.R = g.R; kp.N = g.N; kp.K = g.K; kp.E = g.E; kp.nkb = g.K / 128;
     kp.a_scale = g.a_scale; kp.as_row = g.as_row; kp.as_kb = g.as_kb;

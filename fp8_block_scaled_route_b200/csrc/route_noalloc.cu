@@ -24,7 +24,7 @@
 
 #include <mutex>
 
-#include "../../include/moefp8.h"
+#include "moefp8.h"
 #include "common.cuh"
 #include "kernels.h"
 
