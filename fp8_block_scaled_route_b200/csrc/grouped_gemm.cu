@@ -73,17 +73,18 @@ struct Cfg {
     static constexpr int AS_TILE_BYTES = SWAP ? 32768 : 0;  // a_scale staging [nkb][BT]
     static constexpr int XCH_BYTES = SWAP ? ((4 * BT + 2 * BT) * 4 + 15) / 16 * 16 : 2 * 128 * 4;
     static constexpr int SCALE_BYTES = SWAP ? 0 : kScaleSlots * kScaleSlotFloats * 4;
-    static constexpr int BAR_BYTES = 512;
+    static constexpr int BAR_BYTES = 1024;
     static constexpr int FIXED =
         1024 + AS_TILE_BYTES + SCALE_BYTES + kTableBytes + XCH_BYTES + BAR_BYTES;
     static constexpr int STAGES_FIT = (kSmemLimit - FIXED) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
     static constexpr int SMEM_BYTES = FIXED + STAGES * STAGE_BYTES;
-    static constexpr uint32_t TMEM_COLS = SWAP ? 4 * BT : 512;
-    // TMEM accumulator slots: two K blocks in flight, each slot holding both
-    // 128-row weight blocks of the tile (direct: one N = 256 MMA per K step;
-    // swapped: two N = BT MMAs).
-    static constexpr int TSLOTS = 2;
+    static constexpr uint32_t TMEM_COLS = 512;
+    // TMEM accumulator slots, each holding both 128-row weight blocks of one
+    // K block: direct = 2 slots of 256 columns (one N = 256 MMA per K step);
+    // swapped = up to 16 slots of 2 x BT columns, so the weight stream keeps
+    // going while the epilogue finishes a tile.
+    static constexpr int TSLOTS = SWAP ? (512 / (2 * BT) > 16 ? 16 : 512 / (2 * BT)) : 2;
     static constexpr int TBUF_COLS = SWAP ? 2 * BT : 256;
     static constexpr int MAX_NKB = SWAP ? AS_TILE_BYTES / (4 * BT) : 1 << 20;
     // TMA boxes per stage, one per issuing producer lane: the token tile in
@@ -156,13 +157,13 @@ __device__ __forceinline__ Smem carve(uint8_t* base) {
     s.full = bars;
     s.empty = bars + 8;
     s.tfull = bars + 16;
-    s.tempty = bars + 20;
-    s.drain = bars + 24;
-    s.epi = bars + 25;
-    s.sfull = bars + 26;
-    s.sempty = bars + 26 + kScaleSlots;
-    s.tmem = reinterpret_cast<uint32_t*>(bars + 26 + 2 * kScaleSlots);
-    s.abort = reinterpret_cast<volatile int*>(bars + 27 + 2 * kScaleSlots);
+    s.tempty = bars + 32;
+    s.drain = bars + 48;
+    s.epi = bars + 49;
+    s.sfull = bars + 50;
+    s.sempty = bars + 50 + kScaleSlots;
+    s.tmem = reinterpret_cast<uint32_t*>(bars + 50 + 2 * kScaleSlots);
+    s.abort = reinterpret_cast<volatile int*>(bars + 51 + 2 * kScaleSlots);
     return s;
 }
 
@@ -337,8 +338,7 @@ __device__ void mma_role(const KParams& p, const Smem& s, const WaitCtl& wc, uin
             }
             umma_commit(&s.empty[stage]);
             umma_commit(&s.tfull[j]);
-            j ^= 1;
-            if (j == 0) jphase ^= 1;
+            if (++j == C::TSLOTS) { j = 0; jphase ^= 1; }
             if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
     }
@@ -553,6 +553,7 @@ __device__ void epilogue_direct(const KParams& p, const Smem& s, const WaitCtl& 
 template <int BT, int EPI>
 __device__ void epilogue_swap(const KParams& p, const Smem& s, const WaitCtl& wc,
                               uint32_t tmem_base) {
+    using C = Cfg<BT>;
     constexpr bool GATED = (EPI == EPI_SWIGLU_BF16 || EPI == EPI_SWIGLU_QUANT);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = warp & 3;
@@ -621,8 +622,7 @@ __device__ void epilogue_swap(const KParams& p, const Smem& s, const WaitCtl& wc
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.tempty[buf]);
-            buf ^= 1;
-            if (buf == 0) bphase ^= 1;
+            if (++buf == C::TSLOTS) { buf = 0; bphase ^= 1; }
         }
 
         if constexpr (EPI == EPI_SWIGLU_QUANT) {

@@ -43,18 +43,26 @@ __global__ void __launch_bounds__(256) route_hist(const int32_t* __restrict__ id
         chunk_hist[static_cast<long long>(blockIdx.x) * E + e] = hist[e];
 }
 
-// blockDim.x = 1024 >= E
+// blockDim.x = 1024 >= E.  Each thread owns one expert; the per-chunk counts
+// are read in batches of independent loads so the loop is not one memory
+// latency per chunk.
 __global__ void __launch_bounds__(1024) route_scan(int nchunks, int E, int32_t* __restrict__ chunk_hist,
                                                    int32_t* __restrict__ m_indptr) {
     __shared__ int warp_tot[32];
+    constexpr int kBatch = 16;
     const int e = threadIdx.x;
     int count = 0;
     if (e < E) {
-        for (int c = 0; c < nchunks; ++c) {
-            const long long i = static_cast<long long>(c) * E + e;
-            const int h = chunk_hist[i];
-            chunk_hist[i] = count;  // rows of e in earlier chunks
-            count += h;
+        for (int c0 = 0; c0 < nchunks; c0 += kBatch) {
+            int h[kBatch];
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i)
+                h[i] = (c0 + i < nchunks) ? chunk_hist[static_cast<long long>(c0 + i) * E + e] : 0;
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) {
+                if (c0 + i < nchunks) chunk_hist[static_cast<long long>(c0 + i) * E + e] = count;  // rows of e in earlier chunks
+                count += h[i];
+            }
         }
     }
     // exclusive scan of count over experts
@@ -86,22 +94,32 @@ __global__ void __launch_bounds__(1024) route_scan(int nchunks, int E, int32_t* 
     if (e == E - 1) m_indptr[E] = excl + count;
 }
 
-// blockDim.x = 32: one warp per chunk
+// blockDim.x = 32: one warp per chunk.  The chunk's expert ids are read up
+// front (one batch of independent loads), then ranked 32 at a time.
 __global__ void __launch_bounds__(32) route_scatter(const int32_t* __restrict__ ids, int R, int E,
                                                     const int32_t* __restrict__ chunk_base,
                                                     int32_t* __restrict__ perm,
                                                     int32_t* __restrict__ inv_perm) {
     extern __shared__ int cursor[];
+    constexpr int kSteps = kRouteChunk / 32;
     const int lane = threadIdx.x;
+    const int base = blockIdx.x * kRouteChunk;
+    const int end = min(R, base + kRouteChunk);
+    int my_ids[kSteps];
+#pragma unroll
+    for (int i = 0; i < kSteps; ++i) {
+        const int p = base + i * 32 + lane;
+        my_ids[i] = p < end ? ids[p] : -1;
+    }
     for (int e = lane; e < E; e += 32)
         cursor[e] = chunk_base[static_cast<long long>(blockIdx.x) * E + e];
     __syncwarp();
-    const int base = blockIdx.x * kRouteChunk;
-    const int end = min(R, base + kRouteChunk);
-    for (int p0 = base; p0 < end; p0 += 32) {
-        const int p = p0 + lane;
+#pragma unroll
+    for (int i = 0; i < kSteps; ++i) {
+        const int p = base + i * 32 + lane;
+        if (base + i * 32 >= end) break;
         const bool live = p < end;
-        const int e = live ? ids[p] : -1;
+        const int e = my_ids[i];
         const bool ok = live && e >= 0 && e < E;
         const unsigned peers = __match_any_sync(0xffffffffu, ok ? e : -1);
         const int rank = __popc(peers & ((1u << lane) - 1u));
