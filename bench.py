@@ -370,6 +370,44 @@ def run_ours(args, cfg):
     return 0
 
 
+def run_swiglu(args):
+    """Standalone SwiGLU + MXFP8 quantisation at the three (M, K) sizes;
+    each iteration timed alone with an L2 flush (256 MB write) in between."""
+    import fp8_block_scaled_route_b200 as moe
+    torch.cuda.set_device(0)
+    hbm, _, _, src = load_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    res = []
+    for (M, K) in synth.SWIGLU_SHAPES:
+        for variant in ("normal", "block_scaled"):
+            x = synth.make_swiglu_input(M, K, variant, seed=0, device="cuda")
+            out = torch.empty(M, K, dtype=torch.uint8, device="cuda")
+            sc = torch.empty(M, K // 32, dtype=torch.uint8, device="cuda")
+            for _ in range(args.warmup):
+                moe.swiglu_mxfp8_quant(x, out, sc)
+            times = []
+            for _ in range(args.steps):
+                flush.fill_(1)
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record()
+                moe.swiglu_mxfp8_quant(x, out, sc)
+                b.record()
+                torch.cuda.synchronize()
+                times.append(a.elapsed_time(b))
+            ms = statistics.median(times)
+            nbytes = 4 * M * K + M * K + M * K // 32
+            res.append({"M": M, "K": K, "input": variant, "us": ms * 1e3,
+                        "gbs": nbytes / (ms * 1e-3) / 1e9, "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / hbm})
+    line = {"metric": "SwiGLU+MXFP8 quantisation µs and GB/s as % of HBM", "unit": "us",
+            "higher_is_better": False, "steps": args.steps, "warmup": args.warmup,
+            "peak_hbm_gbs": hbm, "peak_source": src, "data": "synthetic",
+            "config": {"workload": "bf16 [M,2K] (gate|up) -> FP8 [M,K] + E8M0 per 32",
+                       "l2": "flushed before every timed launch"}, "results": res}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -379,9 +417,13 @@ def main():
                     choices=sorted(synth.CONFIGS) + sorted(PROFILE_SLICES))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", default="moe", choices=["moe", "swiglu_mxfp8"],
+                    help="swiglu_mxfp8: time the standalone SwiGLU+MXFP8 op instead")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.op == "swiglu_mxfp8":
+        return run_swiglu(args)
     cfg = synth.CONFIGS.get(args.workload) or PROFILE_SLICES[args.workload]
     if args.impl == "reference":
         return run_reference(args, cfg)

@@ -218,17 +218,13 @@ __device__ __forceinline__ WTile weight_tile(const Tile& t, int N) {
     return w;
 }
 
-__device__ __forceinline__ float silu_f(float z) {
-    return __fdiv_rn(z, 1.0f + expf(-z));
-}
-
 __device__ __forceinline__ float a_scale_at(const KParams& p, int row, int kb) {
     return p.a_scale[static_cast<long long>(row) * p.as_row + static_cast<long long>(kb) * p.as_kb];
 }
 
-// silu with the hardware exp2 and reciprocal (about 2 ulp); used where the
-// result feeds a requantisation or a bf16 rounding, whose steps are 2^19 times
-// coarser.
+// silu with the hardware exp2 and reciprocal (about 2 ulp); its result feeds
+// an FP8 requantisation or a bf16 rounding, whose steps are 2^19 times
+// coarser than that error.
 __device__ __forceinline__ float silu_fast(float z) {
     return z * __frcp_rn(1.0f + __expf(-z));
 }
@@ -239,6 +235,30 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
                                           int where) {
     const bool ok = wait_bar(bar, parity, wc, where);
     return __all_sync(0xffffffffu, ok) != 0;
+}
+
+// Max over the 32 lanes of each of G values per lane (G = 16 or 32), by a
+// transposing butterfly: afterwards v[0] of lane L holds the maximum of
+// value (L mod G) over all lanes.  G - 1 + (32 / G - 1) * G shuffles instead
+// of 5 * G.
+template <int G>
+__device__ __forceinline__ void warp_transpose_max(float (&v)[G]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 16; o >= G; o >>= 1) {
+#pragma unroll
+        for (int i = 0; i < G; ++i) v[i] = fmaxf(v[i], __shfl_xor_sync(0xffffffffu, v[i], o));
+    }
+#pragma unroll
+    for (int o = G / 2; o >= 1; o >>= 1) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < o; ++i) {
+            const float send = up ? v[i] : v[i + o];
+            const float keep = up ? v[i + o] : v[i];
+            v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, o));
+        }
+    }
 }
 
 __device__ __forceinline__ bool warp_wait_spin(uint64_t* bar, uint32_t parity, const WaitCtl& wc,
@@ -626,29 +646,39 @@ __device__ void epilogue_swap(const KParams& p, const Smem& s, const WaitCtl& wc
         }
 
         if constexpr (EPI == EPI_SWIGLU_QUANT) {
-            float* red = s.xch;  // [4 warps][BT] per-token partial amax
+            float* red = s.xch;             // [4 warps][BT] per-token partial amax
+            float* s_sc = s.xch + 4 * BT;   // [BT] scale of each token's 128-column block
+            float* s_inv = s.xch + 5 * BT;  // [BT] its reciprocal
+            constexpr int G = BT < 32 ? BT : 32;   // tokens per transpose group
 #pragma unroll
-            for (int j = 0; j < BT; ++j) {
-                const float h = silu_f(acc0[j]) * acc1[j];
-                acc0[j] = h;
-                float m = fabsf(h);
+            for (int g0 = 0; g0 < BT; g0 += G) {
+                float m[G];
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                if (lane == 0) red[q * BT + j] = m;
+                for (int i = 0; i < G; ++i) {
+                    const float h = silu_fast(acc0[g0 + i]) * acc1[g0 + i];
+                    acc0[g0 + i] = h;
+                    m[i] = fabsf(h);
+                }
+                // after this lane L holds the warp's max for token g0 + (L mod G)
+                warp_transpose_max<G>(m);
+                if (lane < G) red[q * BT + g0 + lane] = m[0];
+            }
+            if (!epi_sync(s, ephase, wc)) return;
+            if (et < BT) {
+                const float amax = fmaxf(fmaxf(red[et], red[BT + et]), fmaxf(red[2 * BT + et], red[3 * BT + et]));
+                const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+                s_sc[et] = sc;
+                s_inv[et] = __frcp_rn(sc);
+                if (et < tl.rows) p.hs[static_cast<long long>(tl.nt) * p.R + tl.row0 + et] = sc;
             }
             if (!epi_sync(s, ephase, wc)) return;
             const int ldh = p.N >> 1;
             const int col = tl.nt * 128 + w;
 #pragma unroll
             for (int j = 0; j < BT; ++j) {
-                if (j < tl.rows) {
-                    const float amax = fmaxf(fmaxf(red[j], red[BT + j]), fmaxf(red[2 * BT + j], red[3 * BT + j]));
-                    const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-                    const float x = __fdiv_rn(acc0[j], sc);
+                if (j < tl.rows)
                     p.hq[static_cast<long long>(tl.row0 + j) * ldh + col] =
-                        static_cast<uint8_t>(cvt_e4m3x2(x, 0.0f) & 0xFF);
-                    if (w == j) p.hs[static_cast<long long>(tl.nt) * p.R + tl.row0 + j] = sc;
-                }
+                        static_cast<uint8_t>(cvt_e4m3x2(acc0[j] * s_inv[j], 0.0f) & 0xFF);
             }
         } else if constexpr (EPI == EPI_COMBINE) {
             const int colA = tl.nt * 256 + w;
@@ -679,7 +709,7 @@ __device__ void epilogue_swap(const KParams& p, const Smem& s, const WaitCtl& wc
             for (int j = 0; j < BT; ++j) {
                 if (j < tl.rows)
                     p.out_bf16[static_cast<long long>(tl.row0 + j) * ldo + col] =
-                        __float2bfloat16_rn(silu_f(acc0[j]) * acc1[j]);
+                        __float2bfloat16_rn(silu_fast(acc0[j]) * acc1[j]);
             }
         }
     }

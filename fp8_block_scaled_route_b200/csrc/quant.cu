@@ -108,57 +108,70 @@ __device__ __forceinline__ uint32_t e8m0_code(float amax) {
     return static_cast<uint32_t>(c);
 }
 
-__device__ __forceinline__ float e8m0_value(uint32_t c) {
-    // 2^(c-127); c = 0 is the fp32 subnormal 2^-127
-    return c == 0 ? __uint_as_float(0x00400000u) : __uint_as_float(c << 23);
+// 2^(127 - c): the exact reciprocal of the E8M0 value 2^(c - 127).  x * 2^-s
+// and x / 2^s round the same exact value once, so the product is bit-identical
+// to the IEEE quotient for every x (subnormal results included).
+__device__ __forceinline__ float e8m0_reciprocal(uint32_t c) {
+    // c = 0 -> 2^127, c = 254 -> 2^-127 (an fp32 subnormal, exactly representable)
+    return c == 254 ? __uint_as_float(0x00400000u) : __uint_as_float((254u - c) << 23);
 }
 
-__device__ __forceinline__ float silu_q(float z) { return __fdiv_rn(z, 1.0f + expf(-z)); }
+// silu with the hardware exp2 and reciprocal (about 2 ulp); the result feeds
+// an 8-level-per-octave quantisation, so a flip needs the value to sit within
+// a few fp32 ulps of a rounding midpoint.
+__device__ __forceinline__ float silu_q(float z) { return z * __frcp_rn(1.0f + __expf(-z)); }
 
-// Four threads per 32-element block, eight outputs each (16-byte loads).  The
-// loop bound is uniform per warp so every lane reaches the shuffles.
+// Two threads per 32-element block, sixteen outputs each (2 x 16-byte loads
+// of gate and of up).  The loop bound is uniform per warp so every lane
+// reaches the shuffle.
 __global__ void __launch_bounds__(256) swiglu_mxfp8_kernel(const __nv_bfloat16* __restrict__ in,
                                                            uint8_t* __restrict__ out,
                                                            uint8_t* __restrict__ scale, int M, int K) {
-    const long long groups = static_cast<long long>(M) * (K / 8);
-    const int kg = K / 8;
+    const int kg = K / 16;
+    const long long groups = static_cast<long long>(M) * kg;
     for (long long gi = blockIdx.x * 256ll + threadIdx.x; gi - (threadIdx.x & 31) < groups;
          gi += static_cast<long long>(gridDim.x) * 256) {
         const bool live = gi < groups;
-        float v[8];
+        float v[16];
         float amax = 0.0f;
         long long m = 0;
         int c0 = 0;
         if (live) {
             m = gi / kg;
-            c0 = static_cast<int>(gi - m * kg) * 8;
-            const uint4 gr = *reinterpret_cast<const uint4*>(in + m * 2 * K + c0);
-            const uint4 ur = *reinterpret_cast<const uint4*>(in + m * 2 * K + K + c0);
-            const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w};
-            const uint32_t uw[4] = {ur.x, ur.y, ur.z, ur.w};
+            c0 = static_cast<int>(gi - m * kg) * 16;
+            const uint4* g4 = reinterpret_cast<const uint4*>(in + m * 2 * K + c0);
+            const uint4* u4 = reinterpret_cast<const uint4*>(in + m * 2 * K + K + c0);
+            const uint4 gr[2] = {g4[0], g4[1]};
+            const uint4 ur[2] = {u4[0], u4[1]};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                __nv_bfloat162 gb, ub;
-                memcpy(&gb, &gw[i], 4);
-                memcpy(&ub, &uw[i], 4);
-                const float2 gf = __bfloat1622float2(gb);
-                const float2 uf = __bfloat1622float2(ub);
-                v[2 * i] = silu_q(gf.x) * uf.x;
-                v[2 * i + 1] = silu_q(gf.y) * uf.y;
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t gw[4] = {gr[h].x, gr[h].y, gr[h].z, gr[h].w};
+                const uint32_t uw[4] = {ur[h].x, ur[h].y, ur[h].z, ur[h].w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    __nv_bfloat162 gb, ub;
+                    memcpy(&gb, &gw[i], 4);
+                    memcpy(&ub, &uw[i], 4);
+                    const float2 gf = __bfloat1622float2(gb);
+                    const float2 uf = __bfloat1622float2(ub);
+                    v[8 * h + 2 * i] = silu_q(gf.x) * uf.x;
+                    v[8 * h + 2 * i + 1] = silu_q(gf.y) * uf.y;
+                }
             }
 #pragma unroll
-            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
         }
-        // the four threads of a 32-block are lanes 4j..4j+3 of the warp
+        // the two threads of a 32-block are lanes 2j, 2j+1 of the warp
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
         if (live) {
             const uint32_t code = e8m0_code(amax);
-            const float X = e8m0_value(code);
-            uint2 o;
-            o.x = cvt_e4m3x4(__fdiv_rn(v[0], X), __fdiv_rn(v[1], X), __fdiv_rn(v[2], X), __fdiv_rn(v[3], X));
-            o.y = cvt_e4m3x4(__fdiv_rn(v[4], X), __fdiv_rn(v[5], X), __fdiv_rn(v[6], X), __fdiv_rn(v[7], X));
-            *reinterpret_cast<uint2*>(out + m * K + c0) = o;
+            const float r = e8m0_reciprocal(code);
+            uint4 o;
+            o.x = cvt_e4m3x4(v[0] * r, v[1] * r, v[2] * r, v[3] * r);
+            o.y = cvt_e4m3x4(v[4] * r, v[5] * r, v[6] * r, v[7] * r);
+            o.z = cvt_e4m3x4(v[8] * r, v[9] * r, v[10] * r, v[11] * r);
+            o.w = cvt_e4m3x4(v[12] * r, v[13] * r, v[14] * r, v[15] * r);
+            *reinterpret_cast<uint4*>(out + m * K + c0) = o;
             if ((c0 & 31) == 0) scale[m * (K / 32) + c0 / 32] = static_cast<uint8_t>(code);
         }
     }
@@ -166,10 +179,10 @@ __global__ void __launch_bounds__(256) swiglu_mxfp8_kernel(const __nv_bfloat16* 
 
 int launch_swiglu_mxfp8(const void* in, void* out, uint8_t* scale, int M, int K, int num_sms,
                         cudaStream_t stream) {
-    const long long groups = static_cast<long long>(M) * (K / 8);
+    const long long groups = static_cast<long long>(M) * (K / 16);
     if (groups == 0) return ST_OK;
     long long blocks = (groups + 255) / 256;
-    // size band: small problems (M*K < 2^20) use one 256-thread CTA per 2048
+    // size band: small problems (M*K < 2^20) use one 256-thread CTA per 4096
     // outputs so that several CTAs share an SM; larger ones stream with a
     // grid of a few waves of CTAs per SM.
     if (static_cast<long long>(M) * K >= (1ll << 20)) {

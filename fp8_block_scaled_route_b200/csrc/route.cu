@@ -7,7 +7,8 @@
 // counting sort on the pair id p = t*k + j, so the result is unique and
 // bit-reproducible.
 //
-// Three launches, no atomics on the output order:
+// Three launches (one for inputs of at most 8 chunks), no atomics on the
+// output order:
 //  1. route_hist:    one 1024-pair chunk per CTA -> per-chunk expert histogram
 //  2. route_scan:    one CTA: per-expert exclusive scan over chunks, then the
 //                    exclusive scan over experts -> m_indptr and the first
@@ -137,11 +138,138 @@ __global__ void __launch_bounds__(32) route_scatter(const int32_t* __restrict__ 
     }
 }
 
+// Small inputs (at most kSmallChunks chunks): the same three phases in one
+// CTA of 1024 threads, so routing costs one launch.  Warp c owns chunk c in
+// phases 1 and 3; thread e owns expert e in phase 2.  The per-chunk tables
+// live in shared memory.
+constexpr int kSmallChunks = 8;
+
+__global__ void __launch_bounds__(1024) route_small(const int32_t* __restrict__ ids, int R, int E,
+                                                    int32_t* __restrict__ m_indptr,
+                                                    int32_t* __restrict__ perm,
+                                                    int32_t* __restrict__ inv_perm, int* status) {
+    extern __shared__ int tab[];  // [kSmallChunks][E]: histograms, then first rows
+    __shared__ int warp_tot[32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nchunks = (R + kRouteChunk - 1) / kRouteChunk;
+    constexpr int kSteps = kRouteChunk / 32;
+    for (int i = threadIdx.x; i < nchunks * E; i += blockDim.x) tab[i] = 0;
+    __syncthreads();
+    // phase 1: per-chunk histograms
+    int my_ids[kSteps];
+    const int base = warp * kRouteChunk;
+    if (warp < nchunks) {
+        const int end = min(R, base + kRouteChunk);
+        int bad = 0;
+#pragma unroll
+        for (int i = 0; i < kSteps; ++i) {
+            const int p = base + i * 32 + lane;
+            my_ids[i] = p < end ? ids[p] : -1;
+        }
+#pragma unroll
+        for (int i = 0; i < kSteps; ++i) {
+            const int p = base + i * 32 + lane;
+            if (p < end) {
+                const int e = my_ids[i];
+                if (e >= 0 && e < E) atomicAdd(&tab[warp * E + e], 1);
+                else ++bad;
+            }
+        }
+        if (bad) {
+            atomicAdd(&status[2], bad);
+            report_error(status, ST_BAD_EXPERT_ID, 0);
+        }
+    }
+    __syncthreads();
+    // phase 2: scan over chunks and experts
+    const int e = threadIdx.x;
+    int count = 0;
+    if (e < E) {
+        for (int c = 0; c < nchunks; ++c) {
+            const int h = tab[c * E + e];
+            tab[c * E + e] = count;
+            count += h;
+        }
+    }
+    int incl = count;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int t = warp_tot[lane];
+        int ti = t;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, ti, o);
+            if (lane >= o) ti += v;
+        }
+        warp_tot[lane] = ti - t;
+    }
+    __syncthreads();
+    const int excl = warp_tot[warp] + incl - count;
+    if (e < E) {
+        m_indptr[e] = excl;
+        for (int c = 0; c < nchunks; ++c) tab[c * E + e] += excl;
+    }
+    if (e == E - 1) m_indptr[E] = excl + count;
+    __syncthreads();
+    // phase 3: stable scatter, 32 pairs at a time per chunk
+    if (warp < nchunks) {
+        const int end = min(R, base + kRouteChunk);
+        int* cursor = tab + warp * E;
+#pragma unroll
+        for (int i = 0; i < kSteps; ++i) {
+            const int p = base + i * 32 + lane;
+            if (base + i * 32 >= end) break;
+            const bool live = p < end;
+            const int ex = my_ids[i];
+            const bool ok = live && ex >= 0 && ex < E;
+            const unsigned peers = __match_any_sync(0xffffffffu, ok ? ex : -1);
+            const int rank = __popc(peers & ((1u << lane) - 1u));
+            const int first = cursor[ok ? ex : 0];
+            __syncwarp();
+            if (ok) {
+                const int row = first + rank;
+                perm[row] = p;
+                if (inv_perm) inv_perm[p] = row;
+                if (rank == 0) cursor[ex] = first + __popc(peers);
+            } else if (live && inv_perm) {
+                inv_perm[p] = -1;
+            }
+            __syncwarp();
+        }
+    }
+}
+
 int launch_route_permute(const RouteArgs& r, cudaStream_t stream) {
     const int R = r.T * r.k;
     const int nchunks = (R + kRouteChunk - 1) / kRouteChunk;
     const size_t hist_smem = static_cast<size_t>(r.E) * sizeof(int);
-    if (nchunks > 0) {
+    if (nchunks <= kSmallChunks) {
+        const size_t smem = static_cast<size_t>(kSmallChunks) * r.E * sizeof(int);
+        if (smem > 48 * 1024) {
+            // above the default dynamic shared-memory limit: opt in (per device)
+            static bool attr_set[64] = {};
+            int dev = 0;
+            cudaGetDevice(&dev);
+            if (dev < 0 || dev >= 64) return ST_CUDA;
+            if (!attr_set[dev]) {
+                if (cudaFuncSetAttribute(route_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmallChunks * 1024 * static_cast<int>(sizeof(int))) !=
+                    cudaSuccess)
+                    return ST_CUDA;
+                attr_set[dev] = true;
+            }
+        }
+        route_small<<<1, 1024, smem, stream>>>(r.topk_ids, R, r.E, r.m_indptr, r.perm, r.inv_perm,
+                                               r.status);
+        return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
+    }
+    {
         route_hist<<<nchunks, 256, hist_smem, stream>>>(r.topk_ids, R, r.E, r.chunk_hist, r.status);
         if (cudaGetLastError() != cudaSuccess) return ST_CUDA;
     }

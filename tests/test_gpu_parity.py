@@ -63,6 +63,21 @@ def test_route_permute_empty():
     assert st == moe.MOE_OK and np.all(m_g == 0)
 
 
+def test_route_bad_ids_multi_chunk():
+    """More than eight 1024-pair chunks: the three-launch path, with bad ids."""
+    g = torch.Generator().manual_seed(77)
+    ids, _ = synth.make_routing(2000, 64, 8, "normal", g, "cpu")
+    ids[5, 3] = -2
+    ids[1999, 0] = 64
+    m_g, p_g, i_g, st = _route_gpu(ids, 64)
+    m_o, p_o, i_o, bad = O.route_permute(ids.numpy(), 64)
+    assert st == moe.MOE_ERR_BAD_EXPERT_ID and bad == 2
+    assert np.array_equal(m_g, m_o)
+    n = int(m_o[-1])
+    assert np.array_equal(p_g[:n], p_o[:n])
+    assert np.array_equal(i_g, i_o)
+
+
 def test_route_bad_ids_dropped_and_reported():
     ids = torch.tensor([[0, 5], [1, -1], [2, 3], [9, 1]], dtype=torch.int32)
     m_g, p_g, i_g, st = _route_gpu(ids, 4)
