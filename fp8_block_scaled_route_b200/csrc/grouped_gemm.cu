@@ -289,12 +289,14 @@ __device__ __forceinline__ void tmem_load_cols(uint32_t taddr, float (&v)[BT]) {
 }
 
 // ---------------------------------------------------------------- roles
-// Producer: lane l < NBOX of warp 0 issues box l of every stage.
+// Producer (all of warp 0, converged): lane l < NBOX issues box l of every
+// stage.
 template <int BT, bool GATED>
 __device__ void producer_role(const CUtensorMap* tmA, const CUtensorMap* tmB, const KParams& p,
                               const Smem& s, const WaitCtl& wc) {
     using C = Cfg<BT>;
     const int l = threadIdx.x & 31;
+    const bool issuer = l < C::NBOX;
     // this lane's box: which map, smem offset inside the stage, row offset, bytes
     const bool is_a = l < C::A_BOXES;
     const int b = l - C::A_BOXES;  // weight box 0..3: block b/2, half b%2
@@ -309,10 +311,13 @@ __device__ void producer_role(const CUtensorMap* tmA, const CUtensorMap* tmB, co
         const int row = is_a ? tl.row0 + l * C::A_BOX_ROWS
                              : ((b >> 1) ? wt.wrow1 : wt.wrow0) + (b & 1) * 64;
         for (int kb = 0; kb < p.nkb; ++kb) {
-            if (!wait_bar_spin(&s.empty[stage], phase ^ 1, wc, 1)) { ok = false; break; }
+            if (!warp_wait_spin(&s.empty[stage], phase ^ 1, wc, 1)) { ok = false; break; }
             uint8_t* st = s.stages + stage * C::STAGE_BYTES;
-            mbar_arrive_expect_tx(&s.full[stage], bytes);
-            tma_load_2d(st + off, is_a ? tmA : tmB, &s.full[stage], kb * 128, row);
+            if (issuer) {
+                mbar_arrive_expect_tx(&s.full[stage], bytes);
+                tma_load_2d(st + off, is_a ? tmA : tmB, &s.full[stage], kb * 128, row);
+            }
+            __syncwarp();
             armed |= 1u << stage;
             armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
             if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
@@ -321,11 +326,12 @@ __device__ void producer_role(const CUtensorMap* tmA, const CUtensorMap* tmB, co
     // make sure no copy is still writing into shared memory when the CTA exits
     for (int st = 0; st < C::STAGES; ++st)
         if ((armed >> st) & 1u) wait_bar(&s.full[st], (armed_par >> st) & 1u, wc, 2, /*drain=*/true);
+    __syncwarp();
 }
 
-// MMA issue (one thread).  Each K block goes into TMEM slot j (two slots
-// alternate): direct = one 128 x 256 MMA per K step (both weight blocks);
-// swapped = one 128 x BT MMA per weight block per K step.
+// MMA issue (all of warp 1, converged; one elected lane issues).  Each K
+// block goes into TMEM slot j: direct = one 128 x 256 MMA per K step (both
+// weight blocks); swapped = one 128 x BT MMA per weight block per K step.
 template <int BT>
 __device__ void mma_role(const KParams& p, const Smem& s, const WaitCtl& wc, uint32_t tmem_base) {
     using C = Cfg<BT>;
@@ -335,13 +341,15 @@ __device__ void mma_role(const KParams& p, const Smem& s, const WaitCtl& wc, uin
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         for (int kb = 0; kb < p.nkb; ++kb) {
-            if (!wait_bar_spin(&s.tempty[j], jphase ^ 1, wc, 3)) { ok = false; break; }
-            if (!wait_bar_spin(&s.full[stage], phase, wc, 4)) { ok = false; break; }
+            if (!warp_wait_spin(&s.tempty[j], jphase ^ 1, wc, 3)) { ok = false; break; }
+            if (!warp_wait_spin(&s.full[stage], phase, wc, 4)) { ok = false; break; }
             tc_fence_after();
             const uint32_t sa = smem_u32(s.stages + stage * C::STAGE_BYTES + C::A_OFF);
             const uint32_t sb = smem_u32(s.stages + stage * C::STAGE_BYTES + C::B_OFF);
             const uint32_t d = tmem_base + j * C::TBUF_COLS;
-            if constexpr (C::SWAP) {
+            if (!elect_one()) {
+                // lanes that do not issue
+            } else if constexpr (C::SWAP) {
                 // weight block 0 into columns [0, BT), block 1 into [BT, 2BT)
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
@@ -350,21 +358,28 @@ __device__ void mma_role(const KParams& p, const Smem& s, const WaitCtl& wc, uin
                     umma_f8(d + BT, smem_desc_k_sw128(sb + 16384 + kk * 32),
                             smem_desc_k_sw128(sa + kk * 32), idesc, kk);
                 }
+                umma_commit(&s.empty[stage]);
+                umma_commit(&s.tfull[j]);
             } else {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     umma_f8(d, smem_desc_k_sw128(sa + kk * 32), smem_desc_k_sw128(sb + kk * 32),
                             idesc, kk);
+                umma_commit(&s.empty[stage]);
+                umma_commit(&s.tfull[j]);
             }
-            umma_commit(&s.empty[stage]);
-            umma_commit(&s.tfull[j]);
+            __syncwarp();
             if (++j == C::TSLOTS) { j = 0; jphase ^= 1; }
             if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
     }
-    // every MMA this thread issued must be complete before TMEM is freed
-    umma_commit(s.drain);
+    // every MMA this warp issued must be complete before TMEM is freed; the
+    // drain commit comes from the lane that issued (elect.sync picks the same
+    // lane of a converged warp every time)
+    if (elect_one()) umma_commit(s.drain);
+    __syncwarp();
     wait_bar(s.drain, 0, wc, 5, /*drain=*/true);
+    __syncwarp();
 }
 
 // Scale stager of the direct kernel (warp 2): for every K block of every
@@ -791,8 +806,8 @@ __global__ void __launch_bounds__(Cfg<BT>::THREADS, 1)
 
     if (warp < 4) {
         if constexpr (!C::SWAP) setmaxnreg_dec<kDirectLowRegs>();
-        if (warp == 0 && lane < C::NBOX) producer_role<BT, GATED>(&tmA, &tmB, p, s, wc);
-        else if (warp == 1 && lane == 0) mma_role<BT>(p, s, wc, tmem_base);
+        if (warp == 0) producer_role<BT, GATED>(&tmA, &tmB, p, s, wc);
+        else if (warp == 1) mma_role<BT>(p, s, wc, tmem_base);
         else if (warp == 2) { if constexpr (!C::SWAP) scale_role<GATED>(p, s, wc); }
     } else {
         if constexpr (!C::SWAP) {
