@@ -73,9 +73,11 @@ struct Cfg {
     static constexpr int AS_TILE_BYTES = SWAP ? 32768 : 0;  // a_scale staging [nkb][BT]
     static constexpr int XCH_BYTES = SWAP ? ((4 * BT + 2 * BT) * 4 + 15) / 16 * 16 : 2 * 128 * 4;
     static constexpr int SCALE_BYTES = SWAP ? 0 : kScaleSlots * kScaleSlotFloats * 4;
+    // direct combine: per epilogue warp a 32-row x 16-column fp32 transpose tile
+    static constexpr int CST_BYTES = SWAP ? 0 : EPI_WARPS * 32 * 16 * 4;
     static constexpr int BAR_BYTES = 1024;
     static constexpr int FIXED =
-        1024 + AS_TILE_BYTES + SCALE_BYTES + kTableBytes + XCH_BYTES + BAR_BYTES;
+        1024 + AS_TILE_BYTES + SCALE_BYTES + CST_BYTES + kTableBytes + XCH_BYTES + BAR_BYTES;
     static constexpr int STAGES_FIT = (kSmemLimit - FIXED) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
     static constexpr int SMEM_BYTES = FIXED + STAGES * STAGE_BYTES;
@@ -125,6 +127,7 @@ struct Smem {
     int* mind;    // [E+1] clamped m_indptr
     float* xch;   // epilogue exchange area
     float* scales;  // direct kernel: kScaleSlots x {a_scale[128], b_scale[2], pad[2]}
+    float* cstage;  // direct combine transpose tiles
     uint64_t* full;
     uint64_t* empty;
     uint64_t* tfull;
@@ -153,6 +156,8 @@ __device__ __forceinline__ Smem carve(uint8_t* base) {
     p += C::XCH_BYTES;
     s.scales = reinterpret_cast<float*>(p);
     p += C::SCALE_BYTES;
+    s.cstage = reinterpret_cast<float*>(p);
+    p += C::CST_BYTES;
     uint64_t* bars = reinterpret_cast<uint64_t*>(p);
     s.full = bars;
     s.empty = bars + 8;
@@ -226,7 +231,7 @@ __device__ __forceinline__ float a_scale_at(const KParams& p, int row, int kb) {
 // an FP8 requantisation or a bf16 rounding, whose steps are 2^19 times
 // coarser than that error.
 __device__ __forceinline__ float silu_fast(float z) {
-    return z * __frcp_rn(1.0f + __expf(-z));
+    return z * rcp_approx(1.0f + __expf(-z));
 }
 
 // Wait of a whole epilogue warp: every lane waits, and the warp proceeds only
@@ -527,19 +532,50 @@ __device__ void epilogue_direct(const KParams& p, const Smem& s, const WaitCtl& 
             }
             if (!epi_sync(s, ephase, wc)) return;
         } else if constexpr (EPI == EPI_COMBINE) {
+            // Scatter-add w * row into the token's output row.  A lane holds
+            // 64 consecutive columns of one row per weight block; passing them
+            // through a shared-memory tile 16 columns at a time lets each
+            // reduction instruction cover 8 rows x 64 contiguous bytes instead
+            // of 32 rows x 16 bytes.  Tile layout: row r at 128-byte line
+            // r / 2, 16-byte slot (r & 1) * 4 + ((c + r / 2) & 3) for column
+            // chunk c, so both the row-wise writes and the column-wise reads
+            // are free of bank conflicts.
+            int tok = -1;
+            float w = 0.0f;
             if (row_ok) {
                 const int pair = p.perm[row];
-                const int tok = pair / p.topk;
-                const float w = p.topk_w[pair];
-                float* dst = p.out_acc + static_cast<long long>(tok) * p.out_ld + tl.nt * 256 + colg;
+                tok = pair / p.topk;
+                w = p.topk_w[pair];
+            }
+            float* const obase = p.out_acc + tl.nt * 256 + colg;
+            float* stg = s.cstage + (warp - 4) * 512;
+            const int rr = lane >> 2, cc = lane & 3;
 #pragma unroll
-                for (int j = 0; j < 64; j += 4)
-                    red_add_v4(dst + j, w * accf[j], w * accf[j + 1], w * accf[j + 2], w * accf[j + 3]);
-                if (v1) {
+            for (int half = 0; half < 2; ++half) {
+                if (half == 1 && !v1) break;
 #pragma unroll
-                    for (int j = 0; j < 64; j += 4)
-                        red_add_v4(dst + 128 + j, w * accf[64 + j], w * accf[65 + j], w * accf[66 + j],
-                                   w * accf[67 + j]);
+                for (int c16 = 0; c16 < 4; ++c16) {
+                    const float* a = accf + half * 64 + c16 * 16;
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const int slot = (lane & 1) * 4 + ((q4 + (lane >> 1)) & 3);
+                        *reinterpret_cast<float4*>(stg + (lane >> 1) * 32 + slot * 4) =
+                            make_float4(w * a[4 * q4], w * a[4 * q4 + 1], w * a[4 * q4 + 2],
+                                        w * a[4 * q4 + 3]);
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int rg = 0; rg < 4; ++rg) {
+                        const int r = rg * 8 + rr;
+                        const int slot = (r & 1) * 4 + ((cc + (r >> 1)) & 3);
+                        const float4 v = *reinterpret_cast<const float4*>(stg + (r >> 1) * 32 + slot * 4);
+                        const int t_r = __shfl_sync(0xffffffffu, tok, r);
+                        if (t_r >= 0)
+                            red_add_v4(obase + static_cast<long long>(t_r) * p.out_ld + half * 128 +
+                                           c16 * 16 + cc * 4,
+                                       v.x, v.y, v.z, v.w);
+                    }
+                    __syncwarp();
                 }
             }
         } else if constexpr (EPI == EPI_BF16) {

@@ -250,6 +250,14 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
 }
 
 // ----------------------------------------------------------------- misc
+// Hardware reciprocal (rcp.approx.ftz.f32, within 1 ulp); for arguments of
+// at least 1, where flushing subnormals cannot matter.
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
 // True in exactly one lane of the (converged) warp.  tcgen05.mma issued from
 // a converged warp through an elected lane reaches the tensor rate; issued from
 // a lone lane of a diverged warp it costs about 100 clk per instruction.

@@ -119,7 +119,7 @@ __device__ __forceinline__ float e8m0_reciprocal(uint32_t c) {
 // silu with the hardware exp2 and reciprocal (about 2 ulp); the result feeds
 // an 8-level-per-octave quantisation, so a flip needs the value to sit within
 // a few fp32 ulps of a rounding midpoint.
-__device__ __forceinline__ float silu_q(float z) { return z * __frcp_rn(1.0f + __expf(-z)); }
+__device__ __forceinline__ float silu_q(float z) { return z * rcp_approx(1.0f + __expf(-z)); }
 
 // Two threads per 32-element block, sixteen outputs each (2 x 16-byte loads
 // of gate and of up).  The loop bound is uniform per warp so every lane
