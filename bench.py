@@ -18,6 +18,7 @@ a bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -38,7 +39,16 @@ METRIC = "fused MoE layer µs & TFLOPS/GB/s as % of B200 FP8-tensor/HBM roofline
 FP8_OVER_BF16 = 2.0        # nominal dense FP8 / BF16 tensor ratio (4.5 / 2.25 PFLOP/s)
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-KERNELS_PER_LAYER = 7      # route hist/scan/scatter, quant, GEMM1, GEMM2, bf16 conversion
+ROUTE_CHUNK = 1024         # (token, slot) pairs per routing chunk
+ROUTE_SMALL_CHUNKS = 8     # up to this many chunks, routing is one single-CTA launch
+
+
+def kernels_per_layer(T: int, k: int) -> int:
+    """Kernel launches of one fused layer: routing (one launch for inputs of
+    at most 8 chunks of 1024 pairs, else histogram/scan/scatter), quant,
+    GEMM1, GEMM2 and the bf16 conversion."""
+    nchunks = (T * k + ROUTE_CHUNK - 1) // ROUTE_CHUNK
+    return (1 if nchunks <= ROUTE_SMALL_CHUNKS else 3) + 4
 
 
 # Slices of the prefill and decode workloads (same H, I, top-k and routing,
@@ -47,6 +57,32 @@ PROFILE_SLICES = {
     "prefill_slice": synth.MoEConfig("prefill_slice", 1024, 7168, 2048, 32, 8, "zipf"),
     "decode_slice": synth.MoEConfig("decode_slice", 64, 7168, 2048, 32, 8),
 }
+
+
+# DRAM bytes (read + write) per launch of the dominant kernel, GEMM1, taken
+# from the ncu launch list of `bench.py --workload <name>` (see the launch-list
+# summaries under profiles/).  A figure is reported only while the GEMM
+# sources still hash to the digest it was taken with.
+GEMM_SOURCES = ("grouped_gemm.cu", "ptx.cuh", "common.cuh", "kernels.h")
+MEASURED_TRAFFIC = {}  # workload -> (source digest, bytes per GEMM1 launch)
+
+
+def gemm_source_digest() -> str:
+    h = hashlib.sha256()
+    for name in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "fp8_block_scaled_route_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload: str):
+    entry = MEASURED_TRAFFIC.get(workload)
+    if entry is None:
+        return None
+    try:
+        return entry[1] if gemm_source_digest() == entry[0] else None
+    except OSError:
+        return None
 
 
 def workload_desc(cfg: synth.MoEConfig) -> str:
@@ -322,7 +358,8 @@ def run_ours(args, cfg):
         else:
             roof = {"bound": "hbm", "achieved": g1_gbs, "peak": hbm, "unit": "GB/s",
                     "frac": g1_gbs / hbm}
-        roof.update({"traffic": None, "kernel": "grouped GEMM1 (gate/up + SwiGLU + FP8 requant)",
+        roof.update({"traffic": measured_traffic(cfg.name),
+                     "kernel": "grouped GEMM1 (gate/up + SwiGLU + FP8 requant)",
                      "peak_source": f"{src} (FP8 = bf16 burst x {FP8_OVER_BF16:g})"
                      if roof["bound"] == "tensor" else f"{src} copy bandwidth"})
         layer_gbs = counts["bytes"] / (ms_step * 1e-3) / 1e9
@@ -346,7 +383,7 @@ def run_ours(args, cfg):
             "roofline": roof,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": T * H * 2 + T * k * 8, "d2h_bytes_per_step": T * H * 2},
-            "gpu_launches": KERNELS_PER_LAYER * args.steps,
+            "gpu_launches": kernels_per_layer(T, k) * args.steps,
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

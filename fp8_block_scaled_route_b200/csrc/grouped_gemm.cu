@@ -47,6 +47,7 @@ namespace moe {
 
 constexpr int kSmemLimit = 232448;  // 227 KB of opt-in dynamic shared memory per CTA
 constexpr int kMaxE = 1024;
+constexpr long long kCombineRangeBytes = 64ll << 20;  // half of the 126 MB L2
 constexpr int kTableBytes = ((2 * (kMaxE + 1) * 4) + 15) / 16 * 16;
 constexpr int kScaleSlots = 8;        // depth of the direct kernel's scale ring
 constexpr int kScaleSlotFloats = 132;  // a_scale of 128 rows, then b_scale of the two blocks
@@ -104,6 +105,9 @@ struct Cfg {
 
 struct KParams {
     int R, N, K, E, nkb;
+    // Tiles are ordered by column range first: nranges ranges of ntn_r
+    // column tiles each, then expert, column tile, row tile.
+    int nranges, ntn_r;
     const float* a_scale;
     long long as_row, as_kb;
     const float* b_scale;
@@ -176,8 +180,17 @@ struct Tile {
     int e, mt, nt, row0, rows;
 };
 
+// Total tiles of the launch: tstart[E] tiles per column range.
+__device__ __forceinline__ int total_tiles(const Smem& s, const KParams& p) {
+    return s.tstart[p.E] * p.nranges;
+}
+
 template <int BT>
-__device__ __forceinline__ Tile decode_tile(int t, const Smem& s, int E) {
+__device__ __forceinline__ Tile decode_tile(int t, const Smem& s, const KParams& p) {
+    const int E = p.E;
+    const int per = s.tstart[E];
+    const int range = t / per;
+    t -= range * per;
     int lo = 0, hi = E;  // tstart[lo] <= t < tstart[hi]
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
@@ -188,8 +201,9 @@ __device__ __forceinline__ Tile decode_tile(int t, const Smem& s, int E) {
     const int local = t - s.tstart[lo];
     const int me = max(0, s.mind[lo + 1] - s.mind[lo]);
     const int mtiles = (me + BT - 1) / BT;
-    r.nt = local / mtiles;
-    r.mt = local - r.nt * mtiles;
+    const int ntl = local / mtiles;
+    r.nt = range * p.ntn_r + ntl;
+    r.mt = local - ntl * mtiles;
     r.row0 = s.mind[lo] + r.mt * BT;
     r.rows = min(BT, me - r.mt * BT);
     return r;
@@ -308,10 +322,10 @@ __device__ void producer_role(const CUtensorMap* tmA, const CUtensorMap* tmB, co
     const uint32_t off = is_a ? C::A_OFF + l * C::A_BOX_ROWS * 128 : C::B_OFF + b * 64 * 128;
     const uint32_t bytes = is_a ? C::A_BOX_ROWS * 128 : 64 * 128;
     uint32_t stage = 0, phase = 0, armed = 0, armed_par = 0;
-    const int total = s.tstart[p.E];
+    const int total = total_tiles(s, p);
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const Tile tl = decode_tile<BT>(t, s, p.E);
+        const Tile tl = decode_tile<BT>(t, s, p);
         const WTile wt = weight_tile<GATED>(tl, p.N);
         const int row = is_a ? tl.row0 + l * C::A_BOX_ROWS
                              : ((b >> 1) ? wt.wrow1 : wt.wrow0) + (b & 1) * 64;
@@ -342,7 +356,7 @@ __device__ void mma_role(const KParams& p, const Smem& s, const WaitCtl& wc, uin
     using C = Cfg<BT>;
     constexpr uint32_t idesc = C::SWAP ? idesc_e4m3_f32(128, BT) : idesc_e4m3_f32(128, 256);
     uint32_t stage = 0, phase = 0, j = 0, jphase = 0;
-    const int total = s.tstart[p.E];
+    const int total = total_tiles(s, p);
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         for (int kb = 0; kb < p.nkb; ++kb) {
@@ -396,11 +410,11 @@ __device__ void mma_role(const KParams& p, const Smem& s, const WaitCtl& wc, uin
 template <bool GATED>
 __device__ void scale_role(const KParams& p, const Smem& s, const WaitCtl& wc) {
     const int lane = threadIdx.x & 31;
-    const int total = s.tstart[p.E];
+    const int total = total_tiles(s, p);
     const int nkb = p.nkb;
     uint32_t slot = 0, sphase = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
-        const Tile tl = decode_tile<128>(t, s, p.E);
+        const Tile tl = decode_tile<128>(t, s, p);
         const WTile wt = weight_tile<GATED>(tl, p.N);
         const float* bs0 = p.b_scale + static_cast<long long>(wt.sb0) * nkb;
         const float* bs1 = p.b_scale + static_cast<long long>(wt.sb1) * nkb;
@@ -450,12 +464,12 @@ __device__ void epilogue_direct(const KParams& p, const Smem& s, const WaitCtl& 
     // second 128 output columns).
     const int colg = g * 64;
     uint32_t tj = 0, tjphase = 0, ephase = 0, slot = 0, sphase = 0;
-    const int total = s.tstart[p.E];
+    const int total = total_tiles(s, p);
     const int nkb = p.nkb;
     float2 acc[64];
     uint32_t va[32], vb[32];
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
-        const Tile tl = decode_tile<128>(t, s, p.E);
+        const Tile tl = decode_tile<128>(t, s, p);
         const WTile wt = weight_tile<GATED>(tl, p.N);
         const bool row_ok = rl < tl.rows;
         const int row = tl.row0 + rl;
@@ -463,7 +477,15 @@ __device__ void epilogue_direct(const KParams& p, const Smem& s, const WaitCtl& 
 #pragma unroll
         for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
         const uint32_t tlane = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + colg;
+        // combine: the row's pair id and top-k weight are fetched during the
+        // main loop (two dependent loads that may miss L2), not in the tail
+        int c_pair = -1;
+        float c_w = 0.0f;
+        if constexpr (EPI == EPI_COMBINE) c_pair = row_ok ? __ldg(p.perm + row) : -1;
         for (int kb = 0; kb < nkb; ++kb) {
+            if constexpr (EPI == EPI_COMBINE) {
+                if (kb == (nkb > 1 ? 1 : 0) && c_pair >= 0) c_w = __ldg(p.topk_w + c_pair);
+            }
             if (!warp_wait(&s.tfull[tj], tjphase, wc, 6)) return;
             tc_fence_after();
             const uint32_t tb = tlane + tj * 256;
@@ -540,13 +562,8 @@ __device__ void epilogue_direct(const KParams& p, const Smem& s, const WaitCtl& 
             // r / 2, 16-byte slot (r & 1) * 4 + ((c + r / 2) & 3) for column
             // chunk c, so both the row-wise writes and the column-wise reads
             // are free of bank conflicts.
-            int tok = -1;
-            float w = 0.0f;
-            if (row_ok) {
-                const int pair = p.perm[row];
-                tok = pair / p.topk;
-                w = p.topk_w[pair];
-            }
+            const int tok = c_pair >= 0 ? c_pair / p.topk : -1;
+            const float w = c_w;
             float* const obase = p.out_acc + tl.nt * 256 + colg;
             float* stg = s.cstage + (warp - 4) * 512;
             const int rr = lane >> 2, cc = lane & 3;
@@ -631,13 +648,13 @@ __device__ void epilogue_swap(const KParams& p, const Smem& s, const WaitCtl& wc
     const int w = q * 32 + lane;          // weight row inside each block
     const int et = threadIdx.x - 128;     // epilogue thread index 0..127
     uint32_t buf = 0, bphase = 0, ephase = 0;
-    const int total = s.tstart[p.E];
+    const int total = total_tiles(s, p);
     const int nkb = p.nkb;
     int* s_tok = reinterpret_cast<int*>(s.xch + 4 * BT);
     float* s_wt = s.xch + 5 * BT;
     float acc0[BT], acc1[BT];
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
-        const Tile tl = decode_tile<BT>(t, s, p.E);
+        const Tile tl = decode_tile<BT>(t, s, p);
         const WTile wt = weight_tile<GATED>(tl, p.N);
         // stage this tile's activation scales (and combine metadata)
         if (!epi_sync(s, ephase, wc)) return;
@@ -806,7 +823,7 @@ __global__ void __launch_bounds__(Cfg<BT>::THREADS, 1)
     if (warp == 2) {
         // per-expert tile table: tiles of expert e = ceil(rows_e / BT) * n_tiles
         const int E = p.E;
-        const int ntn = GATED ? (p.N >> 8) : ((p.N + 255) >> 8);
+        const int ntn = p.ntn_r;  // column tiles per range
         const int per = (E + 31) >> 5;
         const int lo = min(E, lane * per), hi = min(E, lo + per);
         int sum = 0;
@@ -986,6 +1003,25 @@ int launch_grouped_gemm(const GemmArgs& g, cudaStream_t stream) {
     kp.out_bf16 = static_cast<__nv_bfloat16*>(g.out_bf16);
     kp.status = g.status;
     kp.timeout_ns = g.timeout_ns;
+    // Column ranges: the combine's fp32 reductions go to out_acc[token, n];
+    // rows of every expert touch tokens all over out_acc, so when out_acc
+    // exceeds L2 each reduction would miss.  Walking the tiles one column
+    // range at a time keeps the range's slice of out_acc resident; it costs
+    // one extra read of the activations per extra range.
+    const bool gated = g.epi == EPI_SWIGLU_BF16 || g.epi == EPI_SWIGLU_QUANT;
+    const int ntn = gated ? (g.N >> 8) : ((g.N + 255) >> 8);
+    int nranges = 1;
+    if (g.epi == EPI_COMBINE && g.tile_m == 128 && ntn > 0) {
+        const long long acc_bytes =
+            static_cast<long long>(g.R / (g.topk > 0 ? g.topk : 1)) * g.out_ld * 4;
+        for (int d = 1; d <= ntn; ++d) {
+            if (ntn % d) continue;
+            nranges = d;
+            if (acc_bytes / d <= kCombineRangeBytes) break;
+        }
+    }
+    kp.nranges = nranges;
+    kp.ntn_r = ntn / nranges;
     switch (g.tile_m) {
         case 16: return launch_bt<16>(g.epi, ma, mb, kp, g.num_sms, stream);
         case 32: return launch_bt<32>(g.epi, ma, mb, kp, g.num_sms, stream);
