@@ -64,7 +64,10 @@ PROFILE_SLICES = {
 # summaries under profiles/).  A figure is reported only while the GEMM
 # sources still hash to the digest it was taken with.
 GEMM_SOURCES = ("grouped_gemm.cu", "ptx.cuh", "common.cuh", "kernels.h")
-MEASURED_TRAFFIC = {}  # workload -> (source digest, bytes per GEMM1 launch)
+MEASURED_TRAFFIC = {  # workload -> (source digest, bytes per GEMM1 launch)
+    "prefill": ("5dd440abe3e85069", 5686449109),
+    "decode": ("5dd440abe3e85069", 6528205696),
+}
 
 
 def gemm_source_digest() -> str:
