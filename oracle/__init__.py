@@ -73,6 +73,12 @@ def lib():
         L.oracle_groupwise_gemm_bf16.argtypes = [P, P, P, P, P, i, i, i, i, i, P]
         L.oracle_swiglu_mxfp8.restype = None
         L.oracle_swiglu_mxfp8.argtypes = [P, i, i, P, P]
+        L.oracle_quant_rows_mx_bf16.restype = None
+        L.oracle_quant_rows_mx_bf16.argtypes = [P, i, i, P, P]
+        L.oracle_mx_grouped_gemm.restype = None
+        L.oracle_mx_grouped_gemm.argtypes = [P, P, P, P, P, i, i, i, i, P]
+        L.oracle_mx_gemm_bf16.restype = None
+        L.oracle_mx_gemm_bf16.argtypes = [P, P, P, P, P, i, i, i, i, i, P]
         L.oracle_num_threads.restype = i
         L.oracle_num_threads.argtypes = []
     return _lib
@@ -246,6 +252,40 @@ def swiglu_mxfp8(in_bits):
     sc = np.zeros((M, K // 32), np.uint8)
     lib().oracle_swiglu_mxfp8(_p(x), M, K, _p(out), _p(sc))
     return out, sc
+
+
+# ---------------------------------------------------------------- MXFP8 variant
+def quant_rows_mx_bf16(x_bits):
+    """[rows, cols] bf16 bits -> (E4M3 codes [rows, cols], E8M0 codes [rows, cols/32])."""
+    x = _c(x_bits, np.uint16)
+    rows, cols = x.shape
+    q = np.zeros((rows, cols), np.uint8)
+    sf = np.zeros((rows, cols // 32), np.uint8)
+    lib().oracle_quant_rows_mx_bf16(_p(x), rows, cols, _p(q), _p(sf))
+    return q, sf
+
+
+def mx_grouped_gemm(a, a_sf, b, b_sf, m_indptr):
+    """fp32 [R, N]: per 32-wide K block, 2^(sa-127) 2^(sb-127) times the block dot."""
+    a = _u8(a); b = _u8(b); a_sf = _u8(a_sf); b_sf = _u8(b_sf)
+    m_indptr = _c(m_indptr, np.int32)
+    R, K = a.shape
+    E, N, _ = b.shape
+    out = np.zeros((R, N), np.float32)
+    lib().oracle_mx_grouped_gemm(_p(a), _p(a_sf), _p(b), _p(b_sf), _p(m_indptr), R, N, K, E,
+                                 _p(out))
+    return out
+
+
+def mx_gemm_bf16(a, a_sf, b, b_sf, m_indptr, is_gated: bool):
+    a = _u8(a); b = _u8(b); a_sf = _u8(a_sf); b_sf = _u8(b_sf)
+    m_indptr = _c(m_indptr, np.int32)
+    R, K = a.shape
+    E, N, _ = b.shape
+    out = np.zeros((R, N // 2 if is_gated else N), np.uint16)
+    lib().oracle_mx_gemm_bf16(_p(a), _p(a_sf), _p(b), _p(b_sf), _p(m_indptr), R, N, K, E,
+                              int(bool(is_gated)), _p(out))
+    return out
 
 
 # ---------------------------------------------------------------- tile selection

@@ -432,6 +432,95 @@ void oracle_swiglu_mxfp8(const uint16_t* in, int M, int K, uint8_t* out, uint8_t
     }
 }
 
+/* ------------------------------------------------------------------ */
+/* MXFP8 variant: one E8M0 scale per 32 consecutive K elements          */
+/* ------------------------------------------------------------------ */
+/*
+ * The Wave page names FP8 and MXFP8 as the two formats of its grouped MoE
+ * GEMM (section "들어가며"; "mxfp8 grouped MoE" timings in "왜 이게 좋은가?").
+ * MXFP8 scales every 32 consecutive elements along K with a power of two
+ * (E8M0), on both operands; the scale rule is the one above (the Cake-act
+ * page's SwiGLU + MXFP8 kernel).  Products of two E4M3 values and their sum
+ * over a 32-element block are exact in double, and so is the power-of-two
+ * scaling; the blocks are accumulated in double and the result rounded to
+ * fp32 once.  The tensor core accumulates in fp32, so the two agree to a
+ * tolerance, not bit for bit.
+ */
+
+/* x: [rows, cols] bf16 bits, cols a multiple of 32.  q: [rows, cols] E4M3
+ * codes; sf: [rows, cols/32] E8M0 codes (row-major). */
+void oracle_quant_rows_mx_bf16(const uint16_t* x, int rows, int cols, uint8_t* q, uint8_t* sf) {
+    #pragma omp parallel for schedule(static)
+    for (int r = 0; r < rows; ++r) {
+        for (int b = 0; b < cols / 32; ++b) {
+            float v[32];
+            float amax = 0.0f;
+            for (int i = 0; i < 32; ++i) {
+                v[i] = bf16_to_f32(x[(size_t)r * cols + b * 32 + i]);
+                float a = fabsf(v[i]);
+                if (a > amax) amax = a;
+            }
+            uint8_t code = oracle_e8m0_scale_code(amax);
+            float X = oracle_e8m0_decode(code);
+            sf[(size_t)r * (cols / 32) + b] = code;
+            for (int i = 0; i < 32; ++i)
+                q[(size_t)r * cols + b * 32 + i] = oracle_e4m3_encode(v[i] / X);
+        }
+    }
+}
+
+/* Grouped MXFP8 GEMM in the m_indptr layout.  a: [R, K] codes, a_sf [R, K/32];
+ * b: [E, N, K] codes, b_sf [E, N, K/32]; rows [m_indptr[e], m_indptr[e+1])
+ * use expert e.  out: [R, N] fp32 (rows outside every group untouched). */
+void oracle_mx_grouped_gemm(const uint8_t* a, const uint8_t* a_sf, const uint8_t* b,
+                            const uint8_t* b_sf, const int32_t* m_indptr, int R, int N, int K,
+                            int E, float* out) {
+    float dec[256];
+    make_decode_table(dec);
+    const int nb = K / 32;
+    (void)R;
+    for (int e = 0; e < E; ++e) {
+        #pragma omp parallel for schedule(static)
+        for (int r = m_indptr[e]; r < m_indptr[e + 1]; ++r) {
+            const uint8_t* ar = a + (size_t)r * K;
+            for (int n = 0; n < N; ++n) {
+                const size_t wrow = (size_t)e * N + n;
+                const uint8_t* br = b + wrow * K;
+                double acc = 0.0;
+                for (int blk = 0; blk < nb; ++blk) {
+                    double s = 0.0;
+                    for (int i = 0; i < 32; ++i)
+                        s += (double)dec[ar[blk * 32 + i]] * (double)dec[br[blk * 32 + i]];
+                    const int ex = (int)a_sf[(size_t)r * nb + blk] + (int)b_sf[wrow * nb + blk] - 254;
+                    acc += ldexp(s, ex);
+                }
+                out[(size_t)r * N + n] = (float)acc;
+            }
+        }
+    }
+}
+
+/* bf16 output of the MXFP8 GEMM: plain out [R, N], or gated out [R, N/2] =
+ * bf16(silu(G[:, :N/2]) * G[:, N/2:]) with G rounded to fp32 first. */
+void oracle_mx_gemm_bf16(const uint8_t* a, const uint8_t* a_sf, const uint8_t* b,
+                         const uint8_t* b_sf, const int32_t* m_indptr, int R, int N, int K, int E,
+                         int is_gated, uint16_t* out) {
+    float* g = (float*)malloc(sizeof(float) * ((size_t)R * N + 1));
+    for (size_t i = 0; i < (size_t)R * N; ++i) g[i] = 0.0f;
+    oracle_mx_grouped_gemm(a, a_sf, b, b_sf, m_indptr, R, N, K, E, g);
+    int Rg = m_indptr[E];
+    if (!is_gated) {
+        for (size_t i = 0; i < (size_t)Rg * N; ++i) out[i] = f32_to_bf16(g[i]);
+    } else {
+        int I = N / 2;
+        float* h = (float*)malloc(sizeof(float) * ((size_t)R * I + 1));
+        oracle_swiglu(g, Rg, I, h);
+        for (size_t i = 0; i < (size_t)Rg * I; ++i) out[i] = f32_to_bf16(h[i]);
+        free(h);
+    }
+    free(g);
+}
+
 /* Threads an OpenMP parallel region would use (0 when built without it). */
 int oracle_num_threads(void) {
 #ifdef _OPENMP
