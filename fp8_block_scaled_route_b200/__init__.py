@@ -23,7 +23,7 @@ __all__ = [
     "moe_route_permute", "moe_fp8_fused", "moe_fp8_fused_debug", "fp8_groupwise_moe_gemm",
     "swiglu_mxfp8_quant", "moe_select_tile_m", "moe_workspace_size", "moe_route_workspace_size",
     "moe_get_device_status", "moe_set_wait_timeout_ns", "moe_status_string",
-    "moe_set_stage_events", "moe_route_permute_noalloc",
+    "moe_set_stage_events", "moe_route_permute_noalloc", "mxfp8_moe_gemm",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -42,7 +42,7 @@ EXPORTS = (
     "moe_status_string", "moe_route_workspace_size", "moe_route_permute", "moe_workspace_size",
     "moe_fp8_fused", "moe_fp8_fused_debug", "fp8_groupwise_moe_gemm", "moe_select_tile_m",
     "swiglu_mxfp8_quant", "moe_get_device_status", "moe_set_wait_timeout_ns",
-    "moe_set_stage_events", "moe_route_permute_noalloc",
+    "moe_set_stage_events", "moe_route_permute_noalloc", "mxfp8_moe_gemm",
 )
 
 _lib = None
@@ -86,6 +86,8 @@ def lib():
     L.moe_select_tile_m.argtypes = [I] * 6 + [ctypes.POINTER(I), ctypes.POINTER(I)]
     L.swiglu_mxfp8_quant.restype = I
     L.swiglu_mxfp8_quant.argtypes = [P, P, P, I, I, P]
+    L.mxfp8_moe_gemm.restype = I
+    L.mxfp8_moe_gemm.argtypes = [P] * 6 + [I] * 5 + [P]
     L.moe_get_device_status.restype = I
     L.moe_get_device_status.argtypes = [P, P]
     L.moe_set_wait_timeout_ns.restype = None
@@ -215,6 +217,21 @@ def fp8_groupwise_moe_gemm(a, b, a_scale, b_scale, m_indptr, out, scale_major_mo
                                       _ptr(m_indptr), _ptr(out), R, N, K, E, mode, sg_m, sg_n,
                                       sg_k, int(bool(is_gated)), tile_m, tile_n, _stream(stream))
     return _check(st, "fp8_groupwise_moe_gemm", check)
+
+
+def mxfp8_moe_gemm(a, b, a_sf, b_sf, m_indptr, out, is_gated=False, *, dims=None, stream=None,
+                   check=True) -> int:
+    """a [R,K] fp8, b [E,N,K] fp8, a_sf [R,K/32] / b_sf [E,N,K/32] uint8 E8M0,
+    out bf16 [R, N/2 if gated else N].  dims = (R, N, K, E) when raw addresses
+    are passed."""
+    if dims is None:
+        R, K = a.shape
+        E, N, _ = b.shape
+    else:
+        R, N, K, E = dims
+    st = lib().mxfp8_moe_gemm(_ptr(a), _ptr(b), _ptr(a_sf), _ptr(b_sf), _ptr(m_indptr), _ptr(out),
+                              R, N, K, E, int(bool(is_gated)), _stream(stream))
+    return _check(st, "mxfp8_moe_gemm", check)
 
 
 def swiglu_mxfp8_quant(inp, out, scale, *, dims=None, stream=None, check=True) -> int:

@@ -347,6 +347,32 @@ int fp8_groupwise_moe_gemm(const void* a, const void* b, const float* a_scale, c
     return launch_grouped_gemm(g, s);
 }
 
+int mxfp8_moe_gemm(const void* a, const void* b, const uint8_t* a_sf, const uint8_t* b_sf,
+                   const int32_t* m_indptr, void* out, int R, int N, int K, int E, int is_gated,
+                   moe_stream_t stream) {
+    if (R < 0 || N <= 0 || K <= 0 || E < 1 || N % 128 || K % 128) return MOE_ERR_INVALID_ARG;
+    if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+    if (is_gated && (N % 2 || (N / 2) % 128)) return MOE_ERR_INVALID_ARG;
+    if (!m_indptr || (R > 0 && (!a || !b || !a_sf || !b_sf || !out))) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(b) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(a_sf) | reinterpret_cast<uintptr_t>(b_sf)) & 3)
+        return MOE_ERR_INVALID_ARG;
+    const DevInfo* d = dev_info();
+    if (int st = check_device(d)) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(d->lib_status, 0, sizeof(int) * kStatusInts, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (R == 0) return MOE_OK;
+    MxGemmArgs g{};
+    g.a = a; g.b = b; g.a_sf = a_sf; g.b_sf = b_sf; g.m_indptr = m_indptr;
+    g.R = R; g.N = N; g.K = K; g.E = E; g.gated = is_gated ? 1 : 0;
+    g.out = out;
+    g.status = d->lib_status;
+    g.timeout_ns = g_timeout_ns.load();
+    g.num_sms = d->sms;
+    return launch_mx_gemm(g, s);
+}
+
 int swiglu_mxfp8_quant(const void* in, void* out, uint8_t* scale, int M, int K, moe_stream_t stream) {
     if (M < 0 || K <= 0 || K % 32) return MOE_ERR_INVALID_ARG;
     if (M > 0 && (!in || !out || !scale)) return MOE_ERR_INVALID_ARG;

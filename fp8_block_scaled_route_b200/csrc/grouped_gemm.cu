@@ -937,6 +937,15 @@ bool make_map(CUtensorMap* out, const void* ptr, long long rows, long long cols,
     return true;
 }
 
+}  // namespace
+
+bool make_tma_map_fp8(CUtensorMap* out, const void* ptr, long long rows, long long cols,
+                      int box_rows) {
+    return make_map(out, ptr, rows, cols, box_rows);
+}
+
+namespace {
+
 template <int BT, int EPI>
 int launch_inst(const CUtensorMap& ma, const CUtensorMap& mb, const KParams& kp, int num_sms,
                 cudaStream_t stream) {

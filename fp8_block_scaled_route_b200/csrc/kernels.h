@@ -70,4 +70,21 @@ int launch_f32_to_bf16(const float* in, void* out, long long n, int num_sms, cud
 int launch_swiglu_mxfp8(const void* in, void* out, uint8_t* scale, int M, int K, int num_sms,
                         cudaStream_t stream);
 
+// Grouped MXFP8 GEMM on the block-scaled tensor core path: E4M3 operands with
+// one E8M0 scale per 32 K elements of every row of A and of B.
+struct MxGemmArgs {
+    const void* a;            // [R, K] E4M3, grouped rows
+    const void* b;            // [E, N, K] E4M3
+    const uint8_t* a_sf;      // [R, K/32] E8M0, row-major
+    const uint8_t* b_sf;      // [E, N, K/32] E8M0, row-major
+    const int32_t* m_indptr;  // [E+1]
+    int R, N, K, E;
+    int gated;                // out [R, N/2] = bf16(silu(G_gate) * G_up), else [R, N] = bf16(G)
+    void* out;
+    int* status;
+    uint64_t timeout_ns;
+    int num_sms;
+};
+int launch_mx_gemm(const MxGemmArgs& g, cudaStream_t stream);
+
 }  // namespace moe

@@ -1,0 +1,427 @@
+// Grouped MXFP8 GEMM on the block-scaled tensor core path.
+//
+// Format: E4M3 operands with one E8M0 (power-of-two) scale per 32 consecutive
+// K elements of every row of A and of B -- the MXFP8 format that the page
+// "FlashInfer SM120 MoE GEMM 최적화: 웨이브+잔여물 비용 모델 도입" names beside
+// FP8 for its grouped MoE GEMM (section "들어가며"; "mxfp8 grouped MoE" timings
+// in "왜 이게 좋은가?"), with the scale rule of the SwiGLU + MXFP8 kernel of the
+// page "NVIDIA R200(SM107)을 위한 SwiGLU + MXFP8 커널 최적화".
+//
+// Because the scales are powers of two, tcgen05.mma kind::mxf8f6f4.block_scale
+// applies them inside the tensor core: the accumulator stays in TMEM for the
+// whole K loop and the epilogue reads it once per tile (the FP8 kernel with
+// fp32 block scales has to read and promote every 128-wide K block).
+//
+// Tile: 128 grouped rows (MMA M) x 256 weight rows (MMA N; gated: 128 gate +
+// 128 up rows), persistent CTAs, 4-stage ring of 50 KB stages:
+//   A  128 x 128 B  (TMA, 128-byte swizzle)        16 KB
+//   B  256 x 128 B  (TMA, 128-byte swizzle)        32 KB
+//   SF A 128 rows x 4 scales, B 256 rows x 4 scales, each 128-row group in
+//      the 512-byte layout byte(r, j) = (r % 32) * 16 + (r / 32) * 4 + j
+//      (j = 32-wide K step), copied from row-major [rows, K/32] by cp.async
+// Warps: 0 TMA producer, 1 MMA issuer (elected lane), 2 scale-factor loader,
+// 3 idle, 4-11 epilogue.  TMEM: accumulator columns [0, 256), A scale factors
+// [256, 260), B scale factors [264, 272); one tcgen05.cp per 128 rows moves a
+// stage's scale factors into TMEM ahead of its four MMAs (issued by the same
+// thread, so they are ordered).
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+bool make_tma_map_fp8(CUtensorMap* out, const void* ptr, long long rows, long long cols,
+                      int box_rows);
+
+namespace {
+
+constexpr int kMxStages = 4;
+constexpr int kMxA = 128 * 128;
+constexpr int kMxB = 256 * 128;
+constexpr int kMxSfOff = kMxA + kMxB;
+constexpr int kMxStage = kMxA + kMxB + 2048;  // scale factors: 512 (A) + 1024 (B), padded
+constexpr int kMxMaxE = 1024;
+constexpr int kMxTable = ((2 * (kMxMaxE + 1) * 4) + 15) / 16 * 16;
+constexpr int kMxSmem = 1024 + kMxStages * kMxStage + kMxTable + 256;
+constexpr int kMxThreads = 384;
+constexpr int kMxEpiWarps = 8;
+constexpr int kMxBoxes = 6;  // TMA boxes per stage: 2 x 64 token rows, 4 x 64 weight rows
+constexpr uint32_t kMxTmemCols = 512;
+constexpr uint32_t kMxSfaCol = 256;
+constexpr uint32_t kMxSfbCol = 264;
+static_assert(kMxStage % 1024 == 0, "stages must stay 1024-byte aligned for the swizzle");
+static_assert(kMxSmem <= 232448, "shared memory budget");
+
+struct MxParams {
+    int R, N, K, E, nkb, gated;
+    const uint8_t* a_sf;
+    const uint8_t* b_sf;
+    const int32_t* m_indptr;
+    __nv_bfloat16* out;
+    int* status;
+    unsigned long long timeout_ns;
+};
+
+struct MxSmem {
+    uint8_t* stages;
+    int* tstart;  // [E+1] first tile of each expert
+    int* mind;    // [E+1] clamped m_indptr
+    uint64_t* full;
+    uint64_t* empty;
+    uint64_t* tfull;
+    uint64_t* tempty;
+    uint64_t* drain;
+    uint32_t* tmem;
+    volatile int* abort;
+};
+
+__device__ __forceinline__ MxSmem mx_carve(uint8_t* base) {
+    MxSmem s;
+    s.stages = base;
+    uint8_t* p = base + kMxStages * kMxStage;
+    s.tstart = reinterpret_cast<int*>(p);
+    s.mind = s.tstart + (kMxMaxE + 1);
+    p += kMxTable;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(p);
+    s.full = bars;
+    s.empty = bars + kMxStages;
+    s.tfull = bars + 2 * kMxStages;
+    s.tempty = bars + 2 * kMxStages + 1;
+    s.drain = bars + 2 * kMxStages + 2;
+    s.tmem = reinterpret_cast<uint32_t*>(bars + 2 * kMxStages + 3);
+    s.abort = reinterpret_cast<volatile int*>(bars + 2 * kMxStages + 4);
+    return s;
+}
+
+struct MxTile {
+    int e, nt, row0, rows;
+};
+
+// Tile t -> (expert, column tile, 128-row tile); column tiles outer within an
+// expert so that consecutive CTAs share the weight tile.
+__device__ __forceinline__ MxTile mx_decode(int t, const MxSmem& s, int E) {
+    int lo = 0, hi = E;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s.tstart[mid] <= t) lo = mid; else hi = mid;
+    }
+    MxTile r;
+    r.e = lo;
+    const int local = t - s.tstart[lo];
+    const int me = max(0, s.mind[lo + 1] - s.mind[lo]);
+    const int mtiles = (me + 127) / 128;
+    r.nt = local / mtiles;
+    const int mt = local - r.nt * mtiles;
+    r.row0 = s.mind[lo] + mt * 128;
+    r.rows = min(128, me - mt * 128);
+    return r;
+}
+
+// Global weight rows of the tile's two 128-row blocks.
+__device__ __forceinline__ void mx_weight_rows(const MxTile& t, const MxParams& p, int& w0, int& w1) {
+    if (p.gated) {
+        w0 = t.e * p.N + t.nt * 128;
+        w1 = t.e * p.N + (p.N >> 1) + t.nt * 128;
+    } else {
+        w0 = t.e * p.N + t.nt * 256;
+        w1 = w0 + 128;
+    }
+}
+
+__device__ __forceinline__ bool mx_warp_wait_spin(uint64_t* bar, uint32_t parity, const WaitCtl& wc,
+                                                  int where) {
+    return __all_sync(0xffffffffu, wait_bar_spin(bar, parity, wc, where)) != 0;
+}
+__device__ __forceinline__ bool mx_warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& wc,
+                                             int where) {
+    return __all_sync(0xffffffffu, wait_bar(bar, parity, wc, where)) != 0;
+}
+
+// Warp 0: lane l < 6 issues TMA box l of every stage.
+__device__ void mx_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const MxParams& p,
+                            const MxSmem& s, const WaitCtl& wc, int total) {
+    const int l = threadIdx.x & 31;
+    const bool issuer = l < kMxBoxes;
+    const bool is_a = l < 2;
+    const int b = l - 2;  // weight box 0..3: block b/2, half b%2
+    const uint32_t off = is_a ? l * 64 * 128 : kMxA + b * 64 * 128;
+    uint32_t stage = 0, phase = 0, armed = 0, armed_par = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const MxTile tl = mx_decode(t, s, p.E);
+        int w0, w1;
+        mx_weight_rows(tl, p, w0, w1);
+        const int row = is_a ? tl.row0 + l * 64 : ((b >> 1) ? w1 : w0) + (b & 1) * 64;
+        for (int kb = 0; kb < p.nkb; ++kb) {
+            if (!mx_warp_wait_spin(&s.empty[stage], phase ^ 1, wc, 1)) { ok = false; break; }
+            if (issuer) {
+                mbar_arrive_expect_tx(&s.full[stage], 64 * 128);
+                tma_load_2d(s.stages + stage * kMxStage + off, is_a ? tmA : tmB, &s.full[stage],
+                            kb * 128, row);
+            }
+            __syncwarp();
+            armed |= 1u << stage;
+            armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+            if (++stage == kMxStages) { stage = 0; phase ^= 1; }
+        }
+    }
+    for (int st = 0; st < kMxStages; ++st)
+        if ((armed >> st) & 1u) wait_bar(&s.full[st], (armed_par >> st) & 1u, wc, 2, /*drain=*/true);
+    __syncwarp();
+}
+
+// Warp 2: per stage, the 4 E8M0 scales (one 32-bit word of a row-major
+// [rows, K/32] array) of each of the tile's 128 token rows and 256 weight rows,
+// written into the 512-byte tcgen05.cp layout; completion arrives on the
+// stage's full barrier.  Rows past the ends read as 0 (scale 2^-127).
+__device__ void mx_sf_loader(const MxParams& p, const MxSmem& s, const WaitCtl& wc, int total) {
+    const int lane = threadIdx.x & 31;
+    const int nsf = p.K >> 5;  // scale bytes per row
+    const long long wrows = static_cast<long long>(p.E) * p.N;
+    uint32_t stage = 0, phase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const MxTile tl = mx_decode(t, s, p.E);
+        int w0, w1;
+        mx_weight_rows(tl, p, w0, w1);
+        for (int kb = 0; kb < p.nkb; ++kb) {
+            if (!mx_warp_wait(&s.empty[stage], phase ^ 1, wc, 8)) { ok = false; break; }
+            uint8_t* sf = s.stages + stage * kMxStage + kMxSfOff;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {  // token row lane + 32 i
+                const int r = tl.row0 + lane + 32 * i;
+                const bool v = r < p.R;
+                const uint8_t* src = v ? p.a_sf + static_cast<long long>(r) * nsf + kb * 4 : p.a_sf;
+                cp_async_4(sf + lane * 16 + i * 4, src, v ? 4u : 0u);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {  // weight row lane + 32 i of the tile
+                const int j = lane + 32 * i;
+                const long long w = (j < 128 ? w0 + j : w1 + (j - 128));
+                const bool v = w < wrows;
+                const uint8_t* src = v ? p.b_sf + w * nsf + kb * 4 : p.b_sf;
+                cp_async_4(sf + 512 + (i >> 2) * 512 + lane * 16 + (i & 3) * 4, src, v ? 4u : 0u);
+            }
+            cp_async_arrive_noinc(&s.full[stage]);
+            if (++stage == kMxStages) { stage = 0; phase ^= 1; }
+        }
+    }
+    cp_async_wait_all();
+    __syncwarp();
+}
+
+// Warp 1: per stage, the scale factors into TMEM and four K=32 block-scaled
+// MMAs (elected lane); the accumulator is released by the epilogue per tile.
+__device__ void mx_mma(const MxParams& p, const MxSmem& s, const WaitCtl& wc, uint32_t tmem_base,
+                       int total) {
+    uint32_t stage = 0, phase = 0, it = 0;
+    bool ok = true;
+    const uint32_t sfa_t = tmem_base + kMxSfaCol;
+    const uint32_t sfb_t = tmem_base + kMxSfbCol;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+        if (!mx_warp_wait_spin(s.tempty, (it & 1) ^ 1, wc, 3)) break;
+        tc_fence_after();
+        for (int kb = 0; kb < p.nkb; ++kb) {
+            if (!mx_warp_wait_spin(&s.full[stage], phase, wc, 4)) { ok = false; break; }
+            tc_fence_after();
+            uint8_t* st = s.stages + stage * kMxStage;
+            const uint32_t sa = smem_u32(st);
+            const uint32_t sb = smem_u32(st + kMxA);
+            const uint32_t ssf = smem_u32(st + kMxSfOff);
+            if (elect_one()) {
+                tmem_cp_32x128b_x4(sfa_t, smem_desc_k_noswizzle(ssf, 16, 128));
+                tmem_cp_32x128b_x4(sfb_t, smem_desc_k_noswizzle(ssf + 512, 16, 128));
+                tmem_cp_32x128b_x4(sfb_t + 4, smem_desc_k_noswizzle(ssf + 1024, 16, 128));
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_mx(tmem_base, smem_desc_k_sw128(sa + kk * 32), smem_desc_k_sw128(sb + kk * 32),
+                            idesc_mx_e4m3(128, 256, kk, kk), sfa_t | (static_cast<uint32_t>(kk) << 30),
+                            sfb_t | (static_cast<uint32_t>(kk) << 30), (kb | kk) != 0);
+                umma_commit(&s.empty[stage]);
+                if (kb == p.nkb - 1) umma_commit(s.tfull);
+            }
+            __syncwarp();
+            if (++stage == kMxStages) { stage = 0; phase ^= 1; }
+        }
+    }
+    if (elect_one()) umma_commit(s.drain);
+    __syncwarp();
+    wait_bar(s.drain, 0, wc, 5, /*drain=*/true);
+    __syncwarp();
+}
+
+__device__ __forceinline__ float mx_silu(float z) { return z * rcp_approx(1.0f + __expf(-z)); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    uint32_t u;
+    memcpy(&u, &h, 4);
+    return u;
+}
+
+// Warps 4-11: thread = one row of the tile, 64 columns of each weight block
+// (warp w: rows 32 (w % 4) .. +31, column half (w - 4) / 4).
+__device__ void mx_epilogue(const MxParams& p, const MxSmem& s, const WaitCtl& wc,
+                            uint32_t tmem_base, int total) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = warp & 3;
+    const int g = (warp - 4) >> 2;
+    const int rl = q * 32 + lane;
+    const int colg = g * 64;
+    const uint32_t tl_addr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + colg;
+    uint32_t it = 0;
+    uint32_t v[4][32];
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+        const MxTile tl = mx_decode(t, s, p.E);
+        if (!mx_warp_wait(s.tfull, it & 1, wc, 6)) return;
+        tc_fence_after();
+        tmem_ld32_async(tl_addr, v[0]);
+        tmem_ld32_async(tl_addr + 32, v[1]);
+        tmem_ld32_async(tl_addr + 128, v[2]);
+        tmem_ld32_async(tl_addr + 160, v[3]);
+        tmem_wait_ld(v[0]);
+        tmem_wait_ld(v[1]);
+        tmem_wait_ld(v[2]);
+        tmem_wait_ld(v[3]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s.tempty);
+        if (rl >= tl.rows) continue;
+        const long long row = tl.row0 + rl;
+        if (p.gated) {
+            // h = silu(gate) * up, 64 bf16 values per row
+            uint4* dst = reinterpret_cast<uint4*>(p.out + row * (p.N >> 1) + tl.nt * 128 + colg);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                float h[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int j = 8 * c + i;
+                    h[i] = mx_silu(__uint_as_float(v[j >> 5][j & 31])) *
+                           __uint_as_float(v[2 + (j >> 5)][j & 31]);
+                }
+                dst[c] = make_uint4(pack_bf16(h[0], h[1]), pack_bf16(h[2], h[3]),
+                                    pack_bf16(h[4], h[5]), pack_bf16(h[6], h[7]));
+            }
+        } else {
+            const int n0 = tl.nt * 256;
+            __nv_bfloat16* rowp = p.out + row * p.N + n0 + colg;
+#pragma unroll
+            for (int blk = 0; blk < 2; ++blk) {
+                if (n0 + blk * 128 >= p.N) break;
+                uint4* dst = reinterpret_cast<uint4*>(rowp + blk * 128);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint32_t* a = v[2 * blk + (c >> 2)] + (c & 3) * 8;
+                    dst[c] = make_uint4(pack_bf16(__uint_as_float(a[0]), __uint_as_float(a[1])),
+                                        pack_bf16(__uint_as_float(a[2]), __uint_as_float(a[3])),
+                                        pack_bf16(__uint_as_float(a[4]), __uint_as_float(a[5])),
+                                        pack_bf16(__uint_as_float(a[6]), __uint_as_float(a[7])));
+                }
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kMxThreads, 1)
+    mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const MxParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const MxSmem s = mx_carve(base);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kMxStages; ++i) {
+            mbar_init(&s.full[i], kMxBoxes + 32);
+            mbar_init(&s.empty[i], 1);
+        }
+        mbar_init(s.tfull, 1);
+        mbar_init(s.tempty, kMxEpiWarps);
+        mbar_init(s.drain, 1);
+        *s.abort = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(s.tmem, kMxTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 2) {
+        // per-expert tile table: tiles of expert e = ceil(rows_e / 128) * column tiles
+        const int E = p.E;
+        const int ntn = p.gated ? (p.N >> 8) : ((p.N + 255) >> 8);
+        const int per = (E + 31) >> 5;
+        const int lo = min(E, lane * per), hi = min(E, lo + per);
+        int sum = 0;
+        for (int e = lo; e < hi; ++e) {
+            const int m0 = min(max(p.m_indptr[e], 0), p.R);
+            const int m1 = min(max(p.m_indptr[e + 1], 0), p.R);
+            s.mind[e] = m0;
+            sum += ((max(0, m1 - m0) + 127) / 128) * ntn;
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int x = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += x;
+        }
+        int run = incl - sum;
+        for (int e = lo; e < hi; ++e) {
+            s.tstart[e] = run;
+            const int m0 = s.mind[e];
+            const int m1 = min(max(p.m_indptr[e + 1], 0), p.R);
+            run += ((max(0, m1 - m0) + 127) / 128) * ntn;
+        }
+        if (lane == 31) {
+            s.tstart[E] = incl;
+            s.mind[E] = min(max(p.m_indptr[E], 0), p.R);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *s.tmem;
+    const WaitCtl wc{s.abort, p.status, p.timeout_ns};
+    const int total = s.tstart[p.E];
+    if (warp == 0) mx_producer(&tmA, &tmB, p, s, wc, total);
+    else if (warp == 1) mx_mma(p, s, wc, tmem_base, total);
+    else if (warp == 2) mx_sf_loader(p, s, wc, total);
+    else if (warp >= 4) mx_epilogue(p, s, wc, tmem_base, total);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, kMxTmemCols);
+}
+
+}  // namespace
+
+int launch_mx_gemm(const MxGemmArgs& g, cudaStream_t stream) {
+    if (g.R <= 0 || g.E <= 0) return ST_OK;
+    if (g.E > kMxMaxE) return ST_INVALID_ARG;
+    CUtensorMap ma, mb;
+    if (!make_tma_map_fp8(&ma, g.a, g.R, g.K, 64)) return ST_CUDA;
+    if (!make_tma_map_fp8(&mb, g.b, static_cast<long long>(g.E) * g.N, g.K, 64)) return ST_CUDA;
+    MxParams p;
+    p.R = g.R; p.N = g.N; p.K = g.K; p.E = g.E; p.nkb = g.K / 128; p.gated = g.gated ? 1 : 0;
+    p.a_sf = g.a_sf; p.b_sf = g.b_sf; p.m_indptr = g.m_indptr;
+    p.out = static_cast<__nv_bfloat16*>(g.out);
+    p.status = g.status;
+    p.timeout_ns = g.timeout_ns;
+    static int configured_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+        if (cudaFuncSetAttribute(mx_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kMxSmem) != cudaSuccess)
+            return ST_CUDA;
+        configured_dev = dev;
+    }
+    mx_gemm_kernel<<<g.num_sms, kMxThreads, kMxSmem, stream>>>(ma, mb, p);
+    return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
+}
+
+}  // namespace moe

@@ -226,6 +226,57 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t smem_addr) {
     return d;
 }
 
+// Descriptor of an unswizzled K-major shared-memory operand: core matrices of
+// 8 rows x 16 bytes (rows 16 bytes apart), `lbo` bytes between core matrices
+// along K, `sbo` bytes between groups of 8 rows.
+__device__ __forceinline__ uint64_t smem_desc_k_noswizzle(uint32_t smem_addr, uint32_t lbo,
+                                                          uint32_t sbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((smem_addr & 0x3FFFF) >> 4);
+    d |= static_cast<uint64_t>((lbo & 0x3FFFF) >> 4) << 16;
+    d |= static_cast<uint64_t>((sbo & 0x3FFFF) >> 4) << 32;
+    d |= static_cast<uint64_t>(1) << 46;  // descriptor version (sm_100); layout 0 = no swizzle
+    return d;
+}
+
+// Block-scaled MMA, kind::mxf8f6f4: D (+)= (A . 2^SFA) x (B . 2^SFB)^T for one
+// K=32 step, with one E8M0 scale per row of A and per row of B read from the
+// TMEM columns at sfa_tmem / sfb_tmem (byte `sf id` of each column, also in
+// bits 30-31 of the address).
+__device__ __forceinline__ void umma_mx(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                        uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                        uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem),
+        "r"(accumulate)
+        : "memory");
+}
+
+// Shared -> TMEM copy of 32 rows x 16 bytes into 4 columns of lanes 0-31,
+// replicated to the four 32-lane quarters (the scale-factor layout the
+// block-scaled MMA reads).  Asynchronous; ordered before later tcgen05.mma of
+// the same thread.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+                 : "memory");
+}
+
+// Instruction descriptor, block-scaled kind::mxf8f6f4: E4M3 x E4M3 -> fp32,
+// E8M0 scale factors, K-major operands; a_id / b_id select the byte of each
+// scale-factor column.
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3(int M, int N, int a_id, int b_id) {
+    return (static_cast<uint32_t>(b_id & 3) << 4)          // B scale factor id
+           | (0u << 7) | (0u << 10)                        // A, B format E4M3
+           | (0u << 15) | (0u << 16)                       // A, B K-major
+           | (static_cast<uint32_t>(N >> 3) << 17)         // N / 8
+           | (1u << 23)                                    // scale format E8M0
+           | (static_cast<uint32_t>(M >> 4) << 24)         // M / 16
+           | (static_cast<uint32_t>(a_id & 3) << 29);      // A scale factor id
+}
+
 // Instruction descriptor: E4M3 x E4M3 -> fp32, both operands K-major.
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
     return (1u << 4)                                   // D format fp32
@@ -237,6 +288,9 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
 
 // ----------------------------------------------------------------- cp.async
 // 4-byte asynchronous global -> shared copy; src_bytes = 0 writes zeros.
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
 __device__ __forceinline__ void cp_async_4(void* smem_dst, const void* gmem_src, uint32_t src_bytes) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(smem_dst)),
                  "l"(gmem_src), "r"(src_bytes)

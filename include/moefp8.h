@@ -185,6 +185,35 @@ MOE_API int moe_select_tile_m(int total_rows, int n, int k, int E, int num_sms, 
                       int* tile_m, int* tile_n);
 
 /* ------------------------------------------------------------------ */
+/* Grouped MXFP8 GEMM (block-scaled tensor core path)                   */
+/* ------------------------------------------------------------------ */
+
+/* The MXFP8 grouped MoE GEMM that the page "FlashInfer SM120 MoE GEMM 최적화:
+ * 웨이브+잔여물 비용 모델 도입" names beside FP8 (section "들어가며"; "mxfp8
+ * grouped MoE" in "왜 이게 좋은가?"): E4M3 operands with one E8M0 scale per 32
+ * consecutive K elements of every row of A and of B, in the grouped layout of
+ * fp8_groupwise_moe_gemm:
+ *   G[r, n] = sum over 32-wide K blocks b of
+ *             2^(a_sf[r,b]-127) * 2^(b_sf[e,n,b]-127) * sum_k a[r,k] * b[e,n,k],
+ *   e = the expert with m_indptr[e] <= r < m_indptr[e+1];
+ * accumulated in fp32 by the tensor core (the scales are applied inside it).
+ *  a       device FP8  [R, K] grouped rows
+ *  b       device FP8  [E, N, K]
+ *  a_sf    device uint8 [R, K/32] E8M0 codes, row-major (4-byte aligned)
+ *  b_sf    device uint8 [E, N, K/32] E8M0 codes, row-major (4-byte aligned)
+ *  m_indptr device int32 [E+1]
+ *  out     device bf16: plain [R, N] = bf16(G); gated [R, N/2] =
+ *          bf16(silu(G[:, :N/2]) * G[:, N/2:]) (gate rows then up rows of b)
+ * Rows outside [m_indptr[0], m_indptr[E]) are not written.  K and N must be
+ * multiples of 128 (gated: N/2 too); a, b, out 16-byte aligned.  Returns
+ * MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED on bad arguments before any
+ * launch; device timeouts are read with moe_get_device_status(NULL, stream).
+ * Caller owns all memory; asynchronous on `stream`. */
+MOE_API int mxfp8_moe_gemm(const void* a, const void* b, const uint8_t* a_sf,
+                           const uint8_t* b_sf, const int32_t* m_indptr, void* out,
+                           int R, int N, int K, int E, int is_gated, moe_stream_t stream);
+
+/* ------------------------------------------------------------------ */
 /* Standalone SwiGLU + MXFP8 quantisation                               */
 /* ------------------------------------------------------------------ */
 

@@ -143,3 +143,53 @@ def make_grouped_gemm_inputs(R: int, N: int, K: int, E: int, seed: int = 0, devi
     b, b_scale = _expert_weights(E, N, K, 1.0 / math.sqrt(K), g, device)
     return dict(a=a.contiguous(), a_scale=a_scale.contiguous(), b=b, b_scale=b_scale,
                 m_indptr=m_indptr)
+
+
+def quantize_mx_rows(x: torch.Tensor):
+    """[rows, cols] fp32 -> (float8_e4m3fn [rows, cols], uint8 E8M0 codes
+    [rows, cols/32]): per 32 consecutive values the smallest power of two 2^s
+    with amax <= 448 * 2^s (code s + 127, all-zero blocks code 0), then
+    torch's float8 cast of x / 2^s (exact power-of-two scaling)."""
+    rows, cols = x.shape
+    blocks = x.view(rows, cols // 32, 32)
+    amax = blocks.abs().amax(dim=2).to(torch.float64)
+    s = torch.ceil(torch.log2(torch.clamp(amax, min=1e-300) / 448.0))
+    s = torch.where(amax > torch.ldexp(torch.full_like(amax, 448.0), s), s + 1, s)
+    s = torch.where(amax <= torch.ldexp(torch.full_like(amax, 448.0), s - 1), s - 1, s)
+    code = torch.clamp(s + 127, 0, 254)
+    code = torch.where(amax > 0, code, torch.zeros_like(code))
+    X = torch.ldexp(torch.ones_like(amax), (code - 127).to(torch.int64)).to(torch.float32)
+    q = (blocks / X[:, :, None]).to(torch.float8_e4m3fn).view(rows, cols)
+    return q.contiguous(), code.to(torch.uint8).contiguous()
+
+
+def make_mx_gemm_inputs(R: int, N: int, K: int, E: int, seed: int = 0, device="cpu",
+                        group_sizes=None, spread: int = 4):
+    """Inputs for the MXFP8 grouped GEMM: activations N(0,1) and weights
+    N(0, 1/K), each 32-wide K block of a row multiplied by 2^u with u uniform
+    in [-spread, spread] (so the scales differ from block to block), then
+    quantised to MXFP8 (quantize_mx_rows); m_indptr as in
+    make_grouped_gemm_inputs."""
+    g = _gen(seed, device)
+    if group_sizes is None:
+        idx = torch.randint(0, E, (R,), generator=g, device=device)
+        group_sizes = torch.bincount(idx, minlength=E)
+    group_sizes = torch.as_tensor(group_sizes, device=device, dtype=torch.int64)
+    m_indptr = torch.zeros(E + 1, dtype=torch.int32, device=device)
+    m_indptr[1:] = torch.cumsum(group_sizes, 0).to(torch.int32)
+    R = int(m_indptr[-1])
+
+    def spread_blocks(x):
+        u = torch.randint(-spread, spread + 1, (x.shape[0], x.shape[1] // 32), generator=g,
+                          device=device).to(torch.float32)
+        return (x.view(x.shape[0], -1, 32) * torch.exp2(u)[:, :, None]).view(x.shape)
+
+    a32 = spread_blocks(torch.randn(R, K, generator=g, device=device, dtype=torch.float32))
+    a, a_sf = quantize_mx_rows(a32)
+    b = torch.empty(E, N, K, dtype=torch.float8_e4m3fn, device=device)
+    b_sf = torch.empty(E, N, K // 32, dtype=torch.uint8, device=device)
+    for e in range(E):
+        w = spread_blocks(torch.randn(N, K, generator=g, device=device, dtype=torch.float32)
+                          / math.sqrt(K))
+        b[e], b_sf[e] = quantize_mx_rows(w)
+    return dict(a=a, a_sf=a_sf, b=b, b_sf=b_sf, m_indptr=m_indptr)
