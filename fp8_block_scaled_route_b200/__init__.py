@@ -24,6 +24,7 @@ __all__ = [
     "swiglu_mxfp8_quant", "moe_select_tile_m", "moe_workspace_size", "moe_route_workspace_size",
     "moe_get_device_status", "moe_set_wait_timeout_ns", "moe_status_string",
     "moe_set_stage_events", "moe_route_permute_noalloc", "mxfp8_moe_gemm",
+    "mxfp8_tile_scales",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -42,7 +43,7 @@ EXPORTS = (
     "moe_status_string", "moe_route_workspace_size", "moe_route_permute", "moe_workspace_size",
     "moe_fp8_fused", "moe_fp8_fused_debug", "fp8_groupwise_moe_gemm", "moe_select_tile_m",
     "swiglu_mxfp8_quant", "moe_get_device_status", "moe_set_wait_timeout_ns",
-    "moe_set_stage_events", "moe_route_permute_noalloc", "mxfp8_moe_gemm",
+    "moe_set_stage_events", "moe_route_permute_noalloc", "mxfp8_moe_gemm", "mxfp8_tile_scales",
 )
 
 _lib = None
@@ -88,6 +89,8 @@ def lib():
     L.swiglu_mxfp8_quant.argtypes = [P, P, P, I, I, P]
     L.mxfp8_moe_gemm.restype = I
     L.mxfp8_moe_gemm.argtypes = [P] * 6 + [I] * 5 + [P]
+    L.mxfp8_tile_scales.restype = I
+    L.mxfp8_tile_scales.argtypes = [P, P, I, I, P]
     L.moe_get_device_status.restype = I
     L.moe_get_device_status.argtypes = [P, P]
     L.moe_set_wait_timeout_ns.restype = None
@@ -221,8 +224,8 @@ def fp8_groupwise_moe_gemm(a, b, a_scale, b_scale, m_indptr, out, scale_major_mo
 
 def mxfp8_moe_gemm(a, b, a_sf, b_sf, m_indptr, out, is_gated=False, *, dims=None, stream=None,
                    check=True) -> int:
-    """a [R,K] fp8, b [E,N,K] fp8, a_sf [R,K/32] / b_sf [E,N,K/32] uint8 E8M0,
-    out bf16 [R, N/2 if gated else N].  dims = (R, N, K, E) when raw addresses
+    """a [R,K] fp8, b [E,N,K] fp8, a_sf [R,K/32] uint8 E8M0 row-major, b_sf the
+    weight scales tiled by mxfp8_tile_scales, out bf16 [R, N/2 if gated else N].  dims = (R, N, K, E) when raw addresses
     are passed."""
     if dims is None:
         R, K = a.shape
@@ -232,6 +235,18 @@ def mxfp8_moe_gemm(a, b, a_sf, b_sf, m_indptr, out, is_gated=False, *, dims=None
     st = lib().mxfp8_moe_gemm(_ptr(a), _ptr(b), _ptr(a_sf), _ptr(b_sf), _ptr(m_indptr), _ptr(out),
                               R, N, K, E, int(bool(is_gated)), _stream(stream))
     return _check(st, "mxfp8_moe_gemm", check)
+
+
+def mxfp8_tile_scales(sf_rowmajor, sf_tiled, *, dims=None, stream=None, check=True) -> int:
+    """sf_rowmajor uint8 [rows, K/32] -> sf_tiled uint8 (rows * K/32 bytes, tiled).
+    dims = (rows, K) when raw addresses are passed."""
+    if dims is None:
+        rows = sf_rowmajor.shape[0] if sf_rowmajor.dim() == 2 else sf_rowmajor.shape[0] * sf_rowmajor.shape[1]
+        K = sf_rowmajor.shape[-1] * 32
+    else:
+        rows, K = dims
+    st = lib().mxfp8_tile_scales(_ptr(sf_rowmajor), _ptr(sf_tiled), rows, K, _stream(stream))
+    return _check(st, "mxfp8_tile_scales", check)
 
 
 def swiglu_mxfp8_quant(inp, out, scale, *, dims=None, stream=None, check=True) -> int:

@@ -355,8 +355,7 @@ int mxfp8_moe_gemm(const void* a, const void* b, const uint8_t* a_sf, const uint
     if (is_gated && (N % 2 || (N / 2) % 128)) return MOE_ERR_INVALID_ARG;
     if (!m_indptr || (R > 0 && (!a || !b || !a_sf || !b_sf || !out))) return MOE_ERR_INVALID_ARG;
     if (!aligned16(a) || !aligned16(b) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
-    if ((reinterpret_cast<uintptr_t>(a_sf) | reinterpret_cast<uintptr_t>(b_sf)) & 3)
-        return MOE_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(a_sf) & 3) || !aligned16(b_sf)) return MOE_ERR_INVALID_ARG;
     const DevInfo* d = dev_info();
     if (int st = check_device(d)) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -371,6 +370,18 @@ int mxfp8_moe_gemm(const void* a, const void* b, const uint8_t* a_sf, const uint
     g.timeout_ns = g_timeout_ns.load();
     g.num_sms = d->sms;
     return launch_mx_gemm(g, s);
+}
+
+int mxfp8_tile_scales(const uint8_t* sf_rowmajor, uint8_t* sf_tiled, int rows, int K,
+                      moe_stream_t stream) {
+    if (rows < 0 || K <= 0 || K % 128 || rows % 128) return MOE_ERR_INVALID_ARG;
+    if (rows > 0 && (!sf_rowmajor || !sf_tiled)) return MOE_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(sf_rowmajor) | reinterpret_cast<uintptr_t>(sf_tiled)) & 3)
+        return MOE_ERR_INVALID_ARG;
+    const DevInfo* d = dev_info();
+    if (int st = check_device(d)) return st;
+    return launch_mx_tile_scales(sf_rowmajor, sf_tiled, rows, K, d->sms,
+                                 reinterpret_cast<cudaStream_t>(stream));
 }
 
 int swiglu_mxfp8_quant(const void* in, void* out, uint8_t* scale, int M, int K, moe_stream_t stream) {

@@ -76,7 +76,7 @@ struct MxGemmArgs {
     const void* a;            // [R, K] E4M3, grouped rows
     const void* b;            // [E, N, K] E4M3
     const uint8_t* a_sf;      // [R, K/32] E8M0, row-major
-    const uint8_t* b_sf;      // [E, N, K/32] E8M0, row-major
+    const uint8_t* b_sf;      // [E*N/128, K/128, 512] E8M0, tiled (launch_mx_tile_scales)
     const int32_t* m_indptr;  // [E+1]
     int R, N, K, E;
     int gated;                // out [R, N/2] = bf16(silu(G_gate) * G_up), else [R, N] = bf16(G)
@@ -86,5 +86,11 @@ struct MxGemmArgs {
     int num_sms;
 };
 int launch_mx_gemm(const MxGemmArgs& g, cudaStream_t stream);
+
+// Row-major E8M0 scales [rows, K/32] -> the tiled layout the MXFP8 GEMM reads
+// for weights: [rows/128, K/128, 512], byte (r % 32) * 16 + ((r / 32) % 4) * 4 + j
+// of atom (r / 128, kb) = scale j of row r in K block kb.  rows % 128 == 0.
+int launch_mx_tile_scales(const uint8_t* rm, uint8_t* tiled, int rows, int K, int num_sms,
+                          cudaStream_t stream);
 
 }  // namespace moe

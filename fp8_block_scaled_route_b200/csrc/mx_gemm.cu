@@ -18,9 +18,13 @@
 //   B  256 x 128 B  (TMA, 128-byte swizzle)        32 KB
 //   SF A 128 rows x 4 scales, B 256 rows x 4 scales, each 128-row group in
 //      the 512-byte layout byte(r, j) = (r % 32) * 16 + (r / 32) * 4 + j
-//      (j = 32-wide K step), copied from row-major [rows, K/32] by cp.async
-// Warps: 0 TMA producer, 1 MMA issuer (elected lane), 2 scale-factor loader,
-// 3 idle, 4-11 epilogue.  TMEM: accumulator columns [0, 256), A scale factors
+//      (j = 32-wide K step).  Weight scales come pre-tiled in that layout
+//      ([E*N/128, K/128, 512], see mxfp8_tile_scales), one coalesced 16-byte
+//      copy per lane per 128-row block; activation scales are row-major
+//      [R, K/32] because a tile's rows start anywhere, four 4-byte copies per
+//      lane.
+// Warps: 0 TMA producer, 1 MMA issuer (elected lane), 2 weight scale loader,
+// 3 activation scale loader, 4-11 epilogue.  TMEM: accumulator columns [0, 256), A scale factors
 // [256, 260), B scale factors [264, 272); one tcgen05.cp per 128 rows moves a
 // stage's scale factors into TMEM ahead of its four MMAs (issued by the same
 // thread, so they are ordered).
@@ -172,14 +176,15 @@ __device__ void mx_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, cons
     __syncwarp();
 }
 
-// Warp 2: per stage, the 4 E8M0 scales (one 32-bit word of a row-major
-// [rows, K/32] array) of each of the tile's 128 token rows and 256 weight rows,
-// written into the 512-byte tcgen05.cp layout; completion arrives on the
-// stage's full barrier.  Rows past the ends read as 0 (scale 2^-127).
+// Warps 2 (weights) and 3 (activations): per stage, the 4 E8M0 scales of
+// each of the tile's 256 weight rows or 128 token rows, in the 512-byte
+// tcgen05.cp layout; completion arrives on the stage's full barrier.  Rows
+// past the ends read as 0 (scale 2^-127; those outputs are not stored).
+template <bool WEIGHTS>
 __device__ void mx_sf_loader(const MxParams& p, const MxSmem& s, const WaitCtl& wc, int total) {
     const int lane = threadIdx.x & 31;
-    const int nsf = p.K >> 5;  // scale bytes per row
-    const long long wrows = static_cast<long long>(p.E) * p.N;
+    const int nsf = p.K >> 5;  // row-major activation scale bytes per row
+    const long long wblocks = static_cast<long long>(p.E) * p.N / 128;
     uint32_t stage = 0, phase = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
@@ -189,20 +194,22 @@ __device__ void mx_sf_loader(const MxParams& p, const MxSmem& s, const WaitCtl& 
         for (int kb = 0; kb < p.nkb; ++kb) {
             if (!mx_warp_wait(&s.empty[stage], phase ^ 1, wc, 8)) { ok = false; break; }
             uint8_t* sf = s.stages + stage * kMxStage + kMxSfOff;
+            if constexpr (WEIGHTS) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {  // token row lane + 32 i
-                const int r = tl.row0 + lane + 32 * i;
-                const bool v = r < p.R;
-                const uint8_t* src = v ? p.a_sf + static_cast<long long>(r) * nsf + kb * 4 : p.a_sf;
-                cp_async_4(sf + lane * 16 + i * 4, src, v ? 4u : 0u);
-            }
+                for (int blk = 0; blk < 2; ++blk) {
+                    const long long wb = (blk ? w1 : w0) >> 7;
+                    const bool v = wb < wblocks;
+                    const uint8_t* src = v ? p.b_sf + (wb * p.nkb + kb) * 512 + lane * 16 : p.b_sf;
+                    cp_async_16(sf + 512 + blk * 512 + lane * 16, src, v ? 16u : 0u);
+                }
+            } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {  // weight row lane + 32 i of the tile
-                const int j = lane + 32 * i;
-                const long long w = (j < 128 ? w0 + j : w1 + (j - 128));
-                const bool v = w < wrows;
-                const uint8_t* src = v ? p.b_sf + w * nsf + kb * 4 : p.b_sf;
-                cp_async_4(sf + 512 + (i >> 2) * 512 + lane * 16 + (i & 3) * 4, src, v ? 4u : 0u);
+                for (int i = 0; i < 4; ++i) {  // token row lane + 32 i
+                    const int r = tl.row0 + lane + 32 * i;
+                    const bool v = r < p.R;
+                    const uint8_t* src = v ? p.a_sf + static_cast<long long>(r) * nsf + kb * 4 : p.a_sf;
+                    cp_async_4(sf + lane * 16 + i * 4, src, v ? 4u : 0u);
+                }
             }
             cp_async_arrive_noinc(&s.full[stage]);
             if (++stage == kMxStages) { stage = 0; phase ^= 1; }
@@ -335,7 +342,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int i = 0; i < kMxStages; ++i) {
-            mbar_init(&s.full[i], kMxBoxes + 32);
+            mbar_init(&s.full[i], kMxBoxes + 64);  // TMA lanes + two scale-loader warps
             mbar_init(&s.empty[i], 1);
         }
         mbar_init(s.tfull, 1);
@@ -389,7 +396,8 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     const int total = s.tstart[p.E];
     if (warp == 0) mx_producer(&tmA, &tmB, p, s, wc, total);
     else if (warp == 1) mx_mma(p, s, wc, tmem_base, total);
-    else if (warp == 2) mx_sf_loader(p, s, wc, total);
+    else if (warp == 2) mx_sf_loader<true>(p, s, wc, total);
+    else if (warp == 3) mx_sf_loader<false>(p, s, wc, total);
     else if (warp >= 4) mx_epilogue(p, s, wc, tmem_base, total);
     tc_fence_before();
     __syncthreads();
@@ -397,7 +405,35 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     if (warp == 1) tmem_dealloc(tmem_base, kMxTmemCols);
 }
 
+// Row-major E8M0 scales [rows, K/32] -> tiled [rows/128, K/128, 512]: one
+// thread per 4-byte word (the 4 scales of one row in one 128-wide K block).
+__global__ void __launch_bounds__(256) mx_tile_scales_kernel(const uint32_t* __restrict__ rm,
+                                                             uint32_t* __restrict__ tiled,
+                                                             long long words, int nkb) {
+    for (long long w = blockIdx.x * 256ll + threadIdx.x; w < words; w += gridDim.x * 256ll) {
+        const long long atom = w >> 7;  // (128-row block, K block)
+        const int pos = static_cast<int>(w & 127);
+        const long long blk = atom / nkb;
+        const int kb = static_cast<int>(atom - blk * nkb);
+        const int l = pos >> 2, g = pos & 3;
+        const long long row = blk * 128 + g * 32 + l;
+        tiled[w] = rm[row * nkb + kb];
+    }
+}
+
 }  // namespace
+
+int launch_mx_tile_scales(const uint8_t* rm, uint8_t* tiled, int rows, int K, int num_sms,
+                          cudaStream_t stream) {
+    const int nkb = K / 128;
+    const long long words = static_cast<long long>(rows) * nkb;
+    if (words == 0) return ST_OK;
+    const long long blocks = (words + 255) / 256;
+    const int grid = static_cast<int>(blocks < num_sms * 8ll ? blocks : num_sms * 8ll);
+    mx_tile_scales_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint32_t*>(rm),
+                                                    reinterpret_cast<uint32_t*>(tiled), words, nkb);
+    return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
+}
 
 int launch_mx_gemm(const MxGemmArgs& g, cudaStream_t stream) {
     if (g.R <= 0 || g.E <= 0) return ST_OK;

@@ -288,6 +288,13 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
 
 // ----------------------------------------------------------------- cp.async
 // 4-byte asynchronous global -> shared copy; src_bytes = 0 writes zeros.
+// 16-byte asynchronous global -> shared copy (both 16-byte aligned), bypassing
+// L1; src_bytes = 0 writes zeros.
+__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gmem_src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)),
+                 "l"(gmem_src), "r"(src_bytes)
+                 : "memory");
+}
 __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.wait_all;" ::: "memory");
 }

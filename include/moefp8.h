@@ -200,7 +200,9 @@ MOE_API int moe_select_tile_m(int total_rows, int n, int k, int E, int num_sms, 
  *  a       device FP8  [R, K] grouped rows
  *  b       device FP8  [E, N, K]
  *  a_sf    device uint8 [R, K/32] E8M0 codes, row-major (4-byte aligned)
- *  b_sf    device uint8 [E, N, K/32] E8M0 codes, row-major (4-byte aligned)
+ *  b_sf    device uint8 E8M0 codes of the weights in the tiled layout that
+ *          mxfp8_tile_scales produces from [E, N, K/32] row-major
+ *          (16-byte aligned; weights are tiled once, not per call)
  *  m_indptr device int32 [E+1]
  *  out     device bf16: plain [R, N] = bf16(G); gated [R, N/2] =
  *          bf16(silu(G[:, :N/2]) * G[:, N/2:]) (gate rows then up rows of b)
@@ -212,6 +214,17 @@ MOE_API int moe_select_tile_m(int total_rows, int n, int k, int E, int num_sms, 
 MOE_API int mxfp8_moe_gemm(const void* a, const void* b, const uint8_t* a_sf,
                            const uint8_t* b_sf, const int32_t* m_indptr, void* out,
                            int R, int N, int K, int E, int is_gated, moe_stream_t stream);
+
+/* Rearranges row-major E8M0 scales [rows, K/32] into the tiled layout that
+ * mxfp8_moe_gemm reads for the weights: [rows/128, K/128, 512] bytes, where
+ * byte (r % 32) * 16 + ((r / 32) % 4) * 4 + j of block (r / 128, kb) holds
+ * scale j (of the four 32-wide steps) of row r in K block kb -- 128 rows x
+ * 4 scales in the order the tensor core's scale-factor copy reads them.
+ * No counterpart on the pages: it is the storage format of this library's
+ * block-scaled GEMM.  rows and K must be multiples of 128; pointers 4-byte
+ * aligned (16 for use by mxfp8_moe_gemm); asynchronous on `stream`. */
+MOE_API int mxfp8_tile_scales(const uint8_t* sf_rowmajor, uint8_t* sf_tiled, int rows, int K,
+                              moe_stream_t stream);
 
 /* ------------------------------------------------------------------ */
 /* Standalone SwiGLU + MXFP8 quantisation                               */

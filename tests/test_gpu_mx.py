@@ -10,13 +10,21 @@ import fp8_block_scaled_route_b200 as moe
 pytestmark = pytest.mark.gpu
 
 
+def _tiled(sf_rowmajor):
+    rows = sf_rowmajor.numel() // sf_rowmajor.shape[-1]
+    flat = sf_rowmajor.reshape(rows, sf_rowmajor.shape[-1]).contiguous()
+    tiled = torch.empty_like(flat)
+    moe.mxfp8_tile_scales(flat, tiled)
+    return tiled
+
+
 def _run(inp, is_gated):
     a, b = inp["a"], inp["b"]
     R = a.shape[0]
     E, N, _ = b.shape
     out = torch.full((R, N // 2 if is_gated else N), float("nan"), dtype=torch.bfloat16,
                      device=a.device)
-    moe.mxfp8_moe_gemm(a, b, inp["a_sf"], inp["b_sf"], inp["m_indptr"], out, is_gated)
+    moe.mxfp8_moe_gemm(a, b, inp["a_sf"], _tiled(inp["b_sf"]), inp["m_indptr"], out, is_gated)
     torch.cuda.synchronize()
     assert moe.moe_get_device_status(None) == 0
     return out.cpu()
@@ -92,6 +100,20 @@ def test_mx_gemm_scale_placement(oracle):
     got = _run({k: v.cuda() for k, v in inp.items()}, False)
     ref = _oracle(oracle, inp, False)
     _compare(got, ref, R)
+
+
+def test_mx_tile_scales_layout():
+    """Tiled byte (r % 32) * 16 + ((r / 32) % 4) * 4 + j of block (r / 128, kb)
+    = row-major scale [r, 4 kb + j]; bit-exact."""
+    rows, K = 384, 512
+    rm = torch.randint(0, 256, (rows, K // 32), dtype=torch.uint8)
+    got = _tiled(rm.cuda()).cpu().numpy().reshape(rows // 128, K // 128, 512)
+    r = np.arange(rows)[:, None]
+    j = np.arange(K // 32)[None, :]
+    kb, jj = j // 4, j % 4
+    ref = np.zeros_like(got)
+    ref[r // 128, kb, (r % 32) * 16 + ((r // 32) % 4) * 4 + jj] = rm.numpy()
+    np.testing.assert_array_equal(got, ref)
 
 
 def test_mx_gemm_empty_and_bad_args():
