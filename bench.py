@@ -448,6 +448,74 @@ def run_swiglu(args):
     return 0
 
 
+def run_mx_gemm(args, cfg):
+    """MXFP8 grouped GEMM (block-scaled tensor core path) on the gate/up GEMM
+    of a workload: A = the workload's routed rows [T*k, H], B = gated weights
+    [E, 2I, H], group sizes from its routing; activations and weights drawn
+    as N(0,1) / N(0,1/H) with per-32 magnitudes 2^U{-4..4}, quantised to
+    MXFP8.  The same shape through the fp32-block-scaled grouped GEMM
+    (fp8_groupwise_moe_gemm) is timed beside it.  Inputs exceed L2."""
+    import fp8_block_scaled_route_b200 as moe
+    torch.cuda.set_device(0)
+    hbm, bf16, _, src = load_peaks()
+    fp8_peak = bf16 * FP8_OVER_BF16
+    ids = synth.make_moe_inputs(cfg, seed=0, device="cuda", weights=False)["topk_ids"]
+    sizes = torch.bincount(ids.flatten().long(), minlength=cfg.E).cpu().tolist()
+    R, N, K, E = sum(sizes), 2 * cfg.I, cfg.H, cfg.E
+    inp = synth.make_mx_gemm_inputs(R, N, K, E, seed=1, device="cuda", group_sizes=sizes)
+    a_sf = inp["a_sf"].view(R, K // 128, 4).permute(1, 0, 2).contiguous()
+    b_sf = torch.empty(E * N, K // 32, dtype=torch.uint8, device="cuda")
+    moe.mxfp8_tile_scales(inp["b_sf"].view(E * N, K // 32), b_sf)
+    out = torch.empty(R, N // 2, dtype=torch.bfloat16, device="cuda")
+
+    def mx():
+        moe.mxfp8_moe_gemm(inp["a"], inp["b"], a_sf, b_sf, inp["m_indptr"], out, True, "MN")
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / args.steps
+
+    ms_mx = timed(mx)
+    del a_sf
+    fp = synth.make_grouped_gemm_inputs(R, N, K, E, seed=1, device="cuda", group_sizes=sizes)
+    a_mn = fp["a_scale"].t().contiguous()
+
+    def fp32_scaled():
+        moe.fp8_groupwise_moe_gemm(fp["a"], fp["b"], a_mn, fp["b_scale"], fp["m_indptr"], out,
+                                   "MN", (1, 128, 128), True, -1, -1)
+
+    ms_fp = timed(fp32_scaled)
+    flops = 2.0 * R * N * K
+    touched = sum(1 for x in sizes if x > 0)
+    nbytes = touched * N * K * (1 + 1 / 32) + R * K * (1 + 1 / 32) + R * (N // 2) * 2
+    tf = flops / (ms_mx * 1e-3) / 1e12
+    line = {"metric": "MXFP8 grouped GEMM (gate/up + SwiGLU) TFLOP/s", "value": tf,
+            "unit": "TFLOP/s", "higher_is_better": True, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_mx, "n_gpus": 1, "data": "synthetic",
+            "dtype": "mxfp8 e4m3 + e8m0 per 32 (fp32 accumulate)",
+            "config": {"workload": f"{cfg.name} gate/up GEMM: R={R} N={N} K={K} E={E}, "
+                                   f"group sizes from its routing",
+                       "l2": "inputs larger than L2 (no flush)"},
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": fp8_peak, "unit": "TFLOP/s",
+                         "frac": tf / fp8_peak, "traffic": None,
+                         "peak_source": f"{src} (FP8 = bf16 burst x {FP8_OVER_BF16:g})",
+                         "alg_bytes": nbytes, "gbs": nbytes / (ms_mx * 1e-3) / 1e9},
+            "fp32_block_scaled_same_shape": {"ms": ms_fp,
+                                             "tflops": flops / (ms_fp * 1e-3) / 1e12},
+            "gpu_launches": args.steps}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -457,14 +525,16 @@ def main():
                     choices=sorted(synth.CONFIGS) + sorted(PROFILE_SLICES))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", default="moe", choices=["moe", "swiglu_mxfp8"],
-                    help="swiglu_mxfp8: time the standalone SwiGLU+MXFP8 op instead")
+    ap.add_argument("--op", default="moe", choices=["moe", "swiglu_mxfp8", "mxfp8_gemm"],
+                    help="swiglu_mxfp8 / mxfp8_gemm: time that standalone op instead")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.op == "swiglu_mxfp8":
         return run_swiglu(args)
     cfg = synth.CONFIGS.get(args.workload) or PROFILE_SLICES[args.workload]
+    if args.op == "mxfp8_gemm":
+        return run_mx_gemm(args, cfg)
     if args.impl == "reference":
         return run_reference(args, cfg)
     return run_ours(args, cfg)

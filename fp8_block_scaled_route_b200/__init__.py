@@ -88,7 +88,7 @@ def lib():
     L.swiglu_mxfp8_quant.restype = I
     L.swiglu_mxfp8_quant.argtypes = [P, P, P, I, I, P]
     L.mxfp8_moe_gemm.restype = I
-    L.mxfp8_moe_gemm.argtypes = [P] * 6 + [I] * 5 + [P]
+    L.mxfp8_moe_gemm.argtypes = [P] * 6 + [I] * 6 + [P]
     L.mxfp8_tile_scales.restype = I
     L.mxfp8_tile_scales.argtypes = [P, P, I, I, P]
     L.moe_get_device_status.restype = I
@@ -222,8 +222,8 @@ def fp8_groupwise_moe_gemm(a, b, a_scale, b_scale, m_indptr, out, scale_major_mo
     return _check(st, "fp8_groupwise_moe_gemm", check)
 
 
-def mxfp8_moe_gemm(a, b, a_sf, b_sf, m_indptr, out, is_gated=False, *, dims=None, stream=None,
-                   check=True) -> int:
+def mxfp8_moe_gemm(a, b, a_sf, b_sf, m_indptr, out, is_gated=False, a_sf_major="K", *,
+                   dims=None, stream=None, check=True) -> int:
     """a [R,K] fp8, b [E,N,K] fp8, a_sf [R,K/32] uint8 E8M0 row-major, b_sf the
     weight scales tiled by mxfp8_tile_scales, out bf16 [R, N/2 if gated else N].  dims = (R, N, K, E) when raw addresses
     are passed."""
@@ -232,8 +232,9 @@ def mxfp8_moe_gemm(a, b, a_sf, b_sf, m_indptr, out, is_gated=False, *, dims=None
         E, N, _ = b.shape
     else:
         R, N, K, E = dims
+    mode = {"K": 0, "MN": 1}.get(a_sf_major, a_sf_major)
     st = lib().mxfp8_moe_gemm(_ptr(a), _ptr(b), _ptr(a_sf), _ptr(b_sf), _ptr(m_indptr), _ptr(out),
-                              R, N, K, E, int(bool(is_gated)), _stream(stream))
+                              R, N, K, E, mode, int(bool(is_gated)), _stream(stream))
     return _check(st, "mxfp8_moe_gemm", check)
 
 

@@ -348,9 +348,10 @@ int fp8_groupwise_moe_gemm(const void* a, const void* b, const float* a_scale, c
 }
 
 int mxfp8_moe_gemm(const void* a, const void* b, const uint8_t* a_sf, const uint8_t* b_sf,
-                   const int32_t* m_indptr, void* out, int R, int N, int K, int E, int is_gated,
-                   moe_stream_t stream) {
+                   const int32_t* m_indptr, void* out, int R, int N, int K, int E,
+                   int a_sf_major, int is_gated, moe_stream_t stream) {
     if (R < 0 || N <= 0 || K <= 0 || E < 1 || N % 128 || K % 128) return MOE_ERR_INVALID_ARG;
+    if (a_sf_major != 0 && a_sf_major != 1) return MOE_ERR_INVALID_ARG;
     if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
     if (is_gated && (N % 2 || (N / 2) % 128)) return MOE_ERR_INVALID_ARG;
     if (!m_indptr || (R > 0 && (!a || !b || !a_sf || !b_sf || !out))) return MOE_ERR_INVALID_ARG;
@@ -364,6 +365,7 @@ int mxfp8_moe_gemm(const void* a, const void* b, const uint8_t* a_sf, const uint
     if (R == 0) return MOE_OK;
     MxGemmArgs g{};
     g.a = a; g.b = b; g.a_sf = a_sf; g.b_sf = b_sf; g.m_indptr = m_indptr;
+    g.a_sf_mn = a_sf_major;
     g.R = R; g.N = N; g.K = K; g.E = E; g.gated = is_gated ? 1 : 0;
     g.out = out;
     g.status = d->lib_status;

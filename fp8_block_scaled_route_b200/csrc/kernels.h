@@ -75,7 +75,8 @@ int launch_swiglu_mxfp8(const void* in, void* out, uint8_t* scale, int M, int K,
 struct MxGemmArgs {
     const void* a;            // [R, K] E4M3, grouped rows
     const void* b;            // [E, N, K] E4M3
-    const uint8_t* a_sf;      // [R, K/32] E8M0, row-major
+    const uint8_t* a_sf;      // E8M0: [R, K/32] row-major (a_sf_mn = 0) or [K/128, R, 4] (1)
+    int a_sf_mn;
     const uint8_t* b_sf;      // [E*N/128, K/128, 512] E8M0, tiled (launch_mx_tile_scales)
     const int32_t* m_indptr;  // [E+1]
     int R, N, K, E;

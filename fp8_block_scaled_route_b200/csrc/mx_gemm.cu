@@ -21,8 +21,8 @@
 //      (j = 32-wide K step).  Weight scales come pre-tiled in that layout
 //      ([E*N/128, K/128, 512], see mxfp8_tile_scales), one coalesced 16-byte
 //      copy per lane per 128-row block; activation scales are row-major
-//      [R, K/32] because a tile's rows start anywhere, four 4-byte copies per
-//      lane.
+//      [R, K/32] or K-block-major [K/128, R, 4] (a tile's rows start anywhere,
+//      so four 4-byte copies per lane; coalesced in the second layout).
 // Warps: 0 TMA producer, 1 MMA issuer (elected lane), 2 weight scale loader,
 // 3 activation scale loader, 4-11 epilogue.  TMEM: accumulator columns [0, 256), A scale factors
 // [256, 260), B scale factors [264, 272); one tcgen05.cp per 128 rows moves a
@@ -59,7 +59,7 @@ static_assert(kMxStage % 1024 == 0, "stages must stay 1024-byte aligned for the 
 static_assert(kMxSmem <= 232448, "shared memory budget");
 
 struct MxParams {
-    int R, N, K, E, nkb, gated;
+    int R, N, K, E, nkb, gated, a_sf_mn;
     const uint8_t* a_sf;
     const uint8_t* b_sf;
     const int32_t* m_indptr;
@@ -207,8 +207,10 @@ __device__ void mx_sf_loader(const MxParams& p, const MxSmem& s, const WaitCtl& 
                 for (int i = 0; i < 4; ++i) {  // token row lane + 32 i
                     const int r = tl.row0 + lane + 32 * i;
                     const bool v = r < p.R;
-                    const uint8_t* src = v ? p.a_sf + static_cast<long long>(r) * nsf + kb * 4 : p.a_sf;
-                    cp_async_4(sf + lane * 16 + i * 4, src, v ? 4u : 0u);
+                    // [K/128, R, 4]: a warp's 32 rows are 128 contiguous bytes
+                    const long long off = p.a_sf_mn ? (static_cast<long long>(kb) * p.R + r) * 4
+                                                    : static_cast<long long>(r) * nsf + kb * 4;
+                    cp_async_4(sf + lane * 16 + i * 4, v ? p.a_sf + off : p.a_sf, v ? 4u : 0u);
                 }
             }
             cp_async_arrive_noinc(&s.full[stage]);
@@ -443,6 +445,7 @@ int launch_mx_gemm(const MxGemmArgs& g, cudaStream_t stream) {
     if (!make_tma_map_fp8(&mb, g.b, static_cast<long long>(g.E) * g.N, g.K, 64)) return ST_CUDA;
     MxParams p;
     p.R = g.R; p.N = g.N; p.K = g.K; p.E = g.E; p.nkb = g.K / 128; p.gated = g.gated ? 1 : 0;
+    p.a_sf_mn = g.a_sf_mn ? 1 : 0;
     p.a_sf = g.a_sf; p.b_sf = g.b_sf; p.m_indptr = g.m_indptr;
     p.out = static_cast<__nv_bfloat16*>(g.out);
     p.status = g.status;

@@ -199,7 +199,10 @@ MOE_API int moe_select_tile_m(int total_rows, int n, int k, int E, int num_sms, 
  * accumulated in fp32 by the tensor core (the scales are applied inside it).
  *  a       device FP8  [R, K] grouped rows
  *  b       device FP8  [E, N, K]
- *  a_sf    device uint8 [R, K/32] E8M0 codes, row-major (4-byte aligned)
+ *  a_sf    device uint8 E8M0 codes of the activations (4-byte aligned):
+ *          a_sf_major = 0: [R, K/32] row-major; 1: [K/128, R, 4], the four
+ *          scales of a 128-wide K block of each row together, rows
+ *          consecutive (the rows of a tile are then read contiguously)
  *  b_sf    device uint8 E8M0 codes of the weights in the tiled layout that
  *          mxfp8_tile_scales produces from [E, N, K/32] row-major
  *          (16-byte aligned; weights are tiled once, not per call)
@@ -213,7 +216,8 @@ MOE_API int moe_select_tile_m(int total_rows, int n, int k, int E, int num_sms, 
  * Caller owns all memory; asynchronous on `stream`. */
 MOE_API int mxfp8_moe_gemm(const void* a, const void* b, const uint8_t* a_sf,
                            const uint8_t* b_sf, const int32_t* m_indptr, void* out,
-                           int R, int N, int K, int E, int is_gated, moe_stream_t stream);
+                           int R, int N, int K, int E, int a_sf_major, int is_gated,
+                           moe_stream_t stream);
 
 /* Rearranges row-major E8M0 scales [rows, K/32] into the tiled layout that
  * mxfp8_moe_gemm reads for the weights: [rows/128, K/128, 512] bytes, where

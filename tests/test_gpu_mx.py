@@ -18,13 +18,21 @@ def _tiled(sf_rowmajor):
     return tiled
 
 
-def _run(inp, is_gated):
+def _mn(a_sf):
+    """[R, K/32] -> [K/128, R, 4] (the four scales of a K block together)."""
+    R, nsf = a_sf.shape
+    return a_sf.view(R, nsf // 4, 4).permute(1, 0, 2).contiguous()
+
+
+def _run(inp, is_gated, a_mn=False):
     a, b = inp["a"], inp["b"]
     R = a.shape[0]
     E, N, _ = b.shape
     out = torch.full((R, N // 2 if is_gated else N), float("nan"), dtype=torch.bfloat16,
                      device=a.device)
-    moe.mxfp8_moe_gemm(a, b, inp["a_sf"], _tiled(inp["b_sf"]), inp["m_indptr"], out, is_gated)
+    a_sf = _mn(inp["a_sf"]) if a_mn else inp["a_sf"]
+    moe.mxfp8_moe_gemm(a, b, a_sf, _tiled(inp["b_sf"]), inp["m_indptr"], out, is_gated,
+                       "MN" if a_mn else "K")
     torch.cuda.synchronize()
     assert moe.moe_get_device_status(None) == 0
     return out.cpu()
@@ -84,9 +92,10 @@ def test_mx_gemm_exact_small_integers(oracle):
 def test_mx_gemm_random(oracle, R, N, K, E, gated, sizes):
     inp = synth.make_mx_gemm_inputs(R, N, K, E, seed=R + K, group_sizes=sizes)
     rows = int(inp["m_indptr"][-1])
-    got = _run({k: v.cuda() for k, v in inp.items()}, gated)
+    dev = {k: v.cuda() for k, v in inp.items()}
     ref = _oracle(oracle, inp, gated)
-    _compare(got, ref, rows)
+    _compare(_run(dev, gated), ref, rows)
+    _compare(_run(dev, gated, a_mn=True), ref, rows)
 
 
 def test_mx_gemm_scale_placement(oracle):
@@ -97,9 +106,10 @@ def test_mx_gemm_scale_placement(oracle):
     inp = synth.make_mx_gemm_inputs(R, N, K, E, seed=7, group_sizes=[R], spread=0)
     inp["a_sf"][37, 5] += 8
     inp["b_sf"][0, 200, 2] += 8
-    got = _run({k: v.cuda() for k, v in inp.items()}, False)
     ref = _oracle(oracle, inp, False)
-    _compare(got, ref, R)
+    for a_mn in (False, True):
+        got = _run({k: v.cuda() for k, v in inp.items()}, False, a_mn)
+        _compare(got, ref, R)
 
 
 def test_mx_tile_scales_layout():
