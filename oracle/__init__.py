@@ -79,6 +79,8 @@ def lib():
         L.oracle_mx_grouped_gemm.argtypes = [P, P, P, P, P, i, i, i, i, P]
         L.oracle_mx_gemm_bf16.restype = None
         L.oracle_mx_gemm_bf16.argtypes = [P, P, P, P, P, i, i, i, i, i, P]
+        L.oracle_moe_mx_fused.restype = i
+        L.oracle_moe_mx_fused.argtypes = [P] * 8 + [i] * 5 + [P] * 4
         L.oracle_num_threads.restype = i
         L.oracle_num_threads.argtypes = []
     return _lib
@@ -285,6 +287,32 @@ def mx_gemm_bf16(a, a_sf, b, b_sf, m_indptr, is_gated: bool):
     out = np.zeros((R, N // 2 if is_gated else N), np.uint16)
     lib().oracle_mx_gemm_bf16(_p(a), _p(a_sf), _p(b), _p(b_sf), _p(m_indptr), R, N, K, E,
                               int(bool(is_gated)), _p(out))
+    return out
+
+
+def moe_mx_fused(x_bits, topk_ids, topk_w, w13, w13_sf, w2, w2_sf, want_dump=False):
+    """The fused layer with MXFP8 operands.  x_bits [T,H] bf16 bits; w13 [E,2I,H]
+    codes, w13_sf [E,2I,H/32]; w2 [E,H,I] codes, w2_sf [E,H,I/32].  Returns bf16
+    bits [T,H] (and m_indptr, perm, hq [R,I], hsf [R,I/32] when want_dump)."""
+    x = _c(x_bits, np.uint16)
+    ids = _c(topk_ids, np.int32)
+    w = _c(topk_w, np.float32)
+    w13 = _u8(w13); w2 = _u8(w2); w13_sf = _u8(w13_sf); w2_sf = _u8(w2_sf)
+    T, H = x.shape
+    k = ids.shape[1]
+    E, I2, _ = w13.shape
+    I = I2 // 2
+    R = T * k
+    out = np.zeros((T, H), np.uint16)
+    m_indptr = np.zeros(E + 1, np.int32)
+    perm = np.zeros(max(R, 1), np.int32)
+    hq = np.zeros((max(R, 1), I), np.uint8)
+    hsf = np.zeros((max(R, 1), I // 32), np.uint8)
+    lib().oracle_moe_mx_fused(_p(x), _p(ids), _p(w), _p(w13), _p(w13_sf), _p(w2), _p(w2_sf),
+                              _p(out), T, H, I, E, k, _p(m_indptr), _p(perm), _p(hq), _p(hsf))
+    if want_dump:
+        Rg = int(m_indptr[E])
+        return out, m_indptr, perm[:Rg], hq[:Rg], hsf[:Rg]
     return out
 
 

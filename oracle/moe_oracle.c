@@ -469,6 +469,26 @@ void oracle_quant_rows_mx_bf16(const uint16_t* x, int rows, int cols, uint8_t* q
     }
 }
 
+/* fp32 rows -> MXFP8 (same rule as oracle_quant_rows_mx_bf16). */
+static void quant_rows_mx_f32(const float* x, int rows, int cols, uint8_t* q, uint8_t* sf) {
+    #pragma omp parallel for schedule(static)
+    for (int r = 0; r < rows; ++r) {
+        for (int b = 0; b < cols / 32; ++b) {
+            const float* v = x + (size_t)r * cols + b * 32;
+            float amax = 0.0f;
+            for (int i = 0; i < 32; ++i) {
+                float a = fabsf(v[i]);
+                if (a > amax) amax = a;
+            }
+            uint8_t code = oracle_e8m0_scale_code(amax);
+            float X = oracle_e8m0_decode(code);
+            sf[(size_t)r * (cols / 32) + b] = code;
+            for (int i = 0; i < 32; ++i)
+                q[(size_t)r * cols + b * 32 + i] = oracle_e4m3_encode(v[i] / X);
+        }
+    }
+}
+
 /* Grouped MXFP8 GEMM in the m_indptr layout.  a: [R, K] codes, a_sf [R, K/32];
  * b: [E, N, K] codes, b_sf [E, N, K/32]; rows [m_indptr[e], m_indptr[e+1])
  * use expert e.  out: [R, N] fp32 (rows outside every group untouched). */
@@ -519,6 +539,66 @@ void oracle_mx_gemm_bf16(const uint8_t* a, const uint8_t* a_sf, const uint8_t* b
         free(h);
     }
     free(g);
+}
+
+/* The fused layer in the MXFP8 variant: the five stages of the AlphaMoE
+ * page's pipeline ("문제점: MoE Expert 계산의 병목", stages 1-5) with every FP8
+ * operand in MXFP8 (E8M0 per 32 K elements): activations quantised per
+ * token per 32 columns and gathered into grouped rows, GEMM1 gate/up, SwiGLU
+ * in fp32, requantisation of the intermediate to MXFP8 per row per 32
+ * columns (the Cake-act page's SwiGLU + MXFP8 rule), GEMM2 down, combine in
+ * fp32 (ascending slot) and bf16.  Weight scales row-major:
+ * w13_sf [E, 2I, H/32], w2_sf [E, H, I/32].  Optional dumps: m_indptr [E+1],
+ * perm [R], hq [R, I] codes, hsf [R, I/32]. */
+int oracle_moe_mx_fused(const uint16_t* x, const int32_t* topk_ids, const float* topk_w,
+                        const uint8_t* w13, const uint8_t* w13_sf,
+                        const uint8_t* w2, const uint8_t* w2_sf,
+                        uint16_t* out, int T, int H, int I, int E, int k,
+                        int32_t* m_indptr_out, int32_t* perm_out,
+                        uint8_t* hq_out, uint8_t* hsf_out) {
+    int R = T * k;
+    int32_t* m_indptr = (int32_t*)malloc(sizeof(int32_t) * (E + 1));
+    int32_t* perm = (int32_t*)malloc(sizeof(int32_t) * (R > 0 ? R : 1));
+    int32_t* inv_perm = (int32_t*)malloc(sizeof(int32_t) * (R > 0 ? R : 1));
+    int bad = oracle_route_permute(topk_ids, T, k, E, m_indptr, perm, inv_perm);
+    int Rg = m_indptr[E];
+
+    uint8_t* xq_tok = (uint8_t*)malloc((size_t)T * H + 1);
+    uint8_t* xsf_tok = (uint8_t*)malloc((size_t)T * (H / 32) + 1);
+    oracle_quant_rows_mx_bf16(x, T, H, xq_tok, xsf_tok);
+    uint8_t* xq = (uint8_t*)malloc((size_t)R * H + 1);
+    uint8_t* xsf = (uint8_t*)malloc((size_t)R * (H / 32) + 1);
+    for (int r = 0; r < Rg; ++r) {
+        int t = perm[r] / k;
+        memcpy(xq + (size_t)r * H, xq_tok + (size_t)t * H, H);
+        memcpy(xsf + (size_t)r * (H / 32), xsf_tok + (size_t)t * (H / 32), H / 32);
+    }
+    float* g = (float*)malloc(sizeof(float) * ((size_t)R * 2 * I + 1));
+    oracle_mx_grouped_gemm(xq, xsf, w13, w13_sf, m_indptr, R, 2 * I, H, E, g);
+    float* h = (float*)malloc(sizeof(float) * ((size_t)R * I + 1));
+    oracle_swiglu(g, Rg, I, h);
+    uint8_t* hq = (uint8_t*)malloc((size_t)R * I + 1);
+    uint8_t* hsf = (uint8_t*)malloc((size_t)R * (I / 32) + 1);
+    quant_rows_mx_f32(h, Rg, I, hq, hsf);
+    float* y = (float*)malloc(sizeof(float) * ((size_t)R * H + 1));
+    oracle_mx_grouped_gemm(hq, hsf, w2, w2_sf, m_indptr, R, H, I, E, y);
+    for (int t = 0; t < T; ++t)
+        for (int c = 0; c < H; ++c) {
+            float acc = 0.0f;
+            for (int j = 0; j < k; ++j) {
+                int row = inv_perm[t * k + j];
+                if (row < 0) continue;
+                acc += topk_w[t * k + j] * y[(size_t)row * H + c];
+            }
+            out[(size_t)t * H + c] = f32_to_bf16(acc);
+        }
+    if (m_indptr_out) memcpy(m_indptr_out, m_indptr, sizeof(int32_t) * (E + 1));
+    if (perm_out) memcpy(perm_out, perm, sizeof(int32_t) * Rg);
+    if (hq_out) memcpy(hq_out, hq, (size_t)Rg * I);
+    if (hsf_out) memcpy(hsf_out, hsf, (size_t)Rg * (I / 32));
+    free(m_indptr); free(perm); free(inv_perm); free(xq_tok); free(xsf_tok);
+    free(xq); free(xsf); free(g); free(h); free(hq); free(hsf); free(y);
+    return bad;
 }
 
 /* Threads an OpenMP parallel region would use (0 when built without it). */

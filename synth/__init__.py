@@ -193,3 +193,24 @@ def make_mx_gemm_inputs(R: int, N: int, K: int, E: int, seed: int = 0, device="c
                           / math.sqrt(K))
         b[e], b_sf[e] = quantize_mx_rows(w)
     return dict(a=a, a_sf=a_sf, b=b, b_sf=b_sf, m_indptr=m_indptr)
+
+
+def make_mx_moe_inputs(cfg: MoEConfig, seed: int = 0, device="cpu"):
+    """The fused layer's inputs with MXFP8 weights: routing and x as in
+    make_moe_inputs; w13 [E,2I,H] and w2 [E,H,I] drawn N(0, 1/fan_in) and
+    quantised per row per 32 (quantize_mx_rows); scales row-major
+    w13_sf [E,2I,H/32], w2_sf [E,H,I/32]."""
+    base = make_moe_inputs(cfg, seed, device, weights=False)
+    g = _gen(seed + 7919, device)
+    E, H, I = cfg.E, cfg.H, cfg.I
+    w13 = torch.empty(E, 2 * I, H, dtype=torch.float8_e4m3fn, device=device)
+    w13_sf = torch.empty(E, 2 * I, H // 32, dtype=torch.uint8, device=device)
+    w2 = torch.empty(E, H, I, dtype=torch.float8_e4m3fn, device=device)
+    w2_sf = torch.empty(E, H, I // 32, dtype=torch.uint8, device=device)
+    for e in range(E):
+        w13[e], w13_sf[e] = quantize_mx_rows(
+            torch.randn(2 * I, H, generator=g, device=device) / math.sqrt(H))
+        w2[e], w2_sf[e] = quantize_mx_rows(
+            torch.randn(H, I, generator=g, device=device) / math.sqrt(I))
+    base.update(w13=w13, w13_sf=w13_sf, w2=w2, w2_sf=w2_sf)
+    return base

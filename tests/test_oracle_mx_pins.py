@@ -144,3 +144,68 @@ def test_mx_gemm_bf16_gated_is_swiglu_of_plain(oracle):
     assert torch.all(diff <= ulp)
     np.testing.assert_array_equal(plain.view(np.int16),
                                   torch.from_numpy(g).to(torch.bfloat16).view(torch.int16).numpy())
+
+
+# ------------------------------------------------------------ fused MXFP8 layer
+def _mx_layer_inputs(seed=0):
+    import synth
+    cfg = synth.MoEConfig("mx_pin", 12, 256, 128, 4, 2)
+    return cfg, synth.make_mx_moe_inputs(cfg, seed=seed)
+
+
+def _mx_layer(oracle, inp, topk_w=None, perm_tokens=None):
+    x = inp["x"]
+    ids = inp["topk_ids"]
+    w = inp["topk_w"] if topk_w is None else topk_w
+    if perm_tokens is not None:
+        x, ids, w = x[perm_tokens], ids[perm_tokens], w[perm_tokens]
+    bits = oracle.moe_mx_fused(_bf16_bits(x), ids.numpy(), w.numpy(),
+                               inp["w13"].view(torch.uint8).numpy(), inp["w13_sf"].numpy(),
+                               inp["w2"].view(torch.uint8).numpy(), inp["w2_sf"].numpy())
+    return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+
+
+def test_mx_layer_close_to_float64_ffn(oracle):
+    # the decoded weights in float64 with unquantised activations: the layer
+    # differs from it only by the MXFP8 rounding of x and of the intermediate
+    cfg, inp = _mx_layer_inputs(1)
+    got = _mx_layer(oracle, inp).to(torch.float64)
+    w13 = torch.from_numpy(_dequant(inp["w13"].view(torch.uint8).numpy(), inp["w13_sf"].numpy()))
+    w2 = torch.from_numpy(_dequant(inp["w2"].view(torch.uint8).numpy(), inp["w2_sf"].numpy()))
+    x = inp["x"].to(torch.float64)
+    ref = torch.zeros(cfg.T, cfg.H, dtype=torch.float64)
+    for t in range(cfg.T):
+        for j in range(cfg.k):
+            e = int(inp["topk_ids"][t, j])
+            gu = w13[e] @ x[t]
+            h = torch.nn.functional.silu(gu[:cfg.I]) * gu[cfg.I:]
+            ref[t] += float(inp["topk_w"][t, j]) * (w2[e] @ h)
+    rel = ((got - ref).norm() / ref.norm()).item()
+    assert rel < 0.06, rel
+    # and clearly farther from a layer with a wrong expert choice
+    wrong = torch.zeros_like(ref)
+    for t in range(cfg.T):
+        for j in range(cfg.k):
+            e = (int(inp["topk_ids"][t, j]) + 1) % cfg.E
+            gu = w13[e] @ x[t]
+            wrong[t] += float(inp["topk_w"][t, j]) * (w2[e] @ (torch.nn.functional.silu(gu[:cfg.I]) * gu[cfg.I:]))
+    assert ((got - wrong).norm() / ref.norm()).item() > 5 * rel
+
+
+def test_mx_layer_linear_in_router_weight(oracle):
+    # doubling every router weight doubles every fp32 sum exactly, so the
+    # bf16 outputs double exactly
+    _, inp = _mx_layer_inputs(2)
+    base = _mx_layer(oracle, inp).to(torch.float32)
+    dbl = _mx_layer(oracle, inp, topk_w=inp["topk_w"] * 2).to(torch.float32)
+    assert torch.equal(dbl, 2 * base)
+
+
+def test_mx_layer_token_order(oracle):
+    # each token's result depends only on its own row: permuting the tokens
+    # permutes the outputs bit for bit
+    cfg, inp = _mx_layer_inputs(3)
+    base = _mx_layer(oracle, inp)
+    p = torch.randperm(cfg.T, generator=torch.Generator().manual_seed(0))
+    got = _mx_layer(oracle, inp, perm_tokens=p)
+    assert torch.equal(got.view(torch.int16), base[p].view(torch.int16))
