@@ -24,7 +24,7 @@ __all__ = [
     "swiglu_mxfp8_quant", "moe_select_tile_m", "moe_workspace_size", "moe_route_workspace_size",
     "moe_get_device_status", "moe_set_wait_timeout_ns", "moe_status_string",
     "moe_set_stage_events", "moe_route_permute_noalloc", "mxfp8_moe_gemm",
-    "mxfp8_tile_scales",
+    "mxfp8_tile_scales", "moe_mxfp8_fused", "moe_mxfp8_fused_debug",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -44,6 +44,7 @@ EXPORTS = (
     "moe_fp8_fused", "moe_fp8_fused_debug", "fp8_groupwise_moe_gemm", "moe_select_tile_m",
     "swiglu_mxfp8_quant", "moe_get_device_status", "moe_set_wait_timeout_ns",
     "moe_set_stage_events", "moe_route_permute_noalloc", "mxfp8_moe_gemm", "mxfp8_tile_scales",
+    "moe_mxfp8_fused", "moe_mxfp8_fused_debug",
 )
 
 _lib = None
@@ -91,6 +92,10 @@ def lib():
     L.mxfp8_moe_gemm.argtypes = [P] * 6 + [I] * 6 + [P]
     L.mxfp8_tile_scales.restype = I
     L.mxfp8_tile_scales.argtypes = [P, P, I, I, P]
+    L.moe_mxfp8_fused.restype = I
+    L.moe_mxfp8_fused.argtypes = [P] * 8 + [I] * 5 + [P, ctypes.c_size_t, P]
+    L.moe_mxfp8_fused_debug.restype = I
+    L.moe_mxfp8_fused_debug.argtypes = [P] * 8 + [I] * 5 + [P, ctypes.c_size_t, P] + [P] * 4
     L.moe_get_device_status.restype = I
     L.moe_get_device_status.argtypes = [P, P]
     L.moe_set_wait_timeout_ns.restype = None
@@ -236,6 +241,32 @@ def mxfp8_moe_gemm(a, b, a_sf, b_sf, m_indptr, out, is_gated=False, a_sf_major="
     st = lib().mxfp8_moe_gemm(_ptr(a), _ptr(b), _ptr(a_sf), _ptr(b_sf), _ptr(m_indptr), _ptr(out),
                               R, N, K, E, mode, int(bool(is_gated)), _stream(stream))
     return _check(st, "mxfp8_moe_gemm", check)
+
+
+def moe_mxfp8_fused(x, topk_ids, topk_w, w13, w13_sf, w2, w2_sf, out, ws, ws_bytes=None, *,
+                    dims=None, stream=None, check=True) -> int:
+    """w13_sf / w2_sf: weight scales tiled by mxfp8_tile_scales.  dims = (T, H, I, E, k)
+    when raw addresses are passed."""
+    T, H, I, E, k = dims if dims is not None else _fused_dims(x, topk_ids, w13)
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size()
+    st = lib().moe_mxfp8_fused(_ptr(x), _ptr(topk_ids), _ptr(topk_w), _ptr(w13), _ptr(w13_sf),
+                               _ptr(w2), _ptr(w2_sf), _ptr(out), T, H, I, E, k, _ptr(ws), ws_bytes,
+                               _stream(stream))
+    return _check(st, "moe_mxfp8_fused", check)
+
+
+def moe_mxfp8_fused_debug(x, topk_ids, topk_w, w13, w13_sf, w2, w2_sf, out, ws, m_indptr=None,
+                          perm=None, h_fp8=None, h_sf=None, ws_bytes=None, *, dims=None,
+                          stream=None, check=True) -> int:
+    T, H, I, E, k = dims if dims is not None else _fused_dims(x, topk_ids, w13)
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size()
+    st = lib().moe_mxfp8_fused_debug(_ptr(x), _ptr(topk_ids), _ptr(topk_w), _ptr(w13),
+                                     _ptr(w13_sf), _ptr(w2), _ptr(w2_sf), _ptr(out), T, H, I, E,
+                                     k, _ptr(ws), ws_bytes, _stream(stream), _ptr(m_indptr),
+                                     _ptr(perm), _ptr(h_fp8), _ptr(h_sf))
+    return _check(st, "moe_mxfp8_fused_debug", check)
 
 
 def mxfp8_tile_scales(sf_rowmajor, sf_tiled, *, dims=None, stream=None, check=True) -> int:

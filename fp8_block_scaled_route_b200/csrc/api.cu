@@ -288,6 +288,108 @@ static int fused_impl(const void* x, const int32_t* topk_ids, const float* topk_
     return MOE_OK;
 }
 
+// The fused layer with MXFP8 operands.  Same workspace layout as the FP8
+// path: the fp32 scale regions (4 bytes per 128 columns per row) hold the
+// E8M0 scales (one byte per 32 columns per row) in [K/128, R, 4] order.
+static int mx_fused_impl(const void* x, const int32_t* topk_ids, const float* topk_w,
+                         const void* w13, const uint8_t* w13_sf, const void* w2,
+                         const uint8_t* w2_sf, void* out, int T, int H, int I, int E, int k,
+                         void* ws, size_t ws_bytes, moe_stream_t stream, int32_t* dbg_m_indptr,
+                         int32_t* dbg_perm, uint8_t* dbg_hq, uint8_t* dbg_hsf) {
+    if (T < 0 || H <= 0 || I <= 0 || H % 128 || I % 128 || k < 1) return MOE_ERR_INVALID_ARG;
+    if (E < 1) return MOE_ERR_INVALID_ARG;
+    if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+    if (k > E) return MOE_ERR_INVALID_ARG;
+    if (!ws) return MOE_ERR_INVALID_ARG;
+    const FusedWs L = fused_layout(T, H, I, E, k);
+    if (ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+    if (T > 0) {
+        if (!x || !topk_ids || !topk_w || !w13 || !w13_sf || !w2 || !w2_sf || !out)
+            return MOE_ERR_INVALID_ARG;
+        if (!aligned16(x) || !aligned16(w13) || !aligned16(w2) || !aligned16(out) ||
+            !aligned16(w13_sf) || !aligned16(w2_sf))
+            return MOE_ERR_INVALID_ARG;
+    }
+    const DevInfo* d = dev_info();
+    if (int st = check_device(d)) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    char* b = static_cast<char*>(ws);
+    int* status = reinterpret_cast<int*>(b + L.status);
+    int32_t* m_indptr = reinterpret_cast<int32_t*>(b + L.m_indptr);
+    int32_t* perm = reinterpret_cast<int32_t*>(b + L.perm);
+    int32_t* inv_perm = reinterpret_cast<int32_t*>(b + L.inv_perm);
+    uint8_t* xq = reinterpret_cast<uint8_t*>(b + L.xq);
+    uint8_t* xsf = reinterpret_cast<uint8_t*>(b + L.xs);
+    uint8_t* hq = reinterpret_cast<uint8_t*>(b + L.hq);
+    uint8_t* hsf = reinterpret_cast<uint8_t*>(b + L.hs);
+    float* out_acc = reinterpret_cast<float*>(b + L.out_acc);
+    if (cudaMemsetAsync(status, 0, sizeof(int) * kStatusInts, s) != cudaSuccess) return MOE_ERR_CUDA;
+    const int R = T * k;
+    RouteArgs ra{topk_ids, T, k, E, m_indptr, perm, inv_perm,
+                 reinterpret_cast<int32_t*>(b + L.chunk_hist), status};
+    stage_mark(0, s);
+    int st = launch_route_permute(ra, s);
+    if (st) return st;
+    stage_mark(1, s);
+    if (T > 0) {
+        st = launch_mx_quant_scatter(x, T, H, k, R, inv_perm, xq, xsf, out_acc, s);
+        if (st) return st;
+        stage_mark(2, s);
+        const unsigned long long tmo = g_timeout_ns.load();
+        MxGemmArgs g1{};
+        g1.a = xq; g1.b = w13; g1.a_sf = xsf; g1.a_sf_mn = 1; g1.b_sf = w13_sf;
+        g1.m_indptr = m_indptr; g1.R = R; g1.N = 2 * I; g1.K = H; g1.E = E; g1.gated = 1;
+        g1.epi = MX_EPI_SWIGLU_MXQUANT; g1.hq = hq; g1.hsf = hsf;
+        g1.status = status; g1.timeout_ns = tmo; g1.num_sms = d->sms;
+        st = launch_mx_gemm(g1, s);
+        if (st) return st;
+        stage_mark(3, s);
+        MxGemmArgs g2{};
+        g2.a = hq; g2.b = w2; g2.a_sf = hsf; g2.a_sf_mn = 1; g2.b_sf = w2_sf;
+        g2.m_indptr = m_indptr; g2.R = R; g2.N = H; g2.K = I; g2.E = E; g2.gated = 0;
+        g2.epi = MX_EPI_COMBINE; g2.perm = perm; g2.topk_w = topk_w; g2.topk = k;
+        g2.out_acc = out_acc; g2.out_ld = H;
+        g2.status = status; g2.timeout_ns = tmo; g2.num_sms = d->sms;
+        st = launch_mx_gemm(g2, s);
+        if (st) return st;
+        stage_mark(4, s);
+        st = launch_f32_to_bf16(out_acc, out, static_cast<long long>(T) * H, d->sms, s);
+        if (st) return st;
+        stage_mark(5, s);
+    }
+    if (dbg_m_indptr &&
+        cudaMemcpyAsync(dbg_m_indptr, m_indptr, sizeof(int32_t) * (E + 1), cudaMemcpyDeviceToDevice, s))
+        return MOE_ERR_CUDA;
+    if (R > 0) {
+        if (dbg_perm &&
+            cudaMemcpyAsync(dbg_perm, perm, sizeof(int32_t) * R, cudaMemcpyDeviceToDevice, s))
+            return MOE_ERR_CUDA;
+        if (dbg_hq &&
+            cudaMemcpyAsync(dbg_hq, hq, static_cast<size_t>(R) * I, cudaMemcpyDeviceToDevice, s))
+            return MOE_ERR_CUDA;
+        if (dbg_hsf &&
+            cudaMemcpyAsync(dbg_hsf, hsf, static_cast<size_t>(R) * (I / 32), cudaMemcpyDeviceToDevice, s))
+            return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+}
+
+int moe_mxfp8_fused(const void* x, const int32_t* topk_ids, const float* topk_w, const void* w13,
+                    const uint8_t* w13_sf, const void* w2, const uint8_t* w2_sf, void* out, int T,
+                    int H, int I, int E, int k, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    return mx_fused_impl(x, topk_ids, topk_w, w13, w13_sf, w2, w2_sf, out, T, H, I, E, k, ws,
+                         ws_bytes, stream, nullptr, nullptr, nullptr, nullptr);
+}
+
+int moe_mxfp8_fused_debug(const void* x, const int32_t* topk_ids, const float* topk_w,
+                          const void* w13, const uint8_t* w13_sf, const void* w2,
+                          const uint8_t* w2_sf, void* out, int T, int H, int I, int E, int k,
+                          void* ws, size_t ws_bytes, moe_stream_t stream, int32_t* m_indptr,
+                          int32_t* perm, uint8_t* h_fp8, uint8_t* h_sf) {
+    return mx_fused_impl(x, topk_ids, topk_w, w13, w13_sf, w2, w2_sf, out, T, H, I, E, k, ws,
+                         ws_bytes, stream, m_indptr, perm, h_fp8, h_sf);
+}
+
 int moe_fp8_fused(const void* x, const int32_t* topk_ids, const float* topk_w, const void* w13,
                   const float* w13_scale, const void* w2, const float* w2_scale, void* out, int T,
                   int H, int I, int E, int k, void* ws, size_t ws_bytes, moe_stream_t stream) {
@@ -367,6 +469,7 @@ int mxfp8_moe_gemm(const void* a, const void* b, const uint8_t* a_sf, const uint
     g.a = a; g.b = b; g.a_sf = a_sf; g.b_sf = b_sf; g.m_indptr = m_indptr;
     g.a_sf_mn = a_sf_major;
     g.R = R; g.N = N; g.K = K; g.E = E; g.gated = is_gated ? 1 : 0;
+    g.epi = MX_EPI_BF16;
     g.out = out;
     g.status = d->lib_status;
     g.timeout_ns = g_timeout_ns.load();

@@ -93,4 +93,34 @@ __device__ __forceinline__ bool wait_bar_spin(uint64_t* bar, uint32_t parity, co
     }
 }
 
+// E8M0 code of the smallest power of two X = 2^s with amax <= 448 * X.
+// With amax = m * 2^e, m in [1, 2): 448 = 1.75 * 2^8, so s = e - 8 when
+// m <= 1.75 and s = e - 7 otherwise; computed exactly from the fp32 bits.
+__device__ __forceinline__ uint32_t e8m0_code(float amax) {
+    if (!(amax > 0.0f)) return 0u;
+    uint32_t u = __float_as_uint(amax);
+    int e;
+    uint32_t mant;
+    if ((u >> 23) == 0) {  // subnormal: normalise
+        const int lz = __clz(u) - 8;  // leading zeros within the 24-bit significand
+        mant = (u << lz) & 0x7FFFFFu;
+        e = -126 - lz;
+    } else {
+        e = static_cast<int>(u >> 23) - 127;
+        mant = u & 0x7FFFFFu;
+    }
+    const int s = e - 8 + (mant > 0x600000u ? 1 : 0);
+    int c = s + 127;
+    c = c < 0 ? 0 : (c > 254 ? 254 : c);
+    return static_cast<uint32_t>(c);
+}
+
+// 2^(127 - c): the exact reciprocal of the E8M0 value 2^(c - 127).  x * 2^-s
+// and x / 2^s round the same exact value once, so the product is bit-identical
+// to the IEEE quotient for every x (subnormal results included).
+__device__ __forceinline__ float e8m0_reciprocal(uint32_t c) {
+    // c = 0 -> 2^127, c = 254 -> 2^-127 (an fp32 subnormal, exactly representable)
+    return c == 254 ? __uint_as_float(0x00400000u) : __uint_as_float((254u - c) << 23);
+}
+
 }  // namespace moe

@@ -64,6 +64,10 @@ int launch_route_permute(const RouteArgs& r, cudaStream_t stream);
 int launch_quant_scatter(const void* x, int T, int H, int k, int R, const int32_t* inv_perm,
                          uint8_t* xq, float* xs, float* out_acc, cudaStream_t stream);
 
+// MXFP8 variant: xq as above, xsf [H/128, R, 4] E8M0 codes (one per 32 columns).
+int launch_mx_quant_scatter(const void* x, int T, int H, int k, int R, const int32_t* inv_perm,
+                            uint8_t* xq, uint8_t* xsf, float* out_acc, cudaStream_t stream);
+
 // out [n] bf16 = in [n] fp32
 int launch_f32_to_bf16(const float* in, void* out, long long n, int num_sms, cudaStream_t stream);
 
@@ -72,6 +76,12 @@ int launch_swiglu_mxfp8(const void* in, void* out, uint8_t* scale, int M, int K,
 
 // Grouped MXFP8 GEMM on the block-scaled tensor core path: E4M3 operands with
 // one E8M0 scale per 32 K elements of every row of A and of B.
+enum MxEpilogue : int {
+    MX_EPI_BF16 = 0,            // plain bf16 G, or gated bf16 silu(gate) * up
+    MX_EPI_SWIGLU_MXQUANT = 1,  // gated: h to MXFP8 (hq [R, N/2], hsf [N/256, R, 4])
+    MX_EPI_COMBINE = 2,         // plain: out_acc[token, n] += topk_w * G (fp32 reduction)
+};
+
 struct MxGemmArgs {
     const void* a;            // [R, K] E4M3, grouped rows
     const void* b;            // [E, N, K] E4M3
@@ -81,7 +91,15 @@ struct MxGemmArgs {
     const int32_t* m_indptr;  // [E+1]
     int R, N, K, E;
     int gated;                // out [R, N/2] = bf16(silu(G_gate) * G_up), else [R, N] = bf16(G)
+    int epi;                  // MxEpilogue
     void* out;
+    uint8_t* hq;
+    uint8_t* hsf;
+    const int32_t* perm;
+    const float* topk_w;
+    int topk;
+    float* out_acc;
+    int out_ld;
     int* status;
     uint64_t timeout_ns;
     int num_sms;

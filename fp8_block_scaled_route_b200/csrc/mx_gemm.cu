@@ -42,15 +42,16 @@ bool make_tma_map_fp8(CUtensorMap* out, const void* ptr, long long rows, long lo
 namespace {
 
 constexpr int kMxStages = 4;
+constexpr int kMxEpiWarps = 8;
 constexpr int kMxA = 128 * 128;
 constexpr int kMxB = 256 * 128;
 constexpr int kMxSfOff = kMxA + kMxB;
 constexpr int kMxStage = kMxA + kMxB + 2048;  // scale factors: 512 (A) + 1024 (B), padded
 constexpr int kMxMaxE = 1024;
 constexpr int kMxTable = ((2 * (kMxMaxE + 1) * 4) + 15) / 16 * 16;
-constexpr int kMxSmem = 1024 + kMxStages * kMxStage + kMxTable + 256;
+constexpr int kMxCst = kMxEpiWarps * 32 * 16 * 4;  // combine: per-warp 32 x 16 fp32 transpose tile
+constexpr int kMxSmem = 1024 + kMxStages * kMxStage + kMxTable + kMxCst + 256;
 constexpr int kMxThreads = 384;
-constexpr int kMxEpiWarps = 8;
 constexpr int kMxBoxes = 6;  // TMA boxes per stage: 2 x 64 token rows, 4 x 64 weight rows
 constexpr uint32_t kMxTmemCols = 512;
 constexpr uint32_t kMxSfaCol = 256;
@@ -63,13 +64,21 @@ struct MxParams {
     const uint8_t* a_sf;
     const uint8_t* b_sf;
     const int32_t* m_indptr;
-    __nv_bfloat16* out;
+    __nv_bfloat16* out;        // MX_EPI_BF16
+    uint8_t* hq;               // MX_EPI_SWIGLU_MXQUANT: [R, N/2] codes
+    uint8_t* hsf;              //   and [N/256, R, 4] E8M0 scales
+    const int32_t* perm;       // MX_EPI_COMBINE: out_acc[perm[r] / topk] += topk_w[perm[r]] * G[r]
+    const float* topk_w;
+    int topk;
+    float* out_acc;
+    int out_ld;
     int* status;
     unsigned long long timeout_ns;
 };
 
 struct MxSmem {
     uint8_t* stages;
+    float* cstage;
     int* tstart;  // [E+1] first tile of each expert
     int* mind;    // [E+1] clamped m_indptr
     uint64_t* full;
@@ -88,6 +97,8 @@ __device__ __forceinline__ MxSmem mx_carve(uint8_t* base) {
     s.tstart = reinterpret_cast<int*>(p);
     s.mind = s.tstart + (kMxMaxE + 1);
     p += kMxTable;
+    s.cstage = reinterpret_cast<float*>(p);
+    p += kMxCst;
     uint64_t* bars = reinterpret_cast<uint64_t*>(p);
     s.full = bars;
     s.empty = bars + kMxStages;
@@ -271,7 +282,15 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 }
 
 // Warps 4-11: thread = one row of the tile, 64 columns of each weight block
-// (warp w: rows 32 (w % 4) .. +31, column half (w - 4) / 4).
+// (warp w: rows 32 (w % 4) .. +31, column half (w - 4) / 4).  The
+// accumulator leaves TMEM once per tile; then, by mode:
+//  MX_EPI_BF16           bf16 G (plain) or bf16 silu(gate) * up (gated)
+//  MX_EPI_SWIGLU_MXQUANT h = silu(gate) * up requantised to MXFP8: the
+//                        thread's 64 columns are two 32-column blocks, each
+//                        with its own E8M0 scale (no exchange needed)
+//  MX_EPI_COMBINE        out_acc[token] += w * G through a shared-memory
+//                        transpose (8 rows x 64 contiguous bytes per reduction)
+template <int MODE>
 __device__ void mx_epilogue(const MxParams& p, const MxSmem& s, const WaitCtl& wc,
                             uint32_t tmem_base, int total) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -284,6 +303,18 @@ __device__ void mx_epilogue(const MxParams& p, const MxSmem& s, const WaitCtl& w
     uint32_t v[4][32];
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
         const MxTile tl = mx_decode(t, s, p.E);
+        const bool row_ok = rl < tl.rows;
+        const long long row = tl.row0 + rl;
+        // combine: the row's pair id and weight, fetched while the tile computes
+        int c_tok = -1;
+        float c_w = 0.0f;
+        if constexpr (MODE == MX_EPI_COMBINE) {
+            if (row_ok) {
+                const int pair = __ldg(p.perm + row);
+                c_tok = pair / p.topk;
+                c_w = __ldg(p.topk_w + pair);
+            }
+        }
         if (!mx_warp_wait(s.tfull, it & 1, wc, 6)) return;
         tc_fence_after();
         tmem_ld32_async(tl_addr, v[0]);
@@ -297,9 +328,74 @@ __device__ void mx_epilogue(const MxParams& p, const MxSmem& s, const WaitCtl& w
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(s.tempty);
-        if (rl >= tl.rows) continue;
-        const long long row = tl.row0 + rl;
-        if (p.gated) {
+        if constexpr (MODE == MX_EPI_COMBINE) {
+            float* stg = s.cstage + (warp - 4) * 512;
+            const int rr = lane >> 2, cc = lane & 3;
+            float* const obase = p.out_acc + tl.nt * 256 + colg;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                if (tl.nt * 256 + half * 128 >= p.N) break;
+#pragma unroll
+                for (int c16 = 0; c16 < 4; ++c16) {
+                    const uint32_t* a = v[2 * half + (c16 >> 1)] + (c16 & 1) * 16;
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const int slot = (lane & 1) * 4 + ((q4 + (lane >> 1)) & 3);
+                        *reinterpret_cast<float4*>(stg + (lane >> 1) * 32 + slot * 4) =
+                            make_float4(c_w * __uint_as_float(a[4 * q4]),
+                                        c_w * __uint_as_float(a[4 * q4 + 1]),
+                                        c_w * __uint_as_float(a[4 * q4 + 2]),
+                                        c_w * __uint_as_float(a[4 * q4 + 3]));
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int rg = 0; rg < 4; ++rg) {
+                        const int r = rg * 8 + rr;
+                        const int slot = (r & 1) * 4 + ((cc + (r >> 1)) & 3);
+                        const float4 x4 = *reinterpret_cast<const float4*>(stg + (r >> 1) * 32 + slot * 4);
+                        const int t_r = __shfl_sync(0xffffffffu, c_tok, r);
+                        if (t_r >= 0)
+                            red_add_v4(obase + static_cast<long long>(t_r) * p.out_ld + half * 128 +
+                                           c16 * 16 + cc * 4,
+                                       x4.x, x4.y, x4.z, x4.w);
+                    }
+                    __syncwarp();
+                }
+            }
+            continue;
+        }
+        if (!row_ok) continue;
+        if constexpr (MODE == MX_EPI_SWIGLU_MXQUANT) {
+            const int I = p.N >> 1;
+            uint4* dst = reinterpret_cast<uint4*>(p.hq + row * I + tl.nt * 128 + colg);
+            uint32_t sf2 = 0;
+#pragma unroll
+            for (int blk = 0; blk < 2; ++blk) {
+                float h[32];
+                float amax = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    h[i] = mx_silu(__uint_as_float(v[blk][i])) * __uint_as_float(v[2 + blk][i]);
+                    amax = fmaxf(amax, fabsf(h[i]));
+                }
+                const uint32_t code = e8m0_code(amax);
+                const float inv = e8m0_reciprocal(code);
+                sf2 |= code << (8 * blk);
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint4 w;
+                    w.x = cvt_e4m3x4(h[16 * c + 0] * inv, h[16 * c + 1] * inv, h[16 * c + 2] * inv, h[16 * c + 3] * inv);
+                    w.y = cvt_e4m3x4(h[16 * c + 4] * inv, h[16 * c + 5] * inv, h[16 * c + 6] * inv, h[16 * c + 7] * inv);
+                    w.z = cvt_e4m3x4(h[16 * c + 8] * inv, h[16 * c + 9] * inv, h[16 * c + 10] * inv, h[16 * c + 11] * inv);
+                    w.w = cvt_e4m3x4(h[16 * c + 12] * inv, h[16 * c + 13] * inv, h[16 * c + 14] * inv, h[16 * c + 15] * inv);
+                    dst[2 * blk + c] = w;
+                }
+            }
+            // scales of h columns nt*128 + colg + [0, 64): bytes 2g, 2g + 1 of
+            // the row's 4-byte entry for K block nt of the next GEMM
+            *reinterpret_cast<uint16_t*>(p.hsf + (static_cast<long long>(tl.nt) * p.R + row) * 4 + 2 * g) =
+                static_cast<uint16_t>(sf2);
+        } else if (p.gated) {
             // h = silu(gate) * up, 64 bf16 values per row
             uint4* dst = reinterpret_cast<uint4*>(p.out + row * (p.N >> 1) + tl.nt * 128 + colg);
 #pragma unroll
@@ -334,6 +430,7 @@ __device__ void mx_epilogue(const MxParams& p, const MxSmem& s, const WaitCtl& w
     }
 }
 
+template <int MODE>
 __global__ void __launch_bounds__(kMxThreads, 1)
     mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const MxParams p) {
@@ -400,7 +497,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     else if (warp == 1) mx_mma(p, s, wc, tmem_base, total);
     else if (warp == 2) mx_sf_loader<true>(p, s, wc, total);
     else if (warp == 3) mx_sf_loader<false>(p, s, wc, total);
-    else if (warp >= 4) mx_epilogue(p, s, wc, tmem_base, total);
+    else if (warp >= 4) mx_epilogue<MODE>(p, s, wc, tmem_base, total);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -437,30 +534,45 @@ int launch_mx_tile_scales(const uint8_t* rm, uint8_t* tiled, int rows, int K, in
     return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
 }
 
+namespace {
+template <int MODE>
+int launch_mx_inst(const CUtensorMap& ma, const CUtensorMap& mb, const MxParams& p, int num_sms,
+                   cudaStream_t stream) {
+    static int configured_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+        if (cudaFuncSetAttribute(mx_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kMxSmem) != cudaSuccess)
+            return ST_CUDA;
+        configured_dev = dev;
+    }
+    mx_gemm_kernel<MODE><<<num_sms, kMxThreads, kMxSmem, stream>>>(ma, mb, p);
+    return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
+}
+}  // namespace
+
 int launch_mx_gemm(const MxGemmArgs& g, cudaStream_t stream) {
     if (g.R <= 0 || g.E <= 0) return ST_OK;
     if (g.E > kMxMaxE) return ST_INVALID_ARG;
     CUtensorMap ma, mb;
     if (!make_tma_map_fp8(&ma, g.a, g.R, g.K, 64)) return ST_CUDA;
     if (!make_tma_map_fp8(&mb, g.b, static_cast<long long>(g.E) * g.N, g.K, 64)) return ST_CUDA;
-    MxParams p;
+    MxParams p{};
     p.R = g.R; p.N = g.N; p.K = g.K; p.E = g.E; p.nkb = g.K / 128; p.gated = g.gated ? 1 : 0;
     p.a_sf_mn = g.a_sf_mn ? 1 : 0;
     p.a_sf = g.a_sf; p.b_sf = g.b_sf; p.m_indptr = g.m_indptr;
     p.out = static_cast<__nv_bfloat16*>(g.out);
+    p.hq = g.hq; p.hsf = g.hsf;
+    p.perm = g.perm; p.topk_w = g.topk_w; p.topk = g.topk > 0 ? g.topk : 1;
+    p.out_acc = g.out_acc; p.out_ld = g.out_ld;
     p.status = g.status;
     p.timeout_ns = g.timeout_ns;
-    static int configured_dev = -1;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured_dev != dev) {
-        if (cudaFuncSetAttribute(mx_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kMxSmem) != cudaSuccess)
-            return ST_CUDA;
-        configured_dev = dev;
+    switch (g.epi) {
+        case MX_EPI_SWIGLU_MXQUANT: return launch_mx_inst<MX_EPI_SWIGLU_MXQUANT>(ma, mb, p, g.num_sms, stream);
+        case MX_EPI_COMBINE: return launch_mx_inst<MX_EPI_COMBINE>(ma, mb, p, g.num_sms, stream);
+        default: return launch_mx_inst<MX_EPI_BF16>(ma, mb, p, g.num_sms, stream);
     }
-    mx_gemm_kernel<<<g.num_sms, kMxThreads, kMxSmem, stream>>>(ma, mb, p);
-    return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
 }
 
 }  // namespace moe

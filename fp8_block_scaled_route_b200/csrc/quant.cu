@@ -60,6 +60,59 @@ int launch_quant_scatter(const void* x, int T, int H, int k, int R, const int32_
     return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
 }
 
+// MXFP8 variant of quant_scatter: one warp per (token, 128-column block);
+// lane i owns columns 4i..4i+3 and lanes 8j..8j+7 form 32-column block j,
+// which gets one E8M0 scale (e8m0_code) and codes RNE_sat(x / 2^s).  Scales
+// go to xsf [H/128, R, 4] (the four scales of a row's 128-column block
+// together, rows consecutive).
+__global__ void __launch_bounds__(256) mx_quant_scatter_kernel(
+    const __nv_bfloat16* __restrict__ x, int T, int H, int k, int R,
+    const int32_t* __restrict__ inv_perm, uint8_t* __restrict__ xq, uint8_t* __restrict__ xsf,
+    float* __restrict__ out_acc) {
+    const int nkb = H >> 7;
+    const long long item = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    if (item >= static_cast<long long>(T) * nkb) return;
+    const int lane = threadIdx.x & 31;
+    const int t = static_cast<int>(item / nkb);
+    const int kb = static_cast<int>(item - static_cast<long long>(t) * nkb);
+    const long long off = static_cast<long long>(t) * H + kb * 128 + lane * 4;
+    uint2 raw = *reinterpret_cast<const uint2*>(x + off);
+    __nv_bfloat162 b01, b23;
+    memcpy(&b01, &raw.x, 4);
+    memcpy(&b23, &raw.y, 4);
+    const float2 f01 = __bfloat1622float2(b01);
+    const float2 f23 = __bfloat1622float2(b23);
+    float amax = fmaxf(fmaxf(fabsf(f01.x), fabsf(f01.y)), fmaxf(fabsf(f23.x), fabsf(f23.y)));
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const uint32_t code = e8m0_code(amax);
+    const float inv = e8m0_reciprocal(code);
+    const uint32_t codes = cvt_e4m3x4(f01.x * inv, f01.y * inv, f23.x * inv, f23.y * inv);
+    // the four block scales of this 128-column block, one byte each
+    const uint32_t c1 = __shfl_sync(0xffffffffu, code, 8);
+    const uint32_t c2 = __shfl_sync(0xffffffffu, code, 16);
+    const uint32_t c3 = __shfl_sync(0xffffffffu, code, 24);
+    const uint32_t sf4 = code | (c1 << 8) | (c2 << 16) | (c3 << 24);
+    for (int j = 0; j < k; ++j) {
+        const int row = inv_perm[t * k + j];
+        if (row < 0) continue;
+        *reinterpret_cast<uint32_t*>(xq + static_cast<long long>(row) * H + kb * 128 + lane * 4) = codes;
+        if (lane == 0)
+            *reinterpret_cast<uint32_t*>(xsf + (static_cast<long long>(kb) * R + row) * 4) = sf4;
+    }
+    if (out_acc) *reinterpret_cast<float4*>(out_acc + off) = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+int launch_mx_quant_scatter(const void* x, int T, int H, int k, int R, const int32_t* inv_perm,
+                            uint8_t* xq, uint8_t* xsf, float* out_acc, cudaStream_t stream) {
+    const long long items = static_cast<long long>(T) * (H / 128);
+    if (items == 0) return ST_OK;
+    const long long blocks = (items + 7) / 8;
+    mx_quant_scatter_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(x), T, H, k, R, inv_perm, xq, xsf, out_acc);
+    return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
+}
+
 __global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float* __restrict__ in,
                                                           __nv_bfloat16* __restrict__ out,
                                                           long long n4) {
@@ -86,35 +139,6 @@ int launch_f32_to_bf16(const float* in, void* out, long long n, int num_sms, cud
 }
 
 // ------------------------------------------------------------ SwiGLU + MXFP8
-// E8M0 code of the smallest power of two X = 2^s with amax <= 448 * X.
-// With amax = m * 2^e, m in [1, 2): 448 = 1.75 * 2^8, so s = e - 8 when
-// m <= 1.75 and s = e - 7 otherwise; computed exactly from the fp32 bits.
-__device__ __forceinline__ uint32_t e8m0_code(float amax) {
-    if (!(amax > 0.0f)) return 0u;
-    uint32_t u = __float_as_uint(amax);
-    int e;
-    uint32_t mant;
-    if ((u >> 23) == 0) {  // subnormal: normalise
-        const int lz = __clz(u) - 8;  // leading zeros within the 24-bit significand
-        mant = (u << lz) & 0x7FFFFFu;
-        e = -126 - lz;
-    } else {
-        e = static_cast<int>(u >> 23) - 127;
-        mant = u & 0x7FFFFFu;
-    }
-    const int s = e - 8 + (mant > 0x600000u ? 1 : 0);
-    int c = s + 127;
-    c = c < 0 ? 0 : (c > 254 ? 254 : c);
-    return static_cast<uint32_t>(c);
-}
-
-// 2^(127 - c): the exact reciprocal of the E8M0 value 2^(c - 127).  x * 2^-s
-// and x / 2^s round the same exact value once, so the product is bit-identical
-// to the IEEE quotient for every x (subnormal results included).
-__device__ __forceinline__ float e8m0_reciprocal(uint32_t c) {
-    // c = 0 -> 2^127, c = 254 -> 2^-127 (an fp32 subnormal, exactly representable)
-    return c == 254 ? __uint_as_float(0x00400000u) : __uint_as_float((254u - c) << 23);
-}
 
 // silu with the hardware exp2 and reciprocal (about 2 ulp); the result feeds
 // an 8-level-per-octave quantisation, so a flip needs the value to sit within

@@ -219,6 +219,36 @@ MOE_API int mxfp8_moe_gemm(const void* a, const void* b, const uint8_t* a_sf,
                            int R, int N, int K, int E, int a_sf_major, int is_gated,
                            moe_stream_t stream);
 
+/* The fused layer of moe_fp8_fused in the MXFP8 variant: every FP8 operand
+ * carries one E8M0 scale per 32 K elements (the Wave page's MXFP8 grouped
+ * MoE GEMM format; the intermediate is requantised with the SwiGLU + MXFP8
+ * rule of the page "NVIDIA R200(SM107)을 위한 SwiGLU + MXFP8 커널 최적화").
+ * Stages: routing, x quantised per token per 32 columns and scattered into
+ * the k grouped rows, GEMM1 gate/up (block-scaled tensor cores) with
+ * SwiGLU and MXFP8 requantisation in its epilogue, GEMM2 down with the
+ * top-k weighted fp32 combine in its epilogue, bf16 output.
+ *  w13     device FP8 [E, 2I, H] (gate rows then up rows)
+ *  w13_sf  device uint8: E8M0 scales of w13 ([E*2I, H/32] row-major)
+ *          tiled by mxfp8_tile_scales (16-byte aligned)
+ *  w2      device FP8 [E, H, I];  w2_sf: [E*H, I/32] tiled the same way
+ *  x, topk_ids, topk_w, out, T, H, I, E, k, ws, ws_bytes, stream: as for
+ *  moe_fp8_fused; the workspace size is moe_workspace_size(T, H, I, E, k).
+ * Errors as for moe_fp8_fused. */
+MOE_API int moe_mxfp8_fused(const void* x, const int32_t* topk_ids, const float* topk_w,
+                            const void* w13, const uint8_t* w13_sf, const void* w2,
+                            const uint8_t* w2_sf, void* out, int T, int H, int I, int E, int k,
+                            void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_mxfp8_fused plus copies of m_indptr [E+1], perm [T*k], the FP8
+ * intermediate h_fp8 [T*k, I] and its E8M0 scales h_sf [I/128, T*k, 4]
+ * (any may be NULL). */
+MOE_API int moe_mxfp8_fused_debug(const void* x, const int32_t* topk_ids, const float* topk_w,
+                                  const void* w13, const uint8_t* w13_sf, const void* w2,
+                                  const uint8_t* w2_sf, void* out, int T, int H, int I, int E,
+                                  int k, void* ws, size_t ws_bytes, moe_stream_t stream,
+                                  int32_t* m_indptr, int32_t* perm, uint8_t* h_fp8,
+                                  uint8_t* h_sf);
+
 /* Rearranges row-major E8M0 scales [rows, K/32] into the tiled layout that
  * mxfp8_moe_gemm reads for the weights: [rows/128, K/128, 512] bytes, where
  * byte (r % 32) * 16 + ((r / 32) % 4) * 4 + j of block (r / 128, kb) holds
