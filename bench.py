@@ -516,6 +516,80 @@ def run_mx_gemm(args, cfg):
     return 0
 
 
+def run_mx_moe(args, cfg):
+    """The fused layer in the MXFP8 variant (moe_mxfp8_fused) on a workload:
+    same routing and x as the FP8 layer, MXFP8 weights; the FP8 layer with
+    fp32 block scales is timed on the same routing beside it."""
+    import fp8_block_scaled_route_b200 as moe
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    _, bf16, _, src = load_peaks()
+    fp8_peak = bf16 * FP8_OVER_BF16
+    inp = synth.make_mx_moe_inputs(cfg, seed=0, device=dev)
+    T, H, I, E, k = cfg.T, cfg.H, cfg.I, cfg.E, cfg.k
+    w13_sf = torch.empty(E * 2 * I, H // 32, dtype=torch.uint8, device=dev)
+    w2_sf = torch.empty(E * H, I // 32, dtype=torch.uint8, device=dev)
+    moe.mxfp8_tile_scales(inp["w13_sf"].view(E * 2 * I, H // 32), w13_sf)
+    moe.mxfp8_tile_scales(inp["w2_sf"].view(E * H, I // 32), w2_sf)
+    ws = torch.empty(moe.moe_workspace_size(T, H, I, E, k), dtype=torch.uint8, device=dev)
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    counts = work_counts(cfg, inp["topk_ids"])
+
+    def timed(step):
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize(dev)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+        for evs in ev:
+            for e in evs:
+                e.record(stream)
+        torch.cuda.synchronize(dev)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(args.steps):
+            moe.moe_set_stage_events(ev[i])
+            step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        moe.moe_set_stage_events(None)
+        st = moe.moe_get_device_status(ws, stream=stream)
+        if st != moe.MOE_OK:
+            raise RuntimeError(f"device status: {moe.moe_status_string(st)}")
+        stages = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(5)] for e in ev]).mean(axis=0)
+        return a.elapsed_time(b) / args.steps, stages
+
+    ms_mx, st_mx = timed(lambda: moe.moe_mxfp8_fused(
+        inp["x"], inp["topk_ids"], inp["topk_w"], inp["w13"], w13_sf, inp["w2"], w2_sf, out, ws,
+        stream=stream))
+    del w13_sf, w2_sf
+    fp = synth.make_moe_inputs(cfg, seed=0, device=dev)
+    ms_fp, st_fp = timed(lambda: moe.moe_fp8_fused(
+        fp["x"], fp["topk_ids"], fp["topk_w"], fp["w13"], fp["w13_scale"], fp["w2"],
+        fp["w2_scale"], out, ws, stream=stream))
+    g1_tf = counts["g1_flops"] / (st_mx[2] * 1e-3) / 1e12
+    line = {"metric": "fused MoE layer, MXFP8 variant: TFLOP/s", "unit": "TFLOP/s",
+            "value": counts["flops"] / (ms_mx * 1e-3) / 1e12, "ms_per_step": ms_mx,
+            "higher_is_better": True, "steps": args.steps, "warmup": args.warmup, "n_gpus": 1,
+            "dtype": "mxfp8 e4m3 + e8m0 per 32 (fp32 accumulate)", "data": "synthetic",
+            "config": {"workload": workload_desc(cfg) + "; MXFP8 weights and activations",
+                       "l2": "inputs larger than L2 (no flush)"},
+            "stages_us": {n: float(v) * 1e3 for n, v in
+                          zip(["route", "quant", "gemm1", "gemm2", "finish"], st_mx)},
+            "roofline": {"bound": "tensor", "achieved": g1_tf, "peak": fp8_peak,
+                         "unit": "TFLOP/s", "frac": g1_tf / fp8_peak, "traffic": None,
+                         "kernel": "MXFP8 GEMM1 (gate/up + SwiGLU + MXFP8 requant)",
+                         "peak_source": f"{src} (FP8 = bf16 burst x {FP8_OVER_BF16:g})"},
+            "fp8_fp32_scaled_layer_same_routing": {
+                "ms_per_step": ms_fp,
+                "stages_us": {n: float(v) * 1e3 for n, v in
+                              zip(["route", "quant", "gemm1", "gemm2", "finish"], st_fp)}},
+            "gpu_launches": kernels_per_layer(T, k) * args.steps}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -525,8 +599,8 @@ def main():
                     choices=sorted(synth.CONFIGS) + sorted(PROFILE_SLICES))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", default="moe", choices=["moe", "swiglu_mxfp8", "mxfp8_gemm"],
-                    help="swiglu_mxfp8 / mxfp8_gemm: time that standalone op instead")
+    ap.add_argument("--op", default="moe", choices=["moe", "swiglu_mxfp8", "mxfp8_gemm", "mxfp8_moe"],
+                    help="swiglu_mxfp8 / mxfp8_gemm / mxfp8_moe: time that op instead")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -535,6 +609,8 @@ def main():
     cfg = synth.CONFIGS.get(args.workload) or PROFILE_SLICES[args.workload]
     if args.op == "mxfp8_gemm":
         return run_mx_gemm(args, cfg)
+    if args.op == "mxfp8_moe":
+        return run_mx_moe(args, cfg)
     if args.impl == "reference":
         return run_reference(args, cfg)
     return run_ours(args, cfg)
