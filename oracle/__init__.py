@@ -55,6 +55,8 @@ def lib():
         L.oracle_e8m0_scale_code.argtypes = [ctypes.c_float]
         L.oracle_f32_to_bf16.restype = ctypes.c_uint16
         L.oracle_f32_to_bf16.argtypes = [ctypes.c_float]
+        L.oracle_router_topk.restype = None
+        L.oracle_router_topk.argtypes = [P, i, i, i, P, P]
         L.oracle_route_permute.restype = i
         L.oracle_route_permute.argtypes = [P, i, i, i, P, P, P]
         L.oracle_quant_rows_128.restype = None
@@ -131,6 +133,16 @@ def f32_to_bf16_bits(values) -> np.ndarray:
 
 
 # ---------------------------------------------------------------- stages
+def router_topk(logits, k: int):
+    """logits fp32 [T, E] -> (ids int32 [T, k], weights fp32 [T, k])."""
+    l = _c(logits, np.float32)
+    T, E = l.shape
+    ids = np.zeros((T, k), np.int32)
+    w = np.zeros((T, k), np.float32)
+    lib().oracle_router_topk(_p(l), T, E, k, _p(ids), _p(w))
+    return ids, w
+
+
 def route_permute(topk_ids, E: int):
     """Stage a1.  Returns (m_indptr[E+1], perm[R], inv_perm[R], n_bad)."""
     ids = _c(topk_ids, np.int32)

@@ -109,6 +109,38 @@ uint16_t oracle_f32_to_bf16(float f) { return f32_to_bf16(f); }
 /* Stage a1: routing and permutation                                     */
 /* ------------------------------------------------------------------ */
 
+/* Router, the step before the expert computation (the AlphaMoE page's
+ * five-stage pipeline, "문제점: MoE Expert 계산의 병목", starts from each token's
+ * experts and weights).  Reading: a token's k largest logits in descending
+ * order, ties to the lower expert index; weights = softmax over those k
+ * logits in fp32 with the largest one subtracted (expf), summed in slot
+ * order, w_j = e_j / sum. */
+void oracle_router_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w) {
+    #pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        const float* l = logits + (size_t)t * E;
+        int32_t* id = ids + (size_t)t * k;
+        for (int j = 0; j < k; ++j) {
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                int taken = 0;
+                for (int i = 0; i < j; ++i) taken |= (id[i] == e);
+                if (taken) continue;
+                if (best < 0 || l[e] > l[best]) best = e;  /* strict: ties keep the lower index */
+            }
+            id[j] = best;
+        }
+        float ex[1024];
+        float sum = 0.0f;
+        const float m = l[id[0]];
+        for (int j = 0; j < k; ++j) {
+            ex[j] = expf(l[id[j]] - m);
+            sum += ex[j];
+        }
+        for (int j = 0; j < k; ++j) w[(size_t)t * k + j] = ex[j] / sum;
+    }
+}
+
 /* Group the T*k (token, slot) pairs by expert with a stable counting sort.
  * m_indptr[E+1] is the exclusive prefix of per-expert counts; perm maps a
  * grouped row to its pair id p = t*k + j (ascending p inside each group);

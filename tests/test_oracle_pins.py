@@ -362,3 +362,34 @@ def test_balanced_tile_count_bruteforce(oracle):
         want = sum(-(-s // tm) for s in sizes) * (-(-n // 128))
         assert oracle.balanced_tile_count(R, n, E, tm, 128) == want
         assert oracle.balanced_max_rows(R, E) == max(sizes)
+
+
+# ------------------------------------------------------------ router (top-k + softmax)
+@pytest.mark.parametrize("T,E,k,seed", [(64, 256, 8, 0), (17, 5, 5, 1), (40, 1024, 3, 2), (9, 4, 1, 3)])
+def test_router_topk_bruteforce(oracle, T, E, k, seed):
+    g = torch.Generator().manual_seed(seed)
+    logits = torch.randn(T, E, generator=g)
+    # a few exact ties inside the selected set and at its edge
+    logits[0, 1] = logits[0, 0]
+    logits[1, E - 1] = logits[1, 0]
+    ids, w = oracle.router_topk(logits.numpy(), k)
+    for t in range(T):
+        # descending logit, ties to the lower index: a stable sort on -logit
+        order = np.argsort(-logits[t].numpy().astype(np.float64), kind="stable")[:k]
+        np.testing.assert_array_equal(ids[t], order)
+        sel = logits[t].numpy().astype(np.float64)[order]
+        ref = np.exp(sel - sel.max())
+        ref /= ref.sum()
+        np.testing.assert_allclose(w[t], ref, rtol=2e-6, atol=1e-9)
+    assert np.allclose(w.sum(axis=1), 1.0, atol=1e-6)
+
+
+def test_router_matches_generator_for_normal_logits(oracle):
+    # the input generator draws routing with torch.topk + softmax; with
+    # continuous logits (no ties) the oracle's router gives the same ids
+    g = torch.Generator().manual_seed(5)
+    logits = torch.randn(32, 64, generator=g)
+    top_v, top_i = torch.topk(logits, 4, dim=1, largest=True, sorted=True)
+    ids, w = oracle.router_topk(logits.numpy(), 4)
+    np.testing.assert_array_equal(ids, top_i.numpy())
+    np.testing.assert_allclose(w, torch.softmax(top_v, dim=1).numpy(), rtol=2e-6)
