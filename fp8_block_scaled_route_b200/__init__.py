@@ -24,7 +24,7 @@ __all__ = [
     "swiglu_mxfp8_quant", "moe_select_tile_m", "moe_workspace_size", "moe_route_workspace_size",
     "moe_get_device_status", "moe_set_wait_timeout_ns", "moe_status_string",
     "moe_set_stage_events", "moe_route_permute_noalloc", "mxfp8_moe_gemm",
-    "mxfp8_tile_scales", "moe_mxfp8_fused", "moe_mxfp8_fused_debug",
+    "mxfp8_tile_scales", "moe_mxfp8_fused", "moe_mxfp8_fused_debug", "moe_router_topk",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -44,7 +44,7 @@ EXPORTS = (
     "moe_fp8_fused", "moe_fp8_fused_debug", "fp8_groupwise_moe_gemm", "moe_select_tile_m",
     "swiglu_mxfp8_quant", "moe_get_device_status", "moe_set_wait_timeout_ns",
     "moe_set_stage_events", "moe_route_permute_noalloc", "mxfp8_moe_gemm", "mxfp8_tile_scales",
-    "moe_mxfp8_fused", "moe_mxfp8_fused_debug",
+    "moe_mxfp8_fused", "moe_mxfp8_fused_debug", "moe_router_topk",
 )
 
 _lib = None
@@ -90,6 +90,8 @@ def lib():
     L.swiglu_mxfp8_quant.argtypes = [P, P, P, I, I, P]
     L.mxfp8_moe_gemm.restype = I
     L.mxfp8_moe_gemm.argtypes = [P] * 6 + [I] * 6 + [P]
+    L.moe_router_topk.restype = I
+    L.moe_router_topk.argtypes = [P, I, I, I, P, P, P]
     L.mxfp8_tile_scales.restype = I
     L.mxfp8_tile_scales.argtypes = [P, P, I, I, P]
     L.moe_mxfp8_fused.restype = I
@@ -241,6 +243,18 @@ def mxfp8_moe_gemm(a, b, a_sf, b_sf, m_indptr, out, is_gated=False, a_sf_major="
     st = lib().mxfp8_moe_gemm(_ptr(a), _ptr(b), _ptr(a_sf), _ptr(b_sf), _ptr(m_indptr), _ptr(out),
                               R, N, K, E, mode, int(bool(is_gated)), _stream(stream))
     return _check(st, "mxfp8_moe_gemm", check)
+
+
+def moe_router_topk(logits, topk_ids, topk_w, *, dims=None, stream=None, check=True) -> int:
+    """logits fp32 [T, E] -> topk_ids int32 [T, k], topk_w fp32 [T, k].
+    dims = (T, E, k) when raw addresses are passed."""
+    if dims is None:
+        T, E = logits.shape
+        k = topk_ids.shape[1]
+    else:
+        T, E, k = dims
+    st = lib().moe_router_topk(_ptr(logits), T, E, k, _ptr(topk_ids), _ptr(topk_w), _stream(stream))
+    return _check(st, "moe_router_topk", check)
 
 
 def moe_mxfp8_fused(x, topk_ids, topk_w, w13, w13_sf, w2, w2_sf, out, ws, ws_bytes=None, *,

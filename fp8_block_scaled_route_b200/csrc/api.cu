@@ -449,6 +449,17 @@ int fp8_groupwise_moe_gemm(const void* a, const void* b, const float* a_scale, c
     return launch_grouped_gemm(g, s);
 }
 
+int moe_router_topk(const float* logits, int T, int E, int k, int32_t* topk_ids, float* topk_w,
+                    moe_stream_t stream) {
+    if (T < 0 || E < 1 || k < 1 || k > E || k > MOE_ROUTER_MAX_K) return MOE_ERR_INVALID_ARG;
+    if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+    if (T > 0 && (!logits || !topk_ids || !topk_w)) return MOE_ERR_INVALID_ARG;
+    const DevInfo* d = dev_info();
+    if (int st = check_device(d)) return st;
+    return launch_router_topk(logits, T, E, k, topk_ids, topk_w,
+                              reinterpret_cast<cudaStream_t>(stream));
+}
+
 int mxfp8_moe_gemm(const void* a, const void* b, const uint8_t* a_sf, const uint8_t* b_sf,
                    const int32_t* m_indptr, void* out, int R, int N, int K, int E,
                    int a_sf_major, int is_gated, moe_stream_t stream) {

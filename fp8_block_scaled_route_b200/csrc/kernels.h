@@ -59,6 +59,11 @@ struct RouteArgs {
 constexpr int kRouteChunk = 1024;
 int launch_route_permute(const RouteArgs& r, cudaStream_t stream);
 
+// logits fp32 [T, E] -> ids int32 [T, k] (descending logit, ties to the lower
+// expert), w fp32 [T, k] = softmax of the selected logits.  E <= 1024, k <= 32.
+int launch_router_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
+                       cudaStream_t stream);
+
 // x [T, H] bf16 -> xq rows inv_perm[t*k + j] of [R, H], xs [H/128, R];
 // also zeroes out_acc [T, H] when not null.
 int launch_quant_scatter(const void* x, int T, int H, int k, int R, const int32_t* inv_perm,

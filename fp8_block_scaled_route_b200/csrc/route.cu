@@ -245,6 +245,70 @@ __global__ void __launch_bounds__(1024) route_small(const int32_t* __restrict__ 
     }
 }
 
+// Router (the step before the expert computation): one warp per token.
+// Lane l holds logits l + 32 i; the k winners are taken one at a time by a
+// warp-wide argmax (larger logit first, then the lower expert index), so the
+// ids come out in descending logit order.  Lane j keeps the j-th winner's
+// logit; the softmax subtracts the largest, takes expf per slot and sums the
+// slots in order (every lane runs the same sequential sum), w_j = e_j / sum.
+template <int PER>
+__global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ logits, int T,
+                                                          int E, int k, int32_t* __restrict__ ids,
+                                                          float* __restrict__ w) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * 8 + warp;
+    if (t >= T) return;
+    const float* l = logits + static_cast<long long>(t) * E;
+    float v[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = e < E ? l[e] : 0.0f;
+    }
+    uint32_t taken = 0;
+    float mine = 0.0f;  // logit of slot `lane`
+    for (int j = 0; j < k; ++j) {
+        float bv = 0.0f;
+        int be = E;  // E = none
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E && !((taken >> i) & 1u) && (be == E || v[i] > bv)) {
+                bv = v[i];
+                be = e;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            if (oe != E && (be == E || ov > bv || (ov == bv && oe < be))) {
+                bv = ov;
+                be = oe;
+            }
+        }
+        if (lane == (be & 31)) taken |= 1u << (be >> 5);
+        if (lane == j) mine = bv;
+        if (lane == 0) ids[static_cast<long long>(t) * k + j] = be;
+    }
+    const float m = __shfl_sync(0xffffffffu, mine, 0);
+    const float ex = lane < k ? expf(mine - m) : 0.0f;
+    float sum = 0.0f;
+    for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, ex, j);
+    if (lane < k) w[static_cast<long long>(t) * k + lane] = __fdiv_rn(ex, sum);
+}
+
+int launch_router_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
+                       cudaStream_t stream) {
+    if (T == 0) return ST_OK;
+    const unsigned blocks = static_cast<unsigned>((T + 7) / 8);
+    if (E <= 256)
+        router_topk_kernel<8><<<blocks, 256, 0, stream>>>(logits, T, E, k, ids, w);
+    else
+        router_topk_kernel<32><<<blocks, 256, 0, stream>>>(logits, T, E, k, ids, w);
+    return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
+}
+
 int launch_route_permute(const RouteArgs& r, cudaStream_t stream) {
     const int R = r.T * r.k;
     const int nchunks = (R + kRouteChunk - 1) / kRouteChunk;

@@ -61,6 +61,7 @@ typedef enum {
 
 /* Maximum number of experts. */
 #define MOE_MAX_EXPERTS 1024
+#define MOE_ROUTER_MAX_K 32
 
 /* Human-readable name of a status code (static string). */
 MOE_API const char* moe_status_string(int status);
@@ -105,6 +106,21 @@ MOE_API int moe_route_permute(const int32_t* topk_ids, int T, int k, int E,
 MOE_API int moe_route_permute_noalloc(const int32_t* topk_ids, int T, int k, int E,
                                       int32_t* m_indptr, int32_t* perm, int32_t* inv_perm,
                                       moe_stream_t stream);
+
+/* Router: the step before the expert computation (the AlphaMoE page's
+ * five-stage pipeline, section "문제점: MoE Expert 계산의 병목", starts from
+ * each token's experts and weights; the pages do not define the router, so
+ * this is the plainest reading): for each token the k largest logits in
+ * descending order, ties to the lower expert index, and their softmax in
+ * fp32 with the largest subtracted (expf per slot, slots summed in order,
+ * w_j = e_j / sum).  Its outputs feed moe_route_permute / moe_fp8_fused.
+ *  logits    device fp32 [T, E] (finite)
+ *  topk_ids  device int32 [T, k] out;  topk_w device fp32 [T, k] out
+ * 1 <= k <= min(E, MOE_ROUTER_MAX_K); E <= MOE_MAX_EXPERTS; T = 0 is a
+ * no-op.  Caller owns all memory; asynchronous on `stream`; argument errors
+ * are returned before any launch. */
+MOE_API int moe_router_topk(const float* logits, int T, int E, int k, int32_t* topk_ids,
+                            float* topk_w, moe_stream_t stream);
 
 /* ------------------------------------------------------------------ */
 /* The fused layer                                                      */
