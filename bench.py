@@ -177,6 +177,16 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def max_over_ranks(values, pg=None, device="cpu"):
+    """Element-wise maximum of a list of floats over all ranks of the default
+    process group (a collective: every rank must call it, in the same order);
+    the values unchanged when there is no group."""
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if pg is not None:
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -339,10 +349,7 @@ def run_ours(args, cfg):
     e2e_ms = e_start.elapsed_time(e_end)
 
     # max over ranks
-    tvec = torch.tensor([elapsed_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if pg:
-        pg.all_reduce(tvec, op=pg.ReduceOp.MAX)
-    elapsed_ms, e2e_ms = float(tvec[0]), float(tvec[1])
+    elapsed_ms, e2e_ms = max_over_ranks([elapsed_ms, e2e_ms], pg, dev)
 
     if rank == 0:
         ms_step = elapsed_ms / args.steps

@@ -116,6 +116,43 @@ def test_swiglu_and_route_reject_bad_arguments(L):
                                  check=False) == moe.MOE_ERR_INVALID_ARG
 
 
+def test_mxfp8_entry_points_reject_bad_arguments(L):
+    def mx(R=64, N=256, K=256, E=4, mode=0, gated=0, a_sf=FAKE, b_sf=FAKE):
+        return moe.mxfp8_moe_gemm(FAKE, FAKE, a_sf, b_sf, FAKE, FAKE, gated, mode,
+                                  dims=(R, N, K, E), stream=0, check=False)
+    assert mx(K=96) == moe.MOE_ERR_INVALID_ARG          # K not a multiple of 128
+    assert mx(N=200) == moe.MOE_ERR_INVALID_ARG
+    assert mx(gated=1, N=384) == moe.MOE_ERR_INVALID_ARG
+    assert mx(mode=2) == moe.MOE_ERR_INVALID_ARG
+    assert mx(a_sf=FAKE + 2) == moe.MOE_ERR_INVALID_ARG  # activation scales 4-byte aligned
+    assert mx(b_sf=FAKE + 4) == moe.MOE_ERR_INVALID_ARG  # tiled weight scales 16-byte aligned
+    assert mx(E=4096) == moe.MOE_ERR_UNSUPPORTED
+    assert moe.mxfp8_tile_scales(FAKE, FAKE, dims=(100, 256), stream=0, check=False) == \
+        moe.MOE_ERR_INVALID_ARG                          # rows not a multiple of 128
+    assert moe.mxfp8_tile_scales(FAKE, FAKE, dims=(128, 96), stream=0, check=False) == \
+        moe.MOE_ERR_INVALID_ARG
+    ws = moe.moe_workspace_size(8, 256, 128, 4, 2)
+    assert moe.moe_mxfp8_fused(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws,
+                               dims=(8, 200, 128, 4, 2), stream=0, check=False) == \
+        moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_mxfp8_fused(FAKE, FAKE, FAKE, FAKE, FAKE + 4, FAKE, FAKE, FAKE, FAKE, ws,
+                               dims=(8, 256, 128, 4, 2), stream=0, check=False) == \
+        moe.MOE_ERR_INVALID_ARG                          # weight scales 16-byte aligned
+    assert moe.moe_mxfp8_fused(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 10,
+                               dims=(8, 256, 128, 4, 2), stream=0, check=False) == \
+        moe.MOE_ERR_INVALID_ARG                          # workspace too small
+
+
+def test_router_rejects_bad_arguments(L):
+    def r(T=8, E=64, k=4):
+        return moe.moe_router_topk(FAKE, FAKE, FAKE, dims=(T, E, k), stream=0, check=False)
+    assert r(k=0) == moe.MOE_ERR_INVALID_ARG
+    assert r(k=65) == moe.MOE_ERR_INVALID_ARG            # k > E
+    assert r(E=128, k=33) == moe.MOE_ERR_INVALID_ARG     # k above the router's limit
+    assert r(T=-1) == moe.MOE_ERR_INVALID_ARG
+    assert r(E=2048, k=4) == moe.MOE_ERR_UNSUPPORTED
+
+
 def test_product_path_does_not_touch_oracle():
     """The binding and the CUDA sources never import, link or name the oracle."""
     pkg = os.path.join(ROOT, "fp8_block_scaled_route_b200")
