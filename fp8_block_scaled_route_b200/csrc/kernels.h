@@ -97,6 +97,7 @@ struct MxGemmArgs {
     int R, N, K, E;
     int gated;                // out [R, N/2] = bf16(silu(G_gate) * G_up), else [R, N] = bf16(G)
     int epi;                  // MxEpilogue
+    int tile_m;               // 32 (swapped) or 128; <= 0: by group size
     void* out;
     uint8_t* hq;
     uint8_t* hsf;

@@ -88,6 +88,9 @@ def test_mx_gemm_exact_small_integers(oracle):
     (517, 384, 256, 5, False, [0, 130, 1, 0, 386]),  # odd number of 128-column blocks, empty experts
     (1000, 1024, 1024, 8, True, None),
     (640, 512, 7168, 3, False, None),         # 56 K blocks
+    (64, 512, 256, 8, True, None),            # small groups: 32-token swapped tiles
+    (100, 384, 512, 5, False, [0, 40, 1, 0, 59]),  # swapped, groups over one token tile
+    (48, 256, 7168, 6, False, None),          # swapped, 56 K blocks
 ])
 def test_mx_gemm_random(oracle, R, N, K, E, gated, sizes):
     inp = synth.make_mx_gemm_inputs(R, N, K, E, seed=R + K, group_sizes=sizes)
@@ -96,6 +99,24 @@ def test_mx_gemm_random(oracle, R, N, K, E, gated, sizes):
     ref = _oracle(oracle, inp, gated)
     _compare(_run(dev, gated), ref, rows)
     _compare(_run(dev, gated, a_mn=True), ref, rows)
+
+
+def test_mx_gemm_exact_small_integers_swapped(oracle):
+    """As above on the swapped (32-token) tile: groups of at most 32 rows."""
+    torch.manual_seed(1)
+    R, N, K, E = 60, 256, 256, 3
+    table = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).float()
+    ints = {int(v): c for c, v in enumerate(table.tolist()) if v == v and v == int(v) and abs(v) <= 4}
+    lut = torch.tensor([ints[v] for v in range(-4, 5)], dtype=torch.uint8)
+    inp = dict(a=lut[torch.randint(0, 9, (R, K))].view(torch.float8_e4m3fn),
+               b=lut[torch.randint(0, 9, (E, N, K))].view(torch.float8_e4m3fn),
+               a_sf=torch.full((R, K // 32), 127, dtype=torch.uint8),
+               b_sf=torch.full((E, N, K // 32), 127, dtype=torch.uint8),
+               m_indptr=torch.tensor([0, 20, 21, 57], dtype=torch.int32))
+    got = _run({k: v.cuda() for k, v in inp.items()}, False)
+    ref = _oracle(oracle, inp, False)
+    assert torch.equal(got[:57].view(torch.int16), ref[:57].view(torch.int16))
+    assert torch.isnan(got[57:].float()).all()
 
 
 def test_mx_gemm_scale_placement(oracle):
