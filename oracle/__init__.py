@@ -81,6 +81,8 @@ def lib():
         L.oracle_mx_grouped_gemm.argtypes = [P, P, P, P, P, i, i, i, i, P]
         L.oracle_mx_gemm_bf16.restype = None
         L.oracle_mx_gemm_bf16.argtypes = [P, P, P, P, P, i, i, i, i, i, P]
+        L.oracle_moe_mx_tokens.restype = None
+        L.oracle_moe_mx_tokens.argtypes = [P] * 7 + [i] * 5 + [P, i, P, P, P]
         L.oracle_moe_mx_fused.restype = i
         L.oracle_moe_mx_fused.argtypes = [P] * 8 + [i] * 5 + [P] * 4
         L.oracle_num_threads.restype = i
@@ -326,6 +328,27 @@ def moe_mx_fused(x_bits, topk_ids, topk_w, w13, w13_sf, w2, w2_sf, want_dump=Fal
         Rg = int(m_indptr[E])
         return out, m_indptr, perm[:Rg], hq[:Rg], hsf[:Rg]
     return out
+
+
+def moe_mx_tokens(x_bits, topk_ids, topk_w, w13, w13_sf, w2, w2_sf, tokens, want_h=False):
+    """Per-token form of moe_mx_fused for the listed tokens: bf16 bits [n, H]
+    (and hq [n, k, I], hsf [n, k, I/32] when want_h)."""
+    x = _c(x_bits, np.uint16)
+    ids = _c(topk_ids, np.int32)
+    w = _c(topk_w, np.float32)
+    w13 = _u8(w13); w2 = _u8(w2); w13_sf = _u8(w13_sf); w2_sf = _u8(w2_sf)
+    tok = _c(tokens, np.int32)
+    T, H = x.shape
+    k = ids.shape[1]
+    E, I2, _ = w13.shape
+    I = I2 // 2
+    n = len(tok)
+    out = np.zeros((n, H), np.uint16)
+    hq = np.zeros((n, k, I), np.uint8)
+    hsf = np.zeros((n, k, I // 32), np.uint8)
+    lib().oracle_moe_mx_tokens(_p(x), _p(ids), _p(w), _p(w13), _p(w13_sf), _p(w2), _p(w2_sf),
+                               T, H, I, E, k, _p(tok), n, _p(out), _p(hq), _p(hsf))
+    return (out, hq, hsf) if want_h else out
 
 
 # ---------------------------------------------------------------- tile selection

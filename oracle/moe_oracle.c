@@ -633,6 +633,67 @@ int oracle_moe_mx_fused(const uint16_t* x, const int32_t* topk_ids, const float*
     return bad;
 }
 
+/* One 32-wide-block-scaled dot product of length K, as in
+ * oracle_mx_grouped_gemm (block sums and power-of-two scaling exact in
+ * double, blocks accumulated in double). */
+static double mx_dot(const uint8_t* a, const uint8_t* a_sf, const uint8_t* b, const uint8_t* b_sf,
+                     int K, const float* dec) {
+    double acc = 0.0;
+    for (int blk = 0; blk < K / 32; ++blk) {
+        double s = 0.0;
+        for (int i = 0; i < 32; ++i)
+            s += (double)dec[a[blk * 32 + i]] * (double)dec[b[blk * 32 + i]];
+        acc += ldexp(s, (int)a_sf[blk] + (int)b_sf[blk] - 254);
+    }
+    return acc;
+}
+
+/* The MXFP8 layer for selected tokens only, one token at a time (no
+ * grouping): same arithmetic as oracle_moe_mx_fused for each of their rows.
+ * w13_sf [E, 2I, H/32], w2_sf [E, H, I/32] row-major.  out [n_tok, H] bf16;
+ * optional hq [n_tok*k, I], hsf [n_tok*k, I/32] (slot order). */
+void oracle_moe_mx_tokens(const uint16_t* x, const int32_t* topk_ids, const float* topk_w,
+                          const uint8_t* w13, const uint8_t* w13_sf,
+                          const uint8_t* w2, const uint8_t* w2_sf,
+                          int T, int H, int I, int E, int k,
+                          const int32_t* tokens, int n_tok, uint16_t* out,
+                          uint8_t* hq_out, uint8_t* hsf_out) {
+    float dec[256];
+    make_decode_table(dec);
+    (void)T;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int it = 0; it < n_tok; ++it) {
+        int t = tokens[it];
+        uint8_t* xq = (uint8_t*)malloc(H);
+        uint8_t* xsf = (uint8_t*)malloc(H / 32);
+        float* g = (float*)malloc(sizeof(float) * 2 * I);
+        float* h = (float*)malloc(sizeof(float) * I);
+        uint8_t* hq = (uint8_t*)malloc(I);
+        uint8_t* hsf = (uint8_t*)malloc(I / 32);
+        float* acc = (float*)calloc(H, sizeof(float));
+        oracle_quant_rows_mx_bf16(x + (size_t)t * H, 1, H, xq, xsf);
+        for (int j = 0; j < k; ++j) {
+            int e = topk_ids[t * k + j];
+            if (e < 0 || e >= E) continue;
+            for (int n = 0; n < 2 * I; ++n) {
+                const size_t wr = (size_t)e * 2 * I + n;
+                g[n] = (float)mx_dot(xq, xsf, w13 + wr * H, w13_sf + wr * (H / 32), H, dec);
+            }
+            oracle_swiglu(g, 1, I, h);
+            quant_rows_mx_f32(h, 1, I, hq, hsf);
+            if (hq_out) memcpy(hq_out + ((size_t)it * k + j) * I, hq, I);
+            if (hsf_out) memcpy(hsf_out + ((size_t)it * k + j) * (I / 32), hsf, I / 32);
+            for (int c = 0; c < H; ++c) {
+                const size_t wr = (size_t)e * H + c;
+                float yc = (float)mx_dot(hq, hsf, w2 + wr * I, w2_sf + wr * (I / 32), I, dec);
+                acc[c] += topk_w[t * k + j] * yc;
+            }
+        }
+        for (int c = 0; c < H; ++c) out[(size_t)it * H + c] = f32_to_bf16(acc[c]);
+        free(xq); free(xsf); free(g); free(h); free(hq); free(hsf); free(acc);
+    }
+}
+
 /* Threads an OpenMP parallel region would use (0 when built without it). */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

@@ -88,3 +88,57 @@ def test_mx_fused_zero_tokens():
     ws = torch.empty(moe.moe_workspace_size(0, 256, 128, 4, 2), dtype=torch.uint8, device="cuda")
     assert moe.moe_mxfp8_fused(inp["x"], inp["topk_ids"], inp["topk_w"], inp["w13"],
                                _tile(inp["w13_sf"]), inp["w2"], _tile(inp["w2_sf"]), out, ws) == 0
+
+
+def _compact_mx(inp, tokens):
+    """Host copies of only the experts the listed tokens use (MXFP8 weights and
+    row-major scales), with their routing renumbered into the compact list."""
+    dev = inp["topk_ids"].device
+    sel = torch.as_tensor(tokens, device=dev)
+    ids = inp["topk_ids"][sel]
+    used = torch.unique(ids).to(torch.long)
+    remap = torch.full((inp["w13"].shape[0],), -1, dtype=torch.int32, device=dev)
+    remap[used] = torch.arange(len(used), dtype=torch.int32, device=dev)
+    return dict(x=bf16_bits(inp["x"][sel]), topk_ids=i32(remap[ids]), topk_w=f32(inp["topk_w"][sel]),
+                w13=u8(inp["w13"][used]), w13_sf=u8(inp["w13_sf"][used]),
+                w2=u8(inp["w2"][used]), w2_sf=u8(inp["w2_sf"][used]))
+
+
+def _check_mx_sampled(oracle, inp, tokens, what):
+    out, m_indptr, perm, hq, hsf = _run(inp)
+    E = inp["w13"].shape[0]
+    m_o, p_o, i_o, _ = oracle.route_permute(i32(inp["topk_ids"]), E)
+    np.testing.assert_array_equal(m_indptr, m_o, err_msg=what)
+    np.testing.assert_array_equal(perm, p_o, err_msg=what)
+    sub = _compact_mx(inp, tokens)
+    out_o, hq_o, hsf_o = oracle.moe_mx_tokens(sub["x"], sub["topk_ids"], sub["topk_w"], sub["w13"],
+                                              sub["w13_sf"], sub["w2"], sub["w2_sf"],
+                                              np.arange(len(tokens), dtype=np.int32), want_h=True)
+    k = inp["topk_ids"].shape[1]
+    rows = np.array([[i_o[t * k + j] for j in range(k)] for t in tokens]).ravel()
+    got_sf, ref_sf = hsf[rows], hsf_o.reshape(len(rows), -1)
+    assert float((got_sf == ref_sf).mean()) >= SF_MATCH_MIN, what
+    same = np.repeat(got_sf == ref_sf, 32, axis=1)
+    compare_codes(hq[rows][same], hq_o.reshape(len(rows), -1)[same], what + " codes")
+    compare_out(out[tokens], out_o, what + " output")
+
+
+def test_mx_fused_decode_full_size_sampled(oracle):
+    inp = synth.make_mx_moe_inputs(synth.CONFIGS["decode"], seed=0, device="cuda")
+    _check_mx_sampled(oracle, inp, [0, 17, 42, 63], "mx decode")
+    del inp
+    torch.cuda.empty_cache()
+
+
+def test_mx_fused_prefill_full_size_sampled(oracle):
+    inp = synth.make_mx_moe_inputs(synth.CONFIGS["prefill"], seed=0, device="cuda")
+    ids = inp["topk_ids"]
+    counts = torch.bincount(ids.flatten().long(), minlength=256)
+    big = int(torch.argmax(counts))
+    nz = torch.nonzero(counts).flatten()
+    small = int(nz[torch.argmin(counts[nz])])
+    t_big = int(torch.nonzero((ids == big).any(1)).flatten()[0])
+    t_small = int(torch.nonzero((ids == small).any(1)).flatten()[0])
+    _check_mx_sampled(oracle, inp, sorted({0, t_big, t_small, 8191}), "mx prefill")
+    del inp
+    torch.cuda.empty_cache()

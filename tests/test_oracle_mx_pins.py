@@ -209,3 +209,23 @@ def test_mx_layer_token_order(oracle):
     p = torch.randperm(cfg.T, generator=torch.Generator().manual_seed(0))
     got = _mx_layer(oracle, inp, perm_tokens=p)
     assert torch.equal(got.view(torch.int16), base[p].view(torch.int16))
+
+
+def test_mx_layer_per_token_form_equals_grouped(oracle):
+    # the per-token form (used for sampled checks at full size) computes every
+    # row with the same arithmetic as the grouped layer: identical bits
+    cfg, inp = _mx_layer_inputs(4)
+    args = (_bf16_bits(inp["x"]), inp["topk_ids"].numpy(), inp["topk_w"].numpy(),
+            inp["w13"].view(torch.uint8).numpy(), inp["w13_sf"].numpy(),
+            inp["w2"].view(torch.uint8).numpy(), inp["w2_sf"].numpy())
+    full, m_indptr, perm, hq, hsf = oracle.moe_mx_fused(*args, want_dump=True)
+    tokens = np.array([0, 5, cfg.T - 1], np.int32)
+    out, hq_t, hsf_t = oracle.moe_mx_tokens(*args, tokens, want_h=True)
+    np.testing.assert_array_equal(out, full[tokens])
+    inv = np.empty(len(perm), np.int64)
+    inv[perm] = np.arange(len(perm))
+    for i, t in enumerate(tokens):
+        for j in range(cfg.k):
+            r = inv[t * cfg.k + j]
+            np.testing.assert_array_equal(hq_t[i, j], hq[r])
+            np.testing.assert_array_equal(hsf_t[i, j], hsf[r])
