@@ -81,6 +81,14 @@ def lib():
         L.oracle_mx_grouped_gemm.argtypes = [P, P, P, P, P, i, i, i, i, P]
         L.oracle_mx_gemm_bf16.restype = None
         L.oracle_mx_gemm_bf16.argtypes = [P, P, P, P, P, i, i, i, i, i, P]
+        L.oracle_e2m1_decode.restype = ctypes.c_float
+        L.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
+        L.oracle_e2m1_encode.restype = ctypes.c_uint8
+        L.oracle_e2m1_encode.argtypes = [ctypes.c_float]
+        L.oracle_quant_rows_nvfp4.restype = None
+        L.oracle_quant_rows_nvfp4.argtypes = [P, i, i, ctypes.c_float, P, P]
+        L.oracle_nvfp4_grouped_gemm.restype = None
+        L.oracle_nvfp4_grouped_gemm.argtypes = [P, P, ctypes.c_float, P, P, P, P, i, i, i, i, P]
         L.oracle_moe_mx_tokens.restype = None
         L.oracle_moe_mx_tokens.argtypes = [P] * 7 + [i] * 5 + [P, i, P, P, P]
         L.oracle_moe_mx_fused.restype = i
@@ -349,6 +357,38 @@ def moe_mx_tokens(x_bits, topk_ids, topk_w, w13, w13_sf, w2, w2_sf, tokens, want
     lib().oracle_moe_mx_tokens(_p(x), _p(ids), _p(w), _p(w13), _p(w13_sf), _p(w2), _p(w2_sf),
                                T, H, I, E, k, _p(tok), n, _p(out), _p(hq), _p(hsf))
     return (out, hq, hsf) if want_h else out
+
+
+# ---------------------------------------------------------------- NVFP4 variant
+def e2m1_decode(codes) -> np.ndarray:
+    return np.array([lib().oracle_e2m1_decode(int(c)) for c in np.asarray(codes).ravel()],
+                    np.float32).reshape(np.shape(codes))
+
+
+def e2m1_encode(values) -> np.ndarray:
+    return np.array([lib().oracle_e2m1_encode(float(v)) for v in np.asarray(values).ravel()],
+                    np.uint8).reshape(np.shape(values))
+
+
+def quant_rows_nvfp4(x, g: float):
+    """[rows, cols] fp32 -> (E2M1 codes [rows, cols], E4M3 block scales [rows, cols/16])."""
+    x = _c(x, np.float32)
+    rows, cols = x.shape
+    q = np.zeros((rows, cols), np.uint8)
+    sf = np.zeros((rows, cols // 16), np.uint8)
+    lib().oracle_quant_rows_nvfp4(_p(x), rows, cols, float(g), _p(q), _p(sf))
+    return q, sf
+
+
+def nvfp4_grouped_gemm(a, a_sf, ga, b, b_sf, gb, m_indptr):
+    a = _u8(a); b = _u8(b); a_sf = _u8(a_sf); b_sf = _u8(b_sf)
+    gb = _c(gb, np.float32); m_indptr = _c(m_indptr, np.int32)
+    R, K = a.shape
+    E, N, _ = b.shape
+    out = np.zeros((R, N), np.float32)
+    lib().oracle_nvfp4_grouped_gemm(_p(a), _p(a_sf), float(ga), _p(b), _p(b_sf), _p(gb),
+                                    _p(m_indptr), R, N, K, E, _p(out))
+    return out
 
 
 # ---------------------------------------------------------------- tile selection

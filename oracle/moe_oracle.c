@@ -694,6 +694,97 @@ void oracle_moe_mx_tokens(const uint16_t* x, const int32_t* topk_ids, const floa
     }
 }
 
+/* ------------------------------------------------------------------ */
+/* NVFP4 variant: FP4 E2M1 values, one E4M3 scale per 16 elements and   */
+/* one fp32 global scale per tensor (per expert for weights)            */
+/* ------------------------------------------------------------------ */
+/*
+ * The cuTile page ("FlashInfer에 cuTile 기반 Fused MoE 백엔드 도입", section
+ * "2. cuTile NVFP4 양자화 지원") quantises the experts to NVFP4 (W4A4) with
+ * fp4_quantize(weight, global_scale=<per expert>, sf_vec_size=16); it gives
+ * no formulas.  Reading taken here (the format's published definition):
+ *  - E2M1: sign, 2 exponent bits (bias 1), 1 mantissa bit; magnitudes
+ *    0, 0.5, 1, 1.5, 2, 3, 4, 6 (0.5 is the subnormal); no inf/NaN.
+ *  - the global scale g multiplies the data into range (g = 448*6/amax of
+ *    the tensor is the usual choice, passed in);
+ *  - per 16 consecutive elements: scale code c = E4M3_RNE_sat(amax_block * g / 6)
+ *    (an all-zero block gets c = 0);
+ *  - codes q = E2M1_RNE_sat(x * g / dec(c)) (q = 0 where dec(c) = 0);
+ *  - dequantised value = dec_e2m1(q) * dec_e4m3(c) / g.
+ */
+static const float kE2M1[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+
+float oracle_e2m1_decode(uint8_t c) {
+    float v = kE2M1[c & 7];
+    return (c & 8) ? -v : v;
+}
+
+/* Round to the nearest E2M1 value, ties to the even code, saturating at 6. */
+uint8_t oracle_e2m1_encode(float v) {
+    uint8_t sign = (v < 0.0f || (v == 0.0f && signbit(v))) ? 8 : 0;
+    float a = fabsf(v);
+    if (!(a == a)) return sign;  /* NaN: not produced by finite inputs */
+    uint8_t best = 0;
+    for (uint8_t c = 1; c < 8; ++c) {
+        float d = fabsf(a - kE2M1[c]), db = fabsf(a - kE2M1[best]);
+        if (d < db || (d == db && (c & 1) == 0)) best = c;
+    }
+    return (uint8_t)(sign | best);
+}
+
+/* x [rows, cols] fp32, cols a multiple of 16; g the global scale.
+ * q [rows, cols] E2M1 codes (one per byte, low 4 bits); sf [rows, cols/16]
+ * E4M3 codes. */
+void oracle_quant_rows_nvfp4(const float* x, int rows, int cols, float g, uint8_t* q, uint8_t* sf) {
+    #pragma omp parallel for schedule(static)
+    for (int r = 0; r < rows; ++r) {
+        for (int b = 0; b < cols / 16; ++b) {
+            const float* v = x + (size_t)r * cols + b * 16;
+            float amax = 0.0f;
+            for (int i = 0; i < 16; ++i) {
+                float a = fabsf(v[i]);
+                if (a > amax) amax = a;
+            }
+            uint8_t c = oracle_e4m3_encode(amax * g / 6.0f);
+            float s = oracle_e4m3_decode(c);
+            sf[(size_t)r * (cols / 16) + b] = c;
+            for (int i = 0; i < 16; ++i)
+                q[(size_t)r * cols + b * 16 + i] = s > 0.0f ? oracle_e2m1_encode(v[i] * g / s) : 0;
+        }
+    }
+}
+
+/* Grouped NVFP4 GEMM in the m_indptr layout: per 16-wide K block,
+ * dec(sa) dec(sb) / (ga gb_e) times the block dot of the E2M1 values, in
+ * double, rounded to fp32 once.  a [R, K] codes, a_sf [R, K/16], ga;
+ * b [E, N, K] codes, b_sf [E, N, K/16], gb [E]. */
+void oracle_nvfp4_grouped_gemm(const uint8_t* a, const uint8_t* a_sf, float ga, const uint8_t* b,
+                               const uint8_t* b_sf, const float* gb, const int32_t* m_indptr,
+                               int R, int N, int K, int E, float* out) {
+    float dec[256];
+    make_decode_table(dec);
+    const int nb = K / 16;
+    (void)R;
+    for (int e = 0; e < E; ++e) {
+        #pragma omp parallel for schedule(static)
+        for (int r = m_indptr[e]; r < m_indptr[e + 1]; ++r) {
+            for (int n = 0; n < N; ++n) {
+                const size_t wrow = (size_t)e * N + n;
+                double acc = 0.0;
+                for (int blk = 0; blk < nb; ++blk) {
+                    double s = 0.0;
+                    for (int i = 0; i < 16; ++i)
+                        s += (double)oracle_e2m1_decode(a[(size_t)r * K + blk * 16 + i]) *
+                             (double)oracle_e2m1_decode(b[wrow * K + blk * 16 + i]);
+                    acc += s * (double)dec[a_sf[(size_t)r * nb + blk]] *
+                           (double)dec[b_sf[wrow * nb + blk]];
+                }
+                out[(size_t)r * N + n] = (float)(acc / ((double)ga * (double)gb[e]));
+            }
+        }
+    }
+}
+
 /* Threads an OpenMP parallel region would use (0 when built without it). */
 int oracle_num_threads(void) {
 #ifdef _OPENMP
