@@ -89,6 +89,8 @@ def lib():
         L.oracle_quant_rows_nvfp4.argtypes = [P, i, i, ctypes.c_float, P, P]
         L.oracle_nvfp4_grouped_gemm.restype = None
         L.oracle_nvfp4_grouped_gemm.argtypes = [P, P, ctypes.c_float, P, P, P, P, i, i, i, i, P]
+        L.oracle_nvfp4_gemm_bf16.restype = None
+        L.oracle_nvfp4_gemm_bf16.argtypes = [P, P, ctypes.c_float, P, P, P, P, i, i, i, i, i, P]
         L.oracle_moe_mx_tokens.restype = None
         L.oracle_moe_mx_tokens.argtypes = [P] * 7 + [i] * 5 + [P, i, P, P, P]
         L.oracle_moe_mx_fused.restype = i
@@ -388,6 +390,18 @@ def nvfp4_grouped_gemm(a, a_sf, ga, b, b_sf, gb, m_indptr):
     out = np.zeros((R, N), np.float32)
     lib().oracle_nvfp4_grouped_gemm(_p(a), _p(a_sf), float(ga), _p(b), _p(b_sf), _p(gb),
                                     _p(m_indptr), R, N, K, E, _p(out))
+    return out
+
+
+def nvfp4_gemm_bf16(a, a_sf, ga, b, b_sf, gb, m_indptr, is_gated: bool):
+    """bf16 bits of the NVFP4 GEMM: [R, N], or gated [R, N/2] = silu(gate) * up."""
+    a = _u8(a); b = _u8(b); a_sf = _u8(a_sf); b_sf = _u8(b_sf)
+    gb = _c(gb, np.float32); m_indptr = _c(m_indptr, np.int32)
+    R, K = a.shape
+    E, N, _ = b.shape
+    out = np.zeros((R, N // 2 if is_gated else N), np.uint16)
+    lib().oracle_nvfp4_gemm_bf16(_p(a), _p(a_sf), float(ga), _p(b), _p(b_sf), _p(gb),
+                                 _p(m_indptr), R, N, K, E, int(bool(is_gated)), _p(out))
     return out
 
 

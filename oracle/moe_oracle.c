@@ -785,6 +785,28 @@ void oracle_nvfp4_grouped_gemm(const uint8_t* a, const uint8_t* a_sf, float ga, 
     }
 }
 
+/* bf16 output of the NVFP4 GEMM, as oracle_mx_gemm_bf16: plain out [R, N],
+ * or gated out [R, N/2] = bf16(silu(G[:, :N/2]) * G[:, N/2:]) with G (global
+ * scales applied) rounded to fp32 first. */
+void oracle_nvfp4_gemm_bf16(const uint8_t* a, const uint8_t* a_sf, float ga, const uint8_t* b,
+                            const uint8_t* b_sf, const float* gb, const int32_t* m_indptr,
+                            int R, int N, int K, int E, int is_gated, uint16_t* out) {
+    float* g = (float*)malloc(sizeof(float) * ((size_t)R * N + 1));
+    for (size_t i = 0; i < (size_t)R * N; ++i) g[i] = 0.0f;
+    oracle_nvfp4_grouped_gemm(a, a_sf, ga, b, b_sf, gb, m_indptr, R, N, K, E, g);
+    int Rg = m_indptr[E];
+    if (!is_gated) {
+        for (size_t i = 0; i < (size_t)Rg * N; ++i) out[i] = f32_to_bf16(g[i]);
+    } else {
+        int I = N / 2;
+        float* h = (float*)malloc(sizeof(float) * ((size_t)R * I + 1));
+        oracle_swiglu(g, Rg, I, h);
+        for (size_t i = 0; i < (size_t)Rg * I; ++i) out[i] = f32_to_bf16(h[i]);
+        free(h);
+    }
+    free(g);
+}
+
 /* Threads an OpenMP parallel region would use (0 when built without it). */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

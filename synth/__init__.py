@@ -214,3 +214,76 @@ def make_mx_moe_inputs(cfg: MoEConfig, seed: int = 0, device="cpu"):
             torch.randn(H, I, generator=g, device=device) / math.sqrt(I))
     base.update(w13=w13, w13_sf=w13_sf, w2=w2, w2_sf=w2_sf)
     return base
+
+
+E2M1_VALUES = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
+
+
+def _e2m1_codes(v: torch.Tensor) -> torch.Tensor:
+    """Nearest E2M1 code (sign bit 8, magnitude code 0..7), ties to the even
+    code, saturating at 6."""
+    mags = torch.tensor(E2M1_VALUES, device=v.device, dtype=torch.float32)
+    a = v.abs().clamp(max=6.0)
+    d = (a[..., None] - mags).abs()
+    best = d.min(dim=-1, keepdim=True).values
+    cand = d == best
+    # among tied candidates prefer the even code
+    even = torch.arange(8, device=v.device) % 2 == 0
+    pick = torch.where(cand & even, 1, 0) * 16 + torch.where(cand, 1, 0)
+    code = pick.argmax(dim=-1).to(torch.uint8)
+    sign = (v < 0).to(torch.uint8) * 8
+    return code | sign
+
+
+def quantize_nvfp4_rows(x: torch.Tensor, g: float):
+    """[rows, cols] fp32, global scale g -> (E2M1 codes [rows, cols] one per
+    byte, E4M3 block scales [rows, cols/16] as float8_e4m3fn): per 16 values
+    c = E4M3(amax * g / 6) (torch's float8 cast), codes E2M1(x * g / dec(c))."""
+    rows, cols = x.shape
+    blocks = x.view(rows, cols // 16, 16)
+    amax = blocks.abs().amax(dim=2)
+    sc = (amax * g / 6.0).to(torch.float8_e4m3fn)
+    dec = sc.to(torch.float32)
+    scaled = torch.where(dec[:, :, None] > 0, blocks * g / dec[:, :, None].clamp(min=1e-30),
+                         torch.zeros_like(blocks))
+    return _e2m1_codes(scaled).view(rows, cols), sc.contiguous()
+
+
+def pack_e2m1(codes: torch.Tensor) -> torch.Tensor:
+    """[rows, cols] codes -> [rows, cols/2] bytes, element 2i in the low nibble."""
+    c = codes.view(codes.shape[0], -1, 2).to(torch.uint8)
+    return (c[..., 0] | (c[..., 1] << 4)).contiguous()
+
+
+def make_nvfp4_gemm_inputs(R: int, N: int, K: int, E: int, seed: int = 0, device="cpu",
+                           group_sizes=None):
+    """Inputs for the NVFP4 grouped GEMM: activations N(0,1) and weights
+    N(0,1/K), with per-16 magnitudes 2^U{-3..3}; global scales 448*6/amax of
+    the activations and of each expert's weights; codes unpacked (one per
+    byte, for the oracle) and packed (two per byte)."""
+    g = _gen(seed, device)
+    if group_sizes is None:
+        idx = torch.randint(0, E, (R,), generator=g, device=device)
+        group_sizes = torch.bincount(idx, minlength=E)
+    group_sizes = torch.as_tensor(group_sizes, device=device, dtype=torch.int64)
+    m_indptr = torch.zeros(E + 1, dtype=torch.int32, device=device)
+    m_indptr[1:] = torch.cumsum(group_sizes, 0).to(torch.int32)
+    R = int(m_indptr[-1])
+
+    def spread(x):
+        u = torch.randint(-3, 4, (x.shape[0], x.shape[1] // 16), generator=g, device=device)
+        return (x.view(x.shape[0], -1, 16) * torch.exp2(u.float())[:, :, None]).view(x.shape)
+
+    a32 = spread(torch.randn(max(R, 1), K, generator=g, device=device))[:R]
+    ga = 448.0 * 6.0 / max(float(a32.abs().max()) if R else 1.0, 1e-30)
+    a, a_sf = quantize_nvfp4_rows(a32, ga)
+    b = torch.empty(E, N, K, dtype=torch.uint8, device=device)
+    b_sf = torch.empty(E, N, K // 16, dtype=torch.float8_e4m3fn, device=device)
+    gb = torch.empty(E, dtype=torch.float32, device=device)
+    for e in range(E):
+        w = spread(torch.randn(N, K, generator=g, device=device) / math.sqrt(K))
+        gb[e] = 448.0 * 6.0 / float(w.abs().max())
+        b[e], b_sf[e] = quantize_nvfp4_rows(w, float(gb[e]))
+    return dict(a=a, a_packed=pack_e2m1(a) if R else a.view(0, K // 2), a_sf=a_sf, ga=ga,
+                b=b, b_packed=pack_e2m1(b.view(E * N, K)).view(E, N, K // 2), b_sf=b_sf, gb=gb,
+                m_indptr=m_indptr)

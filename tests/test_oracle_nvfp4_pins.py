@@ -90,3 +90,52 @@ def test_nvfp4_gemm_exact_small_values(oracle):
                                     np.full((E, N, 2), 0x38, np.uint8), np.ones(1, np.float32),
                                     np.array([0, R], np.int32))
     np.testing.assert_array_equal(got, (dec[q_a] @ dec[q_b[0]].T).astype(np.float32))
+
+
+def _e4m3_code_of(v):
+    table = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    hits = np.flatnonzero(table == v)
+    assert len(hits), v
+    return int(hits[0])
+
+
+def test_nvfp4_bf16_reduces_to_mxfp8_bf16(oracle):
+    """Every E2M1 value is an E4M3 value and a power-of-two E4M3 block scale is
+    an E8M0 scale: with unit global scales and the same scale on both 16-wide
+    halves of every 32-wide block, the NVFP4 GEMM is an MXFP8 GEMM, so the
+    bf16 outputs (plain and gated) are bit-identical to the pinned MXFP8 ones."""
+    rng = np.random.default_rng(3)
+    R, N, K, E = 40, 64, 128, 3
+    m_indptr = np.array([0, 11, 11, 40], np.int32)
+    q_a = rng.integers(0, 16, (R, K)).astype(np.uint8)
+    q_b = rng.integers(0, 16, (E, N, K)).astype(np.uint8)
+    exp_a = rng.integers(-3, 4, (R, K // 32))
+    exp_b = rng.integers(-3, 4, (E, N, K // 32))
+    to_e4 = np.vectorize(lambda e: _e4m3_code_of(2.0 ** e))
+    sf_a = np.repeat(to_e4(exp_a), 2, axis=-1).astype(np.uint8)
+    sf_b = np.repeat(to_e4(exp_b), 2, axis=-1).astype(np.uint8)
+    e2m1_to_e4m3 = np.array([_e4m3_code_of(v) if v != 0 else (0x80 if c & 8 else 0)
+                             for c, v in enumerate(_e2m1_from_bits(c) for c in range(16))], np.uint8)
+    mx_a, mx_b = e2m1_to_e4m3[q_a], e2m1_to_e4m3[q_b]
+    for gated in (False, True):
+        got = oracle.nvfp4_gemm_bf16(q_a, sf_a, 1.0, q_b, sf_b, np.ones(E, np.float32), m_indptr, gated)
+        want = oracle.mx_gemm_bf16(mx_a, (exp_a + 127).astype(np.uint8), mx_b,
+                                   (exp_b + 127).astype(np.uint8), m_indptr, gated)
+        np.testing.assert_array_equal(got[:40], want[:40])
+
+
+def test_nvfp4_bf16_global_scales(oracle):
+    """Global scales divide the output: halving ga doubles every output (exact
+    in bf16, a power of two)."""
+    rng = np.random.default_rng(4)
+    R, N, K, E = 16, 32, 64, 2
+    q_a = rng.integers(0, 16, (R, K)).astype(np.uint8)
+    q_b = rng.integers(0, 16, (E, N, K)).astype(np.uint8)
+    sf_a = rng.integers(0x30, 0x48, (R, K // 16)).astype(np.uint8)
+    sf_b = rng.integers(0x30, 0x48, (E, N, K // 16)).astype(np.uint8)
+    gb = np.array([3.0, 0.5], np.float32)
+    m = np.array([0, 7, 16], np.int32)
+    one = oracle.nvfp4_gemm_bf16(q_a, sf_a, 4.0, q_b, sf_b, gb, m, False).view(np.int16)
+    two = oracle.nvfp4_gemm_bf16(q_a, sf_a, 2.0, q_b, sf_b, gb, m, False).view(np.int16)
+    f = lambda b: torch.from_numpy(b.copy()).view(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(f(two), 2.0 * f(one))
