@@ -37,6 +37,7 @@ import synth  # noqa: E402
 
 METRIC = "fused MoE layer µs & TFLOPS/GB/s as % of B200 FP8-tensor/HBM roofline"
 FP8_OVER_BF16 = 2.0        # nominal dense FP8 / BF16 tensor ratio (4.5 / 2.25 PFLOP/s)
+FP4_OVER_BF16 = 4.0        # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 PFLOP/s)
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 ROUTE_CHUNK = 1024         # (token, slot) pairs per routing chunk
@@ -523,6 +524,66 @@ def run_mx_gemm(args, cfg):
     return 0
 
 
+def run_nvfp4_gemm(args, cfg):
+    """NVFP4 grouped GEMM (packed E2M1 operands, E4M3 scales per 16 K
+    elements, per-expert alpha) on the gate/up GEMM of a workload: A = the
+    workload's routed rows [T*k, H], B = gated weights [E, 2I, H], group sizes
+    from its routing; activations N(0,1) and weights N(0,1/H) with per-16
+    magnitudes 2^U{-3..3}, quantised to NVFP4 with global scales
+    448*6/amax.  Inputs exceed L2."""
+    import fp8_block_scaled_route_b200 as moe
+    torch.cuda.set_device(0)
+    _, bf16, _, src = load_peaks()
+    fp4_peak = bf16 * FP4_OVER_BF16
+    ids = synth.make_moe_inputs(cfg, seed=0, device="cuda", weights=False)["topk_ids"]
+    sizes = torch.bincount(ids.flatten().long(), minlength=cfg.E).cpu().tolist()
+    R, N, K, E = sum(sizes), 2 * cfg.I, cfg.H, cfg.E
+    inp = synth.make_nvfp4_gemm_inputs(R, N, K, E, seed=1, device="cuda", group_sizes=sizes)
+    a, b = inp["a_packed"], inp["b_packed"]
+    del inp["a"], inp["b"]
+    a_sf = inp["a_sf"].view(torch.uint8)
+    b_sf = torch.empty(E * N, K // 16, dtype=torch.uint8, device="cuda")
+    moe.nvfp4_tile_scales(inp["b_sf"].view(torch.uint8).view(E * N, K // 16), b_sf)
+    alpha = (1.0 / (inp["ga"] * inp["gb"].double())).float()
+    out = torch.empty(R, N // 2, dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        moe.nvfp4_moe_gemm(a, b, a_sf, b_sf, alpha, inp["m_indptr"], out, True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for _ in range(args.steps):
+        step()
+    ev1.record()
+    torch.cuda.synchronize()
+    st = moe.moe_get_device_status(None)
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device status: {moe.moe_status_string(st)}")
+    ms = ev0.elapsed_time(ev1) / args.steps
+    flops = 2.0 * R * N * K
+    touched = sum(1 for x in sizes if x > 0)
+    nbytes = touched * N * K * (0.5 + 1 / 16) + R * K * (0.5 + 1 / 16) + R * (N // 2) * 2
+    tf = flops / (ms * 1e-3) / 1e12
+    line = {"metric": "NVFP4 grouped GEMM (gate/up + SwiGLU) TFLOP/s", "value": tf,
+            "unit": "TFLOP/s", "higher_is_better": True, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "n_gpus": 1, "data": "synthetic",
+            "dtype": "nvfp4 e2m1 + e4m3 per 16 + fp32 global (fp32 accumulate)",
+            "config": {"workload": f"{cfg.name} gate/up GEMM: R={R} N={N} K={K} E={E}, "
+                                   f"group sizes from its routing",
+                       "l2": "inputs larger than L2 (no flush)"},
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": fp4_peak, "unit": "TFLOP/s",
+                         "frac": tf / fp4_peak, "traffic": None,
+                         "peak_source": f"{src} (FP4 = bf16 burst x {FP4_OVER_BF16:g})",
+                         "alg_bytes": nbytes, "gbs": nbytes / (ms * 1e-3) / 1e9},
+            "gpu_launches": args.steps}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_mx_moe(args, cfg):
     """The fused layer in the MXFP8 variant (moe_mxfp8_fused) on a workload:
     same routing and x as the FP8 layer, MXFP8 weights; the FP8 layer with
@@ -606,7 +667,8 @@ def main():
                     choices=sorted(synth.CONFIGS) + sorted(PROFILE_SLICES))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", default="moe", choices=["moe", "swiglu_mxfp8", "mxfp8_gemm", "mxfp8_moe"],
+    ap.add_argument("--op", default="moe", choices=["moe", "swiglu_mxfp8", "mxfp8_gemm", "mxfp8_moe",
+                                                     "nvfp4_gemm"],
                     help="swiglu_mxfp8 / mxfp8_gemm / mxfp8_moe: time that op instead")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -616,6 +678,8 @@ def main():
     cfg = synth.CONFIGS.get(args.workload) or PROFILE_SLICES[args.workload]
     if args.op == "mxfp8_gemm":
         return run_mx_gemm(args, cfg)
+    if args.op == "nvfp4_gemm":
+        return run_nvfp4_gemm(args, cfg)
     if args.op == "mxfp8_moe":
         return run_mx_moe(args, cfg)
     if args.impl == "reference":

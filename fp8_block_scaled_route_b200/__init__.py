@@ -25,6 +25,7 @@ __all__ = [
     "moe_get_device_status", "moe_set_wait_timeout_ns", "moe_status_string",
     "moe_set_stage_events", "moe_route_permute_noalloc", "mxfp8_moe_gemm",
     "mxfp8_tile_scales", "moe_mxfp8_fused", "moe_mxfp8_fused_debug", "moe_router_topk",
+    "nvfp4_moe_gemm", "nvfp4_tile_scales",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -44,7 +45,8 @@ EXPORTS = (
     "moe_fp8_fused", "moe_fp8_fused_debug", "fp8_groupwise_moe_gemm", "moe_select_tile_m",
     "swiglu_mxfp8_quant", "moe_get_device_status", "moe_set_wait_timeout_ns",
     "moe_set_stage_events", "moe_route_permute_noalloc", "mxfp8_moe_gemm", "mxfp8_tile_scales",
-    "moe_mxfp8_fused", "moe_mxfp8_fused_debug", "moe_router_topk",
+    "moe_mxfp8_fused", "moe_mxfp8_fused_debug", "moe_router_topk", "nvfp4_moe_gemm",
+    "nvfp4_tile_scales",
 )
 
 _lib = None
@@ -94,6 +96,10 @@ def lib():
     L.moe_router_topk.argtypes = [P, I, I, I, P, P, P]
     L.mxfp8_tile_scales.restype = I
     L.mxfp8_tile_scales.argtypes = [P, P, I, I, P]
+    L.nvfp4_moe_gemm.restype = I
+    L.nvfp4_moe_gemm.argtypes = [P] * 7 + [I] * 5 + [P]
+    L.nvfp4_tile_scales.restype = I
+    L.nvfp4_tile_scales.argtypes = [P, P, I, I, P]
     L.moe_mxfp8_fused.restype = I
     L.moe_mxfp8_fused.argtypes = [P] * 8 + [I] * 5 + [P, ctypes.c_size_t, P]
     L.moe_mxfp8_fused_debug.restype = I
@@ -293,6 +299,35 @@ def mxfp8_tile_scales(sf_rowmajor, sf_tiled, *, dims=None, stream=None, check=Tr
         rows, K = dims
     st = lib().mxfp8_tile_scales(_ptr(sf_rowmajor), _ptr(sf_tiled), rows, K, _stream(stream))
     return _check(st, "mxfp8_tile_scales", check)
+
+
+def nvfp4_moe_gemm(a, b, a_sf, b_sf, alpha, m_indptr, out, is_gated=False, *, dims=None,
+                   stream=None, check=True) -> int:
+    """a uint8 [R, K/2] packed E2M1, b uint8 [E, N, K/2], a_sf uint8 [R, K/16] E4M3
+    row-major, b_sf the weight scales tiled by nvfp4_tile_scales, alpha fp32 [E],
+    out bf16 [R, N/2 if gated else N].  dims = (R, N, K, E) when raw addresses
+    are passed."""
+    if dims is None:
+        R = a.shape[0]
+        K = a.shape[1] * 2
+        E, N = b.shape[0], b.shape[1]
+    else:
+        R, N, K, E = dims
+    st = lib().nvfp4_moe_gemm(_ptr(a), _ptr(b), _ptr(a_sf), _ptr(b_sf), _ptr(alpha), _ptr(m_indptr),
+                              _ptr(out), R, N, K, E, int(bool(is_gated)), _stream(stream))
+    return _check(st, "nvfp4_moe_gemm", check)
+
+
+def nvfp4_tile_scales(sf_rowmajor, sf_tiled, *, dims=None, stream=None, check=True) -> int:
+    """sf_rowmajor uint8 [rows, K/16] E4M3 -> sf_tiled uint8 (rows * K/16 bytes, tiled).
+    dims = (rows, K) when raw addresses are passed."""
+    if dims is None:
+        rows = sf_rowmajor.numel() // sf_rowmajor.shape[-1]
+        K = sf_rowmajor.shape[-1] * 16
+    else:
+        rows, K = dims
+    st = lib().nvfp4_tile_scales(_ptr(sf_rowmajor), _ptr(sf_tiled), rows, K, _stream(stream))
+    return _check(st, "nvfp4_tile_scales", check)
 
 
 def swiglu_mxfp8_quant(inp, out, scale, *, dims=None, stream=None, check=True) -> int:

@@ -500,6 +500,48 @@ int mxfp8_tile_scales(const uint8_t* sf_rowmajor, uint8_t* sf_tiled, int rows, i
                                  reinterpret_cast<cudaStream_t>(stream));
 }
 
+int nvfp4_moe_gemm(const void* a, const void* b, const uint8_t* a_sf, const uint8_t* b_sf,
+                   const float* alpha, const int32_t* m_indptr, void* out, int R, int N, int K,
+                   int E, int is_gated, moe_stream_t stream) {
+    if (R < 0 || N <= 0 || K <= 0 || E < 1 || N % 128 || K % 256) return MOE_ERR_INVALID_ARG;
+    if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+    if (is_gated && (N % 2 || (N / 2) % 128)) return MOE_ERR_INVALID_ARG;
+    if (!m_indptr || (R > 0 && (!a || !b || !a_sf || !b_sf || !alpha || !out)))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(b) || !aligned16(out) || !aligned16(b_sf))
+        return MOE_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(a_sf) | reinterpret_cast<uintptr_t>(alpha)) & 3)
+        return MOE_ERR_INVALID_ARG;
+    const DevInfo* d = dev_info();
+    if (int st = check_device(d)) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(d->lib_status, 0, sizeof(int) * kStatusInts, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (R == 0) return MOE_OK;
+    NvGemmArgs g{};
+    g.a = a; g.b = b; g.a_sf = a_sf; g.b_sf = b_sf; g.alpha = alpha; g.m_indptr = m_indptr;
+    g.R = R; g.N = N; g.K = K; g.E = E; g.gated = is_gated ? 1 : 0;
+    g.out = out;
+    g.status = d->lib_status;
+    g.timeout_ns = g_timeout_ns.load();
+    g.num_sms = d->sms;
+    return launch_nvfp4_gemm(g, s);
+}
+
+int nvfp4_tile_scales(const uint8_t* sf_rowmajor, uint8_t* sf_tiled, int rows, int K,
+                      moe_stream_t stream) {
+    if (rows < 0 || K <= 0 || K % 64 || rows % 128) return MOE_ERR_INVALID_ARG;
+    if (rows > 0 && (!sf_rowmajor || !sf_tiled)) return MOE_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(sf_rowmajor) | reinterpret_cast<uintptr_t>(sf_tiled)) & 3)
+        return MOE_ERR_INVALID_ARG;
+    const DevInfo* d = dev_info();
+    if (int st = check_device(d)) return st;
+    // K/16 scales per row in groups of four: the MXFP8 tiling of a 2K-wide row
+    // (2K/32 = K/16 scales, 2K/128 = K/64 groups)
+    return launch_mx_tile_scales(sf_rowmajor, sf_tiled, rows, 2 * K, d->sms,
+                                 reinterpret_cast<cudaStream_t>(stream));
+}
+
 int swiglu_mxfp8_quant(const void* in, void* out, uint8_t* scale, int M, int K, moe_stream_t stream) {
     if (M < 0 || K <= 0 || K % 32) return MOE_ERR_INVALID_ARG;
     if (M > 0 && (!in || !out || !scale)) return MOE_ERR_INVALID_ARG;

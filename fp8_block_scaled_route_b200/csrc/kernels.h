@@ -118,4 +118,23 @@ int launch_mx_gemm(const MxGemmArgs& g, cudaStream_t stream);
 int launch_mx_tile_scales(const uint8_t* rm, uint8_t* tiled, int rows, int K, int num_sms,
                           cudaStream_t stream);
 
+// Grouped NVFP4 GEMM on the block-scaled tensor core path: E2M1 operands
+// packed two per byte, one E4M3 scale per 16 K elements of every row of A and
+// of B, G = alpha[e] * (block-scaled product).
+struct NvGemmArgs {
+    const void* a;            // [R, K/2] packed E2M1, grouped rows
+    const void* b;            // [E, N, K/2] packed E2M1
+    const uint8_t* a_sf;      // [R, K/16] E4M3, row-major
+    const uint8_t* b_sf;      // [E*N/128, K/64, 512] E4M3, tiled (launch_mx_tile_scales of 2K)
+    const float* alpha;       // [E] 1 / (global scale of A * global scale of expert e)
+    const int32_t* m_indptr;  // [E+1]
+    int R, N, K, E;
+    int gated;                // out [R, N/2] = bf16(silu(G_gate) * G_up), else [R, N] = bf16(G)
+    void* out;
+    int* status;
+    uint64_t timeout_ns;
+    int num_sms;
+};
+int launch_nvfp4_gemm(const NvGemmArgs& g, cudaStream_t stream);
+
 }  // namespace moe

@@ -277,6 +277,50 @@ MOE_API int mxfp8_tile_scales(const uint8_t* sf_rowmajor, uint8_t* sf_tiled, int
                               moe_stream_t stream);
 
 /* ------------------------------------------------------------------ */
+/* Grouped NVFP4 GEMM (block-scaled tensor core path)                   */
+/* ------------------------------------------------------------------ */
+
+/* The NVFP4 (W4A4) expert GEMM of the page "FlashInfer에 cuTile 기반 Fused
+ * MoE 백엔드 도입" (section "2. cuTile NVFP4 양자화 지원": fp4_quantize with a
+ * per-expert global scale, sf_vec_size=16), in the grouped layout of
+ * fp8_groupwise_moe_gemm.  E2M1 values (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6)
+ * with one E4M3 scale per 16 consecutive K elements of every row and a global
+ * scale per tensor; a real value is e2m1(q) * e4m3(s) / g:
+ *   G[r, n] = alpha[e] * sum over 16-wide K blocks b of
+ *             e4m3(a_sf[r,b]) * e4m3(b_sf[e,n,b]) * sum_k e2m1(a[r,k]) * e2m1(b[e,n,k]),
+ *   alpha[e] = 1 / (g_a * g_b[e]),  e = the expert with m_indptr[e] <= r < m_indptr[e+1];
+ * the block scales are applied inside the tensor core, fp32 accumulation.
+ *  a       device uint8 [R, K/2]: E2M1 codes packed two per byte, element
+ *          2i in the low nibble (sign bit 3 of each nibble)
+ *  b       device uint8 [E, N, K/2], packed the same way
+ *  a_sf    device uint8 [R, K/16] E4M3 codes, row-major (4-byte aligned)
+ *  b_sf    device uint8 E4M3 codes of the weights in the tiled layout that
+ *          nvfp4_tile_scales produces from [E, N, K/16] row-major (16-byte
+ *          aligned; weights are tiled once, not per call)
+ *  alpha   device fp32 [E]
+ *  m_indptr device int32 [E+1]
+ *  out     device bf16: plain [R, N] = bf16(G); gated [R, N/2] =
+ *          bf16(silu(G[:, :N/2]) * G[:, N/2:]) (gate rows then up rows of b)
+ * Rows outside [m_indptr[0], m_indptr[E]) are not written.  K must be a
+ * multiple of 256, N of 128 (gated: N/2 too); a, b, out 16-byte aligned.
+ * Errors and ownership as for mxfp8_moe_gemm. */
+MOE_API int nvfp4_moe_gemm(const void* a, const void* b, const uint8_t* a_sf,
+                           const uint8_t* b_sf, const float* alpha, const int32_t* m_indptr,
+                           void* out, int R, int N, int K, int E, int is_gated,
+                           moe_stream_t stream);
+
+/* Rearranges row-major E4M3 block scales [rows, K/16] into the tiled layout
+ * that nvfp4_moe_gemm reads for the weights: [rows/128, K/64, 512] bytes,
+ * where byte (r % 32) * 16 + ((r / 32) % 4) * 4 + j of block (r / 128, kb)
+ * holds scale j (of the four 16-wide blocks) of row r in K block kb -- the
+ * scales one K = 64 tensor core step reads.  No counterpart on the pages: it
+ * is this library's storage format.  rows a multiple of 128, K of 64;
+ * pointers 4-byte aligned (16 for use by nvfp4_moe_gemm); asynchronous on
+ * `stream`. */
+MOE_API int nvfp4_tile_scales(const uint8_t* sf_rowmajor, uint8_t* sf_tiled, int rows, int K,
+                              moe_stream_t stream);
+
+/* ------------------------------------------------------------------ */
 /* Standalone SwiGLU + MXFP8 quantisation                               */
 /* ------------------------------------------------------------------ */
 

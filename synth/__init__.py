@@ -221,18 +221,14 @@ E2M1_VALUES = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
 
 def _e2m1_codes(v: torch.Tensor) -> torch.Tensor:
     """Nearest E2M1 code (sign bit 8, magnitude code 0..7), ties to the even
-    code, saturating at 6."""
-    mags = torch.tensor(E2M1_VALUES, device=v.device, dtype=torch.float32)
-    a = v.abs().clamp(max=6.0)
-    d = (a[..., None] - mags).abs()
-    best = d.min(dim=-1, keepdim=True).values
-    cand = d == best
-    # among tied candidates prefer the even code
-    even = torch.arange(8, device=v.device) % 2 == 0
-    pick = torch.where(cand & even, 1, 0) * 16 + torch.where(cand, 1, 0)
-    code = pick.argmax(dim=-1).to(torch.uint8)
-    sign = (v < 0).to(torch.uint8) * 8
-    return code | sign
+    code, saturating at 6: the magnitude code counts the midpoints between
+    neighbouring values that |v| passes (a midpoint below an odd code needs
+    |v| strictly above it, one below an even code |v| at or above it)."""
+    a = v.abs()
+    code = torch.zeros(v.shape, dtype=torch.uint8, device=v.device)
+    for i, mid in enumerate((0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0)):
+        code += ((a > mid) if i % 2 == 0 else (a >= mid)).to(torch.uint8)
+    return code | ((v < 0).to(torch.uint8) * 8)
 
 
 def quantize_nvfp4_rows(x: torch.Tensor, g: float):
