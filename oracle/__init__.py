@@ -90,6 +90,11 @@ def lib():
         L.oracle_nvfp4_grouped_gemm.restype = None
         L.oracle_nvfp4_grouped_gemm.argtypes = [P, P, ctypes.c_float, P, P, P, P, i, i, i, i, P]
         L.oracle_nvfp4_gemm_bf16.restype = None
+        L.oracle_moe_nvfp4_fused.restype = i
+        L.oracle_moe_nvfp4_fused.argtypes = [P] * 9 + [ctypes.c_float] * 2 + [P] + [i] * 5 + [P] * 4
+        L.oracle_moe_nvfp4_tokens.restype = None
+        L.oracle_moe_nvfp4_tokens.argtypes = ([P] * 9 + [ctypes.c_float] * 2 + [i] * 5 +
+                                              [P, i, P, P, P])
         L.oracle_nvfp4_gemm_bf16.argtypes = [P, P, ctypes.c_float, P, P, P, P, i, i, i, i, i, P]
         L.oracle_moe_mx_tokens.restype = None
         L.oracle_moe_mx_tokens.argtypes = [P] * 7 + [i] * 5 + [P, i, P, P, P]
@@ -403,6 +408,61 @@ def nvfp4_gemm_bf16(a, a_sf, ga, b, b_sf, gb, m_indptr, is_gated: bool):
     lib().oracle_nvfp4_gemm_bf16(_p(a), _p(a_sf), float(ga), _p(b), _p(b_sf), _p(gb),
                                  _p(m_indptr), R, N, K, E, int(bool(is_gated)), _p(out))
     return out
+
+
+def moe_nvfp4_fused(x_bits, topk_ids, topk_w, w13, w13_sf, w13_g, w2, w2_sf, w2_g, a1_g, a2_g,
+                    want_dump=False):
+    """The fused layer with NVFP4 operands.  x_bits [T,H] bf16 bits; w13 [E,2I,H]
+    E2M1 codes (one per byte), w13_sf [E,2I,H/16] E4M3, w13_g [E]; w2 [E,H,I],
+    w2_sf [E,H,I/16], w2_g [E]; a1_g, a2_g the activations' global scales.
+    Returns bf16 bits [T,H] (and m_indptr, perm, hq [R,I], hsf [R,I/16] when
+    want_dump)."""
+    x = _c(x_bits, np.uint16)
+    ids = _c(topk_ids, np.int32)
+    w = _c(topk_w, np.float32)
+    w13 = _u8(w13); w2 = _u8(w2); w13_sf = _u8(w13_sf); w2_sf = _u8(w2_sf)
+    w13_g = _c(w13_g, np.float32); w2_g = _c(w2_g, np.float32)
+    T, H = x.shape
+    k = ids.shape[1]
+    E, I2, _ = w13.shape
+    I = I2 // 2
+    R = T * k
+    out = np.zeros((T, H), np.uint16)
+    m_indptr = np.zeros(E + 1, np.int32)
+    perm = np.zeros(max(R, 1), np.int32)
+    hq = np.zeros((max(R, 1), I), np.uint8)
+    hsf = np.zeros((max(R, 1), I // 16), np.uint8)
+    lib().oracle_moe_nvfp4_fused(_p(x), _p(ids), _p(w), _p(w13), _p(w13_sf), _p(w13_g), _p(w2),
+                                 _p(w2_sf), _p(w2_g), float(a1_g), float(a2_g), _p(out), T, H, I,
+                                 E, k, _p(m_indptr), _p(perm), _p(hq), _p(hsf))
+    if want_dump:
+        Rg = int(m_indptr[E])
+        return out, m_indptr, perm[:Rg], hq[:Rg], hsf[:Rg]
+    return out
+
+
+def moe_nvfp4_tokens(x_bits, topk_ids, topk_w, w13, w13_sf, w13_g, w2, w2_sf, w2_g, a1_g, a2_g,
+                     tokens, want_h=False):
+    """Per-token form of moe_nvfp4_fused for the listed tokens: bf16 bits [n, H]
+    (and hq [n, k, I], hsf [n, k, I/16] when want_h)."""
+    x = _c(x_bits, np.uint16)
+    ids = _c(topk_ids, np.int32)
+    w = _c(topk_w, np.float32)
+    w13 = _u8(w13); w2 = _u8(w2); w13_sf = _u8(w13_sf); w2_sf = _u8(w2_sf)
+    w13_g = _c(w13_g, np.float32); w2_g = _c(w2_g, np.float32)
+    tok = _c(tokens, np.int32)
+    T, H = x.shape
+    k = ids.shape[1]
+    E, I2, _ = w13.shape
+    I = I2 // 2
+    n = len(tok)
+    out = np.zeros((n, H), np.uint16)
+    hq = np.zeros((n, k, I), np.uint8)
+    hsf = np.zeros((n, k, I // 16), np.uint8)
+    lib().oracle_moe_nvfp4_tokens(_p(x), _p(ids), _p(w), _p(w13), _p(w13_sf), _p(w13_g), _p(w2),
+                                  _p(w2_sf), _p(w2_g), float(a1_g), float(a2_g), T, H, I, E, k,
+                                  _p(tok), n, _p(out), _p(hq), _p(hsf))
+    return (out, hq, hsf) if want_h else out
 
 
 # ---------------------------------------------------------------- tile selection

@@ -807,6 +807,138 @@ void oracle_nvfp4_gemm_bf16(const uint8_t* a, const uint8_t* a_sf, float ga, con
     free(g);
 }
 
+/* x [rows, cols] bf16 bits -> NVFP4 codes and scales with global scale g
+ * (oracle_quant_rows_nvfp4 on the exact fp32 values of x). */
+static void quant_rows_nvfp4_bf16(const uint16_t* x, int rows, int cols, float g, uint8_t* q,
+                                  uint8_t* sf) {
+    float* xf = (float*)malloc(sizeof(float) * ((size_t)rows * cols + 1));
+    for (size_t i = 0; i < (size_t)rows * cols; ++i) xf[i] = bf16_to_f32(x[i]);
+    oracle_quant_rows_nvfp4(xf, rows, cols, g, q, sf);
+    free(xf);
+}
+
+/* The fused layer in the NVFP4 (W4A4) variant: the five stages of the
+ * AlphaMoE page's pipeline ("문제점: MoE Expert 계산의 병목", stages 1-5) with
+ * every operand in NVFP4 as the cuTile page quantises it ("2. cuTile NVFP4
+ * 양자화 지원"): x quantised per token per 16 columns with the global scale
+ * a1_g and gathered into grouped rows, GEMM1 gate/up (weights w13 with
+ * per-expert global scales w13_g), SwiGLU in fp32, the intermediate
+ * requantised per row per 16 columns with the global scale a2_g, GEMM2 down
+ * (w2, w2_g), combine in fp32 (ascending slot) and bf16.  Codes one per byte;
+ * scales row-major: w13_sf [E, 2I, H/16], w2_sf [E, H, I/16].  Optional dumps:
+ * m_indptr [E+1], perm [R], hq [R, I] codes, hsf [R, I/16]. */
+int oracle_moe_nvfp4_fused(const uint16_t* x, const int32_t* topk_ids, const float* topk_w,
+                           const uint8_t* w13, const uint8_t* w13_sf, const float* w13_g,
+                           const uint8_t* w2, const uint8_t* w2_sf, const float* w2_g,
+                           float a1_g, float a2_g, uint16_t* out, int T, int H, int I, int E,
+                           int k, int32_t* m_indptr_out, int32_t* perm_out, uint8_t* hq_out,
+                           uint8_t* hsf_out) {
+    int R = T * k;
+    int32_t* m_indptr = (int32_t*)malloc(sizeof(int32_t) * (E + 1));
+    int32_t* perm = (int32_t*)malloc(sizeof(int32_t) * (R > 0 ? R : 1));
+    int32_t* inv_perm = (int32_t*)malloc(sizeof(int32_t) * (R > 0 ? R : 1));
+    int bad = oracle_route_permute(topk_ids, T, k, E, m_indptr, perm, inv_perm);
+    int Rg = m_indptr[E];
+
+    uint8_t* xq_tok = (uint8_t*)malloc((size_t)T * H + 1);
+    uint8_t* xsf_tok = (uint8_t*)malloc((size_t)T * (H / 16) + 1);
+    quant_rows_nvfp4_bf16(x, T, H, a1_g, xq_tok, xsf_tok);
+    uint8_t* xq = (uint8_t*)malloc((size_t)R * H + 1);
+    uint8_t* xsf = (uint8_t*)malloc((size_t)R * (H / 16) + 1);
+    for (int r = 0; r < Rg; ++r) {
+        int t = perm[r] / k;
+        memcpy(xq + (size_t)r * H, xq_tok + (size_t)t * H, H);
+        memcpy(xsf + (size_t)r * (H / 16), xsf_tok + (size_t)t * (H / 16), H / 16);
+    }
+    float* g = (float*)malloc(sizeof(float) * ((size_t)R * 2 * I + 1));
+    oracle_nvfp4_grouped_gemm(xq, xsf, a1_g, w13, w13_sf, w13_g, m_indptr, R, 2 * I, H, E, g);
+    float* h = (float*)malloc(sizeof(float) * ((size_t)R * I + 1));
+    oracle_swiglu(g, Rg, I, h);
+    uint8_t* hq = (uint8_t*)malloc((size_t)R * I + 1);
+    uint8_t* hsf = (uint8_t*)malloc((size_t)R * (I / 16) + 1);
+    oracle_quant_rows_nvfp4(h, Rg, I, a2_g, hq, hsf);
+    float* y = (float*)malloc(sizeof(float) * ((size_t)R * H + 1));
+    oracle_nvfp4_grouped_gemm(hq, hsf, a2_g, w2, w2_sf, w2_g, m_indptr, R, H, I, E, y);
+    for (int t = 0; t < T; ++t)
+        for (int c = 0; c < H; ++c) {
+            float acc = 0.0f;
+            for (int j = 0; j < k; ++j) {
+                int row = inv_perm[t * k + j];
+                if (row < 0) continue;
+                acc += topk_w[t * k + j] * y[(size_t)row * H + c];
+            }
+            out[(size_t)t * H + c] = f32_to_bf16(acc);
+        }
+    if (m_indptr_out) memcpy(m_indptr_out, m_indptr, sizeof(int32_t) * (E + 1));
+    if (perm_out) memcpy(perm_out, perm, sizeof(int32_t) * Rg);
+    if (hq_out) memcpy(hq_out, hq, (size_t)Rg * I);
+    if (hsf_out) memcpy(hsf_out, hsf, (size_t)Rg * (I / 16));
+    free(m_indptr); free(perm); free(inv_perm); free(xq_tok); free(xsf_tok);
+    free(xq); free(xsf); free(g); free(h); free(hq); free(hsf); free(y);
+    return bad;
+}
+
+/* One NVFP4 dot product of length K, as in oracle_nvfp4_grouped_gemm: block
+ * sums and scale products in double, blocks accumulated in double, then
+ * divided by the product of the global scales and rounded to fp32. */
+static float nvfp4_dot(const uint8_t* a, const uint8_t* a_sf, float ga, const uint8_t* b,
+                       const uint8_t* b_sf, float gb, int K, const float* dec) {
+    double acc = 0.0;
+    for (int blk = 0; blk < K / 16; ++blk) {
+        double s = 0.0;
+        for (int i = 0; i < 16; ++i)
+            s += (double)oracle_e2m1_decode(a[blk * 16 + i]) * (double)oracle_e2m1_decode(b[blk * 16 + i]);
+        acc += s * (double)dec[a_sf[blk]] * (double)dec[b_sf[blk]];
+    }
+    return (float)(acc / ((double)ga * (double)gb));
+}
+
+/* The NVFP4 layer for selected tokens only, one token at a time (no
+ * grouping): same arithmetic as oracle_moe_nvfp4_fused for each of their
+ * rows.  out [n_tok, H] bf16; optional hq [n_tok*k, I], hsf [n_tok*k, I/16]
+ * (slot order). */
+void oracle_moe_nvfp4_tokens(const uint16_t* x, const int32_t* topk_ids, const float* topk_w,
+                             const uint8_t* w13, const uint8_t* w13_sf, const float* w13_g,
+                             const uint8_t* w2, const uint8_t* w2_sf, const float* w2_g,
+                             float a1_g, float a2_g, int T, int H, int I, int E, int k,
+                             const int32_t* tokens, int n_tok, uint16_t* out, uint8_t* hq_out,
+                             uint8_t* hsf_out) {
+    float dec[256];
+    make_decode_table(dec);
+    (void)T;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int it = 0; it < n_tok; ++it) {
+        int t = tokens[it];
+        uint8_t* xq = (uint8_t*)malloc(H);
+        uint8_t* xsf = (uint8_t*)malloc(H / 16);
+        float* g = (float*)malloc(sizeof(float) * 2 * I);
+        float* h = (float*)malloc(sizeof(float) * I);
+        uint8_t* hq = (uint8_t*)malloc(I);
+        uint8_t* hsf = (uint8_t*)malloc(I / 16);
+        float* acc = (float*)calloc(H, sizeof(float));
+        quant_rows_nvfp4_bf16(x + (size_t)t * H, 1, H, a1_g, xq, xsf);
+        for (int j = 0; j < k; ++j) {
+            int e = topk_ids[t * k + j];
+            if (e < 0 || e >= E) continue;
+            for (int n = 0; n < 2 * I; ++n) {
+                const size_t wr = (size_t)e * 2 * I + n;
+                g[n] = nvfp4_dot(xq, xsf, a1_g, w13 + wr * H, w13_sf + wr * (H / 16), w13_g[e], H, dec);
+            }
+            oracle_swiglu(g, 1, I, h);
+            oracle_quant_rows_nvfp4(h, 1, I, a2_g, hq, hsf);
+            if (hq_out) memcpy(hq_out + ((size_t)it * k + j) * I, hq, I);
+            if (hsf_out) memcpy(hsf_out + ((size_t)it * k + j) * (I / 16), hsf, I / 16);
+            for (int c = 0; c < H; ++c) {
+                const size_t wr = (size_t)e * H + c;
+                float yc = nvfp4_dot(hq, hsf, a2_g, w2 + wr * I, w2_sf + wr * (I / 16), w2_g[e], I, dec);
+                acc[c] += topk_w[t * k + j] * yc;
+            }
+        }
+        for (int c = 0; c < H; ++c) out[(size_t)it * H + c] = f32_to_bf16(acc[c]);
+        free(xq); free(xsf); free(g); free(h); free(hq); free(hsf); free(acc);
+    }
+}
+
 /* Threads an OpenMP parallel region would use (0 when built without it). */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

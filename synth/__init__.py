@@ -283,3 +283,44 @@ def make_nvfp4_gemm_inputs(R: int, N: int, K: int, E: int, seed: int = 0, device
     return dict(a=a, a_packed=pack_e2m1(a) if R else a.view(0, K // 2), a_sf=a_sf, ga=ga,
                 b=b, b_packed=pack_e2m1(b.view(E * N, K)).view(E, N, K // 2), b_sf=b_sf, gb=gb,
                 m_indptr=m_indptr)
+
+
+# Calibrated global scales of the NVFP4 layer's activations: 448*6 / the
+# assumed bound of |x| (8; x ~ N(0,1)) and of |silu(gate) * up| (16).
+NVFP4_A1_GSCALE = 448.0 * 6.0 / 8.0
+NVFP4_A2_GSCALE = 448.0 * 6.0 / 16.0
+
+
+def make_nvfp4_moe_inputs(cfg: MoEConfig, seed: int = 0, device="cpu", keep_codes=True):
+    """The fused layer's inputs with NVFP4 weights: routing and x as in
+    make_moe_inputs; w13 [E,2I,H] and w2 [E,H,I] drawn N(0, 1/fan_in),
+    per-expert global scales 448*6/amax, quantised per row per 16
+    (quantize_nvfp4_rows).  Returns packed codes (w13_packed [E,2I,H/2],
+    w2_packed [E,H,I/2]), the codes one per byte when keep_codes (w13, w2),
+    E4M3 scales as uint8 (w13_sf [E,2I,H/16], w2_sf [E,H,I/16]), global
+    scales w13_g, w2_g [E] and the activations' a1_g, a2_g."""
+    base = make_moe_inputs(cfg, seed, device, weights=False)
+    g = _gen(seed + 7919, device)
+    E, H, I = cfg.E, cfg.H, cfg.I
+    out = dict(w13_packed=torch.empty(E, 2 * I, H // 2, dtype=torch.uint8, device=device),
+               w13_sf=torch.empty(E, 2 * I, H // 16, dtype=torch.uint8, device=device),
+               w13_g=torch.empty(E, dtype=torch.float32, device=device),
+               w2_packed=torch.empty(E, H, I // 2, dtype=torch.uint8, device=device),
+               w2_sf=torch.empty(E, H, I // 16, dtype=torch.uint8, device=device),
+               w2_g=torch.empty(E, dtype=torch.float32, device=device))
+    if keep_codes:
+        out["w13"] = torch.empty(E, 2 * I, H, dtype=torch.uint8, device=device)
+        out["w2"] = torch.empty(E, H, I, dtype=torch.uint8, device=device)
+    for name, rows, cols in (("w13", 2 * I, H), ("w2", H, I)):
+        for e in range(E):
+            w = torch.randn(rows, cols, generator=g, device=device) / math.sqrt(cols)
+            ge = 448.0 * 6.0 / float(w.abs().max())
+            q, sf = quantize_nvfp4_rows(w, ge)
+            out[name + "_g"][e] = ge
+            out[name + "_sf"][e] = sf.view(torch.uint8)
+            out[name + "_packed"][e] = pack_e2m1(q)
+            if keep_codes:
+                out[name][e] = q
+    base.update(out)
+    base.update(a1_g=NVFP4_A1_GSCALE, a2_g=NVFP4_A2_GSCALE)
+    return base
