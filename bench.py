@@ -584,6 +584,80 @@ def run_nvfp4_gemm(args, cfg):
     return 0
 
 
+def timed_layer(step, args, ws, stream, dev):
+    """Warm-up, then args.steps timed calls of one fused layer with its five
+    stage events: (ms per step, mean stage times [route, quant, gemm1, gemm2,
+    finish] in ms).  Raises on a device status other than MOE_OK."""
+    import fp8_block_scaled_route_b200 as moe
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    for evs in ev:
+        for e in evs:
+            e.record(stream)
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(args.steps):
+        moe.moe_set_stage_events(ev[i])
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    moe.moe_set_stage_events(None)
+    st = moe.moe_get_device_status(ws, stream=stream)
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device status: {moe.moe_status_string(st)}")
+    stages = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(5)] for e in ev]).mean(axis=0)
+    return a.elapsed_time(b) / args.steps, stages
+
+
+def run_nv_moe(args, cfg):
+    """The fused layer in the NVFP4 variant (moe_nvfp4_fused) on a workload:
+    same routing and x as the FP8 layer, NVFP4 weights (per-expert global
+    scales) and the calibrated activation global scales."""
+    import fp8_block_scaled_route_b200 as moe
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    _, bf16, _, src = load_peaks()
+    fp4_peak = bf16 * FP4_OVER_BF16
+    inp = synth.make_nvfp4_moe_inputs(cfg, seed=0, device=dev, keep_codes=False)
+    T, H, I, E, k = cfg.T, cfg.H, cfg.I, cfg.E, cfg.k
+    w13_sf = torch.empty(E * 2 * I, H // 16, dtype=torch.uint8, device=dev)
+    w2_sf = torch.empty(E * H, I // 16, dtype=torch.uint8, device=dev)
+    moe.nvfp4_tile_scales(inp["w13_sf"].view(E * 2 * I, H // 16), w13_sf)
+    moe.nvfp4_tile_scales(inp["w2_sf"].view(E * H, I // 16), w2_sf)
+    del inp["w13_sf"], inp["w2_sf"]
+    a13 = (1.0 / (inp["a1_g"] * inp["w13_g"].double())).float()
+    a2 = (1.0 / (inp["a2_g"] * inp["w2_g"].double())).float()
+    ws = torch.empty(moe.moe_workspace_size(T, H, I, E, k), dtype=torch.uint8, device=dev)
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    counts = work_counts(cfg, inp["topk_ids"])
+    ms, st = timed_layer(lambda: moe.moe_nvfp4_fused(
+        inp["x"], inp["topk_ids"], inp["topk_w"], inp["w13_packed"], w13_sf, a13,
+        inp["w2_packed"], w2_sf, a2, inp["a1_g"], inp["a2_g"], out, ws, stream=stream),
+        args, ws, stream, dev)
+    g1_tf = counts["g1_flops"] / (st[2] * 1e-3) / 1e12
+    line = {"metric": "fused MoE layer, NVFP4 variant: TFLOP/s", "unit": "TFLOP/s",
+            "value": counts["flops"] / (ms * 1e-3) / 1e12, "ms_per_step": ms,
+            "higher_is_better": True, "steps": args.steps, "warmup": args.warmup, "n_gpus": 1,
+            "dtype": "nvfp4 e2m1 + e4m3 per 16 + fp32 global (fp32 accumulate)",
+            "data": "synthetic",
+            "config": {"workload": workload_desc(cfg) + "; NVFP4 weights and activations",
+                       "l2": "inputs larger than L2 (no flush)"},
+            "stages_us": {n: float(v) * 1e3 for n, v in
+                          zip(["route", "quant", "gemm1", "gemm2", "finish"], st)},
+            "roofline": {"bound": "tensor", "achieved": g1_tf, "peak": fp4_peak,
+                         "unit": "TFLOP/s", "frac": g1_tf / fp4_peak, "traffic": None,
+                         "kernel": "NVFP4 GEMM1 (gate/up + SwiGLU + NVFP4 requant)",
+                         "peak_source": f"{src} (FP4 = bf16 burst x {FP4_OVER_BF16:g})"},
+            "gpu_launches": kernels_per_layer(T, k) * args.steps}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_mx_moe(args, cfg):
     """The fused layer in the MXFP8 variant (moe_mxfp8_fused) on a workload:
     same routing and x as the FP8 layer, MXFP8 weights; the FP8 layer with
@@ -605,28 +679,7 @@ def run_mx_moe(args, cfg):
     counts = work_counts(cfg, inp["topk_ids"])
 
     def timed(step):
-        for _ in range(args.warmup):
-            step()
-        torch.cuda.synchronize(dev)
-        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
-        for evs in ev:
-            for e in evs:
-                e.record(stream)
-        torch.cuda.synchronize(dev)
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for i in range(args.steps):
-            moe.moe_set_stage_events(ev[i])
-            step()
-        b.record(stream)
-        torch.cuda.synchronize(dev)
-        moe.moe_set_stage_events(None)
-        st = moe.moe_get_device_status(ws, stream=stream)
-        if st != moe.MOE_OK:
-            raise RuntimeError(f"device status: {moe.moe_status_string(st)}")
-        stages = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(5)] for e in ev]).mean(axis=0)
-        return a.elapsed_time(b) / args.steps, stages
+        return timed_layer(step, args, ws, stream, dev)
 
     ms_mx, st_mx = timed(lambda: moe.moe_mxfp8_fused(
         inp["x"], inp["topk_ids"], inp["topk_w"], inp["w13"], w13_sf, inp["w2"], w2_sf, out, ws,
@@ -668,8 +721,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op", default="moe", choices=["moe", "swiglu_mxfp8", "mxfp8_gemm", "mxfp8_moe",
-                                                     "nvfp4_gemm"],
-                    help="swiglu_mxfp8 / mxfp8_gemm / mxfp8_moe: time that op instead")
+                                                     "nvfp4_gemm", "nvfp4_moe"],
+                    help="any other than moe: time that op instead")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -682,6 +735,8 @@ def main():
         return run_nvfp4_gemm(args, cfg)
     if args.op == "mxfp8_moe":
         return run_mx_moe(args, cfg)
+    if args.op == "nvfp4_moe":
+        return run_nv_moe(args, cfg)
     if args.impl == "reference":
         return run_reference(args, cfg)
     return run_ours(args, cfg)

@@ -25,7 +25,8 @@ __all__ = [
     "moe_get_device_status", "moe_set_wait_timeout_ns", "moe_status_string",
     "moe_set_stage_events", "moe_route_permute_noalloc", "mxfp8_moe_gemm",
     "mxfp8_tile_scales", "moe_mxfp8_fused", "moe_mxfp8_fused_debug", "moe_router_topk",
-    "nvfp4_moe_gemm", "nvfp4_tile_scales",
+    "nvfp4_moe_gemm", "nvfp4_tile_scales", "moe_nvfp4_fused", "moe_nvfp4_fused_debug",
+    "nvfp4_quantize",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -46,7 +47,7 @@ EXPORTS = (
     "swiglu_mxfp8_quant", "moe_get_device_status", "moe_set_wait_timeout_ns",
     "moe_set_stage_events", "moe_route_permute_noalloc", "mxfp8_moe_gemm", "mxfp8_tile_scales",
     "moe_mxfp8_fused", "moe_mxfp8_fused_debug", "moe_router_topk", "nvfp4_moe_gemm",
-    "nvfp4_tile_scales",
+    "nvfp4_tile_scales", "moe_nvfp4_fused", "moe_nvfp4_fused_debug", "nvfp4_quantize",
 )
 
 _lib = None
@@ -100,6 +101,14 @@ def lib():
     L.nvfp4_moe_gemm.argtypes = [P] * 7 + [I] * 5 + [P]
     L.nvfp4_tile_scales.restype = I
     L.nvfp4_tile_scales.argtypes = [P, P, I, I, P]
+    F = ctypes.c_float
+    L.nvfp4_quantize.restype = I
+    L.nvfp4_quantize.argtypes = [P, F, P, P, I, I, P]
+    L.moe_nvfp4_fused.restype = I
+    L.moe_nvfp4_fused.argtypes = [P] * 9 + [F, F, P] + [I] * 5 + [P, ctypes.c_size_t, P]
+    L.moe_nvfp4_fused_debug.restype = I
+    L.moe_nvfp4_fused_debug.argtypes = ([P] * 9 + [F, F, P] + [I] * 5 +
+                                        [P, ctypes.c_size_t, P] + [P] * 4)
     L.moe_mxfp8_fused.restype = I
     L.moe_mxfp8_fused.argtypes = [P] * 8 + [I] * 5 + [P, ctypes.c_size_t, P]
     L.moe_mxfp8_fused_debug.restype = I
@@ -316,6 +325,50 @@ def nvfp4_moe_gemm(a, b, a_sf, b_sf, alpha, m_indptr, out, is_gated=False, *, di
     st = lib().nvfp4_moe_gemm(_ptr(a), _ptr(b), _ptr(a_sf), _ptr(b_sf), _ptr(alpha), _ptr(m_indptr),
                               _ptr(out), R, N, K, E, int(bool(is_gated)), _stream(stream))
     return _check(st, "nvfp4_moe_gemm", check)
+
+
+def nvfp4_quantize(x, gscale, q, sf, *, dims=None, stream=None, check=True) -> int:
+    """x bf16 [M, K] -> q uint8 [M, K/2] packed E2M1, sf uint8 [M, K/16] E4M3.
+    dims = (M, K) when raw addresses are passed."""
+    M, K = dims if dims is not None else x.shape
+    st = lib().nvfp4_quantize(_ptr(x), float(gscale), _ptr(q), _ptr(sf), M, K, _stream(stream))
+    return _check(st, "nvfp4_quantize", check)
+
+
+def _nv_fused_dims(x, topk_ids, w13):
+    T, H = x.shape
+    return T, H, w13.shape[1] // 2, w13.shape[0], topk_ids.shape[1]
+
+
+def moe_nvfp4_fused(x, topk_ids, topk_w, w13, w13_sf, w13_alpha, w2, w2_sf, w2_alpha, a1_gscale,
+                    a2_gscale, out, ws, ws_bytes=None, *, dims=None, stream=None,
+                    check=True) -> int:
+    """w13 / w2 packed E2M1 [E, 2I, H/2] / [E, H, I/2]; w13_sf / w2_sf tiled by
+    nvfp4_tile_scales; *_alpha fp32 [E]; a1_gscale / a2_gscale floats.
+    dims = (T, H, I, E, k) when raw addresses are passed."""
+    T, H, I, E, k = dims if dims is not None else _nv_fused_dims(x, topk_ids, w13)
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size()
+    st = lib().moe_nvfp4_fused(_ptr(x), _ptr(topk_ids), _ptr(topk_w), _ptr(w13), _ptr(w13_sf),
+                               _ptr(w13_alpha), _ptr(w2), _ptr(w2_sf), _ptr(w2_alpha),
+                               float(a1_gscale), float(a2_gscale), _ptr(out), T, H, I, E, k,
+                               _ptr(ws), ws_bytes, _stream(stream))
+    return _check(st, "moe_nvfp4_fused", check)
+
+
+def moe_nvfp4_fused_debug(x, topk_ids, topk_w, w13, w13_sf, w13_alpha, w2, w2_sf, w2_alpha,
+                          a1_gscale, a2_gscale, out, ws, m_indptr=None, perm=None, h_fp4=None,
+                          h_sf=None, ws_bytes=None, *, dims=None, stream=None, check=True) -> int:
+    T, H, I, E, k = dims if dims is not None else _nv_fused_dims(x, topk_ids, w13)
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size()
+    st = lib().moe_nvfp4_fused_debug(_ptr(x), _ptr(topk_ids), _ptr(topk_w), _ptr(w13),
+                                     _ptr(w13_sf), _ptr(w13_alpha), _ptr(w2), _ptr(w2_sf),
+                                     _ptr(w2_alpha), float(a1_gscale), float(a2_gscale),
+                                     _ptr(out), T, H, I, E, k, _ptr(ws), ws_bytes,
+                                     _stream(stream), _ptr(m_indptr), _ptr(perm), _ptr(h_fp4),
+                                     _ptr(h_sf))
+    return _check(st, "moe_nvfp4_fused_debug", check)
 
 
 def nvfp4_tile_scales(sf_rowmajor, sf_tiled, *, dims=None, stream=None, check=True) -> int:

@@ -390,6 +390,121 @@ int moe_mxfp8_fused_debug(const void* x, const int32_t* topk_ids, const float* t
                          ws_bytes, stream, m_indptr, perm, h_fp8, h_sf);
 }
 
+// The fused layer in the NVFP4 variant.  Workspace: the layout of the FP8
+// layer; packed codes and their E4M3 scales (9/16 of the FP8 code bytes) sit
+// in the code regions, codes first.
+static int nv_fused_impl(const void* x, const int32_t* topk_ids, const float* topk_w,
+                         const void* w13, const uint8_t* w13_sf, const float* w13_alpha,
+                         const void* w2, const uint8_t* w2_sf, const float* w2_alpha,
+                         float a1_gscale, float a2_gscale, void* out, int T, int H, int I, int E,
+                         int k, void* ws, size_t ws_bytes, moe_stream_t stream,
+                         int32_t* dbg_m_indptr, int32_t* dbg_perm, uint8_t* dbg_hq,
+                         uint8_t* dbg_hsf) {
+    if (T < 0 || H <= 0 || I <= 0 || H % 256 || I % 256 || k < 1) return MOE_ERR_INVALID_ARG;
+    if (E < 1) return MOE_ERR_INVALID_ARG;
+    if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+    if (k > E) return MOE_ERR_INVALID_ARG;
+    if (!ws) return MOE_ERR_INVALID_ARG;
+    if (!(a1_gscale > 0.0f) || !(a2_gscale > 0.0f)) return MOE_ERR_INVALID_ARG;
+    const FusedWs L = fused_layout(T, H, I, E, k);
+    if (ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+    if (T > 0) {
+        if (!x || !topk_ids || !topk_w || !w13 || !w13_sf || !w13_alpha || !w2 || !w2_sf ||
+            !w2_alpha || !out)
+            return MOE_ERR_INVALID_ARG;
+        if (!aligned16(x) || !aligned16(w13) || !aligned16(w2) || !aligned16(out) ||
+            !aligned16(w13_sf) || !aligned16(w2_sf))
+            return MOE_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(w13_alpha) | reinterpret_cast<uintptr_t>(w2_alpha)) & 3)
+            return MOE_ERR_INVALID_ARG;
+    }
+    const DevInfo* d = dev_info();
+    if (int st = check_device(d)) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    char* b = static_cast<char*>(ws);
+    const size_t R = static_cast<size_t>(T) * k;
+    const size_t xsf_off = L.xq + up256(R * H / 2);
+    const size_t hsf_off = L.hq + up256(R * I / 2);
+    if (xsf_off + R * H / 16 > L.hq || hsf_off + R * I / 16 > L.out_acc) return MOE_ERR_INVALID_ARG;
+    int* status = reinterpret_cast<int*>(b + L.status);
+    int32_t* m_indptr = reinterpret_cast<int32_t*>(b + L.m_indptr);
+    int32_t* perm = reinterpret_cast<int32_t*>(b + L.perm);
+    int32_t* inv_perm = reinterpret_cast<int32_t*>(b + L.inv_perm);
+    uint8_t* xq = reinterpret_cast<uint8_t*>(b + L.xq);
+    uint8_t* xsf = reinterpret_cast<uint8_t*>(b + xsf_off);
+    uint8_t* hq = reinterpret_cast<uint8_t*>(b + L.hq);
+    uint8_t* hsf = reinterpret_cast<uint8_t*>(b + hsf_off);
+    float* out_acc = reinterpret_cast<float*>(b + L.out_acc);
+    if (cudaMemsetAsync(status, 0, sizeof(int) * kStatusInts, s) != cudaSuccess) return MOE_ERR_CUDA;
+    RouteArgs ra{topk_ids, T, k, E, m_indptr, perm, inv_perm,
+                 reinterpret_cast<int32_t*>(b + L.chunk_hist), status};
+    stage_mark(0, s);
+    int st = launch_route_permute(ra, s);
+    if (st) return st;
+    stage_mark(1, s);
+    if (T > 0) {
+        st = launch_nv_quant_scatter(x, T, H, k, a1_gscale, inv_perm, xq, xsf, out_acc, s);
+        if (st) return st;
+        stage_mark(2, s);
+        const unsigned long long tmo = g_timeout_ns.load();
+        NvGemmArgs g1{};
+        g1.a = xq; g1.b = w13; g1.a_sf = xsf; g1.b_sf = w13_sf; g1.alpha = w13_alpha;
+        g1.m_indptr = m_indptr; g1.R = static_cast<int>(R); g1.N = 2 * I; g1.K = H; g1.E = E;
+        g1.gated = 1; g1.epi = NV_EPI_SWIGLU_NVQUANT; g1.hq = hq; g1.hsf = hsf;
+        g1.h_gscale = a2_gscale;
+        g1.status = status; g1.timeout_ns = tmo; g1.num_sms = d->sms;
+        st = launch_nvfp4_gemm(g1, s);
+        if (st) return st;
+        stage_mark(3, s);
+        NvGemmArgs g2{};
+        g2.a = hq; g2.b = w2; g2.a_sf = hsf; g2.b_sf = w2_sf; g2.alpha = w2_alpha;
+        g2.m_indptr = m_indptr; g2.R = static_cast<int>(R); g2.N = H; g2.K = I; g2.E = E;
+        g2.gated = 0; g2.epi = NV_EPI_COMBINE; g2.perm = perm; g2.topk_w = topk_w; g2.topk = k;
+        g2.out_acc = out_acc; g2.out_ld = H;
+        g2.status = status; g2.timeout_ns = tmo; g2.num_sms = d->sms;
+        st = launch_nvfp4_gemm(g2, s);
+        if (st) return st;
+        stage_mark(4, s);
+        st = launch_f32_to_bf16(out_acc, out, static_cast<long long>(T) * H, d->sms, s);
+        if (st) return st;
+        stage_mark(5, s);
+    }
+    if (dbg_m_indptr &&
+        cudaMemcpyAsync(dbg_m_indptr, m_indptr, sizeof(int32_t) * (E + 1), cudaMemcpyDeviceToDevice, s))
+        return MOE_ERR_CUDA;
+    if (R > 0) {
+        if (dbg_perm &&
+            cudaMemcpyAsync(dbg_perm, perm, sizeof(int32_t) * R, cudaMemcpyDeviceToDevice, s))
+            return MOE_ERR_CUDA;
+        if (dbg_hq && cudaMemcpyAsync(dbg_hq, hq, R * I / 2, cudaMemcpyDeviceToDevice, s))
+            return MOE_ERR_CUDA;
+        if (dbg_hsf && cudaMemcpyAsync(dbg_hsf, hsf, R * I / 16, cudaMemcpyDeviceToDevice, s))
+            return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+}
+
+int moe_nvfp4_fused(const void* x, const int32_t* topk_ids, const float* topk_w, const void* w13,
+                    const uint8_t* w13_sf, const float* w13_alpha, const void* w2,
+                    const uint8_t* w2_sf, const float* w2_alpha, float a1_gscale, float a2_gscale,
+                    void* out, int T, int H, int I, int E, int k, void* ws, size_t ws_bytes,
+                    moe_stream_t stream) {
+    return nv_fused_impl(x, topk_ids, topk_w, w13, w13_sf, w13_alpha, w2, w2_sf, w2_alpha,
+                         a1_gscale, a2_gscale, out, T, H, I, E, k, ws, ws_bytes, stream, nullptr,
+                         nullptr, nullptr, nullptr);
+}
+
+int moe_nvfp4_fused_debug(const void* x, const int32_t* topk_ids, const float* topk_w,
+                          const void* w13, const uint8_t* w13_sf, const float* w13_alpha,
+                          const void* w2, const uint8_t* w2_sf, const float* w2_alpha,
+                          float a1_gscale, float a2_gscale, void* out, int T, int H, int I, int E,
+                          int k, void* ws, size_t ws_bytes, moe_stream_t stream, int32_t* m_indptr,
+                          int32_t* perm, uint8_t* h_fp4, uint8_t* h_sf) {
+    return nv_fused_impl(x, topk_ids, topk_w, w13, w13_sf, w13_alpha, w2, w2_sf, w2_alpha,
+                         a1_gscale, a2_gscale, out, T, H, I, E, k, ws, ws_bytes, stream, m_indptr,
+                         perm, h_fp4, h_sf);
+}
+
 int moe_fp8_fused(const void* x, const int32_t* topk_ids, const float* topk_w, const void* w13,
                   const float* w13_scale, const void* w2, const float* w2_scale, void* out, int T,
                   int H, int I, int E, int k, void* ws, size_t ws_bytes, moe_stream_t stream) {
@@ -526,6 +641,19 @@ int nvfp4_moe_gemm(const void* a, const void* b, const uint8_t* a_sf, const uint
     g.timeout_ns = g_timeout_ns.load();
     g.num_sms = d->sms;
     return launch_nvfp4_gemm(g, s);
+}
+
+int nvfp4_quantize(const void* x, float gscale, uint8_t* q, uint8_t* sf, int M, int K,
+                   moe_stream_t stream) {
+    if (M < 0 || K <= 0 || K % 128 || !(gscale > 0.0f)) return MOE_ERR_INVALID_ARG;
+    if (M > 0 && (!x || !q || !sf)) return MOE_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(q) |
+         reinterpret_cast<uintptr_t>(sf)) & 7)
+        return MOE_ERR_INVALID_ARG;
+    const DevInfo* d = dev_info();
+    if (int st = check_device(d)) return st;
+    return launch_nv_quant_scatter(x, M, K, 1, gscale, nullptr, q, sf, nullptr,
+                                   reinterpret_cast<cudaStream_t>(stream));
 }
 
 int nvfp4_tile_scales(const uint8_t* sf_rowmajor, uint8_t* sf_tiled, int rows, int K,

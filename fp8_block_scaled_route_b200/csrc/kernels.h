@@ -121,6 +121,12 @@ int launch_mx_tile_scales(const uint8_t* rm, uint8_t* tiled, int rows, int K, in
 // Grouped NVFP4 GEMM on the block-scaled tensor core path: E2M1 operands
 // packed two per byte, one E4M3 scale per 16 K elements of every row of A and
 // of B, G = alpha[e] * (block-scaled product).
+enum NvEpilogue : int {
+    NV_EPI_BF16 = 0,            // plain bf16 G, or gated bf16 silu(gate) * up
+    NV_EPI_SWIGLU_NVQUANT = 1,  // gated: h to NVFP4 (hq [R, N/4] packed, hsf [R, N/32])
+    NV_EPI_COMBINE = 2,         // plain: out_acc[token, n] += topk_w * G (fp32 reduction)
+};
+
 struct NvGemmArgs {
     const void* a;            // [R, K/2] packed E2M1, grouped rows
     const void* b;            // [E, N, K/2] packed E2M1
@@ -130,11 +136,26 @@ struct NvGemmArgs {
     const int32_t* m_indptr;  // [E+1]
     int R, N, K, E;
     int gated;                // out [R, N/2] = bf16(silu(G_gate) * G_up), else [R, N] = bf16(G)
+    int epi;                  // NvEpilogue
     void* out;
+    uint8_t* hq;
+    uint8_t* hsf;
+    float h_gscale;           // NV_EPI_SWIGLU_NVQUANT: global scale of h
+    const int32_t* perm;
+    const float* topk_w;
+    int topk;
+    float* out_acc;
+    int out_ld;
     int* status;
     uint64_t timeout_ns;
     int num_sms;
 };
 int launch_nvfp4_gemm(const NvGemmArgs& g, cudaStream_t stream);
+
+// NVFP4 variant of launch_quant_scatter: xq [R, H/2] packed E2M1 codes and
+// xsf [R, H/16] E4M3 scales with global scale g, at rows inv_perm[t*k + j]
+// (row t when inv_perm is null and k = 1).
+int launch_nv_quant_scatter(const void* x, int T, int H, int k, float g, const int32_t* inv_perm,
+                            uint8_t* xq, uint8_t* xsf, float* out_acc, cudaStream_t stream);
 
 }  // namespace moe

@@ -26,8 +26,16 @@
 // Warps: 0 TMA producer, 1 MMA issuer (elected lane), 2 weight scale loader,
 // 3 activation scale loader, 4-11 epilogue.  TMEM: accumulator columns
 // [0, 256), A scale factors [256, 272) (4 per step), B scale factors
-// [272, 304) (8 per step: two 128-row blocks).
+// [272, 304) (8 per step: two 128-row blocks).  Epilogues: bf16 G (plain or
+// gated), SwiGLU + NVFP4 requantisation of the intermediate (GEMM1 of the
+// fused layer), top-k weighted fp32 combine (GEMM2; one stage fewer to make
+// room for its transpose buffer).
+//
+// Also here: the NVFP4 quantise-and-scatter of x (the fused layer's first
+// GEMM input), sharing the quantisation step with the requantising epilogue.
 #include <cuda_bf16.h>
+#include <cuda_fp4.h>
+#include <cuda_fp8.h>
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -62,7 +70,42 @@ __host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
            | (static_cast<uint32_t>(M >> 4) << 24);        // M / 16
 }
 
-constexpr int kNvStages = 4;
+// NVFP4 quantisation of 16 values with global scale g (the cuTile page's
+// fp4_quantize with sf_vec_size=16): scale code c = E4M3_RNE_sat(amax * g / 6),
+// codes E2M1_RNE_sat(v * g / e4m3(c)) (all 0 when the scale decodes to 0), in
+// the same fp32 operation order as the format's definition so that each
+// rounding decision is reproducible.  Returns the scale code; codes[i/2]
+// holds element i in its low nibble when i is even.
+__device__ __forceinline__ uint32_t nv_e4m3_scale(float amax, float g, float& s) {
+    const float t = __fdiv_rn(__fmul_rn(amax, g), 6.0f);
+    const __nv_fp8_storage_t c = __nv_cvt_float_to_fp8(t, __NV_SATFINITE, __NV_E4M3);
+    const __half_raw hr = __nv_cvt_fp8_to_halfraw(c, __NV_E4M3);
+    s = __half2float(__half(hr));
+    return static_cast<uint32_t>(c);
+}
+
+__device__ __forceinline__ uint32_t nv_e2m1(float v) {
+    return static_cast<uint32_t>(__nv_cvt_float_to_fp4(v, __NV_E2M1, cudaRoundNearest)) & 0xFu;
+}
+
+// 16 values -> 8 packed bytes (uint2) and the scale code.
+__device__ __forceinline__ uint32_t nv_quant16(const float (&v)[16], float g, uint2& packed) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    float s;
+    const uint32_t c = nv_e4m3_scale(amax, g, s);
+    uint32_t w[2] = {0u, 0u};
+    if (s > 0.0f) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            w[i >> 3] |= nv_e2m1(__fdiv_rn(__fmul_rn(v[i], g), s)) << (4 * (i & 7));
+    }
+    packed = make_uint2(w[0], w[1]);
+    return c;
+}
+
+
 constexpr int kNvEpiWarps = 8;
 constexpr int kNvA = 128 * 128;
 constexpr int kNvB = 256 * 128;
@@ -71,14 +114,23 @@ constexpr int kNvSfBytes = 4 * 512 + 2 * 4 * 512;  // A: 4 atoms, B: 2 blocks x 
 constexpr int kNvStage = kNvA + kNvB + kNvSfBytes;
 constexpr int kNvMaxE = 1024;
 constexpr int kNvTable = ((2 * (kNvMaxE + 1) * 4) + 15) / 16 * 16;
-constexpr int kNvSmem = 1024 + kNvStages * kNvStage + kNvTable + 256;
+constexpr int kNvCst = kNvEpiWarps * 32 * 16 * 4;  // combine: per-warp 32 x 16 fp32 transpose tile
 constexpr int kNvThreads = 384;
 constexpr int kNvBoxes = 6;  // TMA boxes per stage: 2 x 64 token rows, 4 x 64 weight rows
 constexpr uint32_t kNvTmemCols = 512;
 constexpr uint32_t kNvSfaCol = 256;
 constexpr uint32_t kNvSfbCol = 272;
 static_assert(kNvStage % 1024 == 0, "stages must stay 1024-byte aligned for the swizzle");
-static_assert(kNvSmem <= 232448, "shared memory budget");
+
+// Per epilogue: ring depth and shared memory (the combine's transpose buffer
+// costs one stage).
+template <int MODE>
+struct NvCfg {
+    static constexpr int STAGES = MODE == NV_EPI_COMBINE ? 3 : 4;
+    static constexpr int CST = MODE == NV_EPI_COMBINE ? kNvCst : 0;
+    static constexpr int SMEM = 1024 + STAGES * kNvStage + kNvTable + CST + 256;
+    static_assert(SMEM <= 232448, "shared memory budget");
+};
 
 struct NvParams {
     int R, N, K, E, nkb, gated;  // nkb: 256-element K blocks
@@ -86,13 +138,22 @@ struct NvParams {
     const uint8_t* b_sf;         // [E*N/128, K/64, 512] E4M3, tiled
     const float* alpha;          // [E]
     const int32_t* m_indptr;
-    __nv_bfloat16* out;
+    __nv_bfloat16* out;          // NV_EPI_BF16
+    uint8_t* hq;                 // NV_EPI_SWIGLU_NVQUANT: [R, N/4] packed codes of h
+    uint8_t* hsf;                //   and [R, N/32] E4M3 scales
+    float h_gscale;              //   global scale of h
+    const int32_t* perm;         // NV_EPI_COMBINE: out_acc[perm[r] / topk] += topk_w[perm[r]] * G[r]
+    const float* topk_w;
+    int topk;
+    float* out_acc;
+    int out_ld;
     int* status;
     unsigned long long timeout_ns;
 };
 
 struct NvSmem {
     uint8_t* stages;
+    float* cstage;
     int* tstart;  // [E+1] first tile of each expert
     int* mind;    // [E+1] clamped m_indptr
     uint64_t* full;
@@ -104,21 +165,25 @@ struct NvSmem {
     volatile int* abort;
 };
 
+template <int MODE>
 __device__ __forceinline__ NvSmem nv_carve(uint8_t* base) {
+    constexpr int S = NvCfg<MODE>::STAGES;
     NvSmem s;
     s.stages = base;
-    uint8_t* p = base + kNvStages * kNvStage;
+    uint8_t* p = base + S * kNvStage;
     s.tstart = reinterpret_cast<int*>(p);
     s.mind = s.tstart + (kNvMaxE + 1);
     p += kNvTable;
+    s.cstage = reinterpret_cast<float*>(p);
+    p += NvCfg<MODE>::CST;
     uint64_t* bars = reinterpret_cast<uint64_t*>(p);
     s.full = bars;
-    s.empty = bars + kNvStages;
-    s.tfull = bars + 2 * kNvStages;
-    s.tempty = bars + 2 * kNvStages + 1;
-    s.drain = bars + 2 * kNvStages + 2;
-    s.tmem = reinterpret_cast<uint32_t*>(bars + 2 * kNvStages + 3);
-    s.abort = reinterpret_cast<volatile int*>(bars + 2 * kNvStages + 4);
+    s.empty = bars + S;
+    s.tfull = bars + 2 * S;
+    s.tempty = bars + 2 * S + 1;
+    s.drain = bars + 2 * S + 2;
+    s.tmem = reinterpret_cast<uint32_t*>(bars + 2 * S + 3);
+    s.abort = reinterpret_cast<volatile int*>(bars + 2 * S + 4);
     return s;
 }
 
@@ -168,6 +233,7 @@ __device__ __forceinline__ bool nv_warp_wait(uint64_t* bar, uint32_t parity, con
 
 // Warp 0: lane l < 6 issues TMA box l of every stage (x = byte offset of the
 // stage's 256 K elements, a multiple of 128).
+template <int S>
 __device__ void nv_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const NvParams& p,
                             const NvSmem& s, const WaitCtl& wc, int total) {
     const int l = threadIdx.x & 31;
@@ -192,10 +258,10 @@ __device__ void nv_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, cons
             __syncwarp();
             armed |= 1u << stage;
             armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-            if (++stage == kNvStages) { stage = 0; phase ^= 1; }
+            if (++stage == S) { stage = 0; phase ^= 1; }
         }
     }
-    for (int st = 0; st < kNvStages; ++st)
+    for (int st = 0; st < S; ++st)
         if ((armed >> st) & 1u) wait_bar(&s.full[st], (armed_par >> st) & 1u, wc, 2, /*drain=*/true);
     __syncwarp();
 }
@@ -204,7 +270,7 @@ __device__ void nv_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, cons
 // each of the tile's 256 weight rows or 128 token rows, as four 512-byte
 // atoms (one per K = 64 step); completion arrives on the stage's full
 // barrier.  Rows past the ends read as 0 (those outputs are not stored).
-template <bool WEIGHTS>
+template <bool WEIGHTS, int S>
 __device__ void nv_sf_loader(const NvParams& p, const NvSmem& s, const WaitCtl& wc, int total) {
     const int lane = threadIdx.x & 31;
     const int nsf = p.K >> 4;  // activation scale bytes per row
@@ -244,7 +310,7 @@ __device__ void nv_sf_loader(const NvParams& p, const NvSmem& s, const WaitCtl& 
                 }
             }
             cp_async_arrive_noinc(&s.full[stage]);
-            if (++stage == kNvStages) { stage = 0; phase ^= 1; }
+            if (++stage == S) { stage = 0; phase ^= 1; }
         }
     }
     cp_async_wait_all();
@@ -254,6 +320,7 @@ __device__ void nv_sf_loader(const NvParams& p, const NvSmem& s, const WaitCtl& 
 // Warp 1: per stage, the 12 scale-factor atoms into TMEM and four K = 64
 // block-scaled MMAs (elected lane); the accumulator is released by the
 // epilogue per tile.
+template <int S>
 __device__ void nv_mma(const NvParams& p, const NvSmem& s, const WaitCtl& wc, uint32_t tmem_base,
                        int total) {
     uint32_t stage = 0, phase = 0, it = 0;
@@ -288,7 +355,7 @@ __device__ void nv_mma(const NvParams& p, const NvSmem& s, const WaitCtl& wc, ui
                 if (kb == p.nkb - 1) umma_commit(s.tfull);
             }
             __syncwarp();
-            if (++stage == kNvStages) { stage = 0; phase ^= 1; }
+            if (++stage == S) { stage = 0; phase ^= 1; }
         }
     }
     if (elect_one()) umma_commit(s.drain);
@@ -308,7 +375,14 @@ __device__ __forceinline__ uint32_t nv_pack_bf16(float a, float b) {
 
 // Warps 4-11: thread = one row of the tile, 64 columns of each weight block
 // (warp w: rows 32 (w % 4) .. +31, column half (w - 4) / 4).  G = alpha_e *
-// accumulator; bf16 G (plain) or bf16 silu(G_gate) * G_up (gated).
+// accumulator; then, by mode:
+//  NV_EPI_BF16            bf16 G (plain) or bf16 silu(G_gate) * G_up (gated)
+//  NV_EPI_SWIGLU_NVQUANT  h = silu(G_gate) * G_up requantised to NVFP4 with
+//                         the global scale h_gscale: the thread's 64 columns
+//                         are four 16-column blocks, each with its own scale
+//  NV_EPI_COMBINE         out_acc[token] += w * G through a shared-memory
+//                         transpose (8 rows x 64 contiguous bytes per reduction)
+template <int MODE>
 __device__ void nv_epilogue(const NvParams& p, const NvSmem& s, const WaitCtl& wc,
                             uint32_t tmem_base, int total) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -324,6 +398,16 @@ __device__ void nv_epilogue(const NvParams& p, const NvSmem& s, const WaitCtl& w
         const bool row_ok = rl < tl.rows;
         const long long row = tl.row0 + rl;
         const float al = __ldg(p.alpha + tl.e);
+        // combine: the row's pair id and weight, fetched while the tile computes
+        int c_tok = -1;
+        float c_w = 0.0f;
+        if constexpr (MODE == NV_EPI_COMBINE) {
+            if (row_ok) {
+                const int pair = __ldg(p.perm + row);
+                c_tok = pair / p.topk;
+                c_w = __ldg(p.topk_w + pair) * al;
+            }
+        }
         if (!nv_warp_wait(s.tfull, it & 1, wc, 6)) return;
         tc_fence_after();
         tmem_ld32_async(tl_addr, v[0]);
@@ -337,8 +421,64 @@ __device__ void nv_epilogue(const NvParams& p, const NvSmem& s, const WaitCtl& w
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(s.tempty);
+        if constexpr (MODE == NV_EPI_COMBINE) {
+            float* stg = s.cstage + (warp - 4) * 512;
+            const int rr = lane >> 2, cc = lane & 3;
+            float* const obase = p.out_acc + tl.nt * 256 + colg;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                if (tl.nt * 256 + half * 128 >= p.N) break;
+#pragma unroll
+                for (int c16 = 0; c16 < 4; ++c16) {
+                    const uint32_t* a = v[2 * half + (c16 >> 1)] + (c16 & 1) * 16;
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const int slot = (lane & 1) * 4 + ((q4 + (lane >> 1)) & 3);
+                        *reinterpret_cast<float4*>(stg + (lane >> 1) * 32 + slot * 4) =
+                            make_float4(c_w * __uint_as_float(a[4 * q4]),
+                                        c_w * __uint_as_float(a[4 * q4 + 1]),
+                                        c_w * __uint_as_float(a[4 * q4 + 2]),
+                                        c_w * __uint_as_float(a[4 * q4 + 3]));
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int rg = 0; rg < 4; ++rg) {
+                        const int r = rg * 8 + rr;
+                        const int slot = (r & 1) * 4 + ((cc + (r >> 1)) & 3);
+                        const float4 x4 = *reinterpret_cast<const float4*>(stg + (r >> 1) * 32 + slot * 4);
+                        const int t_r = __shfl_sync(0xffffffffu, c_tok, r);
+                        if (t_r >= 0)
+                            red_add_v4(obase + static_cast<long long>(t_r) * p.out_ld + half * 128 +
+                                           c16 * 16 + cc * 4,
+                                       x4.x, x4.y, x4.z, x4.w);
+                    }
+                    __syncwarp();
+                }
+            }
+            continue;
+        }
         if (!row_ok) continue;
-        if (p.gated) {
+        if constexpr (MODE == NV_EPI_SWIGLU_NVQUANT) {
+            const int I = p.N >> 1;
+            const long long col0 = static_cast<long long>(tl.nt) * 128 + colg;  // first h column
+            uint2 packed[4];
+            uint32_t sf4 = 0;
+#pragma unroll
+            for (int b16 = 0; b16 < 4; ++b16) {
+                float h[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int j = 16 * b16 + i;
+                    h[i] = nv_silu(al * __uint_as_float(v[j >> 5][j & 31])) *
+                           (al * __uint_as_float(v[2 + (j >> 5)][j & 31]));
+                }
+                sf4 |= nv_quant16(h, p.h_gscale, packed[b16]) << (8 * b16);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(p.hq + row * (I >> 1) + (col0 >> 1));
+            dst[0] = make_uint4(packed[0].x, packed[0].y, packed[1].x, packed[1].y);
+            dst[1] = make_uint4(packed[2].x, packed[2].y, packed[3].x, packed[3].y);
+            *reinterpret_cast<uint32_t*>(p.hsf + row * (I >> 4) + (col0 >> 4)) = sf4;
+        } else if (p.gated) {
             uint4* dst = reinterpret_cast<uint4*>(p.out + row * (p.N >> 1) + tl.nt * 128 + colg);
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
@@ -373,16 +513,18 @@ __device__ void nv_epilogue(const NvParams& p, const NvSmem& s, const WaitCtl& w
     }
 }
 
+template <int MODE>
 __global__ void __launch_bounds__(kNvThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const NvParams p) {
+    constexpr int S = NvCfg<MODE>::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    const NvSmem s = nv_carve(base);
+    const NvSmem s = nv_carve<MODE>(base);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kNvStages; ++i) {
+        for (int i = 0; i < S; ++i) {
             mbar_init(&s.full[i], kNvBoxes + 64);  // TMA lanes + two scale-loader warps
             mbar_init(&s.empty[i], 1);
         }
@@ -435,15 +577,83 @@ __global__ void __launch_bounds__(kNvThreads, 1)
     const uint32_t tmem_base = *s.tmem;
     const WaitCtl wc{s.abort, p.status, p.timeout_ns};
     const int total = s.tstart[p.E];
-    if (warp == 0) nv_producer(&tmA, &tmB, p, s, wc, total);
-    else if (warp == 1) nv_mma(p, s, wc, tmem_base, total);
-    else if (warp == 2) nv_sf_loader<true>(p, s, wc, total);
-    else if (warp == 3) nv_sf_loader<false>(p, s, wc, total);
-    else nv_epilogue(p, s, wc, tmem_base, total);
+    if (warp == 0) nv_producer<S>(&tmA, &tmB, p, s, wc, total);
+    else if (warp == 1) nv_mma<S>(p, s, wc, tmem_base, total);
+    else if (warp == 2) nv_sf_loader<true, S>(p, s, wc, total);
+    else if (warp == 3) nv_sf_loader<false, S>(p, s, wc, total);
+    else nv_epilogue<MODE>(p, s, wc, tmem_base, total);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem_base, kNvTmemCols);
+}
+
+// x [T, H] bf16 -> NVFP4 codes xq [R, H/2] and scales xsf [R, H/16] at rows
+// inv_perm[t*k + j] (row t when inv_perm is null and k = 1; global scale g);
+// also zeroes out_acc [T, H] when not null.  Warp per (token, 128-column
+// block); lane quad = one 16-column block, lane = 4 columns.
+__global__ void __launch_bounds__(256) nv_quant_scatter_kernel(
+    const __nv_bfloat16* __restrict__ x, int T, int H, int k, float g,
+    const int32_t* __restrict__ inv_perm, uint8_t* __restrict__ xq, uint8_t* __restrict__ xsf,
+    float* __restrict__ out_acc) {
+    const int nkb = H >> 7;
+    const long long item = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    if (item >= static_cast<long long>(T) * nkb) return;
+    const int lane = threadIdx.x & 31;
+    const int t = static_cast<int>(item / nkb);
+    const int kb = static_cast<int>(item - static_cast<long long>(t) * nkb);
+    const long long off = static_cast<long long>(t) * H + kb * 128 + lane * 4;
+    uint2 raw = *reinterpret_cast<const uint2*>(x + off);
+    __nv_bfloat162 b01, b23;
+    memcpy(&b01, &raw.x, 4);
+    memcpy(&b23, &raw.y, 4);
+    const float2 f01 = __bfloat1622float2(b01);
+    const float2 f23 = __bfloat1622float2(b23);
+    float amax = fmaxf(fmaxf(fabsf(f01.x), fabsf(f01.y)), fmaxf(fabsf(f23.x), fabsf(f23.y)));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    float sc;
+    const uint32_t code = nv_e4m3_scale(amax, g, sc);
+    uint32_t codes = 0;
+    if (sc > 0.0f) {
+        codes = nv_e2m1(__fdiv_rn(__fmul_rn(f01.x, g), sc)) |
+                (nv_e2m1(__fdiv_rn(__fmul_rn(f01.y, g), sc)) << 4) |
+                (nv_e2m1(__fdiv_rn(__fmul_rn(f23.x, g), sc)) << 8) |
+                (nv_e2m1(__fdiv_rn(__fmul_rn(f23.y, g), sc)) << 12);
+    }
+    // the eight block scales of this 128-column block, one byte each
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        lo |= __shfl_sync(0xffffffffu, code, 4 * b) << (8 * b);
+        hi |= __shfl_sync(0xffffffffu, code, 16 + 4 * b) << (8 * b);
+    }
+    for (int j = 0; j < k; ++j) {
+        const int row = inv_perm ? inv_perm[t * k + j] : t;
+        if (row < 0) continue;
+        *reinterpret_cast<uint16_t*>(xq + static_cast<long long>(row) * (H >> 1) + kb * 64 + lane * 2) =
+            static_cast<uint16_t>(codes);
+        if (lane == 0)
+            *reinterpret_cast<uint2*>(xsf + static_cast<long long>(row) * (H >> 4) + kb * 8) =
+                make_uint2(lo, hi);
+    }
+    if (out_acc) *reinterpret_cast<float4*>(out_acc + off) = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+template <int MODE>
+int launch_nv_inst(const CUtensorMap& ma, const CUtensorMap& mb, const NvParams& p, int num_sms,
+                   cudaStream_t stream) {
+    static int configured_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+        if (cudaFuncSetAttribute(nvfp4_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 NvCfg<MODE>::SMEM) != cudaSuccess)
+            return ST_CUDA;
+        configured_dev = dev;
+    }
+    nvfp4_gemm_kernel<MODE><<<num_sms, kNvThreads, NvCfg<MODE>::SMEM, stream>>>(ma, mb, p);
+    return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
 }
 
 }  // namespace
@@ -459,18 +669,28 @@ int launch_nvfp4_gemm(const NvGemmArgs& g, cudaStream_t stream) {
     p.R = g.R; p.N = g.N; p.K = g.K; p.E = g.E; p.nkb = g.K / 256; p.gated = g.gated ? 1 : 0;
     p.a_sf = g.a_sf; p.b_sf = g.b_sf; p.alpha = g.alpha; p.m_indptr = g.m_indptr;
     p.out = static_cast<__nv_bfloat16*>(g.out);
+    p.hq = g.hq; p.hsf = g.hsf; p.h_gscale = g.h_gscale;
+    p.perm = g.perm; p.topk_w = g.topk_w; p.topk = g.topk > 0 ? g.topk : 1;
+    p.out_acc = g.out_acc; p.out_ld = g.out_ld;
     p.status = g.status;
     p.timeout_ns = g.timeout_ns;
-    static int configured_dev = -1;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured_dev != dev) {
-        if (cudaFuncSetAttribute(nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kNvSmem) != cudaSuccess)
-            return ST_CUDA;
-        configured_dev = dev;
+    switch (g.epi) {
+        case NV_EPI_SWIGLU_NVQUANT:
+            return launch_nv_inst<NV_EPI_SWIGLU_NVQUANT>(ma, mb, p, g.num_sms, stream);
+        case NV_EPI_COMBINE:
+            return launch_nv_inst<NV_EPI_COMBINE>(ma, mb, p, g.num_sms, stream);
+        default:
+            return launch_nv_inst<NV_EPI_BF16>(ma, mb, p, g.num_sms, stream);
     }
-    nvfp4_gemm_kernel<<<g.num_sms, kNvThreads, kNvSmem, stream>>>(ma, mb, p);
+}
+
+int launch_nv_quant_scatter(const void* x, int T, int H, int k, float g, const int32_t* inv_perm,
+                            uint8_t* xq, uint8_t* xsf, float* out_acc, cudaStream_t stream) {
+    const long long items = static_cast<long long>(T) * (H / 128);
+    if (items == 0) return ST_OK;
+    const long long blocks = (items + 7) / 8;
+    nv_quant_scatter_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(x), T, H, k, g, inv_perm, xq, xsf, out_acc);
     return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
 }
 

@@ -309,6 +309,55 @@ MOE_API int nvfp4_moe_gemm(const void* a, const void* b, const uint8_t* a_sf,
                            void* out, int R, int N, int K, int E, int is_gated,
                            moe_stream_t stream);
 
+/* The fused layer of moe_fp8_fused in the NVFP4 (W4A4) variant of the cuTile
+ * page ("2. cuTile NVFP4 양자화 지원"): activations and weights in NVFP4 (E2M1,
+ * an E4M3 scale per 16 elements, a global scale per tensor).  Stages: routing,
+ * x quantised per token per 16 columns with the global scale a1_gscale and
+ * scattered into the k grouped rows, GEMM1 gate/up on the block-scaled tensor
+ * cores with SwiGLU (fp32) and NVFP4 requantisation of the intermediate
+ * (global scale a2_gscale) in its epilogue, GEMM2 down with the top-k
+ * weighted fp32 combine in its epilogue, bf16 output.
+ *  w13       device uint8 [E, 2I, H/2] packed E2M1 (gate rows then up rows)
+ *  w13_sf    device uint8 E4M3 scales of w13 ([E*2I, H/16] row-major) tiled
+ *            by nvfp4_tile_scales (16-byte aligned)
+ *  w13_alpha device fp32 [E] = 1 / (a1_gscale * global scale of w13[e])
+ *  w2, w2_sf, w2_alpha: the same for the down weights [E, H, I/2], with
+ *            w2_alpha[e] = 1 / (a2_gscale * global scale of w2[e])
+ *  a1_gscale, a2_gscale  host fp32 > 0: global scales of x and of the
+ *            intermediate (calibrated; values beyond 6 * 448 / g saturate)
+ *  x, topk_ids, topk_w, out, T, E, k, ws, ws_bytes, stream: as for
+ *  moe_fp8_fused; the workspace size is moe_workspace_size(T, H, I, E, k).
+ * H and I must be multiples of 256.  Errors as for moe_fp8_fused. */
+MOE_API int moe_nvfp4_fused(const void* x, const int32_t* topk_ids, const float* topk_w,
+                            const void* w13, const uint8_t* w13_sf, const float* w13_alpha,
+                            const void* w2, const uint8_t* w2_sf, const float* w2_alpha,
+                            float a1_gscale, float a2_gscale, void* out, int T, int H, int I,
+                            int E, int k, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_nvfp4_fused plus copies of m_indptr [E+1], perm [T*k], the packed
+ * NVFP4 intermediate h_fp4 [T*k, I/2] and its E4M3 scales h_sf [T*k, I/16]
+ * (any may be NULL). */
+MOE_API int moe_nvfp4_fused_debug(const void* x, const int32_t* topk_ids, const float* topk_w,
+                                  const void* w13, const uint8_t* w13_sf, const float* w13_alpha,
+                                  const void* w2, const uint8_t* w2_sf, const float* w2_alpha,
+                                  float a1_gscale, float a2_gscale, void* out, int T, int H, int I,
+                                  int E, int k, void* ws, size_t ws_bytes, moe_stream_t stream,
+                                  int32_t* m_indptr, int32_t* perm, uint8_t* h_fp4,
+                                  uint8_t* h_sf);
+
+/* NVFP4 quantisation of bf16 rows, as the cuTile page's fp4_quantize(x,
+ * global_scale, sf_vec_size=16, is_sf_swizzled_layout=False): per 16
+ * consecutive values of a row, scale code c = E4M3_RNE_sat(amax * g / 6) and
+ * codes E2M1_RNE_sat(v * g / e4m3(c)) (0 where the scale decodes to 0), each
+ * step rounded in fp32 in that order.
+ *  x   device bf16 [M, K]
+ *  q   device uint8 [M, K/2] packed codes (element 2i in the low nibble)
+ *  sf  device uint8 [M, K/16] E4M3 scale codes, row-major
+ * K must be a multiple of 128, gscale > 0; pointers 8-byte aligned.
+ * Asynchronous on `stream`. */
+MOE_API int nvfp4_quantize(const void* x, float gscale, uint8_t* q, uint8_t* sf, int M, int K,
+                           moe_stream_t stream);
+
 /* Rearranges row-major E4M3 block scales [rows, K/16] into the tiled layout
  * that nvfp4_moe_gemm reads for the weights: [rows/128, K/64, 512] bytes,
  * where byte (r % 32) * 16 + ((r / 32) % 4) * 4 + j of block (r / 128, kb)
