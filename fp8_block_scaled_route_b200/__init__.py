@@ -26,7 +26,8 @@ __all__ = [
     "moe_set_stage_events", "moe_route_permute_noalloc", "mxfp8_moe_gemm",
     "mxfp8_tile_scales", "moe_mxfp8_fused", "moe_mxfp8_fused_debug", "moe_router_topk",
     "nvfp4_moe_gemm", "nvfp4_tile_scales", "moe_nvfp4_fused", "moe_nvfp4_fused_debug",
-    "nvfp4_quantize",
+    "nvfp4_quantize", "moe_tactic_tune_gemm", "moe_tactic_lookup", "moe_tactic_store",
+    "moe_tactic_clear",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -48,6 +49,7 @@ EXPORTS = (
     "moe_set_stage_events", "moe_route_permute_noalloc", "mxfp8_moe_gemm", "mxfp8_tile_scales",
     "moe_mxfp8_fused", "moe_mxfp8_fused_debug", "moe_router_topk", "nvfp4_moe_gemm",
     "nvfp4_tile_scales", "moe_nvfp4_fused", "moe_nvfp4_fused_debug", "nvfp4_quantize",
+    "moe_tactic_tune_gemm", "moe_tactic_lookup", "moe_tactic_store", "moe_tactic_clear",
 )
 
 _lib = None
@@ -102,6 +104,14 @@ def lib():
     L.nvfp4_tile_scales.restype = I
     L.nvfp4_tile_scales.argtypes = [P, P, I, I, P]
     F = ctypes.c_float
+    L.moe_tactic_tune_gemm.restype = I
+    L.moe_tactic_tune_gemm.argtypes = [P] * 6 + [I] * 7 + [P, ctypes.POINTER(I)]
+    L.moe_tactic_lookup.restype = I
+    L.moe_tactic_lookup.argtypes = [I] * 5 + [ctypes.POINTER(I)]
+    L.moe_tactic_store.restype = I
+    L.moe_tactic_store.argtypes = [I] * 6
+    L.moe_tactic_clear.restype = None
+    L.moe_tactic_clear.argtypes = []
     L.nvfp4_quantize.restype = I
     L.nvfp4_quantize.argtypes = [P, F, P, P, I, I, P]
     L.moe_nvfp4_fused.restype = I
@@ -325,6 +335,45 @@ def nvfp4_moe_gemm(a, b, a_sf, b_sf, alpha, m_indptr, out, is_gated=False, *, di
     st = lib().nvfp4_moe_gemm(_ptr(a), _ptr(b), _ptr(a_sf), _ptr(b_sf), _ptr(alpha), _ptr(m_indptr),
                               _ptr(out), R, N, K, E, int(bool(is_gated)), _stream(stream))
     return _check(st, "nvfp4_moe_gemm", check)
+
+
+def moe_tactic_tune_gemm(a, b, a_scale, b_scale, m_indptr, out, scale_major="K",
+                         is_gated=False, iters=5, *, dims=None, stream=None) -> int:
+    """Times fp8_groupwise_moe_gemm at every tile_m valid for K on these
+    buffers (out is overwritten), stores the fastest in the tactic table and
+    returns it.  dims = (R, N, K, E) when raw addresses are passed."""
+    if dims is None:
+        R, K = a.shape
+        E, N, _ = b.shape
+    else:
+        R, N, K, E = dims
+    mode = {"K": 0, "MN": 1}.get(scale_major, scale_major)
+    tm = ctypes.c_int(0)
+    st = lib().moe_tactic_tune_gemm(_ptr(a), _ptr(b), _ptr(a_scale), _ptr(b_scale), _ptr(m_indptr),
+                                    _ptr(out), R, N, K, E, mode, int(bool(is_gated)), int(iters),
+                                    _stream(stream), ctypes.byref(tm))
+    _check(st, "moe_tactic_tune_gemm", True)
+    return tm.value
+
+
+def moe_tactic_lookup(R, N, K, E, is_gated=False):
+    """Stored tile_m of the shape class, or None (host only)."""
+    tm = ctypes.c_int(0)
+    st = lib().moe_tactic_lookup(R, N, K, E, int(bool(is_gated)), ctypes.byref(tm))
+    if st == MOE_ERR_NO_TILE_CONFIG:
+        return None
+    _check(st, "moe_tactic_lookup", True)
+    return tm.value
+
+
+def moe_tactic_store(R, N, K, E, is_gated, tile_m, *, check=True) -> int:
+    """Sets the shape class's tile_m (host only)."""
+    return _check(lib().moe_tactic_store(R, N, K, E, int(bool(is_gated)), tile_m),
+                  "moe_tactic_store", check)
+
+
+def moe_tactic_clear() -> None:
+    lib().moe_tactic_clear()
 
 
 def nvfp4_quantize(x, gscale, q, sf, *, dims=None, stream=None, check=True) -> int:

@@ -8,6 +8,8 @@
 #include <cstdint>
 #include <cstdio>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "moefp8.h"
 #include "common.cuh"
@@ -120,6 +122,54 @@ void select_tile(int total_rows, int n, int k, int E, int num_sms, int gated, in
     if (k <= 2048) { *tm = max_m < 192 ? 64 : 128; return; }
     auto cost = [&](int t) { return ceil_div(tiles(t), num_sms) * (t + kTileOverheadRows); };
     *tm = cost(64) < cost(128) ? 64 : 128;
+}
+
+// --- tactic table: measured tile choice per GEMM shape class ---------------
+// The cuTile page tunes each GEMM of the pair per architecture and shape
+// ("2. cuTile NVFP4 양자화 지원"); here a process-wide table maps a shape class
+// to the token tile that timed fastest on this GPU (moe_tactic_tune_gemm).
+// Class: (N, K, E, gated, bucket of ceil(R / E)), the bucket being the power
+// of two at or above the balanced rows per expert (8 or fewer -> 0).
+struct TacticKey {
+    int n, k, e, gated, bucket;
+    bool operator==(const TacticKey& o) const {
+        return n == o.n && k == o.k && e == o.e && gated == o.gated && bucket == o.bucket;
+    }
+};
+
+int rows_bucket(long long R, int E) {
+    const long long m = (R + E - 1) / E;
+    int b = 0;
+    for (long long v = 8; v < m && b < 24; v <<= 1) ++b;
+    return b;
+}
+
+std::mutex g_tactic_mu;
+std::vector<std::pair<TacticKey, int>> g_tactics;
+
+bool tactic_lookup(const TacticKey& key, int* tm) {
+    std::lock_guard<std::mutex> lk(g_tactic_mu);
+    for (const auto& kv : g_tactics)
+        if (kv.first == key) { *tm = kv.second; return true; }
+    return false;
+}
+
+void tactic_store(const TacticKey& key, int tm) {
+    std::lock_guard<std::mutex> lk(g_tactic_mu);
+    for (auto& kv : g_tactics)
+        if (kv.first == key) { kv.second = tm; return; }
+    g_tactics.emplace_back(key, tm);
+}
+
+bool valid_tile_m(int tm) { return tm == 16 || tm == 32 || tm == 64 || tm == 128; }
+
+// tile_m for a GEMM launched with tile_m = -1: the tuned entry of its shape
+// class when there is one, else the wave + residue model.
+int choose_tile_m(int R, int N, int K, int E, int gated, int num_sms) {
+    int tm, tn;
+    if (!tactic_lookup(TacticKey{N, K, E, gated ? 1 : 0, rows_bucket(R, E)}, &tm))
+        select_tile(R, N, K, E, num_sms, gated ? 1 : 0, &tm, &tn);
+    return tm;
 }
 
 // Token tiles of the swapped kernels stage K/128 x tile_m scales on chip.
@@ -245,9 +295,8 @@ static int fused_impl(const void* x, const int32_t* topk_ids, const float* topk_
         if (st) return st;
         stage_mark(2, s);
         const unsigned long long tmo = g_timeout_ns.load();
-        int tm1, tn1, tm2, tn2;
-        select_tile(R, 2 * I, H, E, d->sms, 1, &tm1, &tn1);
-        select_tile(R, H, I, E, d->sms, 0, &tm2, &tn2);
+        int tm1 = choose_tile_m(R, 2 * I, H, E, 1, d->sms);
+        int tm2 = choose_tile_m(R, H, I, E, 0, d->sms);
         tm1 = fit_tile_to_k(tm1, H);
         tm2 = fit_tile_to_k(tm2, I);
         GemmArgs g1{};
@@ -543,8 +592,8 @@ int fp8_groupwise_moe_gemm(const void* a, const void* b, const float* a_scale, c
     if (cudaMemsetAsync(d->lib_status, 0, sizeof(int) * kStatusInts, s) != cudaSuccess)
         return MOE_ERR_CUDA;
     if (R == 0) return MOE_OK;
-    int tm = tile_m, tn = want_tn;
-    if (tm == -1) select_tile(R, N, K, E, d->sms, is_gated ? 1 : 0, &tm, &tn);
+    int tm = tile_m;
+    if (tm == -1) tm = choose_tile_m(R, N, K, E, is_gated, d->sms);
     if (tm < 128 && K > swap_max_k(tm)) {
         if (tile_m != -1) return MOE_ERR_NO_TILE_CONFIG;
         tm = fit_tile_to_k(tm, K);
@@ -562,6 +611,68 @@ int fp8_groupwise_moe_gemm(const void* a, const void* b, const float* a_scale, c
     g.timeout_ns = g_timeout_ns.load();
     g.num_sms = d->sms;
     return launch_grouped_gemm(g, s);
+}
+
+int moe_tactic_tune_gemm(const void* a, const void* b, const float* a_scale, const float* b_scale,
+                         const int32_t* m_indptr, void* out, int R, int N, int K, int E,
+                         int scale_major_mode, int is_gated, int iters, moe_stream_t stream,
+                         int* tile_m) {
+    if (!tile_m || iters < 1 || R <= 0 || E < 1) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaEvent_t ev[2];
+    if (cudaEventCreate(&ev[0]) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaEventCreate(&ev[1]) != cudaSuccess) {
+        cudaEventDestroy(ev[0]);
+        return MOE_ERR_CUDA;
+    }
+    int best = -1, st = MOE_OK;
+    float best_ms = 0.0f;
+    for (int tm : {16, 32, 64, 128}) {
+        if (tm < 128 && K > swap_max_k(tm)) continue;
+        auto run = [&]() {
+            return fp8_groupwise_moe_gemm(a, b, a_scale, b_scale, m_indptr, out, R, N, K, E,
+                                          scale_major_mode, 1, 128, 128, is_gated, tm, -1, stream);
+        };
+        if ((st = run()) != MOE_OK) break;  // warm-up
+        if (cudaEventRecord(ev[0], s) != cudaSuccess) { st = MOE_ERR_CUDA; break; }
+        for (int i = 0; i < iters && st == MOE_OK; ++i) st = run();
+        if (st != MOE_OK) break;
+        float ms = 0.0f;
+        if (cudaEventRecord(ev[1], s) != cudaSuccess || cudaEventSynchronize(ev[1]) != cudaSuccess ||
+            cudaEventElapsedTime(&ms, ev[0], ev[1]) != cudaSuccess) {
+            st = MOE_ERR_CUDA;
+            break;
+        }
+        if ((st = moe_get_device_status(nullptr, stream)) != MOE_OK) break;
+        if (best < 0 || ms < best_ms) { best = tm; best_ms = ms; }
+    }
+    cudaEventDestroy(ev[0]);
+    cudaEventDestroy(ev[1]);
+    if (st != MOE_OK) return st;
+    if (best < 0) return MOE_ERR_NO_TILE_CONFIG;
+    tactic_store(TacticKey{N, K, E, is_gated ? 1 : 0, rows_bucket(R, E)}, best);
+    *tile_m = best;
+    return MOE_OK;
+}
+
+int moe_tactic_lookup(int R, int N, int K, int E, int is_gated, int* tile_m) {
+    if (!tile_m || R < 0 || N <= 0 || K <= 0 || E < 1) return MOE_ERR_INVALID_ARG;
+    return tactic_lookup(TacticKey{N, K, E, is_gated ? 1 : 0, rows_bucket(R, E)}, tile_m)
+               ? MOE_OK
+               : MOE_ERR_NO_TILE_CONFIG;
+}
+
+int moe_tactic_store(int R, int N, int K, int E, int is_gated, int tile_m) {
+    if (R < 0 || N <= 0 || K <= 0 || E < 1) return MOE_ERR_INVALID_ARG;
+    if (!valid_tile_m(tile_m) || (tile_m < 128 && K > swap_max_k(tile_m)))
+        return MOE_ERR_NO_TILE_CONFIG;
+    tactic_store(TacticKey{N, K, E, is_gated ? 1 : 0, rows_bucket(R, E)}, tile_m);
+    return MOE_OK;
+}
+
+void moe_tactic_clear(void) {
+    std::lock_guard<std::mutex> lk(g_tactic_mu);
+    g_tactics.clear();
 }
 
 int moe_router_topk(const float* logits, int T, int E, int k, int32_t* topk_ids, float* topk_w,

@@ -201,6 +201,39 @@ MOE_API int moe_select_tile_m(int total_rows, int n, int k, int E, int num_sms, 
                       int* tile_m, int* tile_n);
 
 /* ------------------------------------------------------------------ */
+/* Tactic table (measured tile choice)                                  */
+/* ------------------------------------------------------------------ */
+
+/* The staged GEMM-pair autotuning of the cuTile page ("2. cuTile NVFP4 양자화
+ * 지원": each GEMM of the pair tuned per architecture and shape): a
+ * process-wide table maps a GEMM shape class to the token tile (tile_m) that
+ * ran fastest on this GPU.  Class = (N, K, E, is_gated, bucket of ceil(R/E)),
+ * the bucket being the power of two at or above the balanced rows per expert
+ * (8 or fewer share one bucket).  fp8_groupwise_moe_gemm with tile_m = -1 and
+ * both GEMMs of moe_fp8_fused use the class's entry when it exists, else the
+ * wave + residue model of moe_select_tile_m.
+ *
+ * moe_tactic_tune_gemm: runs fp8_groupwise_moe_gemm on the caller's buffers
+ * (arguments as there; `out` is overwritten) once per tile_m valid for K
+ * (16, 32, 64, 128), one warm-up call and `iters` timed calls each (CUDA
+ * events on `stream`; synchronises it), stores the fastest in the table and
+ * writes it to *tile_m.  Errors of the GEMM are returned unchanged; nothing
+ * is stored then.
+ * moe_tactic_lookup: host only; MOE_OK and *tile_m for a stored class, else
+ * MOE_ERR_NO_TILE_CONFIG.
+ * moe_tactic_store: host only; sets a class's entry (e.g. restored from a
+ * file); MOE_ERR_NO_TILE_CONFIG for a tile_m that is not 16/32/64/128 or that
+ * cannot hold K.
+ * moe_tactic_clear: host only; empties the table. */
+MOE_API int moe_tactic_tune_gemm(const void* a, const void* b, const float* a_scale,
+                                 const float* b_scale, const int32_t* m_indptr, void* out, int R,
+                                 int N, int K, int E, int scale_major_mode, int is_gated, int iters,
+                                 moe_stream_t stream, int* tile_m);
+MOE_API int moe_tactic_lookup(int R, int N, int K, int E, int is_gated, int* tile_m);
+MOE_API int moe_tactic_store(int R, int N, int K, int E, int is_gated, int tile_m);
+MOE_API void moe_tactic_clear(void);
+
+/* ------------------------------------------------------------------ */
 /* Grouped MXFP8 GEMM (block-scaled tensor core path)                   */
 /* ------------------------------------------------------------------ */
 
