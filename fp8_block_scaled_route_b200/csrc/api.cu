@@ -758,9 +758,7 @@ int nvfp4_quantize(const void* x, float gscale, uint8_t* q, uint8_t* sf, int M, 
                    moe_stream_t stream) {
     if (M < 0 || K <= 0 || K % 128 || !(gscale > 0.0f)) return MOE_ERR_INVALID_ARG;
     if (M > 0 && (!x || !q || !sf)) return MOE_ERR_INVALID_ARG;
-    if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(q) |
-         reinterpret_cast<uintptr_t>(sf)) & 7)
-        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || (reinterpret_cast<uintptr_t>(q) & 7)) return MOE_ERR_INVALID_ARG;
     const DevInfo* d = dev_info();
     if (int st = check_device(d)) return st;
     return launch_nv_quant_scatter(x, M, K, 1, gscale, nullptr, q, sf, nullptr,

@@ -32,7 +32,8 @@
 // room for its transpose buffer).
 //
 // Also here: the NVFP4 quantise-and-scatter of x (the fused layer's first
-// GEMM input), sharing the quantisation step with the requantising epilogue.
+// GEMM input), sharing the quantisation step (nv_quant16) with the
+// requantising epilogue.
 #include <cuda_bf16.h>
 #include <cuda_fp4.h>
 #include <cuda_fp8.h>
@@ -590,54 +591,47 @@ __global__ void __launch_bounds__(kNvThreads, 1)
 
 // x [T, H] bf16 -> NVFP4 codes xq [R, H/2] and scales xsf [R, H/16] at rows
 // inv_perm[t*k + j] (row t when inv_perm is null and k = 1; global scale g);
-// also zeroes out_acc [T, H] when not null.  Warp per (token, 128-column
-// block); lane quad = one 16-column block, lane = 4 columns.
+// also zeroes out_acc [T, H] when not null.  Warp per (token, 512 columns),
+// lane = one 16-column block: one 32-byte load, one 8-byte code store and
+// one scale byte per destination row (a warp writes 256 + 32 contiguous
+// bytes per row).
 __global__ void __launch_bounds__(256) nv_quant_scatter_kernel(
     const __nv_bfloat16* __restrict__ x, int T, int H, int k, float g,
     const int32_t* __restrict__ inv_perm, uint8_t* __restrict__ xq, uint8_t* __restrict__ xsf,
     float* __restrict__ out_acc) {
-    const int nkb = H >> 7;
+    const int nch = (H + 511) >> 9;
     const long long item = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-    if (item >= static_cast<long long>(T) * nkb) return;
+    if (item >= static_cast<long long>(T) * nch) return;
     const int lane = threadIdx.x & 31;
-    const int t = static_cast<int>(item / nkb);
-    const int kb = static_cast<int>(item - static_cast<long long>(t) * nkb);
-    const long long off = static_cast<long long>(t) * H + kb * 128 + lane * 4;
-    uint2 raw = *reinterpret_cast<const uint2*>(x + off);
-    __nv_bfloat162 b01, b23;
-    memcpy(&b01, &raw.x, 4);
-    memcpy(&b23, &raw.y, 4);
-    const float2 f01 = __bfloat1622float2(b01);
-    const float2 f23 = __bfloat1622float2(b23);
-    float amax = fmaxf(fmaxf(fabsf(f01.x), fabsf(f01.y)), fmaxf(fabsf(f23.x), fabsf(f23.y)));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    float sc;
-    const uint32_t code = nv_e4m3_scale(amax, g, sc);
-    uint32_t codes = 0;
-    if (sc > 0.0f) {
-        codes = nv_e2m1(__fdiv_rn(__fmul_rn(f01.x, g), sc)) |
-                (nv_e2m1(__fdiv_rn(__fmul_rn(f01.y, g), sc)) << 4) |
-                (nv_e2m1(__fdiv_rn(__fmul_rn(f23.x, g), sc)) << 8) |
-                (nv_e2m1(__fdiv_rn(__fmul_rn(f23.y, g), sc)) << 12);
-    }
-    // the eight block scales of this 128-column block, one byte each
-    uint32_t lo = 0, hi = 0;
+    const int t = static_cast<int>(item / nch);
+    const int col = static_cast<int>(item - static_cast<long long>(t) * nch) * 512 + lane * 16;
+    if (col >= H) return;
+    const long long off = static_cast<long long>(t) * H + col;
+    const uint4* src = reinterpret_cast<const uint4*>(x + off);
+    const uint4 r0 = src[0], r1 = src[1];
+    const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+    float v[16];
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-        lo |= __shfl_sync(0xffffffffu, code, 4 * b) << (8 * b);
-        hi |= __shfl_sync(0xffffffffu, code, 16 + 4 * b) << (8 * b);
+    for (int i = 0; i < 8; ++i) {
+        __nv_bfloat162 b2;
+        memcpy(&b2, &w[i], 4);
+        const float2 f = __bfloat1622float2(b2);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
     }
+    uint2 packed;
+    const uint32_t code = nv_quant16(v, g, packed);
     for (int j = 0; j < k; ++j) {
         const int row = inv_perm ? inv_perm[t * k + j] : t;
         if (row < 0) continue;
-        *reinterpret_cast<uint16_t*>(xq + static_cast<long long>(row) * (H >> 1) + kb * 64 + lane * 2) =
-            static_cast<uint16_t>(codes);
-        if (lane == 0)
-            *reinterpret_cast<uint2*>(xsf + static_cast<long long>(row) * (H >> 4) + kb * 8) =
-                make_uint2(lo, hi);
+        *reinterpret_cast<uint2*>(xq + static_cast<long long>(row) * (H >> 1) + (col >> 1)) = packed;
+        xsf[static_cast<long long>(row) * (H >> 4) + (col >> 4)] = static_cast<uint8_t>(code);
     }
-    if (out_acc) *reinterpret_cast<float4*>(out_acc + off) = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (out_acc) {
+        float4* o = reinterpret_cast<float4*>(out_acc + off);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
 }
 
 template <int MODE>
@@ -686,7 +680,7 @@ int launch_nvfp4_gemm(const NvGemmArgs& g, cudaStream_t stream) {
 
 int launch_nv_quant_scatter(const void* x, int T, int H, int k, float g, const int32_t* inv_perm,
                             uint8_t* xq, uint8_t* xsf, float* out_acc, cudaStream_t stream) {
-    const long long items = static_cast<long long>(T) * (H / 128);
+    const long long items = static_cast<long long>(T) * ((H + 511) / 512);
     if (items == 0) return ST_OK;
     const long long blocks = (items + 7) / 8;
     nv_quant_scatter_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(

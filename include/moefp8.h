@@ -386,8 +386,8 @@ MOE_API int moe_nvfp4_fused_debug(const void* x, const int32_t* topk_ids, const 
  *  x   device bf16 [M, K]
  *  q   device uint8 [M, K/2] packed codes (element 2i in the low nibble)
  *  sf  device uint8 [M, K/16] E4M3 scale codes, row-major
- * K must be a multiple of 128, gscale > 0; pointers 8-byte aligned.
- * Asynchronous on `stream`. */
+ * K must be a multiple of 128, gscale > 0; x 16-byte aligned, q 8-byte
+ * aligned.  Asynchronous on `stream`. */
 MOE_API int nvfp4_quantize(const void* x, float gscale, uint8_t* q, uint8_t* sf, int M, int K,
                            moe_stream_t stream);
 

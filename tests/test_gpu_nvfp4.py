@@ -101,6 +101,7 @@ def test_nvfp4_gemm_exact_small_values(oracle, gated):
     (1000, 1024, 1024, 8, True, None),
     (640, 512, 7168, 3, False, None),         # 28 K blocks
     (64, 512, 2048, 8, True, None),           # small groups
+    (130, 128, 256, 64, False, None),         # one 128-column block, most experts empty
 ])
 def test_nvfp4_gemm_random(oracle, R, N, K, E, gated, sizes):
     inp = synth.make_nvfp4_gemm_inputs(R, N, K, E, seed=R + K, group_sizes=sizes)

@@ -44,13 +44,13 @@ def _compare_e2m1(got, ref, what):
     assert int(np.abs(got - ref).max()) <= 1, f"{what}: a code differs by more than one step"
 
 
-def test_nvfp4_quantize_bit_exact(oracle):
+@pytest.mark.parametrize("M,K", [(300, 1024), (37, 384)])  # 384: a warp's last 8 lanes idle
+def test_nvfp4_quantize_bit_exact(oracle, M, K):
     """Codes and scales identical to the oracle's on the exact fp32 values of
     bf16 rows (x N(0,1) with per-16 magnitudes 2^U{-3..3}, a few all-zero
     blocks and values past the saturation point).  +0 and -0 codes are
     treated as equal (both decode to 0)."""
-    g = torch.Generator().manual_seed(0)
-    M, K = 300, 1024
+    g = torch.Generator().manual_seed(K)
     x = torch.randn(M, K, generator=g)
     u = torch.randint(-3, 4, (M, K // 16), generator=g).float()
     x = (x.view(M, K // 16, 16) * torch.exp2(u)[:, :, None]).view(M, K)
