@@ -541,14 +541,14 @@ def run_nvfp4_gemm(args, cfg):
     inp = synth.make_nvfp4_gemm_inputs(R, N, K, E, seed=1, device="cuda", group_sizes=sizes)
     a, b = inp["a_packed"], inp["b_packed"]
     del inp["a"], inp["b"]
-    a_sf = inp["a_sf"].view(torch.uint8)
+    a_sf = inp["a_sf"].view(torch.uint8).view(R, K // 64, 4).permute(1, 0, 2).contiguous()
     b_sf = torch.empty(E * N, K // 16, dtype=torch.uint8, device="cuda")
     moe.nvfp4_tile_scales(inp["b_sf"].view(torch.uint8).view(E * N, K // 16), b_sf)
     alpha = (1.0 / (inp["ga"] * inp["gb"].double())).float()
     out = torch.empty(R, N // 2, dtype=torch.bfloat16, device="cuda")
 
     def step():
-        moe.nvfp4_moe_gemm(a, b, a_sf, b_sf, alpha, inp["m_indptr"], out, True)
+        moe.nvfp4_moe_gemm(a, b, a_sf, b_sf, alpha, inp["m_indptr"], out, True, "MN")
 
     for _ in range(args.warmup):
         step()
@@ -653,7 +653,8 @@ def run_nv_moe(args, cfg):
                          "unit": "TFLOP/s", "frac": g1_tf / fp4_peak, "traffic": None,
                          "kernel": "NVFP4 GEMM1 (gate/up + SwiGLU + NVFP4 requant)",
                          "peak_source": f"{src} (FP4 = bf16 burst x {FP4_OVER_BF16:g})"},
-            "gpu_launches": kernels_per_layer(T, k) * args.steps}
+            # + the K-block-major transpose of x's scales (taken when I >= H / 16)
+            "gpu_launches": (kernels_per_layer(T, k) + (1 if 16 * I >= H else 0)) * args.steps}
     print(json.dumps(line), flush=True)
     return 0
 

@@ -100,7 +100,7 @@ def lib():
     L.mxfp8_tile_scales.restype = I
     L.mxfp8_tile_scales.argtypes = [P, P, I, I, P]
     L.nvfp4_moe_gemm.restype = I
-    L.nvfp4_moe_gemm.argtypes = [P] * 7 + [I] * 5 + [P]
+    L.nvfp4_moe_gemm.argtypes = [P] * 7 + [I] * 6 + [P]
     L.nvfp4_tile_scales.restype = I
     L.nvfp4_tile_scales.argtypes = [P, P, I, I, P]
     F = ctypes.c_float
@@ -320,20 +320,21 @@ def mxfp8_tile_scales(sf_rowmajor, sf_tiled, *, dims=None, stream=None, check=Tr
     return _check(st, "mxfp8_tile_scales", check)
 
 
-def nvfp4_moe_gemm(a, b, a_sf, b_sf, alpha, m_indptr, out, is_gated=False, *, dims=None,
-                   stream=None, check=True) -> int:
-    """a uint8 [R, K/2] packed E2M1, b uint8 [E, N, K/2], a_sf uint8 [R, K/16] E4M3
-    row-major, b_sf the weight scales tiled by nvfp4_tile_scales, alpha fp32 [E],
-    out bf16 [R, N/2 if gated else N].  dims = (R, N, K, E) when raw addresses
-    are passed."""
+def nvfp4_moe_gemm(a, b, a_sf, b_sf, alpha, m_indptr, out, is_gated=False, a_sf_major="K", *,
+                   dims=None, stream=None, check=True) -> int:
+    """a uint8 [R, K/2] packed E2M1, b uint8 [E, N, K/2], a_sf uint8 E4M3
+    [R, K/16] ("K") or [K/64, R, 4] ("MN"), b_sf the weight scales tiled by
+    nvfp4_tile_scales, alpha fp32 [E], out bf16 [R, N/2 if gated else N].
+    dims = (R, N, K, E) when raw addresses are passed."""
     if dims is None:
         R = a.shape[0]
         K = a.shape[1] * 2
         E, N = b.shape[0], b.shape[1]
     else:
         R, N, K, E = dims
+    mode = {"K": 0, "MN": 1}.get(a_sf_major, a_sf_major)
     st = lib().nvfp4_moe_gemm(_ptr(a), _ptr(b), _ptr(a_sf), _ptr(b_sf), _ptr(alpha), _ptr(m_indptr),
-                              _ptr(out), R, N, K, E, int(bool(is_gated)), _stream(stream))
+                              _ptr(out), R, N, K, E, mode, int(bool(is_gated)), _stream(stream))
     return _check(st, "nvfp4_moe_gemm", check)
 
 

@@ -492,12 +492,22 @@ static int nv_fused_impl(const void* x, const int32_t* topk_ids, const float* to
     if (st) return st;
     stage_mark(1, s);
     if (T > 0) {
-        st = launch_nv_quant_scatter(x, T, H, k, a1_gscale, inv_perm, xq, xsf, out_acc, s);
+        // x's scales are written row-major (coalesced per destination row) into the
+        // intermediate's region, free until GEMM1, then made K-block-major; when that
+        // region is too small (I < H/16) the scatter writes them K-block-major itself
+        if (R * H / 16 <= L.out_acc - L.hq) {
+            st = launch_nv_quant_scatter(x, T, H, k, a1_gscale, inv_perm, xq, hq,
+                                         static_cast<int>(R), 0, out_acc, s);
+            if (!st) st = launch_nv_sf_kblock_major(hq, xsf, static_cast<int>(R), H, s);
+        } else {
+            st = launch_nv_quant_scatter(x, T, H, k, a1_gscale, inv_perm, xq, xsf,
+                                         static_cast<int>(R), 1, out_acc, s);
+        }
         if (st) return st;
         stage_mark(2, s);
         const unsigned long long tmo = g_timeout_ns.load();
         NvGemmArgs g1{};
-        g1.a = xq; g1.b = w13; g1.a_sf = xsf; g1.b_sf = w13_sf; g1.alpha = w13_alpha;
+        g1.a = xq; g1.b = w13; g1.a_sf = xsf; g1.a_sf_mn = 1; g1.b_sf = w13_sf; g1.alpha = w13_alpha;
         g1.m_indptr = m_indptr; g1.R = static_cast<int>(R); g1.N = 2 * I; g1.K = H; g1.E = E;
         g1.gated = 1; g1.epi = NV_EPI_SWIGLU_NVQUANT; g1.hq = hq; g1.hsf = hsf;
         g1.h_gscale = a2_gscale;
@@ -506,7 +516,7 @@ static int nv_fused_impl(const void* x, const int32_t* topk_ids, const float* to
         if (st) return st;
         stage_mark(3, s);
         NvGemmArgs g2{};
-        g2.a = hq; g2.b = w2; g2.a_sf = hsf; g2.b_sf = w2_sf; g2.alpha = w2_alpha;
+        g2.a = hq; g2.b = w2; g2.a_sf = hsf; g2.a_sf_mn = 1; g2.b_sf = w2_sf; g2.alpha = w2_alpha;
         g2.m_indptr = m_indptr; g2.R = static_cast<int>(R); g2.N = H; g2.K = I; g2.E = E;
         g2.gated = 0; g2.epi = NV_EPI_COMBINE; g2.perm = perm; g2.topk_w = topk_w; g2.topk = k;
         g2.out_acc = out_acc; g2.out_ld = H;
@@ -728,8 +738,9 @@ int mxfp8_tile_scales(const uint8_t* sf_rowmajor, uint8_t* sf_tiled, int rows, i
 
 int nvfp4_moe_gemm(const void* a, const void* b, const uint8_t* a_sf, const uint8_t* b_sf,
                    const float* alpha, const int32_t* m_indptr, void* out, int R, int N, int K,
-                   int E, int is_gated, moe_stream_t stream) {
+                   int E, int a_sf_major, int is_gated, moe_stream_t stream) {
     if (R < 0 || N <= 0 || K <= 0 || E < 1 || N % 128 || K % 256) return MOE_ERR_INVALID_ARG;
+    if (a_sf_major != 0 && a_sf_major != 1) return MOE_ERR_INVALID_ARG;
     if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
     if (is_gated && (N % 2 || (N / 2) % 128)) return MOE_ERR_INVALID_ARG;
     if (!m_indptr || (R > 0 && (!a || !b || !a_sf || !b_sf || !alpha || !out)))
@@ -745,7 +756,8 @@ int nvfp4_moe_gemm(const void* a, const void* b, const uint8_t* a_sf, const uint
         return MOE_ERR_CUDA;
     if (R == 0) return MOE_OK;
     NvGemmArgs g{};
-    g.a = a; g.b = b; g.a_sf = a_sf; g.b_sf = b_sf; g.alpha = alpha; g.m_indptr = m_indptr;
+    g.a = a; g.b = b; g.a_sf = a_sf; g.a_sf_mn = a_sf_major; g.b_sf = b_sf; g.alpha = alpha;
+    g.m_indptr = m_indptr;
     g.R = R; g.N = N; g.K = K; g.E = E; g.gated = is_gated ? 1 : 0;
     g.out = out;
     g.status = d->lib_status;
@@ -761,7 +773,7 @@ int nvfp4_quantize(const void* x, float gscale, uint8_t* q, uint8_t* sf, int M, 
     if (!aligned16(x) || (reinterpret_cast<uintptr_t>(q) & 7)) return MOE_ERR_INVALID_ARG;
     const DevInfo* d = dev_info();
     if (int st = check_device(d)) return st;
-    return launch_nv_quant_scatter(x, M, K, 1, gscale, nullptr, q, sf, nullptr,
+    return launch_nv_quant_scatter(x, M, K, 1, gscale, nullptr, q, sf, M, 0, nullptr,
                                    reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -123,14 +123,15 @@ int launch_mx_tile_scales(const uint8_t* rm, uint8_t* tiled, int rows, int K, in
 // of B, G = alpha[e] * (block-scaled product).
 enum NvEpilogue : int {
     NV_EPI_BF16 = 0,            // plain bf16 G, or gated bf16 silu(gate) * up
-    NV_EPI_SWIGLU_NVQUANT = 1,  // gated: h to NVFP4 (hq [R, N/4] packed, hsf [R, N/32])
+    NV_EPI_SWIGLU_NVQUANT = 1,  // gated: h to NVFP4 (hq [R, N/4] packed, hsf [N/128, R, 4])
     NV_EPI_COMBINE = 2,         // plain: out_acc[token, n] += topk_w * G (fp32 reduction)
 };
 
 struct NvGemmArgs {
     const void* a;            // [R, K/2] packed E2M1, grouped rows
     const void* b;            // [E, N, K/2] packed E2M1
-    const uint8_t* a_sf;      // [R, K/16] E4M3, row-major
+    const uint8_t* a_sf;      // E4M3: [R, K/16] row-major (a_sf_mn = 0) or [K/64, R, 4] (1)
+    int a_sf_mn;
     const uint8_t* b_sf;      // [E*N/128, K/64, 512] E4M3, tiled (launch_mx_tile_scales of 2K)
     const float* alpha;       // [E] 1 / (global scale of A * global scale of expert e)
     const int32_t* m_indptr;  // [E+1]
@@ -153,9 +154,15 @@ struct NvGemmArgs {
 int launch_nvfp4_gemm(const NvGemmArgs& g, cudaStream_t stream);
 
 // NVFP4 variant of launch_quant_scatter: xq [R, H/2] packed E2M1 codes and
-// xsf [R, H/16] E4M3 scales with global scale g, at rows inv_perm[t*k + j]
-// (row t when inv_perm is null and k = 1).
+// E4M3 scales with global scale g, at rows inv_perm[t*k + j] (row t when
+// inv_perm is null and k = 1); xsf [R, H/16] row-major, or [H/64, R, 4] when
+// sf_mn.
 int launch_nv_quant_scatter(const void* x, int T, int H, int k, float g, const int32_t* inv_perm,
-                            uint8_t* xq, uint8_t* xsf, float* out_acc, cudaStream_t stream);
+                            uint8_t* xq, uint8_t* xsf, int R, int sf_mn, float* out_acc,
+                            cudaStream_t stream);
+
+// Row-major E4M3 scales [R, K/16] -> K-block-major [K/64, R, 4] (4-byte
+// aligned buffers; (R, K/64) up to (2^21, any)).
+int launch_nv_sf_kblock_major(const uint8_t* rm, uint8_t* mn, int R, int K, cudaStream_t stream);
 
 }  // namespace moe

@@ -21,8 +21,10 @@
 //      byte(r, j) = (r % 32) * 16 + (r / 32) * 4 + j (j = 16-wide K block):
 //      A atoms at kk * 512, B atoms at 2048 + blk * 2048 + kk * 512.
 //      Weight scales come pre-tiled in that layout ([E*N/128, K/64, 512]),
-//      activation scales row-major [R, K/16] (four 4-byte copies per row per
-//      step).
+//      activation scales row-major [R, K/16] or K-block-major [K/64, R, 4]
+//      (the four scales of a 64-wide K block of each row together, rows
+//      consecutive: a warp's 32 rows are 128 contiguous bytes); four 4-byte
+//      copies per row per step.
 // Warps: 0 TMA producer, 1 MMA issuer (elected lane), 2 weight scale loader,
 // 3 activation scale loader, 4-11 epilogue.  TMEM: accumulator columns
 // [0, 256), A scale factors [256, 272) (4 per step), B scale factors
@@ -135,13 +137,14 @@ struct NvCfg {
 
 struct NvParams {
     int R, N, K, E, nkb, gated;  // nkb: 256-element K blocks
-    const uint8_t* a_sf;         // [R, K/16] E4M3
+    int a_sf_mn;                 // activation scales [K/64, R, 4] (1) or [R, K/16] (0)
+    const uint8_t* a_sf;         // E4M3
     const uint8_t* b_sf;         // [E*N/128, K/64, 512] E4M3, tiled
     const float* alpha;          // [E]
     const int32_t* m_indptr;
     __nv_bfloat16* out;          // NV_EPI_BF16
     uint8_t* hq;                 // NV_EPI_SWIGLU_NVQUANT: [R, N/4] packed codes of h
-    uint8_t* hsf;                //   and [R, N/32] E4M3 scales
+    uint8_t* hsf;                //   and [N/128, R, 4] E4M3 scales (K-block-major for GEMM2)
     float h_gscale;              //   global scale of h
     const int32_t* perm;         // NV_EPI_COMBINE: out_acc[perm[r] / topk] += topk_w[perm[r]] * G[r]
     const float* topk_w;
@@ -303,11 +306,14 @@ __device__ void nv_sf_loader(const NvParams& p, const NvSmem& s, const WaitCtl& 
                 for (int i = 0; i < 4; ++i) {  // token row lane + 32 i
                     const int r = tl.row0 + lane + 32 * i;
                     const bool v = r < p.R;
-                    const uint8_t* src = p.a_sf + static_cast<long long>(r) * nsf + kb * 16;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        cp_async_4(sf + kk * 512 + lane * 16 + i * 4, v ? src + kk * 4 : p.a_sf,
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const long long off =
+                            p.a_sf_mn ? (static_cast<long long>(kb * 4 + kk) * p.R + r) * 4
+                                      : static_cast<long long>(r) * nsf + kb * 16 + kk * 4;
+                        cp_async_4(sf + kk * 512 + lane * 16 + i * 4, v ? p.a_sf + off : p.a_sf,
                                    v ? 4u : 0u);
+                    }
                 }
             }
             cp_async_arrive_noinc(&s.full[stage]);
@@ -478,7 +484,8 @@ __device__ void nv_epilogue(const NvParams& p, const NvSmem& s, const WaitCtl& w
             uint4* dst = reinterpret_cast<uint4*>(p.hq + row * (I >> 1) + (col0 >> 1));
             dst[0] = make_uint4(packed[0].x, packed[0].y, packed[1].x, packed[1].y);
             dst[1] = make_uint4(packed[2].x, packed[2].y, packed[3].x, packed[3].y);
-            *reinterpret_cast<uint32_t*>(p.hsf + row * (I >> 4) + (col0 >> 4)) = sf4;
+            // the thread's 64 columns are one 64-wide K block of GEMM2
+            *reinterpret_cast<uint32_t*>(p.hsf + ((col0 >> 6) * p.R + row) * 4) = sf4;
         } else if (p.gated) {
             uint4* dst = reinterpret_cast<uint4*>(p.out + row * (p.N >> 1) + tl.nt * 128 + colg);
 #pragma unroll
@@ -589,8 +596,9 @@ __global__ void __launch_bounds__(kNvThreads, 1)
     if (warp == 1) tmem_dealloc(tmem_base, kNvTmemCols);
 }
 
-// x [T, H] bf16 -> NVFP4 codes xq [R, H/2] and scales xsf [R, H/16] at rows
-// inv_perm[t*k + j] (row t when inv_perm is null and k = 1; global scale g);
+// x [T, H] bf16 -> NVFP4 codes xq [R, H/2] and scales xsf at rows
+// inv_perm[t*k + j] (row t when inv_perm is null and k = 1; global scale g),
+// xsf row-major [R, H/16] or, when sf_mn, K-block-major [H/64, R, 4];
 // also zeroes out_acc [T, H] when not null.  Warp per (token, 512 columns),
 // lane = one 16-column block: one 32-byte load, one 8-byte code store and
 // one scale byte per destination row (a warp writes 256 + 32 contiguous
@@ -598,7 +606,7 @@ __global__ void __launch_bounds__(kNvThreads, 1)
 __global__ void __launch_bounds__(256) nv_quant_scatter_kernel(
     const __nv_bfloat16* __restrict__ x, int T, int H, int k, float g,
     const int32_t* __restrict__ inv_perm, uint8_t* __restrict__ xq, uint8_t* __restrict__ xsf,
-    float* __restrict__ out_acc) {
+    int R, int sf_mn, float* __restrict__ out_acc) {
     const int nch = (H + 511) >> 9;
     const long long item = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     if (item >= static_cast<long long>(T) * nch) return;
@@ -625,12 +633,34 @@ __global__ void __launch_bounds__(256) nv_quant_scatter_kernel(
         const int row = inv_perm ? inv_perm[t * k + j] : t;
         if (row < 0) continue;
         *reinterpret_cast<uint2*>(xq + static_cast<long long>(row) * (H >> 1) + (col >> 1)) = packed;
-        xsf[static_cast<long long>(row) * (H >> 4) + (col >> 4)] = static_cast<uint8_t>(code);
+        const long long so = sf_mn ? (static_cast<long long>(col >> 6) * R + row) * 4 + ((col >> 4) & 3)
+                                   : static_cast<long long>(row) * (H >> 4) + (col >> 4);
+        xsf[so] = static_cast<uint8_t>(code);
     }
     if (out_acc) {
         float4* o = reinterpret_cast<float4*>(out_acc + off);
 #pragma unroll
         for (int i = 0; i < 4; ++i) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+// Row-major activation scales [R, A] 4-byte words (A = K/64: the four scales
+// of a 64-wide K block) -> K-block-major [A, R] words, through a 32 x 32
+// shared-memory tile (reads and writes 128 contiguous bytes per warp).
+__global__ void __launch_bounds__(256) nv_sf_kblock_major_kernel(const uint32_t* __restrict__ rm,
+                                                                 uint32_t* __restrict__ mn, int R,
+                                                                 int A) {
+    __shared__ uint32_t tile[32][33];
+    const int a0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    for (int i = ty; i < 32; i += 8) {
+        const int r = r0 + i, a = a0 + tx;
+        if (r < R && a < A) tile[i][tx] = rm[static_cast<long long>(r) * A + a];
+    }
+    __syncthreads();
+    for (int i = ty; i < 32; i += 8) {
+        const int a = a0 + i, r = r0 + tx;
+        if (r < R && a < A) mn[static_cast<long long>(a) * R + r] = tile[tx][i];
     }
 }
 
@@ -661,6 +691,7 @@ int launch_nvfp4_gemm(const NvGemmArgs& g, cudaStream_t stream) {
     if (!make_tma_map_fp8(&mb, g.b, static_cast<long long>(g.E) * g.N, g.K / 2, 64)) return ST_CUDA;
     NvParams p{};
     p.R = g.R; p.N = g.N; p.K = g.K; p.E = g.E; p.nkb = g.K / 256; p.gated = g.gated ? 1 : 0;
+    p.a_sf_mn = g.a_sf_mn ? 1 : 0;
     p.a_sf = g.a_sf; p.b_sf = g.b_sf; p.alpha = g.alpha; p.m_indptr = g.m_indptr;
     p.out = static_cast<__nv_bfloat16*>(g.out);
     p.hq = g.hq; p.hsf = g.hsf; p.h_gscale = g.h_gscale;
@@ -679,12 +710,22 @@ int launch_nvfp4_gemm(const NvGemmArgs& g, cudaStream_t stream) {
 }
 
 int launch_nv_quant_scatter(const void* x, int T, int H, int k, float g, const int32_t* inv_perm,
-                            uint8_t* xq, uint8_t* xsf, float* out_acc, cudaStream_t stream) {
+                            uint8_t* xq, uint8_t* xsf, int R, int sf_mn, float* out_acc,
+                            cudaStream_t stream) {
     const long long items = static_cast<long long>(T) * ((H + 511) / 512);
     if (items == 0) return ST_OK;
     const long long blocks = (items + 7) / 8;
     nv_quant_scatter_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(x), T, H, k, g, inv_perm, xq, xsf, out_acc);
+        static_cast<const __nv_bfloat16*>(x), T, H, k, g, inv_perm, xq, xsf, R, sf_mn, out_acc);
+    return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
+}
+
+int launch_nv_sf_kblock_major(const uint8_t* rm, uint8_t* mn, int R, int K, cudaStream_t stream) {
+    const int A = K / 64;
+    if (R == 0 || A == 0) return ST_OK;
+    const dim3 grid((A + 31) / 32, (R + 31) / 32);
+    nv_sf_kblock_major_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint32_t*>(rm),
+                                                        reinterpret_cast<uint32_t*>(mn), R, A);
     return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
 }
 

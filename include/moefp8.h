@@ -326,7 +326,10 @@ MOE_API int mxfp8_tile_scales(const uint8_t* sf_rowmajor, uint8_t* sf_tiled, int
  *  a       device uint8 [R, K/2]: E2M1 codes packed two per byte, element
  *          2i in the low nibble (sign bit 3 of each nibble)
  *  b       device uint8 [E, N, K/2], packed the same way
- *  a_sf    device uint8 [R, K/16] E4M3 codes, row-major (4-byte aligned)
+ *  a_sf    device uint8 E4M3 codes of the activations (4-byte aligned):
+ *          a_sf_major = 0: [R, K/16] row-major; 1: [K/64, R, 4], the four
+ *          scales of a 64-wide K block of each row together, rows
+ *          consecutive (the rows of a tile are then read contiguously)
  *  b_sf    device uint8 E4M3 codes of the weights in the tiled layout that
  *          nvfp4_tile_scales produces from [E, N, K/16] row-major (16-byte
  *          aligned; weights are tiled once, not per call)
@@ -339,7 +342,7 @@ MOE_API int mxfp8_tile_scales(const uint8_t* sf_rowmajor, uint8_t* sf_tiled, int
  * Errors and ownership as for mxfp8_moe_gemm. */
 MOE_API int nvfp4_moe_gemm(const void* a, const void* b, const uint8_t* a_sf,
                            const uint8_t* b_sf, const float* alpha, const int32_t* m_indptr,
-                           void* out, int R, int N, int K, int E, int is_gated,
+                           void* out, int R, int N, int K, int E, int a_sf_major, int is_gated,
                            moe_stream_t stream);
 
 /* The fused layer of moe_fp8_fused in the NVFP4 (W4A4) variant of the cuTile
@@ -368,8 +371,8 @@ MOE_API int moe_nvfp4_fused(const void* x, const int32_t* topk_ids, const float*
                             int E, int k, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* moe_nvfp4_fused plus copies of m_indptr [E+1], perm [T*k], the packed
- * NVFP4 intermediate h_fp4 [T*k, I/2] and its E4M3 scales h_sf [T*k, I/16]
- * (any may be NULL). */
+ * NVFP4 intermediate h_fp4 [T*k, I/2] and its E4M3 scales h_sf
+ * [I/64, T*k, 4] (K-block-major, as GEMM2 reads them; any may be NULL). */
 MOE_API int moe_nvfp4_fused_debug(const void* x, const int32_t* topk_ids, const float* topk_w,
                                   const void* w13, const uint8_t* w13_sf, const float* w13_alpha,
                                   const void* w2, const uint8_t* w2_sf, const float* w2_alpha,

@@ -23,14 +23,22 @@ def _alpha(inp):
     return (1.0 / (inp["ga"] * inp["gb"].double())).float()
 
 
-def _run(inp, is_gated):
+def _mn(a_sf):
+    """[R, K/16] -> [K/64, R, 4] (the four scales of a 64-wide K block together)."""
+    R, nsf = a_sf.shape
+    return a_sf.view(R, nsf // 4, 4).permute(1, 0, 2).contiguous()
+
+
+def _run(inp, is_gated, a_mn=False):
     a, b = inp["a_packed"], inp["b_packed"]
     R = a.shape[0]
     E, N, _ = b.shape
     out = torch.full((R, N // 2 if is_gated else N), float("nan"), dtype=torch.bfloat16,
                      device=a.device)
-    moe.nvfp4_moe_gemm(a, b, inp["a_sf"].view(torch.uint8), _tiled(inp["b_sf"]),
-                       _alpha(inp).to(a.device), inp["m_indptr"], out, is_gated)
+    a_sf = inp["a_sf"].view(torch.uint8)
+    moe.nvfp4_moe_gemm(a, b, _mn(a_sf) if a_mn else a_sf, _tiled(inp["b_sf"]),
+                       _alpha(inp).to(a.device), inp["m_indptr"], out, is_gated,
+                       "MN" if a_mn else "K")
     torch.cuda.synchronize()
     assert moe.moe_get_device_status(None) == 0
     return out.cpu()
@@ -107,7 +115,9 @@ def test_nvfp4_gemm_random(oracle, R, N, K, E, gated, sizes):
     inp = synth.make_nvfp4_gemm_inputs(R, N, K, E, seed=R + K, group_sizes=sizes)
     rows = int(inp["m_indptr"][-1])
     ref = _oracle(oracle, inp, gated)
-    _compare(_run(_cuda(inp), gated), ref, rows)
+    dev = _cuda(inp)
+    _compare(_run(dev, gated), ref, rows)
+    _compare(_run(dev, gated, a_mn=True), ref, rows)
 
 
 def test_nvfp4_gemm_scale_placement(oracle):
@@ -121,7 +131,8 @@ def test_nvfp4_gemm_scale_placement(oracle):
     a_sf[37, 21] = 0x58
     b_sf[0, 200, 6] = 0x58
     ref = _oracle(oracle, inp, False)
-    _compare(_run(_cuda(inp), False), ref, R)
+    for a_mn in (False, True):
+        _compare(_run(_cuda(inp), False, a_mn), ref, R)
 
 
 def test_nvfp4_tile_scales_layout():
@@ -149,4 +160,6 @@ def test_nvfp4_gemm_empty_and_bad_args():
     assert moe.nvfp4_moe_gemm(a, b, a_sf, b_sf, alpha, m, out, False) == 0
     # K not a multiple of 256
     assert moe.nvfp4_moe_gemm(a, b, a_sf, b_sf, alpha, m, out, False, dims=(0, 256, 192, 2),
+                              check=False) == moe.MOE_ERR_INVALID_ARG
+    assert moe.nvfp4_moe_gemm(a, b, a_sf, b_sf, alpha, m, out, False, 2,
                               check=False) == moe.MOE_ERR_INVALID_ARG

@@ -93,7 +93,7 @@ def _run(inp):
     m_indptr = torch.empty(E + 1, dtype=torch.int32, device=dev)
     perm = torch.empty(max(R, 1), dtype=torch.int32, device=dev)
     hq = torch.empty(max(R, 1), I // 2, dtype=torch.uint8, device=dev)
-    hsf = torch.empty(max(R, 1), I // 16, dtype=torch.uint8, device=dev)
+    hsf = torch.empty(I // 64, max(R, 1), 4, dtype=torch.uint8, device=dev)  # K-block-major
     a13, a2 = _alphas(inp)
     moe.moe_nvfp4_fused_debug(x, inp["topk_ids"], inp["topk_w"], inp["w13_packed"],
                               _tile(inp["w13_sf"], (E * 2 * I, H // 16)), a13,
@@ -102,7 +102,8 @@ def _run(inp):
     torch.cuda.synchronize()
     assert moe.moe_get_device_status(ws) == 0
     Rg = int(m_indptr[-1])
-    return bf16_bits(out), i32(m_indptr), i32(perm[:Rg]), _unpack(u8(hq[:Rg])), u8(hsf[:Rg])
+    hsf_rm = hsf[:, :Rg, :].permute(1, 0, 2).reshape(Rg, I // 16)
+    return bf16_bits(out), i32(m_indptr), i32(perm[:Rg]), _unpack(u8(hq[:Rg])), u8(hsf_rm)
 
 
 # Output rows whose intermediate differs from the oracle's (a code or a block
@@ -181,6 +182,7 @@ def test_nvfp4_fused_tiny(oracle):
     (33, 256, 256, 5, 3, "normal"),     # ragged tiles, odd group sizes
     (200, 512, 512, 16, 4, "zipf"),     # skewed groups
     (300, 768, 256, 8, 2, "normal"),    # GEMM2 with three 256-column tiles
+    (20, 8192, 256, 4, 2, "normal"),    # I < H/16: x's scales scattered K-block-major directly
 ])
 def test_nvfp4_fused_shapes(oracle, T, H, I, E, k, routing):
     cfg = synth.MoEConfig("nv_case", T, H, I, E, k, routing)
