@@ -651,16 +651,21 @@ __global__ void __launch_bounds__(256) nv_sf_kblock_major_kernel(const uint32_t*
                                                                  uint32_t* __restrict__ mn, int R,
                                                                  int A) {
     __shared__ uint32_t tile[32][33];
-    const int a0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+    const int a0 = blockIdx.x * 32;
     const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-    for (int i = ty; i < 32; i += 8) {
-        const int r = r0 + i, a = a0 + tx;
-        if (r < R && a < A) tile[i][tx] = rm[static_cast<long long>(r) * A + a];
-    }
-    __syncthreads();
-    for (int i = ty; i < 32; i += 8) {
-        const int a = a0 + i, r = r0 + tx;
-        if (r < R && a < A) mn[static_cast<long long>(a) * R + r] = tile[tx][i];
+    const int ntiles = (R + 31) / 32;
+    for (int rt = blockIdx.y; rt < ntiles; rt += gridDim.y) {  // row tiles, grid-stride
+        const int r0 = rt * 32;
+        for (int i = ty; i < 32; i += 8) {
+            const int r = r0 + i, a = a0 + tx;
+            if (r < R && a < A) tile[i][tx] = rm[static_cast<long long>(r) * A + a];
+        }
+        __syncthreads();
+        for (int i = ty; i < 32; i += 8) {
+            const int a = a0 + i, r = r0 + tx;
+            if (r < R && a < A) mn[static_cast<long long>(a) * R + r] = tile[tx][i];
+        }
+        __syncthreads();
     }
 }
 
@@ -723,7 +728,8 @@ int launch_nv_quant_scatter(const void* x, int T, int H, int k, float g, const i
 int launch_nv_sf_kblock_major(const uint8_t* rm, uint8_t* mn, int R, int K, cudaStream_t stream) {
     const int A = K / 64;
     if (R == 0 || A == 0) return ST_OK;
-    const dim3 grid((A + 31) / 32, (R + 31) / 32);
+    const int row_tiles = (R + 31) / 32;
+    const dim3 grid((A + 31) / 32, row_tiles < 65535 ? row_tiles : 65535);
     nv_sf_kblock_major_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint32_t*>(rm),
                                                         reinterpret_cast<uint32_t*>(mn), R, A);
     return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
