@@ -204,10 +204,8 @@ def oracle_sample_rate(inp, cfg, n_tok, repeats=1):
     """Times the CPU oracle (per-token form) on n_tok tokens; returns
     (flops per sample, seconds per sample, threads)."""
     import oracle
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from tests import gpu_helpers as G
     toks = sample_tokens(cfg, n_tok)
-    sub = G.compact_experts(inp, toks)
+    sub = synth.compact_experts(inp, toks)
     args = (sub["x"], sub["topk_ids"], sub["topk_w"], sub["w13"], sub["w13_scale"], sub["w2"],
             sub["w2_scale"], np.arange(len(toks), dtype=np.int32))
     valid = int(((sub["topk_ids"] >= 0)).sum())

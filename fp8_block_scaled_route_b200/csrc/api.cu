@@ -17,6 +17,8 @@
 
 using namespace moe;
 
+static_assert(MOE_MAX_EXPERTS == kMaxRouteExperts, "routing kernels and the C ABI disagree on E");
+
 namespace {
 
 // Status word for the entry points that take no workspace.

@@ -57,6 +57,8 @@ struct RouteArgs {
     int* status;
 };
 constexpr int kRouteChunk = 1024;
+// Largest expert count the routing kernels accept (MOE_MAX_EXPERTS of the C ABI).
+constexpr int kMaxRouteExperts = 1024;
 int launch_route_permute(const RouteArgs& r, cudaStream_t stream);
 
 // logits fp32 [T, E] -> ids int32 [T, k] (descending logit, ties to the lower

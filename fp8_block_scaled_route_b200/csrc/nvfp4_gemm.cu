@@ -598,458 +598,6 @@ __global__ void __launch_bounds__(kNvThreads, 1)
     if (warp == 1) tmem_dealloc(tmem_base, kNvTmemCols);
 }
 
-// ------------------------------------------------------------ two-CTA tile
-// A cluster of two CTAs computes 256 grouped rows x 256 weight rows with
-// tcgen05.mma.cta_group::2 (M = 256): CTA c loads its own 128 token rows and
-// weight block c (the gate rows when c = 0 and the up rows when c = 1 for a
-// gated GEMM), so each SM stages 32 KB of operands per 256 K elements instead
-// of 48 KB, and five stages fit.  The leader CTA (rank 0) issues the
-// scale-factor copies and the MMAs for both; each CTA keeps the accumulator of
-// its own 128 rows in its TMEM and runs its own epilogue.
-//   full[s]   leader only: 4 leader TMA lanes (each expecting its box and the
-//             peer's matching box), 64 leader scale-loader lanes, 1 arrive
-//             forwarded by the peer once its scale loads have landed
-//   sfull[s]  peer only: its 64 scale-loader lanes (cp.async)
-//   empty[s]  both: one multicast commit from the leader's MMA thread
-//   tfull     both: one multicast commit per tile
-//   tempty    leader only: 8 local + 8 remote epilogue-warp arrivals
-// Scale factors: each CTA stages its own 128 rows' activation scales and the
-// full 256-row weight scales (both blocks), moved to its TMEM by the leader's
-// tcgen05.cp.cta_group::2.  Both CTAs leave through a cluster barrier, which
-// every path reaches (waits are bounded and failures break out of the loops).
-// Off by default: selected by MOE_NVFP4_TWO_CTA=1 for the bf16 epilogue.
-constexpr int kNv2Stages = 5;
-constexpr int kNv2A = 128 * 128;
-constexpr int kNv2B = 128 * 128;
-constexpr int kNv2SfOff = kNv2A + kNv2B;
-constexpr int kNv2Stage = kNv2A + kNv2B + kNvSfBytes;
-constexpr int kNv2Smem = 1024 + kNv2Stages * kNv2Stage + kNvTable + 256;
-static_assert(kNv2Stage % 1024 == 0, "stages must stay 1024-byte aligned for the swizzle");
-static_assert(kNv2Smem <= 232448, "shared memory budget");
-
-struct Nv2Smem {
-    uint8_t* stages;
-    int* tstart;
-    int* mind;
-    uint64_t* full;
-    uint64_t* sfull;
-    uint64_t* empty;
-    uint64_t* tfull;
-    uint64_t* tempty;
-    uint32_t* tmem;
-    volatile int* abort;
-};
-
-__device__ __forceinline__ Nv2Smem nv2_carve(uint8_t* base) {
-    Nv2Smem s;
-    s.stages = base;
-    uint8_t* p = base + kNv2Stages * kNv2Stage;
-    s.tstart = reinterpret_cast<int*>(p);
-    s.mind = s.tstart + (kNvMaxE + 1);
-    p += kNvTable;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(p);
-    s.full = bars;
-    s.sfull = bars + kNv2Stages;
-    s.empty = bars + 2 * kNv2Stages;
-    s.tfull = bars + 3 * kNv2Stages;
-    s.tempty = bars + 3 * kNv2Stages + 1;
-    s.tmem = reinterpret_cast<uint32_t*>(bars + 3 * kNv2Stages + 2);
-    s.abort = reinterpret_cast<volatile int*>(bars + 3 * kNv2Stages + 3);
-    return s;
-}
-
-__device__ __forceinline__ uint32_t nv2_cta_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-// Address of the same shared-memory object in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t nv2_mapa(const void* p, uint32_t rank) {
-    uint32_t out;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(smem_u32(p)), "r"(rank));
-    return out;
-}
-
-__device__ __forceinline__ void nv2_remote_arrive(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool nv2_test_wait(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait with cluster-scope acquire (arrivals from the peer CTA).
-__device__ bool nv2_wait(uint64_t* bar, uint32_t parity, const WaitCtl& c, int where) {
-    if (nv2_test_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer();
-#pragma unroll 1
-    for (uint32_t round = 1;; ++round) {
-        if (nv2_test_wait(bar, parity)) return true;
-        if ((round & 255) == 0 || c.timeout_ns < 1000000ull) {
-            if (*c.abort) return false;
-            if (globaltimer() - t0 > c.timeout_ns) {
-                *c.abort = 1;
-                report_error(c.status, ST_DEVICE_TIMEOUT, where);
-                return false;
-            }
-        }
-    }
-}
-__device__ __forceinline__ bool nv2_warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& c,
-                                              int where) {
-    return __all_sync(0xffffffffu, nv2_wait(bar, parity, c, where)) != 0;
-}
-
-// TMA load whose completion is counted on the leader CTA's barrier.
-__device__ __forceinline__ void nv2_tma_load(void* smem_dst, const CUtensorMap* map,
-                                             uint32_t leader_bar, int x, int y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(x), "r"(y)
-        : "memory");
-}
-
-__device__ __forceinline__ void nv2_umma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                         uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
-                                         uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %6, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
-        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem),
-        "r"(accumulate)
-        : "memory");
-}
-
-__device__ __forceinline__ void nv2_tmem_cp(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-                 : "memory");
-}
-
-// Commit of the leader's MMAs, arriving on the barrier at this offset in both CTAs.
-__device__ __forceinline__ void nv2_commit_both(uint64_t* bar) {
-    const uint16_t mask = 3;
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-        " [%0], %1;" ::"r"(smem_u32(bar)), "h"(mask)
-        : "memory");
-}
-
-// Tile t -> (expert, column tile, this CTA's 128 rows of a 256-row tile).
-__device__ __forceinline__ NvTile nv2_decode(int t, const Nv2Smem& s, int E, uint32_t rank) {
-    int lo = 0, hi = E;
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (s.tstart[mid] <= t) lo = mid; else hi = mid;
-    }
-    NvTile r;
-    r.e = lo;
-    const int local = t - s.tstart[lo];
-    const int me = max(0, s.mind[lo + 1] - s.mind[lo]);
-    const int mtiles = (me + 255) / 256;
-    r.nt = local / mtiles;
-    const int mt = local - r.nt * mtiles;
-    r.row0 = s.mind[lo] + mt * 256 + 128 * static_cast<int>(rank);
-    r.rows = max(0, min(128, me - mt * 256 - 128 * static_cast<int>(rank)));
-    return r;
-}
-
-__device__ void nv2_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const NvParams& p,
-                             const Nv2Smem& s, const WaitCtl& wc, int total, uint32_t rank) {
-    const int l = threadIdx.x & 31;
-    const bool issuer = l < 4;
-    const bool is_a = l < 2;
-    const uint32_t off = is_a ? l * 64 * 128 : kNv2A + (l - 2) * 64 * 128;
-    const int ncl = gridDim.x >> 1;
-    uint32_t stage = 0, phase = 0;
-    bool ok = true;
-    for (int t = blockIdx.x >> 1; t < total && ok; t += ncl) {
-        const NvTile tl = nv2_decode(t, s, p.E, rank);
-        int w0, w1;
-        nv_weight_rows(tl, p, w0, w1);
-        const int row = is_a ? tl.row0 + l * 64 : (rank ? w1 : w0) + (l - 2) * 64;
-        for (int kb = 0; kb < p.nkb; ++kb) {
-            if (!nv2_warp_wait(&s.empty[stage], phase ^ 1, wc, 1)) { ok = false; break; }
-            if (issuer) {
-                const uint32_t leader_full = smem_u32(&s.full[stage]) & 0xFEFFFFFFu;
-                if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], 2 * 64 * 128);
-                nv2_tma_load(s.stages + stage * kNv2Stage + off, is_a ? tmA : tmB, leader_full,
-                             kb * 128, row);
-            }
-            __syncwarp();
-            if (++stage == kNv2Stages) { stage = 0; phase ^= 1; }
-        }
-    }
-}
-
-// Scale loaders (warps 2, 3): own 128 rows' activation scales, the full
-// 256-row weight scales; completion on full[s] (leader) or sfull[s] (peer).
-template <bool WEIGHTS>
-__device__ void nv2_sf_loader(const NvParams& p, const Nv2Smem& s, const WaitCtl& wc, int total,
-                              uint32_t rank) {
-    const int lane = threadIdx.x & 31;
-    const int nsf = p.K >> 4;
-    const int natoms = p.K >> 6;
-    const long long wblocks = static_cast<long long>(p.E) * p.N / 128;
-    const int ncl = gridDim.x >> 1;
-    uint32_t stage = 0, phase = 0;
-    bool ok = true;
-    for (int t = blockIdx.x >> 1; t < total && ok; t += ncl) {
-        const NvTile tl = nv2_decode(t, s, p.E, rank);
-        int w0, w1;
-        nv_weight_rows(tl, p, w0, w1);
-        for (int kb = 0; kb < p.nkb; ++kb) {
-            if (!nv2_warp_wait(&s.empty[stage], phase ^ 1, wc, 8)) { ok = false; break; }
-            uint8_t* sf = s.stages + stage * kNv2Stage + kNv2SfOff;
-            if constexpr (WEIGHTS) {
-#pragma unroll
-                for (int blk = 0; blk < 2; ++blk) {
-                    const long long wb = (blk ? w1 : w0) >> 7;
-                    const bool v = wb < wblocks;
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint8_t* src =
-                            v ? p.b_sf + (wb * natoms + kb * 4 + kk) * 512 + lane * 16 : p.b_sf;
-                        cp_async_16(sf + 2048 + blk * 2048 + kk * 512 + lane * 16, src, v ? 16u : 0u);
-                    }
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int r = tl.row0 + lane + 32 * i;
-                    const bool v = r < p.R;
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const long long off =
-                            p.a_sf_mn ? (static_cast<long long>(kb * 4 + kk) * p.R + r) * 4
-                                      : static_cast<long long>(r) * nsf + kb * 16 + kk * 4;
-                        cp_async_4(sf + kk * 512 + lane * 16 + i * 4, v ? p.a_sf + off : p.a_sf,
-                                   v ? 4u : 0u);
-                    }
-                }
-            }
-            cp_async_arrive_noinc(rank == 0 ? &s.full[stage] : &s.sfull[stage]);
-            if (++stage == kNv2Stages) { stage = 0; phase ^= 1; }
-        }
-    }
-    cp_async_wait_all();
-    __syncwarp();
-}
-
-// Warp 1.  Leader: scale-factor copies and MMAs for the pair.  Peer: forwards
-// the completion of its scale loads to the leader's full barrier.
-__device__ void nv2_mma(const NvParams& p, const Nv2Smem& s, const WaitCtl& wc, uint32_t tmem_base,
-                        int total, uint32_t rank) {
-    const int ncl = gridDim.x >> 1;
-    uint32_t stage = 0, phase = 0, it = 0;
-    bool ok = true;
-    if (rank != 0) {
-        for (int t = blockIdx.x >> 1; t < total && ok; t += ncl) {
-            for (int kb = 0; kb < p.nkb; ++kb) {
-                if (!nv2_warp_wait(&s.sfull[stage], phase, wc, 9)) { ok = false; break; }
-                if (elect_one()) {
-                    // cp.async writes (generic proxy) read next by the leader's tcgen05.cp
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    nv2_remote_arrive(nv2_mapa(&s.full[stage], 0));
-                }
-                __syncwarp();
-                if (++stage == kNv2Stages) { stage = 0; phase ^= 1; }
-            }
-        }
-        return;
-    }
-    const uint32_t sfa_t = tmem_base + kNvSfaCol;
-    const uint32_t sfb_t = tmem_base + kNvSfbCol;
-    constexpr uint32_t idesc = idesc_nvf4(256, 256);
-    for (int t = blockIdx.x >> 1; t < total && ok; t += ncl, ++it) {
-        if (!nv2_warp_wait(s.tempty, (it & 1) ^ 1, wc, 3)) break;
-        tc_fence_after();
-        for (int kb = 0; kb < p.nkb; ++kb) {
-            if (!nv2_warp_wait(&s.full[stage], phase, wc, 4)) { ok = false; break; }
-            tc_fence_after();
-            uint8_t* st = s.stages + stage * kNv2Stage;
-            const uint32_t sa = smem_u32(st);
-            const uint32_t sb = smem_u32(st + kNv2A);
-            const uint32_t ssf = smem_u32(st + kNv2SfOff);
-            if (elect_one()) {
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    nv2_tmem_cp(sfa_t + 4 * kk, smem_desc_k_noswizzle(ssf + kk * 512, 16, 128));
-                    nv2_tmem_cp(sfb_t + 8 * kk, smem_desc_k_noswizzle(ssf + 2048 + kk * 512, 16, 128));
-                    nv2_tmem_cp(sfb_t + 8 * kk + 4, smem_desc_k_noswizzle(ssf + 4096 + kk * 512, 16, 128));
-                }
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    nv2_umma(tmem_base, smem_desc_k_sw128(sa + kk * 32), smem_desc_k_sw128(sb + kk * 32),
-                             idesc, sfa_t + 4 * kk, sfb_t + 8 * kk, (kb | kk) != 0);
-                nv2_commit_both(&s.empty[stage]);
-                if (kb == p.nkb - 1) nv2_commit_both(s.tfull);
-            }
-            __syncwarp();
-            if (++stage == kNv2Stages) { stage = 0; phase ^= 1; }
-        }
-    }
-}
-
-// Warps 4-11: as the single-CTA bf16 epilogue, on this CTA's 128 rows; the
-// accumulator is released on the leader's tempty barrier.
-__device__ void nv2_epilogue(const NvParams& p, const Nv2Smem& s, const WaitCtl& wc,
-                             uint32_t tmem_base, int total, uint32_t rank) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int q = warp & 3;
-    const int g = (warp - 4) >> 2;
-    const int rl = q * 32 + lane;
-    const int colg = g * 64;
-    const uint32_t tl_addr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + colg;
-    const uint32_t leader_tempty = nv2_mapa(s.tempty, 0);
-    const int ncl = gridDim.x >> 1;
-    uint32_t it = 0;
-    uint32_t v[4][32];
-    for (int t = blockIdx.x >> 1; t < total; t += ncl, ++it) {
-        const NvTile tl = nv2_decode(t, s, p.E, rank);
-        const bool row_ok = rl < tl.rows;
-        const long long row = tl.row0 + rl;
-        const float al = __ldg(p.alpha + tl.e);
-        if (!nv2_warp_wait(s.tfull, it & 1, wc, 6)) break;
-        tc_fence_after();
-        tmem_ld32_async(tl_addr, v[0]);
-        tmem_ld32_async(tl_addr + 32, v[1]);
-        tmem_ld32_async(tl_addr + 128, v[2]);
-        tmem_ld32_async(tl_addr + 160, v[3]);
-        tmem_wait_ld(v[0]);
-        tmem_wait_ld(v[1]);
-        tmem_wait_ld(v[2]);
-        tmem_wait_ld(v[3]);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) nv2_remote_arrive(leader_tempty);
-        if (!row_ok) continue;
-        if (p.gated) {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + row * (p.N >> 1) + tl.nt * 128 + colg);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                float h[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int j = 8 * c + i;
-                    h[i] = nv_silu(al * __uint_as_float(v[j >> 5][j & 31])) *
-                           (al * __uint_as_float(v[2 + (j >> 5)][j & 31]));
-                }
-                dst[c] = make_uint4(nv_pack_bf16(h[0], h[1]), nv_pack_bf16(h[2], h[3]),
-                                    nv_pack_bf16(h[4], h[5]), nv_pack_bf16(h[6], h[7]));
-            }
-        } else {
-            const int n0 = tl.nt * 256;
-            __nv_bfloat16* rowp = p.out + row * p.N + n0 + colg;
-#pragma unroll
-            for (int blk = 0; blk < 2; ++blk) {
-                if (n0 + blk * 128 >= p.N) break;
-                uint4* dst = reinterpret_cast<uint4*>(rowp + blk * 128);
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint32_t* a = v[2 * blk + (c >> 2)] + (c & 3) * 8;
-                    dst[c] = make_uint4(
-                        nv_pack_bf16(al * __uint_as_float(a[0]), al * __uint_as_float(a[1])),
-                        nv_pack_bf16(al * __uint_as_float(a[2]), al * __uint_as_float(a[3])),
-                        nv_pack_bf16(al * __uint_as_float(a[4]), al * __uint_as_float(a[5])),
-                        nv_pack_bf16(al * __uint_as_float(a[6]), al * __uint_as_float(a[7])));
-                }
-            }
-        }
-    }
-}
-
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNvThreads, 1)
-    nvfp4_gemm_2cta_kernel(const __grid_constant__ CUtensorMap tmA,
-                           const __grid_constant__ CUtensorMap tmB, const NvParams p) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* base = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    const Nv2Smem s = nv2_carve(base);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t rank = nv2_cta_rank();
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < kNv2Stages; ++i) {
-            mbar_init(&s.full[i], 4 + 64 + 1);  // leader TMA lanes, leader scale loaders, peer
-            mbar_init(&s.sfull[i], 64);
-            mbar_init(&s.empty[i], 1);
-        }
-        mbar_init(s.tfull, 1);
-        mbar_init(s.tempty, 2 * kNvEpiWarps);
-        *s.abort = 0;
-        fence_mbar_init();
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        tma_prefetch_desc(&tmA);
-        tma_prefetch_desc(&tmB);
-    }
-    if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
-                     ::"r"(smem_u32(s.tmem)), "r"(kNvTmemCols));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
-    }
-    if (warp == 2) {
-        // per-expert tile table: tiles of expert e = ceil(rows_e / 256) * column tiles
-        const int E = p.E;
-        const int ntn = p.gated ? (p.N >> 8) : ((p.N + 255) >> 8);
-        const int per = (E + 31) >> 5;
-        const int lo = min(E, lane * per), hi = min(E, lo + per);
-        int sum = 0;
-        for (int e = lo; e < hi; ++e) {
-            const int m0 = min(max(p.m_indptr[e], 0), p.R);
-            const int m1 = min(max(p.m_indptr[e + 1], 0), p.R);
-            s.mind[e] = m0;
-            sum += ((max(0, m1 - m0) + 255) / 256) * ntn;
-        }
-        int incl = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int x = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += x;
-        }
-        int run = incl - sum;
-        for (int e = lo; e < hi; ++e) {
-            s.tstart[e] = run;
-            const int m0 = s.mind[e];
-            const int m1 = min(max(p.m_indptr[e + 1], 0), p.R);
-            run += ((max(0, m1 - m0) + 255) / 256) * ntn;
-        }
-        if (lane == 31) {
-            s.tstart[E] = incl;
-            s.mind[E] = min(max(p.m_indptr[E], 0), p.R);
-        }
-    }
-    tc_fence_before();
-    // both CTAs' barriers initialised and TMEM allocated before any cross-CTA traffic
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-    tc_fence_after();
-    const uint32_t tmem_base = *s.tmem;
-    const WaitCtl wc{s.abort, p.status, p.timeout_ns};
-    const int total = s.tstart[p.E];
-    if (warp == 0) nv2_producer(&tmA, &tmB, p, s, wc, total, rank);
-    else if (warp == 1) nv2_mma(p, s, wc, tmem_base, total, rank);
-    else if (warp == 2) nv2_sf_loader<true>(p, s, wc, total, rank);
-    else if (warp == 3) nv2_sf_loader<false>(p, s, wc, total, rank);
-    else nv2_epilogue(p, s, wc, tmem_base, total, rank);
-    tc_fence_before();
-    // no CTA leaves while the pair's copies, MMAs or remote arrivals may still touch it
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-    tc_fence_after();
-    if (warp == 1)
-        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                     "r"(kNvTmemCols));
-}
-
 // x [T, H] bf16 -> NVFP4 codes xq [R, H/2] and scales xsf at rows
 // inv_perm[t*k + j] (row t when inv_perm is null and k = 1; global scale g),
 // xsf row-major [R, H/16] or, when sf_mn, K-block-major [H/64, R, 4];
@@ -1141,31 +689,6 @@ int launch_nv_inst(const CUtensorMap& ma, const CUtensorMap& mb, const NvParams&
 
 }  // namespace
 
-namespace {
-// The two-CTA tile is built but has not yet run on a GPU; it is taken only
-// when the process sets MOE_NVFP4_TWO_CTA=1, for the bf16 epilogue.
-bool two_cta_requested() {
-    const char* v = getenv("MOE_NVFP4_TWO_CTA");
-    return v && v[0] == '1' && v[1] == '\0';
-}
-
-int launch_nv2(const CUtensorMap& ma, const CUtensorMap& mb, const NvParams& p, int num_sms,
-               cudaStream_t stream) {
-    static int configured_dev = -1;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured_dev != dev) {
-        if (cudaFuncSetAttribute(nvfp4_gemm_2cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kNv2Smem) != cudaSuccess)
-            return ST_CUDA;
-        configured_dev = dev;
-    }
-    const int grid = (num_sms / 2) * 2;  // whole clusters of two
-    nvfp4_gemm_2cta_kernel<<<grid, kNvThreads, kNv2Smem, stream>>>(ma, mb, p);
-    return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
-}
-}  // namespace
-
 int launch_nvfp4_gemm(const NvGemmArgs& g, cudaStream_t stream) {
     if (g.R <= 0 || g.E <= 0) return ST_OK;
     if (g.E > kNvMaxE) return ST_INVALID_ARG;
@@ -1183,7 +706,6 @@ int launch_nvfp4_gemm(const NvGemmArgs& g, cudaStream_t stream) {
     p.out_acc = g.out_acc; p.out_ld = g.out_ld;
     p.status = g.status;
     p.timeout_ns = g.timeout_ns;
-    if (g.epi == NV_EPI_BF16 && two_cta_requested()) return launch_nv2(ma, mb, p, g.num_sms, stream);
     switch (g.epi) {
         case NV_EPI_SWIGLU_NVQUANT:
             return launch_nv_inst<NV_EPI_SWIGLU_NVQUANT>(ma, mb, p, g.num_sms, stream);

@@ -143,6 +143,8 @@ __global__ void __launch_bounds__(32) route_scatter(const int32_t* __restrict__ 
 // phases 1 and 3; thread e owns expert e in phase 2.  The per-chunk tables
 // live in shared memory.
 constexpr int kSmallChunks = 8;
+static_assert(kSmallChunks * kMaxRouteExperts * sizeof(int) <= 48 * 1024,
+              "route_small's histogram table must fit the default shared-memory limit");
 
 __global__ void __launch_bounds__(1024) route_small(const int32_t* __restrict__ ids, int R, int E,
                                                     int32_t* __restrict__ m_indptr,
@@ -314,21 +316,8 @@ int launch_route_permute(const RouteArgs& r, cudaStream_t stream) {
     const int nchunks = (R + kRouteChunk - 1) / kRouteChunk;
     const size_t hist_smem = static_cast<size_t>(r.E) * sizeof(int);
     if (nchunks <= kSmallChunks) {
+        // at most 8 x 1024 ints = 32 KB: within the default dynamic shared-memory limit
         const size_t smem = static_cast<size_t>(kSmallChunks) * r.E * sizeof(int);
-        if (smem > 48 * 1024) {
-            // above the default dynamic shared-memory limit: opt in (per device)
-            static bool attr_set[64] = {};
-            int dev = 0;
-            cudaGetDevice(&dev);
-            if (dev < 0 || dev >= 64) return ST_CUDA;
-            if (!attr_set[dev]) {
-                if (cudaFuncSetAttribute(route_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmallChunks * 1024 * static_cast<int>(sizeof(int))) !=
-                    cudaSuccess)
-                    return ST_CUDA;
-                attr_set[dev] = true;
-            }
-        }
         route_small<<<1, 1024, smem, stream>>>(r.topk_ids, R, r.E, r.m_indptr, r.perm, r.inv_perm,
                                                r.status);
         return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;

@@ -18,8 +18,10 @@
 //  * every call uses the same array and leaves its contents behind; calls
 //    whose kernels overlap on the GPU (different streams, no ordering
 //    between them) race on it and give undefined results;
-//  * the first call on a device looks up the array's device address on that
-//    device; make that first call before any stream capture begins.
+//  * the first call on a device, and the first after a cudaDeviceReset of
+//    it, looks up the array's device address in that device's context; make
+//    that call before any stream capture begins.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -39,22 +41,63 @@ constexpr int kNoAllocInts = kNoAllocStatusInts + kNoAllocChunks * MOE_MAX_EXPER
 static __device__ __align__(256) int32_t g_route_scratch[kNoAllocInts];
 
 constexpr int kMaxDevices = 64;
-int32_t* g_scratch_addr[kMaxDevices];  // device address of g_route_scratch per device
+
+// The device address of g_route_scratch is looked up once per CUDA context:
+// cudaDeviceReset destroys the device's context (and the module holding the
+// array), and the next context loads the module again, possibly elsewhere.
+// The context's process-unique id (cuCtxGetId) tells the two apart.
+struct ScratchAddr {
+    unsigned long long ctx_id;
+    int32_t* ptr;
+};
+ScratchAddr g_scratch_addr[kMaxDevices];
 std::mutex g_scratch_mu;
 
-// Device address of the scratch array on the current device.  In host code
-// the array's name only stands in for the symbol; the address has to be
-// asked for once per device with that device current.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Id of the context current on this thread, or 0 when it cannot be read.
+unsigned long long current_ctx_id() {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(f);
+    });
+    if (!get_current || !get_id) return 0;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+    if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+// Device address of the scratch array in the current device's context.  In
+// host code the array's name only stands in for the symbol; the address has
+// to be asked for with that device (and context) current.
 int32_t* scratch_on_current_device() {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    // make the device's primary context current (no allocation), so that its id can be read
+    if (cudaSetDevice(dev) != cudaSuccess) return nullptr;
+    const unsigned long long id = current_ctx_id();
     std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (g_scratch_addr[dev] == nullptr) {
+    ScratchAddr& a = g_scratch_addr[dev];
+    if (a.ptr == nullptr || id == 0 || a.ctx_id != id) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || p == nullptr) return nullptr;
-        g_scratch_addr[dev] = static_cast<int32_t*>(p);
+        a.ptr = static_cast<int32_t*>(p);
+        a.ctx_id = id;
     }
-    return g_scratch_addr[dev];
+    return a.ptr;
 }
 
 }  // namespace

@@ -99,8 +99,9 @@ MOE_API int moe_route_permute(const int32_t* topk_ids, int T, int k, int E,
  * GPU, held until the process exits).  Limits: T*k <= 65536 pairs and
  * E <= MOE_MAX_EXPERTS, else MOE_ERR_INVALID_ARG.  All calls share that
  * array: calls whose kernels overlap on the GPU race and give undefined
- * results.  The first call on a device looks up the array's address on that
- * device; make it before any stream capture.  Ids outside [0, E) are
+ * results.  The first call on a device, and the first after a
+ * cudaDeviceReset of it, looks up the array's address in that device's
+ * context; make that call before any stream capture.  Ids outside [0, E) are
  * dropped (m_indptr[E] then counts only valid pairs) and not reported
  * through moe_get_device_status.  Allocates nothing. */
 MOE_API int moe_route_permute_noalloc(const int32_t* topk_ids, int T, int k, int E,

@@ -100,6 +100,8 @@ def lib():
         L.oracle_moe_mx_tokens.argtypes = [P] * 7 + [i] * 5 + [P, i, P, P, P]
         L.oracle_moe_mx_fused.restype = i
         L.oracle_moe_mx_fused.argtypes = [P] * 8 + [i] * 5 + [P] * 4
+        L.oracle_combine.restype = None
+        L.oracle_combine.argtypes = [P, P, P, i, i, i, P]
         L.oracle_num_threads.restype = i
         L.oracle_num_threads.argtypes = []
     return _lib
@@ -260,6 +262,21 @@ def moe_tokens(x_bits, topk_ids, topk_w, w13, w13_scale, w2, w2_scale, tokens, w
                             T, H, I, E, k, _p(tokens), n, _p(out),
                             _p(hq) if want_h else None, _p(hs) if want_h else None)
     return (out, hq, hs) if want_h else out
+
+
+def combine(y, inv_perm, topk_w):
+    """Stage 5 alone: out [T, H] bf16 bits = bf16(sum_j topk_w[t, j] *
+    y[inv_perm[t*k + j]]) in fp32, ascending j, pairs with inv_perm < 0
+    skipped.  y [rows, H] fp32 (grouped rows), inv_perm [T*k], topk_w [T, k]."""
+    y = _c(y, np.float32)
+    w = _c(topk_w, np.float32)
+    T, k = w.shape
+    inv = _c(inv_perm, np.int32).reshape(T * k)
+    H = y.shape[1]
+    assert int(inv.max(initial=-1)) < y.shape[0]
+    out = np.zeros((T, H), np.uint16)
+    lib().oracle_combine(_p(y), _p(inv), _p(w), T, k, H, _p(out))
+    return out
 
 
 def groupwise_gemm_bf16(a, a_scale_kmajor, b, b_scale, m_indptr, is_gated: bool):

@@ -948,3 +948,28 @@ int oracle_num_threads(void) {
     return 1;
 #endif
 }
+
+/* ------------------------------------------------------------------ */
+/* Stage 5 on its own: the top-k weighted combine                        */
+/* ------------------------------------------------------------------ */
+
+/* The AlphaMoE page's last stage ("문제점: MoE Expert 계산의 병목", stage 5):
+ * out[t, c] = bf16( sum_j topk_w[t, j] * y[inv_perm[t*k + j], c] ), the
+ * products and the sum in fp32, slots in ascending j, pairs with
+ * inv_perm < 0 (dropped ids) skipped.  y [rows, H] fp32 in grouped-row order;
+ * out [T, H] bf16 bits.  The same loop ends oracle_moe_fused; here it takes a
+ * y from elsewhere (for example GEMM2 recomputed on another intermediate). */
+void oracle_combine(const float* y, const int32_t* inv_perm, const float* topk_w, int T, int k,
+                    int H, uint16_t* out) {
+    #pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t)
+        for (int c = 0; c < H; ++c) {
+            float acc = 0.0f;
+            for (int j = 0; j < k; ++j) {
+                int row = inv_perm[t * k + j];
+                if (row < 0) continue;
+                acc += topk_w[t * k + j] * y[(size_t)row * H + c];
+            }
+            out[(size_t)t * H + c] = f32_to_bf16(acc);
+        }
+}

@@ -25,6 +25,7 @@ from __future__ import annotations
 import math
 from dataclasses import dataclass
 
+import numpy as np
 import torch
 
 
@@ -106,6 +107,32 @@ def make_moe_inputs(cfg: MoEConfig, seed: int = 0, device="cpu", weights: bool =
         out["w2"], out["w2_scale"] = _expert_weights(cfg.E, cfg.H, cfg.I,
                                                      1.0 / math.sqrt(cfg.I), g, device)
     return out
+
+
+def _host(t: torch.Tensor, dtype) -> "np.ndarray":
+    return t.detach().contiguous().cpu().view(dtype).numpy()
+
+
+def compact_experts(inp: dict, tokens):
+    """Host copies (numpy) of the listed tokens' inputs and of only the
+    experts they use, with their routing renumbered into that compact expert
+    list: x as bf16 bits, topk_ids int32, topk_w fp32, weights as FP8 codes and
+    fp32 scales.  Lets a per-token check of a full-size workload move a few
+    experts to the host instead of all of them.  Ids outside [0, E) are kept
+    as they are."""
+    E = inp["w13"].shape[0]
+    sel = torch.as_tensor(tokens, device=inp["topk_ids"].device)
+    ids = inp["topk_ids"][sel]
+    valid = (ids >= 0) & (ids < E)
+    used = torch.unique(ids[valid]).to(torch.long)
+    remap = torch.full((E,), -1, dtype=torch.int32, device=ids.device)
+    remap[used] = torch.arange(len(used), dtype=torch.int32, device=ids.device)
+    local = torch.where(valid, remap[ids.clamp(0, E - 1)], ids)
+    return dict(
+        x=_host(inp["x"][sel.to(inp["x"].device)], torch.int16).view(np.uint16),
+        topk_ids=_host(local, torch.int32), topk_w=_host(inp["topk_w"][sel], torch.float32),
+        w13=_host(inp["w13"][used], torch.uint8), w13_scale=_host(inp["w13_scale"][used], torch.float32),
+        w2=_host(inp["w2"][used], torch.uint8), w2_scale=_host(inp["w2_scale"][used], torch.float32))
 
 
 def make_swiglu_input(M: int, K: int, variant: str = "normal", seed: int = 0, device="cpu"):

@@ -26,6 +26,37 @@ SCALE_RTOL = 2.0 ** -16
 OUT_REL_L2 = 1e-2
 OUT_MAX_ABS_RMS = 2e-2
 
+# Worst values seen by the comparisons of this test session (written out by
+# tests/conftest.py when MOE_PARITY_STATS names a file).
+STATS = {"scale_rel_max": 0.0, "code_match_min": 1.0, "out_rel_l2_max": 0.0,
+         "out_max_abs_rms_max": 0.0, "calls": 0}
+
+# Guard bytes after every output buffer the helpers hand to the library: any
+# write past the end of a buffer changes them.
+GUARD_BYTES = 4096
+GUARD_FILL = 0xA5
+
+
+def guarded_empty(shape, dtype, device, fill=None):
+    """A tensor of `shape` at the start of a larger buffer whose tail
+    (GUARD_BYTES) holds GUARD_FILL; returns (tensor, guard view)."""
+    n = 1
+    for d in shape:
+        n *= int(d)
+    esize = torch.empty((), dtype=dtype).element_size()
+    raw = torch.empty(n * esize + GUARD_BYTES, dtype=torch.uint8, device=device)
+    raw[n * esize:].fill_(GUARD_FILL)
+    t = raw[:n * esize].view(dtype).view(*shape)
+    if fill is not None:
+        t.fill_(fill)
+    return t, raw[n * esize:]
+
+
+def check_guards(guards: dict, what: str):
+    for name, g in guards.items():
+        bad = int((g != GUARD_FILL).sum())
+        assert bad == 0, f"{what}: {bad} guard bytes after {name} were overwritten"
+
 
 def bf16_bits(t: torch.Tensor) -> np.ndarray:
     return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
@@ -70,6 +101,7 @@ def compare_codes(gpu: np.ndarray, ref: np.ndarray, what: str):
         return 1.0
     same = gpu == ref
     frac = float(same.mean())
+    STATS["code_match_min"] = min(STATS["code_match_min"], frac)
     dist = np.abs(CODE_RANK[gpu] - CODE_RANK[ref])
     assert frac >= CODE_MATCH_MIN, f"{what}: only {frac:.5f} of codes identical"
     assert int(dist.max()) <= 1, f"{what}: a code differs by {int(dist.max())} steps"
@@ -80,6 +112,7 @@ def compare_scales(gpu: np.ndarray, ref: np.ndarray, what: str, rtol: float = SC
     gpu = np.asarray(gpu, np.float64)
     ref = np.asarray(ref, np.float64)
     rel = np.abs(gpu - ref) / np.maximum(np.abs(ref), 1e-30)
+    STATS["scale_rel_max"] = max(STATS["scale_rel_max"], float(rel.max(initial=0.0)))
     assert float(rel.max(initial=0.0)) <= rtol, f"{what}: scale rel diff {rel.max():.3e}"
 
 
@@ -93,6 +126,9 @@ def compare_out(gpu_bits: np.ndarray, ref_bits: np.ndarray, what: str):
         return 0.0, 0.0
     rel_l2 = float(np.linalg.norm(g - r) / np.linalg.norm(r))
     max_abs = float(np.abs(g - r).max() / rms)
+    STATS["out_rel_l2_max"] = max(STATS["out_rel_l2_max"], rel_l2)
+    STATS["out_max_abs_rms_max"] = max(STATS["out_max_abs_rms_max"], max_abs)
+    STATS["calls"] += 1
     assert rel_l2 <= OUT_REL_L2, f"{what}: relative L2 {rel_l2:.3e}"
     assert max_abs <= OUT_MAX_ABS_RMS, f"{what}: max abs {max_abs:.3e} x rms"
     return rel_l2, max_abs
@@ -104,7 +140,9 @@ def oracle_args(inp: dict):
 
 
 def run_fused(inp: dict, debug: bool = True):
-    """Runs moe_fp8_fused(_debug) on device tensors; returns host arrays."""
+    """Runs moe_fp8_fused(_debug) on device tensors; returns host arrays.
+    The workspace and every output buffer are followed by guard bytes that
+    are checked after the call."""
     x = inp["x"]
     T, H = x.shape
     E, I2, _ = inp["w13"].shape
@@ -112,39 +150,27 @@ def run_fused(inp: dict, debug: bool = True):
     k = inp["topk_ids"].shape[1]
     R = T * k
     dev = x.device
-    ws = torch.empty(moe.moe_workspace_size(T, H, I, E, k), dtype=torch.uint8, device=dev)
-    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    guards = {}
+    ws, guards["ws"] = guarded_empty((moe.moe_workspace_size(T, H, I, E, k),), torch.uint8, dev)
+    out, guards["out"] = guarded_empty((T, H), torch.bfloat16, dev)
     res = {}
     if debug:
-        m_indptr = torch.empty(E + 1, dtype=torch.int32, device=dev)
-        perm = torch.empty(max(R, 1), dtype=torch.int32, device=dev)
-        hq = torch.empty(max(R, 1), I, dtype=torch.uint8, device=dev)
-        hs = torch.empty(I // 128, max(R, 1), dtype=torch.float32, device=dev)
+        m_indptr, guards["m_indptr"] = guarded_empty((E + 1,), torch.int32, dev)
+        perm, guards["perm"] = guarded_empty((max(R, 1),), torch.int32, dev)
+        hq, guards["hq"] = guarded_empty((max(R, 1), I), torch.uint8, dev)
+        hs, guards["hs"] = guarded_empty((I // 128, max(R, 1)), torch.float32, dev)
         moe.moe_fp8_fused_debug(x, inp["topk_ids"], inp["topk_w"], inp["w13"], inp["w13_scale"],
-                                inp["w2"], inp["w2_scale"], out, ws, m_indptr, perm, hq, hs)
+                                inp["w2"], inp["w2_scale"], out, ws, m_indptr, perm, hq, hs,
+                                ws_bytes=moe.moe_workspace_size(T, H, I, E, k))
         st = moe.moe_get_device_status(ws)
         res.update(m_indptr=i32(m_indptr), perm=i32(perm)[:R], hq=u8(hq)[:R],
                    hs=f32(hs)[:, :R].T.copy())
     else:
         moe.moe_fp8_fused(x, inp["topk_ids"], inp["topk_w"], inp["w13"], inp["w13_scale"],
-                          inp["w2"], inp["w2_scale"], out, ws)
+                          inp["w2"], inp["w2_scale"], out, ws,
+                          ws_bytes=moe.moe_workspace_size(T, H, I, E, k))
         st = moe.moe_get_device_status(ws)
+    check_guards(guards, "fused layer")
     res["status"] = st
     res["out"] = bf16_bits(out)
     return res
-
-
-def compact_experts(inp: dict, tokens):
-    """Host copies of only the experts the listed tokens use, with the
-    routing of those tokens renumbered into the compact expert list."""
-    ids = inp["topk_ids"][torch.as_tensor(tokens, device=inp["topk_ids"].device)]
-    used = torch.unique(ids[(ids >= 0) & (ids < inp["w13"].shape[0])]).to(torch.long)
-    remap = torch.full((inp["w13"].shape[0],), -1, dtype=torch.int32, device=ids.device)
-    remap[used] = torch.arange(len(used), dtype=torch.int32, device=ids.device)
-    local = torch.where((ids >= 0) & (ids < inp["w13"].shape[0]), remap[ids.clamp(0)], ids)
-    sub = dict(
-        x=bf16_bits(inp["x"][torch.as_tensor(tokens, device=inp["x"].device)]),
-        topk_ids=i32(local), topk_w=f32(inp["topk_w"][torch.as_tensor(tokens, device=ids.device)]),
-        w13=u8(inp["w13"][used]), w13_scale=f32(inp["w13_scale"][used]),
-        w2=u8(inp["w2"][used]), w2_scale=f32(inp["w2_scale"][used]))
-    return sub

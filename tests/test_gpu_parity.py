@@ -32,12 +32,15 @@ def _route_gpu(ids_cpu: torch.Tensor, E: int):
     T, k = ids_cpu.shape
     R = T * k
     ids = ids_cpu.to(DEV)
-    m_indptr = torch.full((E + 1,), -7, dtype=torch.int32, device=DEV)
-    perm = torch.full((max(R, 1),), -7, dtype=torch.int32, device=DEV)
-    inv = torch.full((max(R, 1),), -7, dtype=torch.int32, device=DEV)
-    ws = torch.empty(moe.moe_route_workspace_size(T, k, E), dtype=torch.uint8, device=DEV)
-    moe.moe_route_permute(ids, E, m_indptr, perm, inv, ws)
+    guards = {}
+    m_indptr, guards["m_indptr"] = G.guarded_empty((E + 1,), torch.int32, DEV, fill=-7)
+    perm, guards["perm"] = G.guarded_empty((max(R, 1),), torch.int32, DEV, fill=-7)
+    inv, guards["inv_perm"] = G.guarded_empty((max(R, 1),), torch.int32, DEV, fill=-7)
+    ws, guards["ws"] = G.guarded_empty((moe.moe_route_workspace_size(T, k, E),), torch.uint8, DEV)
+    moe.moe_route_permute(ids, E, m_indptr, perm, inv, ws,
+                          ws_bytes=moe.moe_route_workspace_size(T, k, E))
     st = moe.moe_get_device_status(ws)
+    G.check_guards(guards, "routing")
     return G.i32(m_indptr), G.i32(perm)[:R], G.i32(inv)[:R], st
 
 
@@ -150,10 +153,11 @@ def _run_gemm(a, a_s, b, b_s, m_indptr, gated, tile_m, mode):
     bs_d = torch.from_numpy(b_s).to(DEV)
     mi = torch.from_numpy(m_indptr).to(DEV)
     n_out = N // 2 if gated else N
-    out = torch.full((R, n_out), float("nan"), dtype=torch.bfloat16, device=DEV)
+    out, guard = G.guarded_empty((R, n_out), torch.bfloat16, DEV, fill=float("nan"))
     moe.fp8_groupwise_moe_gemm(a_d, b_d, as_d, bs_d, mi, out, mode, (1, 128, 128), gated,
                                tile_m, -1)
     assert moe.moe_get_device_status(None) == moe.MOE_OK
+    G.check_guards({"out": guard}, f"grouped GEMM tile_m={tile_m}")
     return G.bf16_bits(out)
 
 
@@ -252,7 +256,7 @@ def _check_sampled(inp, tokens, what):
     m_o, p_o, i_o, _ = O.route_permute(G.i32(inp["topk_ids"]), E)
     assert np.array_equal(res["m_indptr"], m_o), what
     assert np.array_equal(res["perm"], p_o), what
-    sub = G.compact_experts(inp, tokens)
+    sub = synth.compact_experts(inp, tokens)
     out_o, hq_o, hs_o = O.moe_tokens(sub["x"], sub["topk_ids"], sub["topk_w"], sub["w13"],
                                      sub["w13_scale"], sub["w2"], sub["w2_scale"],
                                      np.arange(len(tokens), dtype=np.int32), want_h=True)
