@@ -373,11 +373,31 @@ def run_ours(args, cfg):
     e2e_run(args.steps)
     e_end.record(stream)
     torch.cuda.synchronize(dev)
-    clocks.stop()
     e2e_ms = e_start.elapsed_time(e_end)
 
+    # the decode workload (weight-streaming, HBM-bound) in the same run: its
+    # own seeded inputs, the same warm-up and number of timed steps
+    dec = None
+    if cfg.name == "prefill" and not args.no_decode:
+        dcfg = synth.CONFIGS["decode"]
+        dinp = synth.make_moe_inputs(dcfg, seed=rank, device=dev)
+        dws = torch.empty(moe.moe_workspace_size(dcfg.T, dcfg.H, dcfg.I, dcfg.E, dcfg.k),
+                          dtype=torch.uint8, device=dev)
+        dout = torch.empty(dcfg.T, dcfg.H, dtype=torch.bfloat16, device=dev)
+        if pg:
+            pg.barrier()
+        dec_ms, dec_stages = timed_layer(
+            lambda: moe.moe_fp8_fused(dinp["x"], dinp["topk_ids"], dinp["topk_w"], dinp["w13"],
+                                      dinp["w13_scale"], dinp["w2"], dinp["w2_scale"], dout, dws,
+                                      stream=stream), args, dws, stream, dev)
+        dec = (dcfg, work_counts(dcfg, dinp["topk_ids"]), dec_stages)
+        del dinp, dws, dout
+    else:
+        dec_ms = 0.0
+    clocks.stop()
+
     # max over ranks
-    elapsed_ms, e2e_ms = max_over_ranks([elapsed_ms, e2e_ms], pg, dev)
+    elapsed_ms, e2e_ms, dec_ms = max_over_ranks([elapsed_ms, e2e_ms, dec_ms], pg, dev)
 
     if rank == 0:
         ms_step = elapsed_ms / args.steps
@@ -424,6 +444,21 @@ def run_ours(args, cfg):
             "gpu_launches": kernels_per_layer(T, k) * args.steps,
             "clocks": clocks.summary(),
         }
+        if dec is not None:
+            dcfg, dc, dst = dec
+            d_gbs = dc["bytes"] / (dec_ms * 1e-3) / 1e9
+            g1_gbs_d = dc["g1_bytes"] / (float(dst[2]) * 1e-3) / 1e9
+            line["decode"] = {
+                "workload": workload_desc(dcfg), "us": dec_ms * 1e3, "steps": args.steps,
+                "tflops": dc["flops"] / (dec_ms * 1e-3) / 1e12, "gbs": d_gbs,
+                "hbm_frac": d_gbs / hbm, "alg_bytes": dc["bytes"],
+                "experts_touched": dc["touched"],
+                "stages_us": {n: float(v) * 1e3 for n, v in
+                              zip(["route", "quant", "gemm1", "gemm2", "finish"], dst)},
+                "gemm1_gbs": g1_gbs_d, "gemm1_hbm_frac": g1_gbs_d / hbm,
+                "peak_source": f"{src} copy bandwidth",
+                "l2": "inputs larger than L2 (no flush)",
+                "gpu_launches": kernels_per_layer(dcfg.T, dcfg.k) * args.steps}
         if world == 1 and not args.no_cpu_baseline:
             import oracle
             oracle.build()
@@ -471,14 +506,28 @@ def run_swiglu(args):
                 torch.cuda.synchronize()
                 times.append(a.elapsed_time(b))
             ms = statistics.median(times)
+            # back to back: many launches between two events (no flush), the
+            # per-launch cost of a stream of calls (L2-warm inputs)
+            reps = 1000 if M * K < (1 << 24) else 50
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(reps):
+                moe.swiglu_mxfp8_quant(x, out, sc)
+            b.record()
+            torch.cuda.synchronize()
+            ms_b2b = a.elapsed_time(b) / reps
             nbytes = 4 * M * K + M * K + M * K // 32
             res.append({"M": M, "K": K, "input": variant, "us": ms * 1e3,
-                        "gbs": nbytes / (ms * 1e-3) / 1e9, "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / hbm})
+                        "gbs": nbytes / (ms * 1e-3) / 1e9, "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / hbm,
+                        "us_back_to_back": ms_b2b * 1e3, "back_to_back_launches": reps})
     line = {"metric": "SwiGLU+MXFP8 quantisation µs and GB/s as % of HBM", "unit": "us",
             "higher_is_better": False, "steps": args.steps, "warmup": args.warmup,
             "peak_hbm_gbs": hbm, "peak_source": src, "data": "synthetic",
             "config": {"workload": "bf16 [M,2K] (gate|up) -> FP8 [M,K] + E8M0 per 32",
-                       "l2": "flushed before every timed launch"}, "results": res}
+                       "l2": "us: flushed before every timed launch (median of single launches); "
+                             "us_back_to_back: mean over back-to-back launches, no flush"},
+            "results": res}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -748,6 +797,8 @@ def main():
                     choices=sorted(synth.CONFIGS) + sorted(PROFILE_SLICES))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="with the prefill workload: skip the decode workload's timing")
     ap.add_argument("--op", default="moe", choices=["moe", "swiglu_mxfp8", "mxfp8_gemm", "mxfp8_moe",
                                                      "nvfp4_gemm", "nvfp4_moe"],
                     help="any other than moe: time that op instead")

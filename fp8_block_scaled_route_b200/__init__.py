@@ -27,7 +27,8 @@ __all__ = [
     "mxfp8_tile_scales", "moe_mxfp8_fused", "moe_mxfp8_fused_debug", "moe_router_topk",
     "nvfp4_moe_gemm", "nvfp4_tile_scales", "moe_nvfp4_fused", "moe_nvfp4_fused_debug",
     "nvfp4_quantize", "moe_tactic_tune_gemm", "moe_tactic_lookup", "moe_tactic_store",
-    "moe_tactic_clear",
+    "moe_tactic_clear", "moe_ep_workspace_size", "moe_ep_plan", "moe_ep_pack",
+    "moe_fp8_expert_rows_workspace_size", "moe_fp8_expert_rows", "moe_combine",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -50,6 +51,8 @@ EXPORTS = (
     "moe_mxfp8_fused", "moe_mxfp8_fused_debug", "moe_router_topk", "nvfp4_moe_gemm",
     "nvfp4_tile_scales", "moe_nvfp4_fused", "moe_nvfp4_fused_debug", "nvfp4_quantize",
     "moe_tactic_tune_gemm", "moe_tactic_lookup", "moe_tactic_store", "moe_tactic_clear",
+    "moe_ep_workspace_size", "moe_ep_plan", "moe_ep_pack", "moe_fp8_expert_rows_workspace_size",
+    "moe_fp8_expert_rows", "moe_combine",
 )
 
 _lib = None
@@ -131,6 +134,18 @@ def lib():
     L.moe_route_permute_noalloc.argtypes = [P, I, I, I, P, P, P, P]
     L.moe_set_stage_events.restype = I
     L.moe_set_stage_events.argtypes = [ctypes.POINTER(P), I]
+    L.moe_ep_workspace_size.restype = Z
+    L.moe_ep_workspace_size.argtypes = [I, I, I]
+    L.moe_ep_plan.restype = I
+    L.moe_ep_plan.argtypes = [P, I, I, I, I, P, P, P, P, Z, P]
+    L.moe_ep_pack.restype = I
+    L.moe_ep_pack.argtypes = [P, P, P] + [I] * 7 + [P, P, P, P]
+    L.moe_fp8_expert_rows_workspace_size.restype = Z
+    L.moe_fp8_expert_rows_workspace_size.argtypes = [I] * 4
+    L.moe_fp8_expert_rows.restype = I
+    L.moe_fp8_expert_rows.argtypes = [P, P, P, I, P, P, P, P, P, I, I, I, P, Z, P]
+    L.moe_combine.restype = I
+    L.moe_combine.argtypes = [P, P, P, I, I, I, P, P]
     _lib = L
     return L
 
@@ -454,3 +469,65 @@ def moe_set_stage_events(events) -> int:
 
 def moe_get_device_status(ws=None, *, stream=None) -> int:
     return int(lib().moe_get_device_status(_ptr(ws), _stream(stream)))
+
+
+# ---------------------------------------------------------------- expert parallelism
+def moe_ep_workspace_size(T: int, k: int, G: int) -> int:
+    return int(lib().moe_ep_workspace_size(T, k, G))
+
+
+def moe_ep_plan(topk_ids, E: int, G: int, send_indptr, send_pair, slot_of_pair, ws, ws_bytes=None,
+                *, T=None, k=None, stream=None, check=True) -> int:
+    if T is None or k is None:
+        T, k = topk_ids.shape
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size()
+    st = lib().moe_ep_plan(_ptr(topk_ids), T, k, E, G, _ptr(send_indptr), _ptr(send_pair),
+                           _ptr(slot_of_pair), _ptr(ws), ws_bytes, _stream(stream))
+    return _check(st, "moe_ep_plan", check)
+
+
+def moe_ep_pack(x, topk_ids, slot_of_pair, E: int, G: int, S: int, xq_send, xs_send, eid_send, *,
+                dims=None, stream=None, check=True) -> int:
+    """dims = (T, H, k) when raw addresses are passed."""
+    if dims is None:
+        T, H = x.shape
+        k = topk_ids.shape[1]
+    else:
+        T, H, k = dims
+    st = lib().moe_ep_pack(_ptr(x), _ptr(topk_ids), _ptr(slot_of_pair), T, H, k, E, G, S,
+                           _ptr(xq_send), _ptr(xs_send), _ptr(eid_send), _stream(stream))
+    return _check(st, "moe_ep_pack", check)
+
+
+def moe_fp8_expert_rows_workspace_size(n: int, H: int, I: int, E: int) -> int:
+    return int(lib().moe_fp8_expert_rows_workspace_size(n, H, I, E))
+
+
+def moe_fp8_expert_rows(xq, xs, eid, w13, w13_scale, w2, w2_scale, y, ws, ws_bytes=None, *,
+                        dims=None, stream=None, check=True) -> int:
+    """dims = (n, H, I, E) when raw addresses are passed."""
+    if dims is None:
+        n, H = xq.shape
+        E, I2, _ = w13.shape
+        I = I2 // 2
+    else:
+        n, H, I, E = dims
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size()
+    st = lib().moe_fp8_expert_rows(_ptr(xq), _ptr(xs), _ptr(eid), n, _ptr(w13), _ptr(w13_scale),
+                                   _ptr(w2), _ptr(w2_scale), _ptr(y), H, I, E, _ptr(ws), ws_bytes,
+                                   _stream(stream))
+    return _check(st, "moe_fp8_expert_rows", check)
+
+
+def moe_combine(y, row_of_pair, topk_w, out, *, dims=None, stream=None, check=True) -> int:
+    """dims = (T, k, H) when raw addresses are passed."""
+    if dims is None:
+        T, k = topk_w.shape
+        H = out.shape[1]
+    else:
+        T, k, H = dims
+    st = lib().moe_combine(_ptr(y), _ptr(row_of_pair), _ptr(topk_w), T, k, H, _ptr(out),
+                           _stream(stream))
+    return _check(st, "moe_combine", check)

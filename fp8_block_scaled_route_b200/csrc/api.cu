@@ -86,7 +86,9 @@ FusedWs fused_layout(int T, int H, int I, int E, int k) {
     w.xs = o;         o += up256(sizeof(float) * R * (H / 128));
     w.hq = o;         o += up256(R * I);
     w.hs = o;         o += up256(sizeof(float) * R * (I / 128));
-    w.out_acc = o;    o += up256(sizeof(float) * static_cast<size_t>(T) * H);
+    // FP8 layer: y [R, H] fp32, one row per pair (GEMM2's output); MXFP8 and
+    // NVFP4 layers: their fp32 combine buffer [T, H] at the same place
+    w.out_acc = o;    o += up256(sizeof(float) * R * H);
     w.total = o;
     return w;
 }
@@ -293,7 +295,7 @@ static int fused_impl(const void* x, const int32_t* topk_ids, const float* topk_
     if (st) return st;
     stage_mark(1, s);
     if (T > 0) {
-        st = launch_quant_scatter(x, T, H, k, R, inv_perm, xq, xs, out_acc, s);
+        st = launch_quant_scatter(x, T, H, k, R, inv_perm, xq, xs, nullptr, s);
         if (st) return st;
         stage_mark(2, s);
         const unsigned long long tmo = g_timeout_ns.load();
@@ -309,16 +311,19 @@ static int fused_impl(const void* x, const int32_t* topk_ids, const float* topk_
         st = launch_grouped_gemm(g1, s);
         if (st) return st;
         stage_mark(3, s);
+        // GEMM2 writes each pair's row y once, in grouped order; the combine
+        // then sums each token's k rows in ascending slot order
+        float* y = out_acc;
         GemmArgs g2{};
         g2.a = hq; g2.b = w2; g2.R = R; g2.N = H; g2.K = I; g2.E = E;
         g2.a_scale = hs; g2.as_row = 1; g2.as_kb = R; g2.b_scale = w2_scale;
-        g2.m_indptr = m_indptr; g2.epi = EPI_COMBINE; g2.tile_m = tm2;
-        g2.perm = perm; g2.topk_w = topk_w; g2.topk = k; g2.out_acc = out_acc; g2.out_ld = H;
+        g2.m_indptr = m_indptr; g2.epi = EPI_Y32; g2.tile_m = tm2;
+        g2.y = y; g2.ldy = H;
         g2.status = status; g2.timeout_ns = tmo; g2.num_sms = d->sms;
         st = launch_grouped_gemm(g2, s);
         if (st) return st;
         stage_mark(4, s);
-        st = launch_f32_to_bf16(out_acc, out, static_cast<long long>(T) * H, d->sms, s);
+        st = launch_combine(y, inv_perm, topk_w, T, k, H, out, s);
         if (st) return st;
         stage_mark(5, s);
     }
@@ -803,6 +808,163 @@ int swiglu_mxfp8_quant(const void* in, void* out, uint8_t* scale, int M, int K, 
     if (cudaMemsetAsync(d->lib_status, 0, sizeof(int) * kStatusInts, s) != cudaSuccess)
         return MOE_ERR_CUDA;
     return launch_swiglu_mxfp8(in, out, scale, M, K, d->sms, s);
+}
+
+// ---------------------------------------------------------------- expert parallelism
+namespace {
+
+// Workspace of moe_ep_plan: status word, owner rank per pair, chunk histograms.
+struct EpPlanWs {
+    size_t status, owner, chunk_hist, total;
+};
+EpPlanWs ep_plan_layout(int T, int k, int G) {
+    const size_t R = static_cast<size_t>(T) * k;
+    const size_t nchunks = (R + kRouteChunk - 1) / kRouteChunk;
+    EpPlanWs w{};
+    size_t o = 0;
+    w.status = o;     o += up256(sizeof(int) * kStatusInts);
+    w.owner = o;      o += up256(sizeof(int32_t) * R);
+    w.chunk_hist = o; o += up256(sizeof(int32_t) * nchunks * G);
+    w.total = o;
+    return w;
+}
+
+// Workspace of moe_fp8_expert_rows, in carve order.
+struct ExpertRowsWs {
+    size_t status, m_indptr, chunk_hist, perm, inv_perm, xq, xs, hq, hs, total;
+};
+ExpertRowsWs expert_rows_layout(int n, int H, int I, int E) {
+    const size_t N = static_cast<size_t>(n);
+    const size_t nchunks = (N + kRouteChunk - 1) / kRouteChunk;
+    ExpertRowsWs w{};
+    size_t o = 0;
+    w.status = o;     o += up256(sizeof(int) * kStatusInts);
+    w.m_indptr = o;   o += up256(sizeof(int32_t) * (E + 1));
+    w.chunk_hist = o; o += up256(sizeof(int32_t) * nchunks * E);
+    w.perm = o;       o += up256(sizeof(int32_t) * N);
+    w.inv_perm = o;   o += up256(sizeof(int32_t) * N);
+    w.xq = o;         o += up256(N * H);
+    w.xs = o;         o += up256(sizeof(float) * N * (H / 128));
+    w.hq = o;         o += up256(N * I);
+    w.hs = o;         o += up256(sizeof(float) * N * (I / 128));
+    w.total = o;
+    return w;
+}
+
+}  // namespace
+
+size_t moe_ep_workspace_size(int T, int k, int G) {
+    if (T < 0 || k < 1 || G < 1) return 0;
+    return ep_plan_layout(T, k, G).total;
+}
+
+int moe_ep_plan(const int32_t* topk_ids, int T, int k, int E, int G, int32_t* send_indptr,
+                int32_t* send_pair, int32_t* slot_of_pair, void* ws, size_t ws_bytes,
+                moe_stream_t stream) {
+    if (T < 0 || k < 1 || E < 1 || G < 1 || E % G || G > MOE_MAX_EXPERTS || E > MOE_MAX_EXPERTS)
+        return MOE_ERR_INVALID_ARG;
+    if (!send_indptr || !ws || (T > 0 && (!topk_ids || !send_pair || !slot_of_pair)))
+        return MOE_ERR_INVALID_ARG;
+    const EpPlanWs L = ep_plan_layout(T, k, G);
+    if (ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+    const DevInfo* d = dev_info();
+    if (int st = check_device(d)) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    char* b = static_cast<char*>(ws);
+    int* status = reinterpret_cast<int*>(b + L.status);
+    int32_t* owner = reinterpret_cast<int32_t*>(b + L.owner);
+    if (cudaMemsetAsync(status, 0, sizeof(int) * kStatusInts, s) != cudaSuccess) return MOE_ERR_CUDA;
+    const long long R = static_cast<long long>(T) * k;
+    int st = launch_ep_owner(topk_ids, R, E, E / G, owner, d->sms, s);
+    if (st) return st;
+    RouteArgs ra{owner, T, k, G, send_indptr, send_pair, slot_of_pair,
+                 reinterpret_cast<int32_t*>(b + L.chunk_hist), status};
+    return launch_route_permute(ra, s);
+}
+
+int moe_ep_pack(const void* x, const int32_t* topk_ids, const int32_t* slot_of_pair, int T, int H,
+                int k, int E, int G, int S, uint8_t* xq_send, float* xs_send, int32_t* eid_send,
+                moe_stream_t stream) {
+    if (T < 0 || H <= 0 || H % 128 || k < 1 || E < 1 || G < 1 || E % G || S < 0)
+        return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !topk_ids || !slot_of_pair)) return MOE_ERR_INVALID_ARG;
+    if (S > 0 && (!xq_send || !xs_send || !eid_send)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(xq_send) || (reinterpret_cast<uintptr_t>(xs_send) & 3))
+        return MOE_ERR_INVALID_ARG;
+    const DevInfo* d = dev_info();
+    if (int st = check_device(d)) return st;
+    return launch_ep_pack(x, topk_ids, T, H, k, S, slot_of_pair, E / G, xq_send, xs_send, eid_send,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t moe_fp8_expert_rows_workspace_size(int n, int H, int I, int E) {
+    if (n < 0 || H <= 0 || I <= 0 || E < 1) return 0;
+    return expert_rows_layout(n, H, I, E).total;
+}
+
+int moe_fp8_expert_rows(const uint8_t* xq, const float* xs, const int32_t* eid, int n,
+                        const void* w13, const float* w13_scale, const void* w2,
+                        const float* w2_scale, float* y, int H, int I, int E, void* ws,
+                        size_t ws_bytes, moe_stream_t stream) {
+    if (n < 0 || H <= 0 || I <= 0 || H % 128 || I % 128 || E < 1) return MOE_ERR_INVALID_ARG;
+    if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+    if (!ws) return MOE_ERR_INVALID_ARG;
+    const ExpertRowsWs L = expert_rows_layout(n, H, I, E);
+    if (ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+    if (n > 0) {
+        if (!xq || !xs || !eid || !w13 || !w13_scale || !w2 || !w2_scale || !y)
+            return MOE_ERR_INVALID_ARG;
+        if (!aligned16(xq) || !aligned16(w13) || !aligned16(w2) || !aligned16(y))
+            return MOE_ERR_INVALID_ARG;
+    }
+    const DevInfo* d = dev_info();
+    if (int st = check_device(d)) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    char* b = static_cast<char*>(ws);
+    int* status = reinterpret_cast<int*>(b + L.status);
+    int32_t* m_indptr = reinterpret_cast<int32_t*>(b + L.m_indptr);
+    int32_t* perm = reinterpret_cast<int32_t*>(b + L.perm);
+    int32_t* inv_perm = reinterpret_cast<int32_t*>(b + L.inv_perm);
+    uint8_t* xq_g = reinterpret_cast<uint8_t*>(b + L.xq);
+    float* xs_g = reinterpret_cast<float*>(b + L.xs);
+    uint8_t* hq = reinterpret_cast<uint8_t*>(b + L.hq);
+    float* hs = reinterpret_cast<float*>(b + L.hs);
+    if (cudaMemsetAsync(status, 0, sizeof(int) * kStatusInts, s) != cudaSuccess) return MOE_ERR_CUDA;
+    // rows grouped by local expert (a stable sort of the row index)
+    RouteArgs ra{eid, n, 1, E, m_indptr, perm, inv_perm,
+                 reinterpret_cast<int32_t*>(b + L.chunk_hist), status};
+    int st = launch_route_permute(ra, s);
+    if (st || n == 0) return st;
+    st = launch_gather_rows(xq, xs, n, H, perm, n, m_indptr + E, xq_g, xs_g, s);
+    if (st) return st;
+    const unsigned long long tmo = g_timeout_ns.load();
+    const int tm1 = fit_tile_to_k(choose_tile_m(n, 2 * I, H, E, 1, d->sms), H);
+    const int tm2 = fit_tile_to_k(choose_tile_m(n, H, I, E, 0, d->sms), I);
+    GemmArgs g1{};
+    g1.a = xq_g; g1.b = w13; g1.R = n; g1.N = 2 * I; g1.K = H; g1.E = E;
+    g1.a_scale = xs_g; g1.as_row = 1; g1.as_kb = n; g1.b_scale = w13_scale;
+    g1.m_indptr = m_indptr; g1.epi = EPI_SWIGLU_QUANT; g1.tile_m = tm1;
+    g1.hq = hq; g1.hs = hs; g1.status = status; g1.timeout_ns = tmo; g1.num_sms = d->sms;
+    st = launch_grouped_gemm(g1, s);
+    if (st) return st;
+    // grouped row r is received row perm[r]: GEMM2 writes it there
+    GemmArgs g2{};
+    g2.a = hq; g2.b = w2; g2.R = n; g2.N = H; g2.K = I; g2.E = E;
+    g2.a_scale = hs; g2.as_row = 1; g2.as_kb = n; g2.b_scale = w2_scale;
+    g2.m_indptr = m_indptr; g2.epi = EPI_Y32; g2.tile_m = tm2;
+    g2.y = y; g2.ldy = H; g2.rowmap = perm;
+    g2.status = status; g2.timeout_ns = tmo; g2.num_sms = d->sms;
+    return launch_grouped_gemm(g2, s);
+}
+
+int moe_combine(const float* y, const int32_t* row_of_pair, const float* topk_w, int T, int k, int H,
+                void* out, moe_stream_t stream) {
+    if (T < 0 || k < 1 || H <= 0 || H % 8) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!y || !topk_w || !out)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(y) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    const DevInfo* d = dev_info();
+    if (int st = check_device(d)) return st;
+    return launch_combine(y, row_of_pair, topk_w, T, k, H, out, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int moe_get_device_status(const void* ws, moe_stream_t stream) {

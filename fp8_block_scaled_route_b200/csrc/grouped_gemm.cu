@@ -86,7 +86,10 @@ struct Cfg {
     // TMEM accumulator slots, each holding both 128-row weight blocks of one
     // K block: direct = 2 slots of 256 columns (one N = 256 MMA per K step);
     // swapped = up to 16 slots of 2 x BT columns, so the weight stream keeps
-    // going while the epilogue finishes a tile.
+    // going while the epilogue finishes a tile.  (Four 128-column slots with
+    // two N = 128 MMA groups per K block, each with its own commit and
+    // release, measured 15% slower for GEMM1: twice the handshakes per K
+    // block and the token tile read twice by the tensor core.)
     static constexpr int TSLOTS = SWAP ? (512 / (2 * BT) > 16 ? 16 : 512 / (2 * BT)) : 2;
     static constexpr int TBUF_COLS = SWAP ? 2 * BT : 256;
     static constexpr int MAX_NKB = SWAP ? AS_TILE_BYTES / (4 * BT) : 1 << 20;
@@ -101,6 +104,11 @@ struct Cfg {
     static_assert(SMEM_BYTES <= kSmemLimit, "shared memory budget");
     static_assert(STAGE_BYTES % 1024 == 0 && A_OFF % 1024 == 0 && B_OFF % 1024 == 0,
                   "operand tiles must be 1024-byte aligned for the 128-byte swizzle");
+    // EPI_Y32 (direct): the last pipeline stage and the combine transpose
+    // area, contiguous, become the staging buffers of the output stores: two
+    // 4 KB boxes (32 rows x 32 fp32, 128-byte swizzle) per epilogue warp.
+    static constexpr int Y_STAGE_BYTES = SWAP ? 0 : EPI_WARPS * 2 * 4096;
+    static_assert(SWAP || STAGE_BYTES + CST_BYTES >= Y_STAGE_BYTES, "output staging does not fit");
 };
 
 struct KParams {
@@ -119,9 +127,13 @@ struct KParams {
     int topk;
     float* out_acc;
     int out_ld;
+    float* y;
+    int ldy;
+    const int32_t* rowmap;
     __nv_bfloat16* out_bf16;
     int* status;
     unsigned long long timeout_ns;
+    int nstages;  // pipeline stages in use (EPI_Y32 direct: one less, its space stages the output)
 };
 
 struct Smem {
@@ -132,6 +144,7 @@ struct Smem {
     float* xch;   // epilogue exchange area
     float* scales;  // direct kernel: kScaleSlots x {a_scale[128], b_scale[2], pad[2]}
     float* cstage;  // direct combine transpose tiles
+    uint8_t* ystage;  // direct EPI_Y32 output staging (last stage + cstage)
     uint64_t* full;
     uint64_t* empty;
     uint64_t* tfull;
@@ -151,6 +164,9 @@ __device__ __forceinline__ Smem carve(uint8_t* base) {
     uint8_t* p = base;
     s.stages = p;
     p += C::STAGES * C::STAGE_BYTES;
+    s.cstage = reinterpret_cast<float*>(p);
+    s.ystage = base + (C::STAGES - 1) * C::STAGE_BYTES;
+    p += C::CST_BYTES;
     s.as_tile = reinterpret_cast<float*>(p);
     p += C::AS_TILE_BYTES;
     s.tstart = reinterpret_cast<int*>(p);
@@ -160,8 +176,6 @@ __device__ __forceinline__ Smem carve(uint8_t* base) {
     p += C::XCH_BYTES;
     s.scales = reinterpret_cast<float*>(p);
     p += C::SCALE_BYTES;
-    s.cstage = reinterpret_cast<float*>(p);
-    p += C::CST_BYTES;
     uint64_t* bars = reinterpret_cast<uint64_t*>(p);
     s.full = bars;
     s.empty = bars + 8;
@@ -339,7 +353,7 @@ __device__ void producer_role(const CUtensorMap* tmA, const CUtensorMap* tmB, co
             __syncwarp();
             armed |= 1u << stage;
             armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-            if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+            if (++stage == static_cast<uint32_t>(p.nstages)) { stage = 0; phase ^= 1; }
         }
     }
     // make sure no copy is still writing into shared memory when the CTA exits
@@ -389,7 +403,7 @@ __device__ void mma_role(const KParams& p, const Smem& s, const WaitCtl& wc, uin
             }
             __syncwarp();
             if (++j == C::TSLOTS) { j = 0; jphase ^= 1; }
-            if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+            if (++stage == static_cast<uint32_t>(p.nstages)) { stage = 0; phase ^= 1; }
         }
     }
     // every MMA this warp issued must be complete before TMEM is freed; the
@@ -452,7 +466,7 @@ __device__ __forceinline__ void ffma_chunk(float2* acc, const uint32_t (&v)[32],
 // Direct orientation epilogue: thread = one token row, 128 of 256 columns.
 template <int EPI>
 __device__ void epilogue_direct(const KParams& p, const Smem& s, const WaitCtl& wc,
-                                uint32_t tmem_base) {
+                                uint32_t tmem_base, const CUtensorMap* tmY) {
     constexpr bool GATED = (EPI == EPI_SWIGLU_BF16 || EPI == EPI_SWIGLU_QUANT);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = warp & 3;          // TMEM lane quarter this warp may access
@@ -464,6 +478,7 @@ __device__ void epilogue_direct(const KParams& p, const Smem& s, const WaitCtl& 
     // second 128 output columns).
     const int colg = g * 64;
     uint32_t tj = 0, tjphase = 0, ephase = 0, slot = 0, sphase = 0;
+    uint32_t ybuf = 0;  // EPI_Y32: output boxes staged so far by this warp
     const int total = total_tiles(s, p);
     const int nkb = p.nkb;
     float2 acc[64];
@@ -593,6 +608,54 @@ __device__ void epilogue_direct(const KParams& p, const Smem& s, const WaitCtl& 
                                        v.x, v.y, v.z, v.w);
                     }
                     __syncwarp();
+                }
+            }
+        } else if constexpr (EPI == EPI_Y32) {
+            // The warp's 32 rows x 128 columns leave as four 32 x 32 fp32
+            // boxes through two 4 KB shared-memory buffers and TMA stores,
+            // which the TMA unit drains while the warp goes on with the next
+            // tile.  Buffer layout = the 128-byte swizzle of the tensor map:
+            // 16-byte chunk c of row r sits at chunk c ^ (r % 8), so the eight
+            // lanes of each store phase hit eight different bank groups.  A
+            // quarter with fewer than 32 valid rows (the tile's last rows
+            // belong to the next expert) is written with plain stores.
+            uint8_t* const wbuf = s.ystage + (warp - 4) * 8192;
+            const int rows_here = tl.rows - q * 32;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int blk = c >> 1;
+                if (blk == 1 && !v1) break;
+                const float* a = accf + blk * 64 + (c & 1) * 32;
+                const int col = tl.nt * 256 + blk * 128 + colg + (c & 1) * 32;
+                if (p.rowmap) {
+                    // rows go to scattered places: plain stores of the thread's own row
+                    if (row_ok) {
+                        float4* dst = reinterpret_cast<float4*>(
+                            p.y + static_cast<long long>(__ldg(p.rowmap + row)) * p.ldy + col);
+#pragma unroll
+                        for (int c4 = 0; c4 < 8; ++c4)
+                            dst[c4] = make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]);
+                    }
+                } else if (rows_here >= 32) {
+                    uint8_t* buf = wbuf + (ybuf & 1u) * 4096;
+                    if (lane == 0) bulk_wait_group_read<1>();  // the box staged two boxes ago is read
+                    __syncwarp();
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4)
+                        *reinterpret_cast<float4*>(buf + lane * 128 + ((c4 ^ (lane & 7)) << 4)) =
+                            make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(tmY, buf, col, tl.row0 + q * 32);
+                        bulk_commit_group();
+                    }
+                    ++ybuf;
+                } else if (lane < rows_here) {
+                    float4* dst = reinterpret_cast<float4*>(p.y + static_cast<long long>(row) * p.ldy + col);
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4)
+                        dst[c4] = make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]);
                 }
             }
         } else if constexpr (EPI == EPI_BF16) {
@@ -760,6 +823,17 @@ __device__ void epilogue_swap(const KParams& p, const Smem& s, const WaitCtl& wc
                     if (wt.v1) red_add(rowp + colB, wgt * acc1[j]);
                 }
             }
+        } else if constexpr (EPI == EPI_Y32) {
+            const int colA = tl.nt * 256 + w;
+#pragma unroll
+            for (int j = 0; j < BT; ++j) {
+                if (j < tl.rows) {
+                    const int r = tl.row0 + j;
+                    float* rowp = p.y + static_cast<long long>(p.rowmap ? __ldg(p.rowmap + r) : r) * p.ldy;
+                    rowp[colA] = acc0[j];
+                    if (wt.v1) rowp[colA + 128] = acc1[j];
+                }
+            }
         } else if constexpr (EPI == EPI_BF16) {
             const int colA = tl.nt * 256 + w;
 #pragma unroll
@@ -787,7 +861,8 @@ __device__ void epilogue_swap(const KParams& p, const Smem& s, const WaitCtl& wc
 template <int BT, int EPI>
 __global__ void __launch_bounds__(Cfg<BT>::THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB, const KParams p) {
+                        const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmY, const KParams p) {
     using C = Cfg<BT>;
     constexpr bool GATED = (EPI == EPI_SWIGLU_BF16 || EPI == EPI_SWIGLU_QUANT);
     extern __shared__ uint8_t smem_raw[];
@@ -815,6 +890,7 @@ __global__ void __launch_bounds__(Cfg<BT>::THREADS, 1)
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        if constexpr (EPI == EPI_Y32 && !C::SWAP) tma_prefetch_desc(&tmY);
     }
     if (warp == 1) {
         tmem_alloc(s.tmem, C::TMEM_COLS);
@@ -865,7 +941,12 @@ __global__ void __launch_bounds__(Cfg<BT>::THREADS, 1)
     } else {
         if constexpr (!C::SWAP) {
             setmaxnreg_inc<kDirectHighRegs>();
-            epilogue_direct<EPI>(p, s, wc, tmem_base);
+            epilogue_direct<EPI>(p, s, wc, tmem_base, &tmY);
+            // output boxes still being stored read this CTA's shared memory
+            if constexpr (EPI == EPI_Y32) {
+                if (lane == 0) bulk_wait_group<0>();
+                __syncwarp();
+            }
         } else {
             epilogue_swap<BT, EPI>(p, s, wc, tmem_base);
         }
@@ -937,6 +1018,22 @@ bool make_map(CUtensorMap* out, const void* ptr, long long rows, long long cols,
     return true;
 }
 
+// 2-D map over a row-major fp32 matrix [rows, cols] (cols % 4 == 0, 16-byte
+// aligned rows) with boxes of 32 rows x 32 columns (128 bytes) and the
+// 128-byte swizzle, for the output stores of EPI_Y32.  Not cached: the
+// output buffer changes from call to call more often than the weights.
+bool make_map_f32_out(CUtensorMap* out, const void* ptr, long long rows, long long cols) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 4};
+    cuuint32_t box[2] = {32u, 32u};
+    cuuint32_t es[2] = {1u, 1u};
+    return fn(out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 bool make_tma_map_fp8(CUtensorMap* out, const void* ptr, long long rows, long long cols,
@@ -947,8 +1044,8 @@ bool make_tma_map_fp8(CUtensorMap* out, const void* ptr, long long rows, long lo
 namespace {
 
 template <int BT, int EPI>
-int launch_inst(const CUtensorMap& ma, const CUtensorMap& mb, const KParams& kp, int num_sms,
-                cudaStream_t stream) {
+int launch_inst(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& my,
+                const KParams& kp, int num_sms, cudaStream_t stream) {
     using C = Cfg<BT>;
     auto kern = grouped_gemm_kernel<BT, EPI>;
     static int configured_dev = -1;  // per-instance one-time set-up (device 0 assumed shared)
@@ -969,18 +1066,23 @@ int launch_inst(const CUtensorMap& ma, const CUtensorMap& mb, const KParams& kp,
         configured_dev = dev;
     }
     if (!checked) return ST_UNSUPPORTED;
-    kern<<<num_sms, C::THREADS, C::SMEM_BYTES, stream>>>(ma, mb, kp);
+    kern<<<num_sms, C::THREADS, C::SMEM_BYTES, stream>>>(ma, mb, my, kp);
     return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
 }
 
 template <int BT>
-int launch_bt(int epi, const CUtensorMap& ma, const CUtensorMap& mb, const KParams& kp, int num_sms,
-              cudaStream_t stream) {
+int launch_bt(int epi, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& my,
+              KParams kp, int num_sms, cudaStream_t stream) {
+    // direct EPI_Y32 gives its last pipeline stage to the output staging
+    kp.nstages = (!Cfg<BT>::SWAP && epi == EPI_Y32) ? Cfg<BT>::STAGES - 1 : Cfg<BT>::STAGES;
     switch (epi) {
-        case EPI_BF16: return launch_inst<BT, EPI_BF16>(ma, mb, kp, num_sms, stream);
-        case EPI_SWIGLU_BF16: return launch_inst<BT, EPI_SWIGLU_BF16>(ma, mb, kp, num_sms, stream);
-        case EPI_SWIGLU_QUANT: return launch_inst<BT, EPI_SWIGLU_QUANT>(ma, mb, kp, num_sms, stream);
-        case EPI_COMBINE: return launch_inst<BT, EPI_COMBINE>(ma, mb, kp, num_sms, stream);
+        case EPI_BF16: return launch_inst<BT, EPI_BF16>(ma, mb, my, kp, num_sms, stream);
+        case EPI_SWIGLU_BF16:
+            return launch_inst<BT, EPI_SWIGLU_BF16>(ma, mb, my, kp, num_sms, stream);
+        case EPI_SWIGLU_QUANT:
+            return launch_inst<BT, EPI_SWIGLU_QUANT>(ma, mb, my, kp, num_sms, stream);
+        case EPI_COMBINE: return launch_inst<BT, EPI_COMBINE>(ma, mb, my, kp, num_sms, stream);
+        case EPI_Y32: return launch_inst<BT, EPI_Y32>(ma, mb, my, kp, num_sms, stream);
         default: return ST_INVALID_ARG;
     }
 }
@@ -1009,6 +1111,7 @@ int launch_grouped_gemm(const GemmArgs& g, cudaStream_t stream) {
     kp.hq = g.hq; kp.hs = g.hs;
     kp.perm = g.perm; kp.topk_w = g.topk_w; kp.topk = g.topk > 0 ? g.topk : 1;
     kp.out_acc = g.out_acc; kp.out_ld = g.out_ld;
+    kp.y = g.y; kp.ldy = g.ldy; kp.rowmap = g.rowmap;
     kp.out_bf16 = static_cast<__nv_bfloat16*>(g.out_bf16);
     kp.status = g.status;
     kp.timeout_ns = g.timeout_ns;
@@ -1031,11 +1134,17 @@ int launch_grouped_gemm(const GemmArgs& g, cudaStream_t stream) {
     }
     kp.nranges = nranges;
     kp.ntn_r = ntn / nranges;
+    CUtensorMap my = mb;  // unused unless EPI_Y32
+    if (g.epi == EPI_Y32) {
+        if (!g.y || g.ldy < g.N || g.ldy % 4 || (reinterpret_cast<uintptr_t>(g.y) & 15))
+            return ST_INVALID_ARG;
+        if (!make_map_f32_out(&my, g.y, g.R, g.ldy)) return ST_CUDA;
+    }
     switch (g.tile_m) {
-        case 16: return launch_bt<16>(g.epi, ma, mb, kp, g.num_sms, stream);
-        case 32: return launch_bt<32>(g.epi, ma, mb, kp, g.num_sms, stream);
-        case 64: return launch_bt<64>(g.epi, ma, mb, kp, g.num_sms, stream);
-        case 128: return launch_bt<128>(g.epi, ma, mb, kp, g.num_sms, stream);
+        case 16: return launch_bt<16>(g.epi, ma, mb, my, kp, g.num_sms, stream);
+        case 32: return launch_bt<32>(g.epi, ma, mb, my, kp, g.num_sms, stream);
+        case 64: return launch_bt<64>(g.epi, ma, mb, my, kp, g.num_sms, stream);
+        case 128: return launch_bt<128>(g.epi, ma, mb, my, kp, g.num_sms, stream);
         default: return ST_NO_TILE_CONFIG;
     }
 }

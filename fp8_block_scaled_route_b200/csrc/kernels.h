@@ -11,6 +11,7 @@ enum Epilogue : int {
     EPI_SWIGLU_BF16 = 1,   // gated: out[r, i] = bf16(silu(G_gate) * G_up)
     EPI_SWIGLU_QUANT = 2,  // gated: h = silu(G_gate) * G_up, FP8 per row per 128 cols
     EPI_COMBINE = 3,       // plain: out_acc[token, n] += topk_w * G   (fp32 reduction)
+    EPI_Y32 = 4,           // plain: y[r, n] = G (fp32, grouped row order, each row written once)
 };
 
 struct GemmArgs {
@@ -34,6 +35,10 @@ struct GemmArgs {
     int topk;
     float* out_acc;
     int out_ld;
+    // EPI_Y32: y[r * ldy + n], or y[rowmap[r] * ldy + n] when rowmap is set
+    float* y;
+    int ldy;
+    const int32_t* rowmap;
     // EPI_BF16 / EPI_SWIGLU_BF16
     void* out_bf16;
     int* status;
@@ -71,9 +76,35 @@ int launch_router_topk(const float* logits, int T, int E, int k, int32_t* ids, f
 int launch_quant_scatter(const void* x, int T, int H, int k, int R, const int32_t* inv_perm,
                          uint8_t* xq, float* xs, float* out_acc, cudaStream_t stream);
 
+// Expert-parallel dispatch: quantise x per token per 128 columns and write
+// pair p = t*k + j's row to send slot slot_of_pair[p] (skipped when < 0):
+// xq [S, H] codes, xs [S, H/128] fp32 (row-major), eid [S] = the pair's
+// expert id modulo experts_per_rank (its index on the owning rank).
+int launch_ep_pack(const void* x, const int32_t* ids, int T, int H, int k, int S,
+                   const int32_t* slot_of_pair, int experts_per_rank, uint8_t* xq, float* xs,
+                   int32_t* eid, cudaStream_t stream);
+
+// owner[p] = ids[p] / experts_per_rank for ids in [0, E), else -1.
+int launch_ep_owner(const int32_t* ids, long long R, int E, int experts_per_rank, int32_t* owner,
+                    int num_sms, cudaStream_t stream);
+
+// xq_g[r] = xq[src_of[r]] (rows of H bytes), xs_g[kb * n + r] =
+// xs[src_of[r] * H/128 + kb], for r < rows and r < *rows_dev (when set; n =
+// rows of the source and the column-block stride of xs_g).
+int launch_gather_rows(const uint8_t* xq, const float* xs, int n, int H, const int32_t* src_of,
+                       int rows, const int32_t* rows_dev, uint8_t* xq_g, float* xs_g,
+                       cudaStream_t stream);
+
 // MXFP8 variant: xq as above, xsf [H/128, R, 4] E8M0 codes (one per 32 columns).
 int launch_mx_quant_scatter(const void* x, int T, int H, int k, int R, const int32_t* inv_perm,
                             uint8_t* xq, uint8_t* xsf, float* out_acc, cudaStream_t stream);
+
+// Top-k weighted combine of per-pair rows: out[t, c] = bf16(sum_j
+// fp32(topk_w[t, j] * y[inv_perm[t*k + j], c])) in ascending j (pairs with
+// inv_perm < 0 skipped; inv_perm null = identity).  y [*, H] fp32, out [T, H]
+// bf16, H % 8 == 0.
+int launch_combine(const float* y, const int32_t* inv_perm, const float* topk_w, int T, int k,
+                   int H, void* out, cudaStream_t stream);
 
 // out [n] bf16 = in [n] fp32
 int launch_f32_to_bf16(const float* in, void* out, long long n, int num_sms, cudaStream_t stream);

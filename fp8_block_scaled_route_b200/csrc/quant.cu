@@ -18,10 +18,15 @@
 namespace moe {
 
 // One warp per (token, 128-column block): lane i owns columns 4i..4i+3.
+// Scales go to xs[kb * R + row] (MN-major) or, with xs_kmajor, to
+// xs[row * H/128 + kb].  With eid_out, eid_out[row] = the pair's expert id
+// minus eid_base_div * (id / eid_base_div) (its index inside its owner's
+// expert range).
 __global__ void __launch_bounds__(256) quant_scatter_kernel(
     const __nv_bfloat16* __restrict__ x, int T, int H, int k, int R,
     const int32_t* __restrict__ inv_perm, uint8_t* __restrict__ xq, float* __restrict__ xs,
-    float* __restrict__ out_acc) {
+    float* __restrict__ out_acc, int xs_kmajor, const int32_t* __restrict__ ids,
+    int eid_base_div, int32_t* __restrict__ eid_out) {
     const int nkb = H >> 7;
     const long long item = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     if (item >= static_cast<long long>(T) * nkb) return;
@@ -45,7 +50,14 @@ __global__ void __launch_bounds__(256) quant_scatter_kernel(
         const int row = inv_perm[t * k + j];
         if (row < 0) continue;
         *reinterpret_cast<uint32_t*>(xq + static_cast<long long>(row) * H + kb * 128 + lane * 4) = codes;
-        if (lane == 0) xs[static_cast<long long>(kb) * R + row] = s;
+        if (lane == 0) {
+            if (xs_kmajor) xs[static_cast<long long>(row) * nkb + kb] = s;
+            else xs[static_cast<long long>(kb) * R + row] = s;
+            if (eid_out && kb == 0) {
+                const int e = ids[t * k + j];
+                eid_out[row] = e - eid_base_div * (e / eid_base_div);
+            }
+        }
     }
     if (out_acc) *reinterpret_cast<float4*>(out_acc + off) = make_float4(0.f, 0.f, 0.f, 0.f);
 }
@@ -56,7 +68,20 @@ int launch_quant_scatter(const void* x, int T, int H, int k, int R, const int32_
     if (items == 0) return ST_OK;
     const long long blocks = (items + 7) / 8;
     quant_scatter_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(x), T, H, k, R, inv_perm, xq, xs, out_acc);
+        static_cast<const __nv_bfloat16*>(x), T, H, k, R, inv_perm, xq, xs, out_acc, 0, nullptr,
+        1, nullptr);
+    return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
+}
+
+int launch_ep_pack(const void* x, const int32_t* ids, int T, int H, int k, int S,
+                   const int32_t* slot_of_pair, int experts_per_rank, uint8_t* xq, float* xs,
+                   int32_t* eid, cudaStream_t stream) {
+    const long long items = static_cast<long long>(T) * (H / 128);
+    if (items == 0) return ST_OK;
+    const long long blocks = (items + 7) / 8;
+    quant_scatter_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(x), T, H, k, S, slot_of_pair, xq, xs, nullptr, 1, ids,
+        experts_per_rank, eid);
     return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
 }
 
@@ -135,6 +160,85 @@ int launch_f32_to_bf16(const float* in, void* out, long long n, int num_sms, cud
     if (blocks > cap) blocks = cap;
     f32_to_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
         in, static_cast<__nv_bfloat16*>(out), n4);
+    return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
+}
+
+// ------------------------------------------------------------ combine
+// Stage 5 of the AlphaMoE page's pipeline ("문제점: MoE Expert 계산의 병목"):
+// out[t, c] = bf16(sum_j fp32(topk_w[t, j] * y[inv_perm[t*k + j], c])), the
+// products rounded on their own and added in ascending slot order, so the
+// result depends on nothing but y (no reduction-order freedom).  One CTA per
+// (token, 1024 columns), a thread per 8 columns; the k rows are read four at
+// a time with all their loads issued before the adds.
+constexpr int kCombineCols = 1024;
+
+__global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ y,
+                                                      const int32_t* __restrict__ inv_perm,
+                                                      const float* __restrict__ topk_w, int k,
+                                                      int H, __nv_bfloat16* __restrict__ out) {
+    const int t = blockIdx.y;
+    const int c = blockIdx.x * kCombineCols + threadIdx.x * 8;
+    if (c >= H) return;
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+    const long long pair0 = static_cast<long long>(t) * k;
+    for (int j0 = 0; j0 < k; j0 += 4) {
+        float4 v[4][2];
+        float w[4];
+        bool ok[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = j0 + u;
+            const int row = j < k ? (inv_perm ? __ldg(inv_perm + pair0 + j)
+                                              : static_cast<int>(pair0 + j))
+                                  : -1;
+            ok[u] = row >= 0;
+            w[u] = ok[u] ? __ldg(topk_w + pair0 + j) : 0.0f;
+            const float4* src = reinterpret_cast<const float4*>(
+                y + static_cast<long long>(ok[u] ? row : 0) * H + c);
+            v[u][0] = ok[u] ? __ldg(src) : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[u][1] = ok[u] ? __ldg(src + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (!ok[u]) continue;
+            const float e[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w,
+                                v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], __fmul_rn(w[u], e[i]));
+        }
+    }
+    uint4 o;
+    __nv_bfloat162 b0 = __floats2bfloat162_rn(acc[0], acc[1]);
+    __nv_bfloat162 b1 = __floats2bfloat162_rn(acc[2], acc[3]);
+    __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[4], acc[5]);
+    __nv_bfloat162 b3 = __floats2bfloat162_rn(acc[6], acc[7]);
+    memcpy(&o.x, &b0, 4); memcpy(&o.y, &b1, 4);
+    memcpy(&o.z, &b2, 4); memcpy(&o.w, &b3, 4);
+    *reinterpret_cast<uint4*>(out + static_cast<long long>(t) * H + c) = o;
+}
+
+int launch_combine(const float* y, const int32_t* inv_perm, const float* topk_w, int T, int k,
+                   int H, void* out, cudaStream_t stream) {
+    if (T == 0) return ST_OK;
+    if (H % 8 || k < 1) return ST_INVALID_ARG;
+    const dim3 grid((H + kCombineCols - 1) / kCombineCols, static_cast<unsigned>(T));
+    if (grid.y > 65535u) {
+        // tokens beyond the grid's y limit: one launch per 65535 tokens
+        for (int t0 = 0; t0 < T; t0 += 65535) {
+            const int n = T - t0 < 65535 ? T - t0 : 65535;
+            const long long p0 = static_cast<long long>(t0) * k;
+            // inv_perm holds absolute rows; the identity map counts from this launch's first pair
+            combine_kernel<<<dim3(grid.x, n), 128, 0, stream>>>(
+                inv_perm ? y : y + p0 * H, inv_perm ? inv_perm + p0 : nullptr, topk_w + p0, k, H,
+                static_cast<__nv_bfloat16*>(out) + static_cast<long long>(t0) * H);
+            if (cudaGetLastError() != cudaSuccess) return ST_CUDA;
+        }
+        return ST_OK;
+    }
+    combine_kernel<<<grid, 128, 0, stream>>>(y, inv_perm, topk_w, k, H,
+                                             static_cast<__nv_bfloat16*>(out));
     return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
 }
 

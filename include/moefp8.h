@@ -128,7 +128,8 @@ MOE_API int moe_router_topk(const float* logits, int T, int E, int k, int32_t* t
 /* ------------------------------------------------------------------ */
 
 /* Workspace bytes moe_fp8_fused needs (routing tables, quantised
- * activations, FP8 intermediate, fp32 combine buffer, status word). */
+ * activations, FP8 intermediate, the fp32 down-projection rows of every
+ * (token, slot) pair [T*k, H], status word). */
 MOE_API size_t moe_workspace_size(int T, int H, int I, int E, int k);
 
 /* out[t, :] = bf16( sum_j topk_w[t,j] * Down_e( requant( SwiGLU( GateUp_e(
@@ -145,7 +146,10 @@ MOE_API size_t moe_workspace_size(int T, int H, int I, int E, int k);
  * Activations are quantised per token per 128 columns (scale = amax/448,
  * round-to-nearest-even, saturating); the intermediate is requantised the
  * same way per row per 128 columns; the router weight is applied after the
- * down projection.  T = 0 is a no-op.  Returns MOE_ERR_INVALID_ARG for
+ * down projection: each pair's fp32 down-projection row is written once and
+ * the combine sums a token's k weighted rows in ascending slot order (fp32,
+ * each product rounded, then bf16), so the output does not depend on the
+ * order in which the GEMM's tiles run.  T = 0 is a no-op.  Returns MOE_ERR_INVALID_ARG for
  * sizes that are not multiples of 128, k > E, null pointers, misaligned
  * pointers or a small workspace; MOE_ERR_UNSUPPORTED for E > 1024. */
 MOE_API int moe_fp8_fused(const void* x, const int32_t* topk_ids, const float* topk_w,
@@ -424,6 +428,81 @@ MOE_API int swiglu_mxfp8_quant(const void* in, void* out, uint8_t* scale, int M,
                        moe_stream_t stream);
 
 /* ------------------------------------------------------------------ */
+/* Expert parallelism: the layer with its experts split over G GPUs      */
+/* ------------------------------------------------------------------ */
+/* The AlphaMoE page's five stages ("문제점: MoE Expert 계산의 병목") with rank g
+ * of G owning experts [g*E/G, (g+1)*E/G) and keeping its own tokens.  The
+ * pages do not describe expert parallelism; this follows the plainest
+ * reading: every (token, slot) pair's quantised activation row travels to
+ * the rank that owns its expert, that rank runs the expert FFN on the rows
+ * it received, and the fp32 rows travel back for the combine (the
+ * AG-matmul page, "1. 커널 최적화" and "왜 이게 좋은가", pairs the tensor cores
+ * with NVLink transfers; its "2. API 개선" binds the group and buffers once).
+ * The all-to-all exchanges between the steps are the caller's (for example
+ * NCCL through torch.distributed); each step below is asynchronous on
+ * `stream`.  The output equals the single-GPU moe_fp8_fused output up to the
+ * GEMMs' accumulation order (each row is computed by the same kernels; the
+ * combine order is the same). */
+
+/* Workspace bytes of moe_ep_plan. */
+MOE_API size_t moe_ep_workspace_size(int T, int k, int G);
+
+/* Step 1, on every rank: where each of this rank's T*k pairs goes.
+ *  topk_ids      device int32 [T, k], ids in [0, E); others are dropped and
+ *                reported as MOE_ERR_BAD_EXPERT_ID through
+ *                moe_get_device_status(ws)
+ *  send_indptr   device int32 [G+1] out: pairs for rank g occupy send slots
+ *                [send_indptr[g], send_indptr[g+1]); send_indptr[G] = S, the
+ *                number of valid pairs
+ *  send_pair     device int32 [T*k] out: send slot -> pair id t*k + j,
+ *                ascending pair id within each rank's range
+ *  slot_of_pair  device int32 [T*k] out: pair id -> send slot, -1 if dropped
+ * Requires E % G == 0, E and G <= MOE_MAX_EXPERTS (else
+ * MOE_ERR_INVALID_ARG).  Caller owns all memory. */
+MOE_API int moe_ep_plan(const int32_t* topk_ids, int T, int k, int E, int G,
+                        int32_t* send_indptr, int32_t* send_pair, int32_t* slot_of_pair,
+                        void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Step 2, on every rank: quantise x per token per 128 columns (scale =
+ * amax/448, round-to-nearest-even, as moe_fp8_fused) and write each pair's
+ * row into its send slot s = slot_of_pair[p]:
+ *  xq_send   device FP8 [S, H]; xs_send device fp32 [S, H/128] (row-major);
+ *  eid_send  device int32 [S]: the pair's expert id minus the first expert
+ *            of its owning rank (its local id there).
+ * S = send_indptr[G] from step 1 (read back by the caller to size the
+ * exchange).  H % 128 == 0, E % G == 0. */
+MOE_API int moe_ep_pack(const void* x, const int32_t* topk_ids, const int32_t* slot_of_pair,
+                        int T, int H, int k, int E, int G, int S, uint8_t* xq_send,
+                        float* xs_send, int32_t* eid_send, moe_stream_t stream);
+
+/* Workspace bytes of moe_fp8_expert_rows. */
+MOE_API size_t moe_fp8_expert_rows_workspace_size(int n, int H, int I, int E);
+
+/* Step 3, on the owning rank, after the exchange: the expert FFN on n
+ * received rows in any order,
+ *   y[i, :] = Down_e( requant( SwiGLU( GateUp_e( xq[i, :] * xs[i] ) ) ) ),
+ * e = eid[i] in [0, E) (E = the rank's own experts; w13/w2 and their
+ * scales are those E experts, laid out as for moe_fp8_fused).
+ *  xq device FP8 [n, H], xs device fp32 [n, H/128], eid device int32 [n],
+ *  y  device fp32 [n, H] out, row i for received row i.
+ * Rows are grouped by expert on the device (stable), then run through the
+ * same GEMM1 (SwiGLU + FP8 requant epilogue) and GEMM2 as moe_fp8_fused.
+ * Rows with an eid outside [0, E) are not written; moe_get_device_status(ws)
+ * then reports MOE_ERR_BAD_EXPERT_ID. */
+MOE_API int moe_fp8_expert_rows(const uint8_t* xq, const float* xs, const int32_t* eid, int n,
+                                const void* w13, const float* w13_scale, const void* w2,
+                                const float* w2_scale, float* y, int H, int I, int E,
+                                void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Step 4, on every rank, after the return exchange (and the last stage of
+ * moe_fp8_fused on its own): out[t, :] = bf16( sum_j fp32( topk_w[t, j] *
+ * y[row_of_pair[t*k + j], :] ) ), products rounded on their own and added in
+ * ascending j; pairs with row_of_pair < 0 are skipped; row_of_pair = NULL
+ * means row t*k + j.  y device fp32 [*, H], out device bf16 [T, H], H % 8 == 0. */
+MOE_API int moe_combine(const float* y, const int32_t* row_of_pair, const float* topk_w, int T,
+                        int k, int H, void* out, moe_stream_t stream);
+
+/* ------------------------------------------------------------------ */
 /* Device status                                                        */
 /* ------------------------------------------------------------------ */
 
@@ -439,7 +518,7 @@ MOE_API int moe_get_device_status(const void* ws, moe_stream_t stream);
  * moe_fp8_fused_debug record events[i] (cudaEvent_t handles created by the
  * caller) on the call's stream: 0 before routing, 1 after routing, 2 after
  * activation quantisation, 3 after GEMM1 (gate/up + SwiGLU + requant), 4
- * after GEMM2 (down + combine), 5 after the bf16 conversion.  n must be 6;
+ * after GEMM2 (down projection), 5 after the combine and bf16 output.  n must be 6;
  * events = NULL switches it off.  Process-wide setting. */
 MOE_API int moe_set_stage_events(void* const* events, int n);
 

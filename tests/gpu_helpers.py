@@ -7,10 +7,13 @@ Tolerances (one place, used by every GPU test):
   * FP8 codes of the requantised intermediate and of SwiGLU+MXFP8: at least
     99.9% identical; every other code adjacent (neighbouring representable
     value, same sign) to the oracle's.
-  * fp32 block scales of the intermediate: relative difference <= 2^-16.
-    Both sides take amax/448 of the same fp32 values up to the GEMM's
-    accumulation order: 56 block partials of up to 128 exact products each,
-    added in a different order, move amax by a few fp32 ulps (2^-24 each).
+  * fp32 block scales of the intermediate: relative difference <= 2^-20.
+    Both sides take amax/448 with an IEEE divide of the same fp32 values up
+    to the GEMM's accumulation order (56 block partials of up to 128 exact
+    products each, promoted in a different order) and the kernel's SiLU
+    (hardware exp2 and reciprocal, about 2 ulp): amax moves by a few fp32
+    ulps.  The largest difference over every GPU test is 6.8e-7 (0.71 of
+    the bound).
   * final bf16 output: relative L2 error <= 1e-2 and max abs error
     <= 2e-2 * rms(reference).
 """
@@ -22,7 +25,7 @@ import torch
 import fp8_block_scaled_route_b200 as moe
 
 CODE_MATCH_MIN = 0.999
-SCALE_RTOL = 2.0 ** -16
+SCALE_RTOL = 2.0 ** -20
 OUT_REL_L2 = 1e-2
 OUT_MAX_ABS_RMS = 2e-2
 
