@@ -28,7 +28,7 @@ __all__ = [
     "nvfp4_moe_gemm", "nvfp4_tile_scales", "moe_nvfp4_fused", "moe_nvfp4_fused_debug",
     "nvfp4_quantize", "moe_tactic_tune_gemm", "moe_tactic_lookup", "moe_tactic_store",
     "moe_tactic_clear", "moe_ep_workspace_size", "moe_ep_plan", "moe_ep_pack",
-    "moe_fp8_expert_rows_workspace_size", "moe_fp8_expert_rows", "moe_combine",
+    "moe_fp8_expert_rows_workspace_size", "moe_fp8_expert_rows", "moe_combine", "moe_router_route",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -52,7 +52,7 @@ EXPORTS = (
     "nvfp4_tile_scales", "moe_nvfp4_fused", "moe_nvfp4_fused_debug", "nvfp4_quantize",
     "moe_tactic_tune_gemm", "moe_tactic_lookup", "moe_tactic_store", "moe_tactic_clear",
     "moe_ep_workspace_size", "moe_ep_plan", "moe_ep_pack", "moe_fp8_expert_rows_workspace_size",
-    "moe_fp8_expert_rows", "moe_combine",
+    "moe_fp8_expert_rows", "moe_combine", "moe_router_route",
 )
 
 _lib = None
@@ -139,13 +139,15 @@ def lib():
     L.moe_ep_plan.restype = I
     L.moe_ep_plan.argtypes = [P, I, I, I, I, P, P, P, P, Z, P]
     L.moe_ep_pack.restype = I
-    L.moe_ep_pack.argtypes = [P, P, P] + [I] * 7 + [P, P, P, P]
+    L.moe_ep_pack.argtypes = [P, P, P] + [I] * 6 + [P, P, P, P]
     L.moe_fp8_expert_rows_workspace_size.restype = Z
     L.moe_fp8_expert_rows_workspace_size.argtypes = [I] * 4
     L.moe_fp8_expert_rows.restype = I
     L.moe_fp8_expert_rows.argtypes = [P, P, P, I, P, P, P, P, P, I, I, I, P, Z, P]
     L.moe_combine.restype = I
     L.moe_combine.argtypes = [P, P, P, I, I, I, P, P]
+    L.moe_router_route.restype = I
+    L.moe_router_route.argtypes = [P, I, I, I, P, P, P, P, P, P, Z, P]
     _lib = L
     return L
 
@@ -206,6 +208,19 @@ def moe_route_permute(topk_ids, E: int, m_indptr, perm, inv_perm, ws, ws_bytes=N
     st = lib().moe_route_permute(_ptr(topk_ids), T, k, E, _ptr(m_indptr), _ptr(perm),
                                  _ptr(inv_perm), _ptr(ws), ws_bytes, _stream(stream))
     return _check(st, "moe_route_permute", check)
+
+
+def moe_router_route(logits, k: int, topk_ids, topk_w, m_indptr, perm, inv_perm, ws, ws_bytes=None,
+                     *, dims=None, stream=None, check=True) -> int:
+    """moe_router_topk + moe_route_permute in one call (one launch for up to
+    8192 pairs); dims = (T, E) when raw addresses are passed."""
+    T, E = dims if dims is not None else logits.shape
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size()
+    st = lib().moe_router_route(_ptr(logits), T, E, k, _ptr(topk_ids), _ptr(topk_w),
+                                _ptr(m_indptr), _ptr(perm), _ptr(inv_perm), _ptr(ws), ws_bytes,
+                                _stream(stream))
+    return _check(st, "moe_router_route", check)
 
 
 def moe_route_permute_noalloc(topk_ids, E: int, m_indptr, perm, inv_perm, *, T=None, k=None,

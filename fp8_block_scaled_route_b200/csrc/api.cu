@@ -703,6 +703,25 @@ int moe_router_topk(const float* logits, int T, int E, int k, int32_t* topk_ids,
                               reinterpret_cast<cudaStream_t>(stream));
 }
 
+int moe_router_route(const float* logits, int T, int E, int k, int32_t* topk_ids, float* topk_w,
+                     int32_t* m_indptr, int32_t* perm, int32_t* inv_perm, void* ws, size_t ws_bytes,
+                     moe_stream_t stream) {
+    if (T < 0 || E < 1 || k < 1 || k > E || k > MOE_ROUTER_MAX_K) return MOE_ERR_INVALID_ARG;
+    if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+    if (!m_indptr || !ws || (T > 0 && (!logits || !topk_ids || !topk_w || !perm)))
+        return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < route_ws_bytes(T, k, E) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+    const DevInfo* d = dev_info();
+    if (int st = check_device(d)) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    char* base = static_cast<char*>(ws);
+    int* status = reinterpret_cast<int*>(base);
+    if (cudaMemsetAsync(status, 0, sizeof(int) * kStatusInts, s) != cudaSuccess) return MOE_ERR_CUDA;
+    RouteArgs ra{topk_ids, T, k, E, m_indptr, perm, inv_perm,
+                 reinterpret_cast<int32_t*>(base + up256(sizeof(int) * kStatusInts)), status};
+    return launch_router_route(logits, ra, topk_w, s);
+}
+
 int mxfp8_moe_gemm(const void* a, const void* b, const uint8_t* a_sf, const uint8_t* b_sf,
                    const int32_t* m_indptr, void* out, int R, int N, int K, int E,
                    int a_sf_major, int is_gated, moe_stream_t stream) {
@@ -805,9 +824,10 @@ int swiglu_mxfp8_quant(const void* in, void* out, uint8_t* scale, int M, int K, 
     const DevInfo* d = dev_info();
     if (int st = check_device(d)) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (cudaMemsetAsync(d->lib_status, 0, sizeof(int) * kStatusInts, s) != cudaSuccess)
+    // one launch per call: the kernel clears the status word itself
+    if (M == 0 && cudaMemsetAsync(d->lib_status, 0, sizeof(int) * kStatusInts, s) != cudaSuccess)
         return MOE_ERR_CUDA;
-    return launch_swiglu_mxfp8(in, out, scale, M, K, d->sms, s);
+    return launch_swiglu_mxfp8(in, out, scale, M, K, d->sms, d->lib_status, s);
 }
 
 // ---------------------------------------------------------------- expert parallelism

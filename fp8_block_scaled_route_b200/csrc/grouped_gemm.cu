@@ -47,7 +47,6 @@ namespace moe {
 
 constexpr int kSmemLimit = 232448;  // 227 KB of opt-in dynamic shared memory per CTA
 constexpr int kMaxE = 1024;
-constexpr long long kCombineRangeBytes = 64ll << 20;  // half of the 126 MB L2
 constexpr int kTableBytes = ((2 * (kMaxE + 1) * 4) + 15) / 16 * 16;
 constexpr int kScaleSlots = 8;        // depth of the direct kernel's scale ring
 constexpr int kScaleSlotFloats = 132;  // a_scale of 128 rows, then b_scale of the two blocks
@@ -74,7 +73,8 @@ struct Cfg {
     static constexpr int AS_TILE_BYTES = SWAP ? 32768 : 0;  // a_scale staging [nkb][BT]
     static constexpr int XCH_BYTES = SWAP ? ((4 * BT + 2 * BT) * 4 + 15) / 16 * 16 : 2 * 128 * 4;
     static constexpr int SCALE_BYTES = SWAP ? 0 : kScaleSlots * kScaleSlotFloats * 4;
-    // direct combine: per epilogue warp a 32-row x 16-column fp32 transpose tile
+    // direct: area after the last pipeline stage that, with that stage, stages
+    // the EPI_Y32 output boxes (16 KB)
     static constexpr int CST_BYTES = SWAP ? 0 : EPI_WARPS * 32 * 16 * 4;
     static constexpr int BAR_BYTES = 1024;
     static constexpr int FIXED =
@@ -113,20 +113,15 @@ struct Cfg {
 
 struct KParams {
     int R, N, K, E, nkb;
-    // Tiles are ordered by column range first: nranges ranges of ntn_r
-    // column tiles each, then expert, column tile, row tile.
-    int nranges, ntn_r;
+    // Tiles are ordered by expert, then column tile, then row tile; ntn
+    // column tiles per expert.
+    int ntn;
     const float* a_scale;
     long long as_row, as_kb;
     const float* b_scale;
     const int32_t* m_indptr;
     uint8_t* hq;
     float* hs;
-    const int32_t* perm;
-    const float* topk_w;
-    int topk;
-    float* out_acc;
-    int out_ld;
     float* y;
     int ldy;
     const int32_t* rowmap;
@@ -143,8 +138,7 @@ struct Smem {
     int* mind;    // [E+1] clamped m_indptr
     float* xch;   // epilogue exchange area
     float* scales;  // direct kernel: kScaleSlots x {a_scale[128], b_scale[2], pad[2]}
-    float* cstage;  // direct combine transpose tiles
-    uint8_t* ystage;  // direct EPI_Y32 output staging (last stage + cstage)
+    uint8_t* ystage;  // direct EPI_Y32 output staging (the last stage and the area after it)
     uint64_t* full;
     uint64_t* empty;
     uint64_t* tfull;
@@ -164,7 +158,6 @@ __device__ __forceinline__ Smem carve(uint8_t* base) {
     uint8_t* p = base;
     s.stages = p;
     p += C::STAGES * C::STAGE_BYTES;
-    s.cstage = reinterpret_cast<float*>(p);
     s.ystage = base + (C::STAGES - 1) * C::STAGE_BYTES;
     p += C::CST_BYTES;
     s.as_tile = reinterpret_cast<float*>(p);
@@ -194,17 +187,14 @@ struct Tile {
     int e, mt, nt, row0, rows;
 };
 
-// Total tiles of the launch: tstart[E] tiles per column range.
+// Total tiles of the launch.
 __device__ __forceinline__ int total_tiles(const Smem& s, const KParams& p) {
-    return s.tstart[p.E] * p.nranges;
+    return s.tstart[p.E];
 }
 
 template <int BT>
 __device__ __forceinline__ Tile decode_tile(int t, const Smem& s, const KParams& p) {
     const int E = p.E;
-    const int per = s.tstart[E];
-    const int range = t / per;
-    t -= range * per;
     int lo = 0, hi = E;  // tstart[lo] <= t < tstart[hi]
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
@@ -215,9 +205,8 @@ __device__ __forceinline__ Tile decode_tile(int t, const Smem& s, const KParams&
     const int local = t - s.tstart[lo];
     const int me = max(0, s.mind[lo + 1] - s.mind[lo]);
     const int mtiles = (me + BT - 1) / BT;
-    const int ntl = local / mtiles;
-    r.nt = range * p.ntn_r + ntl;
-    r.mt = local - ntl * mtiles;
+    r.nt = local / mtiles;
+    r.mt = local - r.nt * mtiles;
     r.row0 = s.mind[lo] + r.mt * BT;
     r.rows = min(BT, me - r.mt * BT);
     return r;
@@ -492,15 +481,7 @@ __device__ void epilogue_direct(const KParams& p, const Smem& s, const WaitCtl& 
 #pragma unroll
         for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
         const uint32_t tlane = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + colg;
-        // combine: the row's pair id and top-k weight are fetched during the
-        // main loop (two dependent loads that may miss L2), not in the tail
-        int c_pair = -1;
-        float c_w = 0.0f;
-        if constexpr (EPI == EPI_COMBINE) c_pair = row_ok ? __ldg(p.perm + row) : -1;
         for (int kb = 0; kb < nkb; ++kb) {
-            if constexpr (EPI == EPI_COMBINE) {
-                if (kb == (nkb > 1 ? 1 : 0) && c_pair >= 0) c_w = __ldg(p.topk_w + c_pair);
-            }
             if (!warp_wait(&s.tfull[tj], tjphase, wc, 6)) return;
             tc_fence_after();
             const uint32_t tb = tlane + tj * 256;
@@ -568,48 +549,6 @@ __device__ void epilogue_direct(const KParams& p, const Smem& s, const WaitCtl& 
                 if (g == 0) p.hs[static_cast<long long>(tl.nt) * p.R + row] = sc;
             }
             if (!epi_sync(s, ephase, wc)) return;
-        } else if constexpr (EPI == EPI_COMBINE) {
-            // Scatter-add w * row into the token's output row.  A lane holds
-            // 64 consecutive columns of one row per weight block; passing them
-            // through a shared-memory tile 16 columns at a time lets each
-            // reduction instruction cover 8 rows x 64 contiguous bytes instead
-            // of 32 rows x 16 bytes.  Tile layout: row r at 128-byte line
-            // r / 2, 16-byte slot (r & 1) * 4 + ((c + r / 2) & 3) for column
-            // chunk c, so both the row-wise writes and the column-wise reads
-            // are free of bank conflicts.
-            const int tok = c_pair >= 0 ? c_pair / p.topk : -1;
-            const float w = c_w;
-            float* const obase = p.out_acc + tl.nt * 256 + colg;
-            float* stg = s.cstage + (warp - 4) * 512;
-            const int rr = lane >> 2, cc = lane & 3;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                if (half == 1 && !v1) break;
-#pragma unroll
-                for (int c16 = 0; c16 < 4; ++c16) {
-                    const float* a = accf + half * 64 + c16 * 16;
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const int slot = (lane & 1) * 4 + ((q4 + (lane >> 1)) & 3);
-                        *reinterpret_cast<float4*>(stg + (lane >> 1) * 32 + slot * 4) =
-                            make_float4(w * a[4 * q4], w * a[4 * q4 + 1], w * a[4 * q4 + 2],
-                                        w * a[4 * q4 + 3]);
-                    }
-                    __syncwarp();
-#pragma unroll
-                    for (int rg = 0; rg < 4; ++rg) {
-                        const int r = rg * 8 + rr;
-                        const int slot = (r & 1) * 4 + ((cc + (r >> 1)) & 3);
-                        const float4 v = *reinterpret_cast<const float4*>(stg + (r >> 1) * 32 + slot * 4);
-                        const int t_r = __shfl_sync(0xffffffffu, tok, r);
-                        if (t_r >= 0)
-                            red_add_v4(obase + static_cast<long long>(t_r) * p.out_ld + half * 128 +
-                                           c16 * 16 + cc * 4,
-                                       v.x, v.y, v.z, v.w);
-                    }
-                    __syncwarp();
-                }
-            }
         } else if constexpr (EPI == EPI_Y32) {
             // The warp's 32 rows x 128 columns leave as four 32 x 32 fp32
             // boxes through two 4 KB shared-memory buffers and TMA stores,
@@ -713,30 +652,15 @@ __device__ void epilogue_swap(const KParams& p, const Smem& s, const WaitCtl& wc
     uint32_t buf = 0, bphase = 0, ephase = 0;
     const int total = total_tiles(s, p);
     const int nkb = p.nkb;
-    int* s_tok = reinterpret_cast<int*>(s.xch + 4 * BT);
-    float* s_wt = s.xch + 5 * BT;
     float acc0[BT], acc1[BT];
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
         const Tile tl = decode_tile<BT>(t, s, p);
         const WTile wt = weight_tile<GATED>(tl, p.N);
-        // stage this tile's activation scales (and combine metadata)
+        // stage this tile's activation scales
         if (!epi_sync(s, ephase, wc)) return;
         for (int idx = et; idx < nkb * BT; idx += 128) {
             const int kb = idx / BT, j = idx - kb * BT;
             s.as_tile[idx] = (j < tl.rows) ? a_scale_at(p, tl.row0 + j, kb) : 0.0f;
-        }
-        if constexpr (EPI == EPI_COMBINE) {
-            if (et < BT) {
-                int tok = 0;
-                float wgt = 0.0f;
-                if (et < tl.rows) {
-                    const int pair = p.perm[tl.row0 + et];
-                    tok = pair / p.topk;
-                    wgt = p.topk_w[pair];
-                }
-                s_tok[et] = tok;
-                s_wt[et] = wgt;
-            }
         }
         if (!epi_sync(s, ephase, wc)) return;
         const float* bs0 = p.b_scale + static_cast<long long>(wt.sb0) * nkb;
@@ -810,18 +734,6 @@ __device__ void epilogue_swap(const KParams& p, const Smem& s, const WaitCtl& wc
                 if (j < tl.rows)
                     p.hq[static_cast<long long>(tl.row0 + j) * ldh + col] =
                         static_cast<uint8_t>(cvt_e4m3x2(acc0[j] * s_inv[j], 0.0f) & 0xFF);
-            }
-        } else if constexpr (EPI == EPI_COMBINE) {
-            const int colA = tl.nt * 256 + w;
-            const int colB = colA + 128;
-#pragma unroll
-            for (int j = 0; j < BT; ++j) {
-                if (j < tl.rows) {
-                    float* rowp = p.out_acc + static_cast<long long>(s_tok[j]) * p.out_ld;
-                    const float wgt = s_wt[j];
-                    red_add(rowp + colA, wgt * acc0[j]);
-                    if (wt.v1) red_add(rowp + colB, wgt * acc1[j]);
-                }
             }
         } else if constexpr (EPI == EPI_Y32) {
             const int colA = tl.nt * 256 + w;
@@ -899,7 +811,7 @@ __global__ void __launch_bounds__(Cfg<BT>::THREADS, 1)
     if (warp == 2) {
         // per-expert tile table: tiles of expert e = ceil(rows_e / BT) * n_tiles
         const int E = p.E;
-        const int ntn = p.ntn_r;  // column tiles per range
+        const int ntn = p.ntn;
         const int per = (E + 31) >> 5;
         const int lo = min(E, lane * per), hi = min(E, lo + per);
         int sum = 0;
@@ -1081,7 +993,6 @@ int launch_bt(int epi, const CUtensorMap& ma, const CUtensorMap& mb, const CUten
             return launch_inst<BT, EPI_SWIGLU_BF16>(ma, mb, my, kp, num_sms, stream);
         case EPI_SWIGLU_QUANT:
             return launch_inst<BT, EPI_SWIGLU_QUANT>(ma, mb, my, kp, num_sms, stream);
-        case EPI_COMBINE: return launch_inst<BT, EPI_COMBINE>(ma, mb, my, kp, num_sms, stream);
         case EPI_Y32: return launch_inst<BT, EPI_Y32>(ma, mb, my, kp, num_sms, stream);
         default: return ST_INVALID_ARG;
     }
@@ -1109,31 +1020,12 @@ int launch_grouped_gemm(const GemmArgs& g, cudaStream_t stream) {
     kp.a_scale = g.a_scale; kp.as_row = g.as_row; kp.as_kb = g.as_kb;
     kp.b_scale = g.b_scale; kp.m_indptr = g.m_indptr;
     kp.hq = g.hq; kp.hs = g.hs;
-    kp.perm = g.perm; kp.topk_w = g.topk_w; kp.topk = g.topk > 0 ? g.topk : 1;
-    kp.out_acc = g.out_acc; kp.out_ld = g.out_ld;
     kp.y = g.y; kp.ldy = g.ldy; kp.rowmap = g.rowmap;
     kp.out_bf16 = static_cast<__nv_bfloat16*>(g.out_bf16);
     kp.status = g.status;
     kp.timeout_ns = g.timeout_ns;
-    // Column ranges: the combine's fp32 reductions go to out_acc[token, n];
-    // rows of every expert touch tokens all over out_acc, so when out_acc
-    // exceeds L2 each reduction would miss.  Walking the tiles one column
-    // range at a time keeps the range's slice of out_acc resident; it costs
-    // one extra read of the activations per extra range.
     const bool gated = g.epi == EPI_SWIGLU_BF16 || g.epi == EPI_SWIGLU_QUANT;
-    const int ntn = gated ? (g.N >> 8) : ((g.N + 255) >> 8);
-    int nranges = 1;
-    if (g.epi == EPI_COMBINE && g.tile_m == 128 && ntn > 0) {
-        const long long acc_bytes =
-            static_cast<long long>(g.R / (g.topk > 0 ? g.topk : 1)) * g.out_ld * 4;
-        for (int d = 1; d <= ntn; ++d) {
-            if (ntn % d) continue;
-            nranges = d;
-            if (acc_bytes / d <= kCombineRangeBytes) break;
-        }
-    }
-    kp.nranges = nranges;
-    kp.ntn_r = ntn / nranges;
+    kp.ntn = gated ? (g.N >> 8) : ((g.N + 255) >> 8);
     CUtensorMap my = mb;  // unused unless EPI_Y32
     if (g.epi == EPI_Y32) {
         if (!g.y || g.ldy < g.N || g.ldy % 4 || (reinterpret_cast<uintptr_t>(g.y) & 15))

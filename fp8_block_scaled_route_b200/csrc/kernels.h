@@ -10,7 +10,6 @@ enum Epilogue : int {
     EPI_BF16 = 0,          // plain: out[r, n] = bf16(G)
     EPI_SWIGLU_BF16 = 1,   // gated: out[r, i] = bf16(silu(G_gate) * G_up)
     EPI_SWIGLU_QUANT = 2,  // gated: h = silu(G_gate) * G_up, FP8 per row per 128 cols
-    EPI_COMBINE = 3,       // plain: out_acc[token, n] += topk_w * G   (fp32 reduction)
     EPI_Y32 = 4,           // plain: y[r, n] = G (fp32, grouped row order, each row written once)
 };
 
@@ -29,12 +28,6 @@ struct GemmArgs {
     // EPI_SWIGLU_QUANT: hq [R, N/2] codes, hs [(N/2)/128, R]
     uint8_t* hq;
     float* hs;
-    // EPI_COMBINE: out_acc[token * out_ld + n], token = perm[r] / topk, weight topk_w[perm[r]]
-    const int32_t* perm;
-    const float* topk_w;
-    int topk;
-    float* out_acc;
-    int out_ld;
     // EPI_Y32: y[r * ldy + n], or y[rowmap[r] * ldy + n] when rowmap is set
     float* y;
     int ldy;
@@ -70,6 +63,11 @@ int launch_route_permute(const RouteArgs& r, cudaStream_t stream);
 // expert), w fp32 [T, k] = softmax of the selected logits.  E <= 1024, k <= 32.
 int launch_router_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
                        cudaStream_t stream);
+
+// Router then routing: ids r.topk_ids [T, k] (written) and w [T, k] from
+// logits [T, E] as launch_router_topk, then the tables as
+// launch_route_permute; one launch for at most 8 chunks of pairs.
+int launch_router_route(const float* logits, const RouteArgs& r, float* w, cudaStream_t stream);
 
 // x [T, H] bf16 -> xq rows inv_perm[t*k + j] of [R, H], xs [H/128, R];
 // also zeroes out_acc [T, H] when not null.
@@ -109,8 +107,9 @@ int launch_combine(const float* y, const int32_t* inv_perm, const float* topk_w,
 // out [n] bf16 = in [n] fp32
 int launch_f32_to_bf16(const float* in, void* out, long long n, int num_sms, cudaStream_t stream);
 
+// Also clears the status word `status` (when set) from inside the kernel.
 int launch_swiglu_mxfp8(const void* in, void* out, uint8_t* scale, int M, int K, int num_sms,
-                        cudaStream_t stream);
+                        int* status, cudaStream_t stream);
 
 // Grouped MXFP8 GEMM on the block-scaled tensor core path: E4M3 operands with
 // one E8M0 scale per 32 K elements of every row of A and of B.

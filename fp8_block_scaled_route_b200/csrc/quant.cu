@@ -254,7 +254,10 @@ __device__ __forceinline__ float silu_q(float z) { return z * rcp_approx(1.0f + 
 // reaches the shuffle.
 __global__ void __launch_bounds__(256) swiglu_mxfp8_kernel(const __nv_bfloat16* __restrict__ in,
                                                            uint8_t* __restrict__ out,
-                                                           uint8_t* __restrict__ scale, int M, int K) {
+                                                           uint8_t* __restrict__ scale, int M, int K,
+                                                           int* __restrict__ status) {
+    // the call's status word starts clear (this kernel never reports an error)
+    if (status && blockIdx.x == 0 && threadIdx.x < kStatusInts) status[threadIdx.x] = 0;
     const int kg = K / 16;
     const long long groups = static_cast<long long>(M) * kg;
     for (long long gi = blockIdx.x * 256ll + threadIdx.x; gi - (threadIdx.x & 31) < groups;
@@ -306,7 +309,7 @@ __global__ void __launch_bounds__(256) swiglu_mxfp8_kernel(const __nv_bfloat16* 
 }
 
 int launch_swiglu_mxfp8(const void* in, void* out, uint8_t* scale, int M, int K, int num_sms,
-                        cudaStream_t stream) {
+                        int* status, cudaStream_t stream) {
     const long long groups = static_cast<long long>(M) * (K / 16);
     if (groups == 0) return ST_OK;
     long long blocks = (groups + 255) / 256;
@@ -318,7 +321,7 @@ int launch_swiglu_mxfp8(const void* in, void* out, uint8_t* scale, int M, int K,
         if (blocks > cap) blocks = cap;
     }
     swiglu_mxfp8_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(in), static_cast<uint8_t*>(out), scale, M, K);
+        static_cast<const __nv_bfloat16*>(in), static_cast<uint8_t*>(out), scale, M, K, status);
     return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
 }
 

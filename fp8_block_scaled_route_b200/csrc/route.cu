@@ -146,11 +146,13 @@ constexpr int kSmallChunks = 8;
 static_assert(kSmallChunks * kMaxRouteExperts * sizeof(int) <= 48 * 1024,
               "route_small's histogram table must fit the default shared-memory limit");
 
-__global__ void __launch_bounds__(1024) route_small(const int32_t* __restrict__ ids, int R, int E,
-                                                    int32_t* __restrict__ m_indptr,
-                                                    int32_t* __restrict__ perm,
-                                                    int32_t* __restrict__ inv_perm, int* status) {
-    extern __shared__ int tab[];  // [kSmallChunks][E]: histograms, then first rows
+// The three phases of route_small for a CTA of 1024 threads; tab is
+// [kSmallChunks][E] ints of shared memory.
+__device__ __forceinline__ void route_small_body(const int32_t* __restrict__ ids, int R, int E,
+                                                 int32_t* __restrict__ m_indptr,
+                                                 int32_t* __restrict__ perm,
+                                                 int32_t* __restrict__ inv_perm, int* status,
+                                                 int* tab) {
     __shared__ int warp_tot[32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nchunks = (R + kRouteChunk - 1) / kRouteChunk;
@@ -247,6 +249,14 @@ __global__ void __launch_bounds__(1024) route_small(const int32_t* __restrict__ 
     }
 }
 
+__global__ void __launch_bounds__(1024) route_small(const int32_t* __restrict__ ids, int R, int E,
+                                                    int32_t* __restrict__ m_indptr,
+                                                    int32_t* __restrict__ perm,
+                                                    int32_t* __restrict__ inv_perm, int* status) {
+    extern __shared__ int tab[];  // [kSmallChunks][E]: histograms, then first rows
+    route_small_body(ids, R, E, m_indptr, perm, inv_perm, status, tab);
+}
+
 // Router (the step before the expert computation): one warp per token.
 // Lane l holds logits l + 32 i; the k winners are taken one at a time by a
 // warp-wide argmax (larger logit first, then the lower expert index), so the
@@ -254,12 +264,9 @@ __global__ void __launch_bounds__(1024) route_small(const int32_t* __restrict__ 
 // logit; the softmax subtracts the largest, takes expf per slot and sums the
 // slots in order (every lane runs the same sequential sum), w_j = e_j / sum.
 template <int PER>
-__global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ logits, int T,
-                                                          int E, int k, int32_t* __restrict__ ids,
-                                                          float* __restrict__ w) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = blockIdx.x * 8 + warp;
-    if (t >= T) return;
+__device__ __forceinline__ void router_token(const float* __restrict__ logits, int t, int E, int k,
+                                             int32_t* __restrict__ ids, float* __restrict__ w) {
+    const int lane = threadIdx.x & 31;
     const float* l = logits + static_cast<long long>(t) * E;
     float v[PER];
 #pragma unroll
@@ -300,6 +307,33 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
     if (lane < k) w[static_cast<long long>(t) * k + lane] = __fdiv_rn(ex, sum);
 }
 
+template <int PER>
+__global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ logits, int T,
+                                                          int E, int k, int32_t* __restrict__ ids,
+                                                          float* __restrict__ w) {
+    const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (t >= T) return;
+    router_token<PER>(logits, t, E, k, ids, w);
+}
+
+// Router and routing in one CTA of 1024 threads, for at most kSmallChunks
+// chunks of pairs: each warp routes tokens warp, warp + 32, ..., then the
+// CTA groups the pairs it just wrote (global writes made visible to the
+// whole CTA by the barrier) with route_small's three phases.
+template <int PER>
+__global__ void __launch_bounds__(1024) router_route_small(const float* __restrict__ logits, int T,
+                                                           int E, int k, int32_t* __restrict__ ids,
+                                                           float* __restrict__ w,
+                                                           int32_t* __restrict__ m_indptr,
+                                                           int32_t* __restrict__ perm,
+                                                           int32_t* __restrict__ inv_perm,
+                                                           int* status) {
+    extern __shared__ int tab[];
+    for (int t = threadIdx.x >> 5; t < T; t += 32) router_token<PER>(logits, t, E, k, ids, w);
+    __syncthreads();
+    route_small_body(ids, T * k, E, m_indptr, perm, inv_perm, status, tab);
+}
+
 int launch_router_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
                        cudaStream_t stream) {
     if (T == 0) return ST_OK;
@@ -309,6 +343,26 @@ int launch_router_topk(const float* logits, int T, int E, int k, int32_t* ids, f
     else
         router_topk_kernel<32><<<blocks, 256, 0, stream>>>(logits, T, E, k, ids, w);
     return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
+}
+
+int launch_router_route(const float* logits, const RouteArgs& r, float* w, cudaStream_t stream) {
+    const int R = r.T * r.k;
+    if (R == 0) return launch_route_permute(r, stream);
+    const int nchunks = (R + kRouteChunk - 1) / kRouteChunk;
+    if (nchunks <= kSmallChunks) {
+        int32_t* ids = const_cast<int32_t*>(r.topk_ids);
+        const size_t smem = static_cast<size_t>(kSmallChunks) * r.E * sizeof(int);
+        if (r.E <= 256)
+            router_route_small<8><<<1, 1024, smem, stream>>>(logits, r.T, r.E, r.k, ids, w,
+                                                             r.m_indptr, r.perm, r.inv_perm, r.status);
+        else
+            router_route_small<32><<<1, 1024, smem, stream>>>(logits, r.T, r.E, r.k, ids, w,
+                                                              r.m_indptr, r.perm, r.inv_perm, r.status);
+        return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
+    }
+    int st = launch_router_topk(logits, r.T, r.E, r.k, const_cast<int32_t*>(r.topk_ids), w, stream);
+    if (st) return st;
+    return launch_route_permute(r, stream);
 }
 
 int launch_route_permute(const RouteArgs& r, cudaStream_t stream) {

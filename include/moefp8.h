@@ -123,6 +123,18 @@ MOE_API int moe_route_permute_noalloc(const int32_t* topk_ids, int T, int k, int
 MOE_API int moe_router_topk(const float* logits, int T, int E, int k, int32_t* topk_ids,
                             float* topk_w, moe_stream_t stream);
 
+/* moe_router_topk and moe_route_permute in one call: from the router
+ * logits to the expert grouping, with the same outputs as the two calls
+ * (topk_ids [T, k], topk_w [T, k], m_indptr [E+1], perm [T*k], inv_perm
+ * [T*k] or NULL, all device buffers owned by the caller) and ws of at least
+ * moe_route_workspace_size(T, k, E) bytes.  Up to 8192 pairs (T*k) it is a
+ * single kernel launch: one CTA selects every token's experts and then
+ * groups the pairs it wrote; above that, the router kernel and then the
+ * routing kernels.  Same argument rules as moe_router_topk. */
+MOE_API int moe_router_route(const float* logits, int T, int E, int k, int32_t* topk_ids,
+                             float* topk_w, int32_t* m_indptr, int32_t* perm, int32_t* inv_perm,
+                             void* ws, size_t ws_bytes, moe_stream_t stream);
+
 /* ------------------------------------------------------------------ */
 /* The fused layer                                                      */
 /* ------------------------------------------------------------------ */

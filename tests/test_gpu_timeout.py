@@ -39,3 +39,21 @@ def test_wait_timeout_is_reported_and_context_survives():
     ref = O.groupwise_gemm_bf16(G.u8(inp["a"]), G.f32(inp["a_scale"]), G.u8(inp["b"]),
                                 G.f32(inp["b_scale"]), G.i32(inp["m_indptr"]), True)
     G.compare_out(G.bf16_bits(out), ref, "after timeout")
+
+
+def test_fused_layer_timeout_is_reported_and_context_survives():
+    """The same through the fused layer at a shape whose GEMM2 runs as CTA-pair
+    tiles (both CTAs of each pair give up, drain and leave together)."""
+    cfg = synth.MoEConfig("pairs", 700, 512, 256, 4, 2)
+    inp = synth.make_moe_inputs(cfg, seed=5, device="cuda")
+    moe.moe_set_wait_timeout_ns(1)
+    try:
+        res = G.run_fused(inp, debug=False)
+        assert res["status"] == moe.MOE_ERR_DEVICE_TIMEOUT
+    finally:
+        moe.moe_set_wait_timeout_ns(DEFAULT_TIMEOUT_NS)
+    torch.cuda.synchronize()
+    res = G.run_fused(inp, debug=False)
+    assert res["status"] == moe.MOE_OK
+    ref = O.moe_fused(*G.oracle_args(inp))
+    G.compare_out(res["out"], ref["out"], "fused layer after timeout")

@@ -35,6 +35,28 @@ def test_exports_every_declared_symbol(L):
         assert hasattr(L, name), name
 
 
+def _declared_arg_counts():
+    """name -> number of parameters, from the MOE_API declarations."""
+    counts = {}
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", fn)).read(),
+                         flags=re.S)
+            for m in re.finditer(r"MOE_API\s+[\w\s\*]+?\b(\w+)\s*\(([^)]*)\)", txt):
+                args = m.group(2).strip()
+                counts[m.group(1)] = 0 if args in ("", "void") else args.count(",") + 1
+    return counts
+
+
+def test_binding_signatures_match_header(L):
+    """Every ctypes prototype the binding sets has as many parameters as the
+    header declares (a missing or extra argument would shift every later one)."""
+    for name, n in _declared_arg_counts().items():
+        argtypes = getattr(L, name).argtypes
+        assert argtypes is not None, f"{name}: no ctypes prototype"
+        assert len(argtypes) == n, f"{name}: {len(argtypes)} ctypes arguments, header has {n}"
+
+
 def test_status_strings(L):
     for code, name in [(0, "MOE_OK"), (1, "MOE_ERR_INVALID_ARG"), (4, "MOE_ERR_NO_TILE_CONFIG"),
                        (5, "MOE_ERR_DEVICE_TIMEOUT"), (6, "MOE_ERR_BAD_EXPERT_ID")]:
@@ -161,3 +183,23 @@ def test_product_path_does_not_touch_oracle():
             if fn.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 txt = open(os.path.join(dirpath, fn)).read()
                 assert "oracle" not in txt.lower(), fn
+
+
+def test_expert_parallel_entry_points_reject_bad_arguments(L):
+    ws = 1 << 20
+    assert moe.moe_ep_plan(FAKE, 10, 4, FAKE, FAKE, FAKE, FAKE, ws, T=8, k=2, stream=0,
+                           check=False) == moe.MOE_ERR_INVALID_ARG      # E % G != 0
+    assert moe.moe_ep_plan(FAKE, 8, 4, FAKE, FAKE, FAKE, FAKE, 16, T=8, k=2, stream=0,
+                           check=False) == moe.MOE_ERR_INVALID_ARG      # workspace too small
+    assert moe.moe_ep_pack(FAKE, FAKE, FAKE, 8, 4, 16, FAKE, FAKE, FAKE, dims=(8, 200, 2),
+                           stream=0, check=False) == moe.MOE_ERR_INVALID_ARG  # H % 128
+    assert moe.moe_fp8_expert_rows(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws,
+                                   dims=(16, 256, 100, 4), stream=0, check=False) == \
+        moe.MOE_ERR_INVALID_ARG                                          # I % 128
+    assert moe.moe_fp8_expert_rows(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 64,
+                                   dims=(16, 256, 128, 4), stream=0, check=False) == \
+        moe.MOE_ERR_INVALID_ARG                                          # workspace too small
+    assert moe.moe_combine(FAKE, FAKE, FAKE, FAKE, dims=(4, 2, 12), stream=0, check=False) == \
+        moe.MOE_ERR_INVALID_ARG                                          # H % 8
+    assert moe.moe_ep_workspace_size(16, 2, 4) > 0
+    assert moe.moe_fp8_expert_rows_workspace_size(16, 256, 128, 4) > 0
