@@ -488,7 +488,11 @@ def run_swiglu(args):
     hbm, _, _, src = load_peaks()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     res = []
-    for (M, K) in synth.SWIGLU_SHAPES:
+    shapes = synth.SWIGLU_SHAPES
+    if args.swiglu_shape:
+        M, K = (int(v) for v in args.swiglu_shape.lower().split("x"))
+        shapes = ((M, K),)
+    for (M, K) in shapes:
         for variant in ("normal", "block_scaled"):
             x = synth.make_swiglu_input(M, K, variant, seed=0, device="cuda")
             out = torch.empty(M, K, dtype=torch.uint8, device="cuda")
@@ -539,6 +543,52 @@ def run_swiglu(args):
                        "l2": "us: flushed before every timed launch (median of single launches); "
                              "us_back_to_back: mean over back-to-back calls replayed from one CUDA graph, no flush"},
             "results": res}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_router(args, cfg):
+    """The router (moe_router_topk) and the router with the grouping in one
+    call (moe_router_route) on a workload's routing shape: logits fp32 [T, E]
+    ~ N(0,1) (plus the Zipf bias for the prefill workload), top-k."""
+    import fp8_block_scaled_route_b200 as moe
+    torch.cuda.set_device(0)
+    T, E, k = cfg.T, cfg.E, cfg.k
+    g = torch.Generator().manual_seed(0)
+    logits = torch.randn(T, E, generator=g)
+    if cfg.routing == "zipf":
+        ranks = torch.randperm(E, generator=g).float() + 1.0
+        logits = logits - synth.ZIPF_S * torch.log(ranks)[None, :]
+    logits = logits.cuda()
+    ids = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    m = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    inv = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    ws = torch.empty(moe.moe_route_workspace_size(T, k, E), dtype=torch.uint8, device="cuda")
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / args.steps * 1e3
+
+    us_topk = timed(lambda: moe.moe_router_topk(logits, ids, w))
+    us_route = timed(lambda: moe.moe_route_permute(ids, E, m, perm, inv, ws))
+    us_both = timed(lambda: moe.moe_router_route(logits, k, ids, w, m, perm, inv, ws))
+    line = {"metric": "router and routing latency", "unit": "us", "higher_is_better": False,
+            "steps": args.steps, "warmup": args.warmup, "n_gpus": 1, "data": "synthetic",
+            "config": {"workload": f"{cfg.name} routing: T={T} E={E} top-{k}, logits fp32"},
+            "router_topk_us": us_topk, "route_permute_us": us_route,
+            "router_route_one_call_us": us_both,
+            "logits_read_gbs": T * E * 4 / (us_topk * 1e-6) / 1e9}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -811,14 +861,18 @@ def main():
     ap.add_argument("--no-decode", action="store_true",
                     help="with the prefill workload: skip the decode workload's timing")
     ap.add_argument("--op", default="moe", choices=["moe", "swiglu_mxfp8", "mxfp8_gemm", "mxfp8_moe",
-                                                     "nvfp4_gemm", "nvfp4_moe"],
+                                                     "nvfp4_gemm", "nvfp4_moe", "router"],
                     help="any other than moe: time that op instead")
+    ap.add_argument("--swiglu-shape", default="",
+                    help="with --op swiglu_mxfp8: only this MxK shape (e.g. 8192x7168)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.op == "swiglu_mxfp8":
         return run_swiglu(args)
     cfg = synth.CONFIGS.get(args.workload) or PROFILE_SLICES[args.workload]
+    if args.op == "router":
+        return run_router(args, cfg)
     if args.op == "mxfp8_gemm":
         return run_mx_gemm(args, cfg)
     if args.op == "nvfp4_gemm":

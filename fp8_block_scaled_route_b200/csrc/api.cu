@@ -295,17 +295,25 @@ static int fused_impl(const void* x, const int32_t* topk_ids, const float* topk_
     if (st) return st;
     stage_mark(1, s);
     if (T > 0) {
-        st = launch_quant_scatter(x, T, H, k, R, inv_perm, xq, xs, nullptr, s);
-        if (st) return st;
-        stage_mark(2, s);
-        const unsigned long long tmo = g_timeout_ns.load();
         int tm1 = choose_tile_m(R, 2 * I, H, E, 1, d->sms);
         int tm2 = choose_tile_m(R, H, I, E, 0, d->sms);
         tm1 = fit_tile_to_k(tm1, H);
         tm2 = fit_tile_to_k(tm2, I);
+        // Swapped (small-group) GEMM1 tiles gather each grouped row's token
+        // row through perm (TMA gather4), so x is quantised once per token
+        // ([T, H], scales [H/128, T]).  128-token tiles load their rows as
+        // two tiled boxes per K block, which gathered rows cannot match, so
+        // there the quantiser writes the k grouped copies ([R, H], [H/128, R]).
+        const bool gather = tm1 < 128;
+        st = gather ? launch_quant_scatter(x, T, H, 1, T, nullptr, xq, xs, nullptr, s)
+                    : launch_quant_scatter(x, T, H, k, R, inv_perm, xq, xs, nullptr, s);
+        if (st) return st;
+        stage_mark(2, s);
+        const unsigned long long tmo = g_timeout_ns.load();
         GemmArgs g1{};
         g1.a = xq; g1.b = w13; g1.R = R; g1.N = 2 * I; g1.K = H; g1.E = E;
-        g1.a_scale = xs; g1.as_row = 1; g1.as_kb = R; g1.b_scale = w13_scale;
+        g1.a_scale = xs; g1.as_row = 1; g1.as_kb = gather ? T : R; g1.b_scale = w13_scale;
+        if (gather) { g1.a_rowmap = perm; g1.a_rowdiv = k; g1.a_rows = T; }
         g1.m_indptr = m_indptr; g1.epi = EPI_SWIGLU_QUANT; g1.tile_m = tm1;
         g1.hq = hq; g1.hs = hs; g1.status = status; g1.timeout_ns = tmo; g1.num_sms = d->sms;
         st = launch_grouped_gemm(g1, s);
@@ -945,8 +953,6 @@ int moe_fp8_expert_rows(const uint8_t* xq, const float* xs, const int32_t* eid, 
     int32_t* m_indptr = reinterpret_cast<int32_t*>(b + L.m_indptr);
     int32_t* perm = reinterpret_cast<int32_t*>(b + L.perm);
     int32_t* inv_perm = reinterpret_cast<int32_t*>(b + L.inv_perm);
-    uint8_t* xq_g = reinterpret_cast<uint8_t*>(b + L.xq);
-    float* xs_g = reinterpret_cast<float*>(b + L.xs);
     uint8_t* hq = reinterpret_cast<uint8_t*>(b + L.hq);
     float* hs = reinterpret_cast<float*>(b + L.hs);
     if (cudaMemsetAsync(status, 0, sizeof(int) * kStatusInts, s) != cudaSuccess) return MOE_ERR_CUDA;
@@ -955,19 +961,28 @@ int moe_fp8_expert_rows(const uint8_t* xq, const float* xs, const int32_t* eid, 
                  reinterpret_cast<int32_t*>(b + L.chunk_hist), status};
     int st = launch_route_permute(ra, s);
     if (st || n == 0) return st;
-    st = launch_gather_rows(xq, xs, n, H, perm, n, m_indptr + E, xq_g, xs_g, s);
-    if (st) return st;
     const unsigned long long tmo = g_timeout_ns.load();
     const int tm1 = fit_tile_to_k(choose_tile_m(n, 2 * I, H, E, 1, d->sms), H);
     const int tm2 = fit_tile_to_k(choose_tile_m(n, H, I, E, 0, d->sms), I);
+    // grouped row r is received row perm[r]: swapped GEMM1 tiles read it (and
+    // its row-major scales) there through the row map; 128-token tiles read a
+    // grouped copy; GEMM2 writes the row back at perm[r]
     GemmArgs g1{};
-    g1.a = xq_g; g1.b = w13; g1.R = n; g1.N = 2 * I; g1.K = H; g1.E = E;
-    g1.a_scale = xs_g; g1.as_row = 1; g1.as_kb = n; g1.b_scale = w13_scale;
+    g1.b = w13; g1.R = n; g1.N = 2 * I; g1.K = H; g1.E = E; g1.b_scale = w13_scale;
+    if (tm1 < 128) {
+        g1.a = xq; g1.a_scale = xs; g1.as_row = H / 128; g1.as_kb = 1;
+        g1.a_rowmap = perm; g1.a_rowdiv = 1; g1.a_rows = n;
+    } else {
+        uint8_t* xq_g = reinterpret_cast<uint8_t*>(b + L.xq);
+        float* xs_g = reinterpret_cast<float*>(b + L.xs);
+        st = launch_gather_rows(xq, xs, n, H, perm, n, m_indptr + E, xq_g, xs_g, s);
+        if (st) return st;
+        g1.a = xq_g; g1.a_scale = xs_g; g1.as_row = 1; g1.as_kb = n;
+    }
     g1.m_indptr = m_indptr; g1.epi = EPI_SWIGLU_QUANT; g1.tile_m = tm1;
     g1.hq = hq; g1.hs = hs; g1.status = status; g1.timeout_ns = tmo; g1.num_sms = d->sms;
     st = launch_grouped_gemm(g1, s);
     if (st) return st;
-    // grouped row r is received row perm[r]: GEMM2 writes it there
     GemmArgs g2{};
     g2.a = hq; g2.b = w2; g2.R = n; g2.N = H; g2.K = I; g2.E = E;
     g2.a_scale = hs; g2.as_row = 1; g2.as_kb = n; g2.b_scale = w2_scale;

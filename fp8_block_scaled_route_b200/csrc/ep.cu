@@ -8,8 +8,9 @@
 //  * ep_owner_kernel: owner rank of every pair (-1 for an id outside
 //    [0, E)), the key the routing kernels then sort the pairs by;
 //  * gather_rows_kernel: received rows (any order) into expert-grouped order
-//    for the grouped GEMM: FP8 codes row by row, block scales from row-major
-//    [n, H/128] to column-block-major [H/128, n].
+//    for 128-token GEMM tiles (FP8 codes row by row, block scales from
+//    row-major [n, H/128] to column-block-major [H/128, n]); smaller token
+//    tiles read the received rows in place through the GEMM's row map.
 #include "common.cuh"
 #include "kernels.h"
 

@@ -125,6 +125,11 @@ struct KParams {
     float* y;
     int ldy;
     const int32_t* rowmap;
+    // A row map: grouped row r reads row a_rowmap[r] / a_rowdiv of A and of
+    // its scales (null: row r); a_rows = rows of A
+    const int32_t* a_rowmap;
+    int a_rowdiv;
+    int a_rows;
     __nv_bfloat16* out_bf16;
     int* status;
     unsigned long long timeout_ns;
@@ -240,6 +245,14 @@ __device__ __forceinline__ WTile weight_tile(const Tile& t, int N) {
     return w;
 }
 
+// Row of A (and of its scales) that grouped row `row` reads.
+__device__ __forceinline__ int a_src_row(const KParams& p, int row) {
+    if (!p.a_rowmap) return row;
+    const int r = min(max(row, 0), p.R - 1);
+    const int src = __ldg(p.a_rowmap + r) / p.a_rowdiv;
+    return min(max(src, 0), p.a_rows - 1);
+}
+
 __device__ __forceinline__ float a_scale_at(const KParams& p, int row, int kb) {
     return p.a_scale[static_cast<long long>(row) * p.as_row + static_cast<long long>(kb) * p.as_kb];
 }
@@ -318,10 +331,17 @@ __device__ void producer_role(const CUtensorMap* tmA, const CUtensorMap* tmB, co
                               const Smem& s, const WaitCtl& wc) {
     using C = Cfg<BT>;
     const int l = threadIdx.x & 31;
+    // Tiled A (no row map): lane l < NBOX issues box l: A boxes first, then
+    // the four 64-row weight boxes; each lane arms the barrier with its own
+    // bytes.  Gathered A (row map): lane l < BT/4 loads token rows 4l..4l+3
+    // with one gather4, lanes 0-3 also issue the weight boxes, and lane 0
+    // arms the barrier with the whole stage.
+    const bool gather = p.a_rowmap != nullptr;
     const bool issuer = l < C::NBOX;
-    // this lane's box: which map, smem offset inside the stage, row offset, bytes
     const bool is_a = l < C::A_BOXES;
-    const int b = l - C::A_BOXES;  // weight box 0..3: block b/2, half b%2
+    const int b = gather ? l : l - C::A_BOXES;  // weight box 0..3: block b/2, half b%2
+    const bool b_lane = gather ? l < 4 : (issuer && !is_a);
+    const bool g_lane = gather && l < BT / 4;
     const uint32_t off = is_a ? C::A_OFF + l * C::A_BOX_ROWS * 128 : C::B_OFF + b * 64 * 128;
     const uint32_t bytes = is_a ? C::A_BOX_ROWS * 128 : 64 * 128;
     uint32_t stage = 0, phase = 0, armed = 0, armed_par = 0;
@@ -330,12 +350,29 @@ __device__ void producer_role(const CUtensorMap* tmA, const CUtensorMap* tmB, co
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const Tile tl = decode_tile<BT>(t, s, p);
         const WTile wt = weight_tile<GATED>(tl, p.N);
-        const int row = is_a ? tl.row0 + l * C::A_BOX_ROWS
-                             : ((b >> 1) ? wt.wrow1 : wt.wrow0) + (b & 1) * 64;
+        const int wrow = ((b >> 1) ? wt.wrow1 : wt.wrow0) + (b & 1) * 64;
+        const int row = is_a ? tl.row0 + l * C::A_BOX_ROWS : wrow;
+        // gathered rows of this lane (rows past the tile's end read its first row)
+        int g0 = 0, g1 = 0, g2 = 0, g3 = 0;
+        if (g_lane) {
+            const int r = tl.row0 + 4 * l;
+            g0 = a_src_row(p, 4 * l + 0 < tl.rows ? r + 0 : tl.row0);
+            g1 = a_src_row(p, 4 * l + 1 < tl.rows ? r + 1 : tl.row0);
+            g2 = a_src_row(p, 4 * l + 2 < tl.rows ? r + 2 : tl.row0);
+            g3 = a_src_row(p, 4 * l + 3 < tl.rows ? r + 3 : tl.row0);
+        }
         for (int kb = 0; kb < p.nkb; ++kb) {
             if (!warp_wait_spin(&s.empty[stage], phase ^ 1, wc, 1)) { ok = false; break; }
             uint8_t* st = s.stages + stage * C::STAGE_BYTES;
-            if (issuer) {
+            if (gather) {
+                if (l == 0) mbar_arrive_expect_tx(&s.full[stage], C::STAGE_BYTES);
+                __syncwarp();
+                if (g_lane)
+                    tma_gather4_2d(st + C::A_OFF + l * 4 * 128, tmA, &s.full[stage], kb * 128, g0,
+                                   g1, g2, g3);
+                if (b_lane)
+                    tma_load_2d(st + C::B_OFF + b * 64 * 128, tmB, &s.full[stage], kb * 128, wrow);
+            } else if (issuer) {
                 mbar_arrive_expect_tx(&s.full[stage], bytes);
                 tma_load_2d(st + off, is_a ? tmA : tmB, &s.full[stage], kb * 128, row);
             }
@@ -421,6 +458,10 @@ __device__ void scale_role(const KParams& p, const Smem& s, const WaitCtl& wc) {
         const WTile wt = weight_tile<GATED>(tl, p.N);
         const float* bs0 = p.b_scale + static_cast<long long>(wt.sb0) * nkb;
         const float* bs1 = p.b_scale + static_cast<long long>(wt.sb1) * nkb;
+        int srow[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            srow[i] = lane + 32 * i < tl.rows ? a_src_row(p, tl.row0 + lane + 32 * i) : 0;
         for (int kb = 0; kb < nkb; ++kb) {
             if (!wait_bar(&s.sempty[slot], sphase ^ 1, wc, 8)) return;
             float* f = s.scales + slot * kScaleSlotFloats;
@@ -428,7 +469,7 @@ __device__ void scale_role(const KParams& p, const Smem& s, const WaitCtl& wc) {
             for (int i = 0; i < 4; ++i) {
                 const int r = lane + 32 * i;
                 const bool ok = r < tl.rows;
-                const float* src = ok ? p.a_scale + static_cast<long long>(tl.row0 + r) * p.as_row +
+                const float* src = ok ? p.a_scale + static_cast<long long>(srow[i]) * p.as_row +
                                             static_cast<long long>(kb) * p.as_kb
                                       : p.b_scale;
                 cp_async_4(f + r, src, ok ? 4u : 0u);
@@ -660,7 +701,7 @@ __device__ void epilogue_swap(const KParams& p, const Smem& s, const WaitCtl& wc
         if (!epi_sync(s, ephase, wc)) return;
         for (int idx = et; idx < nkb * BT; idx += 128) {
             const int kb = idx / BT, j = idx - kb * BT;
-            s.as_tile[idx] = (j < tl.rows) ? a_scale_at(p, tl.row0 + j, kb) : 0.0f;
+            s.as_tile[idx] = (j < tl.rows) ? a_scale_at(p, a_src_row(p, tl.row0 + j), kb) : 0.0f;
         }
         if (!epi_sync(s, ephase, wc)) return;
         const float* bs0 = p.b_scale + static_cast<long long>(wt.sb0) * nkb;
@@ -785,7 +826,7 @@ __global__ void __launch_bounds__(Cfg<BT>::THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::STAGES; ++i) {
-            mbar_init(&s.full[i], C::NBOX);
+            mbar_init(&s.full[i], p.a_rowmap ? 1 : C::NBOX);
             mbar_init(&s.empty[i], 1);
         }
         for (int i = 0; i < C::TSLOTS; ++i) {
@@ -1013,7 +1054,10 @@ int launch_grouped_gemm(const GemmArgs& g, cudaStream_t stream) {
     if (g.R <= 0 || g.E <= 0) return ST_OK;
     if (g.tile_m != 128 && g.K > swap_max_k(g.tile_m)) return ST_UNSUPPORTED;
     CUtensorMap ma, mb;
-    if (!make_map(&ma, g.a, g.R, g.K, g.tile_m < 64 ? g.tile_m : 64)) return ST_CUDA;
+    // gathered A: one-row boxes over the A source rows; tiled A: boxes of up to 64 rows
+    const long long a_rows = g.a_rowmap ? (g.a_rows > 0 ? g.a_rows : 1) : g.R;
+    if (!make_map(&ma, g.a, a_rows, g.K, g.a_rowmap ? 1 : (g.tile_m < 64 ? g.tile_m : 64)))
+        return ST_CUDA;
     if (!make_map(&mb, g.b, static_cast<long long>(g.E) * g.N, g.K, 64)) return ST_CUDA;
     KParams kp;
     kp.R = g.R; kp.N = g.N; kp.K = g.K; kp.E = g.E; kp.nkb = g.K / 128;
@@ -1021,6 +1065,8 @@ int launch_grouped_gemm(const GemmArgs& g, cudaStream_t stream) {
     kp.b_scale = g.b_scale; kp.m_indptr = g.m_indptr;
     kp.hq = g.hq; kp.hs = g.hs;
     kp.y = g.y; kp.ldy = g.ldy; kp.rowmap = g.rowmap;
+    kp.a_rowmap = g.a_rowmap; kp.a_rowdiv = g.a_rowdiv > 0 ? g.a_rowdiv : 1;
+    kp.a_rows = static_cast<int>(a_rows);
     kp.out_bf16 = static_cast<__nv_bfloat16*>(g.out_bf16);
     kp.status = g.status;
     kp.timeout_ns = g.timeout_ns;

@@ -28,6 +28,11 @@ struct GemmArgs {
     // EPI_SWIGLU_QUANT: hq [R, N/2] codes, hs [(N/2)/128, R]
     uint8_t* hq;
     float* hs;
+    // When set, grouped row r reads row a_rowmap[r] / a_rowdiv of A (a_rows
+    // rows) and of its scales, through TMA gather4 loads; null: row r of A.
+    const int32_t* a_rowmap;
+    int a_rowdiv;
+    int a_rows;
     // EPI_Y32: y[r * ldy + n], or y[rowmap[r] * ldy + n] when rowmap is set
     float* y;
     int ldy;
@@ -69,7 +74,8 @@ int launch_router_topk(const float* logits, int T, int E, int k, int32_t* ids, f
 // launch_route_permute; one launch for at most 8 chunks of pairs.
 int launch_router_route(const float* logits, const RouteArgs& r, float* w, cudaStream_t stream);
 
-// x [T, H] bf16 -> xq rows inv_perm[t*k + j] of [R, H], xs [H/128, R];
+// x [T, H] bf16 -> xq rows inv_perm[t*k + j] of [R, H] (row t*k + j when
+// inv_perm is null), xs [H/128, R];
 // also zeroes out_acc [T, H] when not null.
 int launch_quant_scatter(const void* x, int T, int H, int k, int R, const int32_t* inv_perm,
                          uint8_t* xq, float* xs, float* out_acc, cudaStream_t stream);

@@ -87,6 +87,19 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
 }
+// Four rows y0..y3 of a 2-D tensor, each one box of one row (the tensor
+// map's box is one row high) starting at column x, into four consecutive
+// 128-byte rows of shared memory (the map's swizzle applies as for a tiled
+// load of those rows); completion counted on `bar` as transaction bytes.
+__device__ __forceinline__ void tma_gather4_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
+                                               int x, int y0, int y1, int y2, int y3) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2),
+        "r"(y3)
+        : "memory");
+}
 // 2-D tiled store of one box from shared memory (bulk-group completion).
 // Rows or columns of the box outside the tensor are not written.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int x,

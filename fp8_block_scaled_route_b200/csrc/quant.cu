@@ -17,40 +17,63 @@
 
 namespace moe {
 
-// One warp per (token, 128-column block): lane i owns columns 4i..4i+3.
-// Scales go to xs[kb * R + row] (MN-major) or, with xs_kmajor, to
-// xs[row * H/128 + kb].  With eid_out, eid_out[row] = the pair's expert id
-// minus eid_base_div * (id / eid_base_div) (its index inside its owner's
-// expert range).
+// One warp per (token, 512 columns): lane l owns columns 16l..16l+15, and
+// lanes 8b..8b+7 form the 128-column block b of the group (its amax by three
+// shuffles).  Codes = RNE_sat(x / s) with s = amax / 448, both IEEE
+// divides (the scale rule's definition); a lane writes 16 codes (16 bytes)
+// per destination row.
+// Pair p = t*k + j is written to row inv_perm[p] (skipped when negative;
+// row p when inv_perm is null).  Scales go to xs[kb * R + row] (MN-major) or,
+// with xs_kmajor, to xs[row * H/128 + kb].  With eid_out, eid_out[row] = the
+// pair's expert id minus eid_base_div * (id / eid_base_div) (its index inside
+// its owner's expert range).
 __global__ void __launch_bounds__(256) quant_scatter_kernel(
     const __nv_bfloat16* __restrict__ x, int T, int H, int k, int R,
     const int32_t* __restrict__ inv_perm, uint8_t* __restrict__ xq, float* __restrict__ xs,
     float* __restrict__ out_acc, int xs_kmajor, const int32_t* __restrict__ ids,
     int eid_base_div, int32_t* __restrict__ eid_out) {
-    const int nkb = H >> 7;
+    const int ng = (H + 511) >> 9;
     const long long item = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-    if (item >= static_cast<long long>(T) * nkb) return;
+    if (item >= static_cast<long long>(T) * ng) return;
     const int lane = threadIdx.x & 31;
-    const int t = static_cast<int>(item / nkb);
-    const int kb = static_cast<int>(item - static_cast<long long>(t) * nkb);
-    const long long off = static_cast<long long>(t) * H + kb * 128 + lane * 4;
-    uint2 raw = *reinterpret_cast<const uint2*>(x + off);
-    __nv_bfloat162 b01, b23;
-    memcpy(&b01, &raw.x, 4);
-    memcpy(&b23, &raw.y, 4);
-    const float2 f01 = __bfloat1622float2(b01);
-    const float2 f23 = __bfloat1622float2(b23);
-    float amax = fmaxf(fmaxf(fabsf(f01.x), fabsf(f01.y)), fmaxf(fabsf(f23.x), fabsf(f23.y)));
+    const int t = static_cast<int>(item / ng);
+    const int c0 = static_cast<int>(item - static_cast<long long>(t) * ng) * 512 + lane * 16;
+    const bool live = c0 < H;   // H % 128 == 0: a block's eight lanes are all live or none
+    const int nkb = H >> 7;
+    const int kb = c0 >> 7;
+    const long long off = static_cast<long long>(t) * H + c0;
+    float f[16];
+    float amax = 0.0f;
+    if (live) {
+        const uint4* src = reinterpret_cast<const uint4*>(x + off);
+        const uint4 r0 = src[0], r1 = src[1];
+        const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        for (int i = 0; i < 8; ++i) {
+            __nv_bfloat162 b2;
+            memcpy(&b2, &w[i], 4);
+            const float2 v = __bfloat1622float2(b2);
+            f[2 * i] = v.x;
+            f[2 * i + 1] = v.y;
+            amax = fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y)));
+        }
+    }
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if (!live) return;
     const float s = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-    const uint32_t codes = cvt_e4m3x4(__fdiv_rn(f01.x, s), __fdiv_rn(f01.y, s),
-                                      __fdiv_rn(f23.x, s), __fdiv_rn(f23.y, s));
+    uint4 codes;
+    uint32_t* cw = reinterpret_cast<uint32_t*>(&codes);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        cw[i] = cvt_e4m3x4(__fdiv_rn(f[4 * i], s), __fdiv_rn(f[4 * i + 1], s),
+                           __fdiv_rn(f[4 * i + 2], s), __fdiv_rn(f[4 * i + 3], s));
+    const bool lead = (lane & 7) == 0;
     for (int j = 0; j < k; ++j) {
-        const int row = inv_perm[t * k + j];
+        const int row = inv_perm ? inv_perm[t * k + j] : t * k + j;
         if (row < 0) continue;
-        *reinterpret_cast<uint32_t*>(xq + static_cast<long long>(row) * H + kb * 128 + lane * 4) = codes;
-        if (lane == 0) {
+        *reinterpret_cast<uint4*>(xq + static_cast<long long>(row) * H + c0) = codes;
+        if (lead) {
             if (xs_kmajor) xs[static_cast<long long>(row) * nkb + kb] = s;
             else xs[static_cast<long long>(kb) * R + row] = s;
             if (eid_out && kb == 0) {
@@ -59,12 +82,15 @@ __global__ void __launch_bounds__(256) quant_scatter_kernel(
             }
         }
     }
-    if (out_acc) *reinterpret_cast<float4*>(out_acc + off) = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (out_acc) {
+        float4* z = reinterpret_cast<float4*>(out_acc + off);
+        z[0] = z[1] = z[2] = z[3] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
 }
 
 int launch_quant_scatter(const void* x, int T, int H, int k, int R, const int32_t* inv_perm,
                          uint8_t* xq, float* xs, float* out_acc, cudaStream_t stream) {
-    const long long items = static_cast<long long>(T) * (H / 128);
+    const long long items = static_cast<long long>(T) * ((H + 511) / 512);
     if (items == 0) return ST_OK;
     const long long blocks = (items + 7) / 8;
     quant_scatter_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
@@ -76,7 +102,7 @@ int launch_quant_scatter(const void* x, int T, int H, int k, int R, const int32_
 int launch_ep_pack(const void* x, const int32_t* ids, int T, int H, int k, int S,
                    const int32_t* slot_of_pair, int experts_per_rank, uint8_t* xq, float* xs,
                    int32_t* eid, cudaStream_t stream) {
-    const long long items = static_cast<long long>(T) * (H / 128);
+    const long long items = static_cast<long long>(T) * ((H + 511) / 512);
     if (items == 0) return ST_OK;
     const long long blocks = (items + 7) / 8;
     quant_scatter_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(

@@ -61,12 +61,16 @@ def _loopback_layer(ranks, inputs):
     return ds, outs
 
 
-@pytest.mark.parametrize("world,E,H,I,k", [(2, 8, 512, 256, 4), (4, 16, 256, 384, 6)])
-def test_expert_parallel_loopback(world, E, H, I, k):
+@pytest.mark.parametrize("world,E,H,I,k,T0", [
+    (2, 8, 512, 256, 4, 40),       # small groups: swapped GEMM tiles reading rows in place
+    (4, 16, 256, 384, 6, 40),
+    (2, 4, 512, 1024, 2, 330),     # ~330 rows per local expert: 128-token GEMM1 tiles on grouped copies
+])
+def test_expert_parallel_loopback(world, E, H, I, k, T0):
     wts = synth.make_moe_inputs(synth.MoEConfig("w", 1, H, I, E, k), seed=11, device="cuda")
     inputs = []
     for r in range(world):
-        cfg = synth.MoEConfig("ep", 40 + 37 * r, H, I, E, k, "zipf" if r % 2 else "normal")
+        cfg = synth.MoEConfig("ep", T0 + 37 * r, H, I, E, k, "zipf" if r % 2 else "normal")
         inputs.append(synth.make_moe_inputs(cfg, seed=200 + r, device="cuda", weights=False))
     inputs[0]["topk_ids"][3, 0] = -1          # dropped pair
     epr = E // world
