@@ -61,13 +61,14 @@ PROFILE_SLICES = {
 
 
 # DRAM bytes (read + write) per launch of the dominant kernel, GEMM1, taken
-# from the ncu launch list of `bench.py --workload <name>` (see the launch-list
-# summaries under profiles/).  A figure is reported only while the GEMM
-# sources still hash to the digest it was taken with.
+# from the one-pass ncu launch list of `bench.py --workload <name>` on the full
+# workload (see the launch-list summaries under profiles/).  A figure is
+# reported only while the GEMM sources still hash to the digest it was taken
+# with.
 GEMM_SOURCES = ("grouped_gemm.cu", "ptx.cuh", "common.cuh")  # the FP8 GEMM kernel's code
 MEASURED_TRAFFIC = {  # workload -> (source digest, bytes per GEMM1 launch)
-    "prefill": ("f399c64eb0773919", 5906985301),
-    "decode": ("f399c64eb0773919", 6528089344),
+    "prefill": ("f2d5aa45afb014b6", 6030000000),
+    "decode": ("f2d5aa45afb014b6", 6525500000),
 }
 
 
@@ -456,6 +457,7 @@ def run_ours(args, cfg):
                 "stages_us": {n: float(v) * 1e3 for n, v in
                               zip(["route", "quant", "gemm1", "gemm2", "finish"], dst)},
                 "gemm1_gbs": g1_gbs_d, "gemm1_hbm_frac": g1_gbs_d / hbm,
+                "gemm1_traffic": measured_traffic(dcfg.name),
                 "peak_source": f"{src} copy bandwidth",
                 "l2": "inputs larger than L2 (no flush)",
                 "gpu_launches": kernels_per_layer(dcfg.T, dcfg.k) * args.steps}

@@ -109,3 +109,32 @@ def test_expert_parallel_loopback(world, E, H, I, k, T0):
         g = G.bits_to_f64(G.bf16_bits(outs[r]))
         f = G.bits_to_f64(fused["out"])
         assert np.all(np.abs(g - f) <= 2 ** -6 * np.abs(f) + 1e-6), f"ep rank {r} vs fused layer"
+
+
+def test_expert_parallel_nccl_single_rank():
+    """The layer called through its NCCL exchanges (a process group of one
+    rank: every exchange is the rank's own rows) equals moe_fp8_fused."""
+    import os
+    import socket
+    import torch.distributed as dist
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        E, H, I, k = 8, 512, 256, 4
+        wts = synth.make_moe_inputs(synth.MoEConfig("w", 1, H, I, E, k), seed=21, device="cuda")
+        inp = synth.make_moe_inputs(synth.MoEConfig("ep1", 150, H, I, E, k), seed=22,
+                                    device="cuda", weights=False)
+        layer = ep.ExpertParallelMoE(E, wts["w13"], wts["w13_scale"], wts["w2"], wts["w2_scale"])
+        out = layer(inp["x"], inp["topk_ids"], inp["topk_w"])
+        torch.cuda.synchronize()
+        fused = G.run_fused(dict(inp, w13=wts["w13"], w13_scale=wts["w13_scale"], w2=wts["w2"],
+                                 w2_scale=wts["w2_scale"]), debug=False)
+        assert fused["status"] == moe.MOE_OK
+        g = G.bits_to_f64(G.bf16_bits(out))
+        f = G.bits_to_f64(fused["out"])
+        assert np.all(np.abs(g - f) <= 2 ** -6 * np.abs(f) + 1e-6)
+    finally:
+        dist.destroy_process_group()
