@@ -41,6 +41,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "gemm_common.cuh"
 #include "kernels.h"
 
 namespace moe {
@@ -257,70 +258,11 @@ __device__ __forceinline__ float a_scale_at(const KParams& p, int row, int kb) {
     return p.a_scale[static_cast<long long>(row) * p.as_row + static_cast<long long>(kb) * p.as_kb];
 }
 
-// silu with the hardware exp2 and reciprocal (about 2 ulp); its result feeds
-// an FP8 requantisation or a bf16 rounding, whose steps are 2^19 times
-// coarser than that error.
-__device__ __forceinline__ float silu_fast(float z) {
-    return z * rcp_approx(1.0f + __expf(-z));
-}
-
-// Wait of a whole epilogue warp: every lane waits, and the warp proceeds only
-// if every lane succeeded, so warp-collective tcgen05.ld never diverges.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& wc,
-                                          int where) {
-    const bool ok = wait_bar(bar, parity, wc, where);
-    return __all_sync(0xffffffffu, ok) != 0;
-}
-
-// Max over the 32 lanes of each of G values per lane (G = 16 or 32), by a
-// transposing butterfly: afterwards v[0] of lane L holds the maximum of
-// value (L mod G) over all lanes.  G - 1 + (32 / G - 1) * G shuffles instead
-// of 5 * G.
-template <int G>
-__device__ __forceinline__ void warp_transpose_max(float (&v)[G]) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int o = 16; o >= G; o >>= 1) {
-#pragma unroll
-        for (int i = 0; i < G; ++i) v[i] = fmaxf(v[i], __shfl_xor_sync(0xffffffffu, v[i], o));
-    }
-#pragma unroll
-    for (int o = G / 2; o >= 1; o >>= 1) {
-        const bool up = (lane & o) != 0;
-#pragma unroll
-        for (int i = 0; i < o; ++i) {
-            const float send = up ? v[i] : v[i + o];
-            const float keep = up ? v[i + o] : v[i];
-            v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, o));
-        }
-    }
-}
-
-__device__ __forceinline__ bool warp_wait_spin(uint64_t* bar, uint32_t parity, const WaitCtl& wc,
-                                               int where) {
-    const bool ok = wait_bar_spin(bar, parity, wc, where);
-    return __all_sync(0xffffffffu, ok) != 0;
-}
-
 __device__ __forceinline__ bool epi_sync(const Smem& s, uint32_t& phase, const WaitCtl& wc) {
     mbar_arrive(s.epi);
     const bool ok = warp_wait(s.epi, phase, wc, 7);
     phase ^= 1;
     return ok;
-}
-
-template <int BT>
-__device__ __forceinline__ void tmem_load_cols(uint32_t taddr, float (&v)[BT]) {
-    if constexpr (BT == 16) {
-        tmem_ld16(taddr, v);
-    } else if constexpr (BT == 32) {
-        tmem_ld32(taddr, v);
-    } else {
-        float* lo = v;
-        float* hi = v + 32;
-        tmem_ld32(taddr, *reinterpret_cast<float(*)[32]>(lo));
-        tmem_ld32(taddr + 32, *reinterpret_cast<float(*)[32]>(hi));
-    }
 }
 
 // ---------------------------------------------------------------- roles
@@ -482,15 +424,6 @@ __device__ void scale_role(const KParams& p, const Smem& s, const WaitCtl& wc) {
     }
     // copies still in flight land before the CTA exits
     asm volatile("cp.async.wait_all;" ::: "memory");
-}
-
-__device__ __forceinline__ void ffma_chunk(float2* acc, const uint32_t (&v)[32], float f) {
-    const float2 f2 = make_float2(f, f);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const float2 x = make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-        acc[i] = __ffma2_rn(x, f2, acc[i]);
-    }
 }
 
 // Direct orientation epilogue: thread = one token row, 128 of 256 columns.

@@ -220,9 +220,8 @@ def test_fused_tiny():
     (24, 256, 128, 6, 6, "normal"),       # every expert chosen by every token
     (200, 256, 256, 64, 2, "zipf"),       # many empty experts
     (1000, 256, 128, 8, 2, "zipf"),       # balanced 250 rows/expert: 128-row tiles
-    (700, 512, 256, 4, 2, "normal"),      # ~350 rows/expert: CTA-pair GEMM2 tiles, one pair's
-                                          # second CTA without rows
-    (1500, 256, 256, 3, 1, "zipf"),       # ~500 rows/expert, skewed: several pair tiles each
+    (700, 512, 256, 4, 2, "normal"),      # ~350 rows/expert: 128-row tiles with a ragged tail
+    (1500, 256, 256, 3, 1, "zipf"),       # ~500 rows/expert, skewed: several tiles each
 ])
 def test_fused_small_shapes(T, H, I, E, k, routing):
     cfg = synth.MoEConfig("case", T, H, I, E, k, routing)

@@ -42,9 +42,9 @@ def test_wait_timeout_is_reported_and_context_survives():
 
 
 def test_fused_layer_timeout_is_reported_and_context_survives():
-    """The same through the fused layer at a shape whose GEMM2 runs as CTA-pair
-    tiles (both CTAs of each pair give up, drain and leave together)."""
-    cfg = synth.MoEConfig("pairs", 700, 512, 256, 4, 2)
+    """The same through the fused layer at a shape with 128-row tiles: every
+    kernel after the first one that gives up still ends and reports."""
+    cfg = synth.MoEConfig("tiles128", 700, 512, 256, 4, 2)
     inp = synth.make_moe_inputs(cfg, seed=5, device="cuda")
     moe.moe_set_wait_timeout_ns(1)
     try:
