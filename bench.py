@@ -44,12 +44,13 @@ ROUTE_CHUNK = 1024         # (token, slot) pairs per routing chunk
 ROUTE_SMALL_CHUNKS = 8     # up to this many chunks, routing is one single-CTA launch
 
 
-def kernels_per_layer(T: int, k: int) -> int:
+def kernels_per_layer(T: int, k: int, fused: bool = False) -> int:
     """Kernel launches of one fused layer: routing (one launch for inputs of
     at most 8 chunks of 1024 pairs, else histogram/scan/scatter), quant,
-    GEMM1, GEMM2 and the bf16 conversion."""
+    GEMM1 and GEMM2 (one fused-expert launch when the plan fuses them) and
+    the combine."""
     nchunks = (T * k + ROUTE_CHUNK - 1) // ROUTE_CHUNK
-    return (1 if nchunks <= ROUTE_SMALL_CHUNKS else 3) + 4
+    return (1 if nchunks <= ROUTE_SMALL_CHUNKS else 3) + (3 if fused else 4)
 
 
 # Slices of the prefill and decode workloads (same H, I, top-k and routing,
@@ -65,10 +66,10 @@ PROFILE_SLICES = {
 # workload (see the launch-list summaries under profiles/).  A figure is
 # reported only while the GEMM sources still hash to the digest it was taken
 # with.
-GEMM_SOURCES = ("grouped_gemm.cu", "ptx.cuh", "common.cuh")  # the FP8 GEMM kernel's code
+GEMM_SOURCES = ("grouped_gemm.cu", "gemm_common.cuh", "ptx.cuh", "common.cuh")  # its code
 MEASURED_TRAFFIC = {  # workload -> (source digest, bytes per GEMM1 launch)
-    "prefill": ("f2d5aa45afb014b6", 6030000000),
-    "decode": ("f2d5aa45afb014b6", 6525500000),
+    "prefill": ("3bc9296fcdf136a7", 6030000000),
+    "decode": ("3bc9296fcdf136a7", 6525500000),
 }
 
 
@@ -107,6 +108,17 @@ def load_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
+FUSION_MODES = {"auto": 0, "on": 1, "off": 2}   # MOE_FUSION_AUTO / ON / OFF
+
+
+def stage_dict(stage_ms, fused: bool) -> dict:
+    """Per-stage device times (µs) from the layer's stage events."""
+    us = [float(v) * 1e3 for v in stage_ms]
+    if fused:   # events 3 and 4 are recorded back to back after the fused launch
+        return {"route": us[0], "quant": us[1], "experts": us[2] + us[3], "finish": us[4]}
+    return dict(zip(["route", "quant", "gemm1", "gemm2", "finish"], us))
+
+
 def work_counts(cfg: synth.MoEConfig, topk_ids: torch.Tensor):
     """Algorithmic flops and bytes of the layer and of GEMM1, from the actual
     routing (only experts with at least one row are read)."""
@@ -123,8 +135,11 @@ def work_counts(cfg: synth.MoEConfig, topk_ids: torch.Tensor):
     # GEMM1 reads the touched gate/up weights, the FP8 activations and their
     # scales, and writes the FP8 intermediate with its scales
     g1_bytes = touched * w13_b + R * H + 4 * R * (H // 128) + R * I + 4 * R * (I // 128)
+    # the fused-expert launch reads the touched weights of both GEMMs and the
+    # FP8 activations once per token, and writes the fp32 pair rows
+    fx_bytes = touched * (w13_b + w2_b) + cfg.T * H + 4 * cfg.T * (H // 128) + 4 * R * H
     return dict(R=R, touched=touched, flops=flops, bytes=layer_bytes, g1_flops=g1_flops,
-                g1_bytes=g1_bytes)
+                g1_bytes=g1_bytes, fx_bytes=fx_bytes)
 
 
 class ClockSampler:
@@ -266,12 +281,14 @@ def run_ours(args, cfg):
                                 device_id=dev)
         pg = dist
     moe.lib()
+    moe.moe_set_expert_fusion(FUSION_MODES[args.fusion])
     inp = synth.make_moe_inputs(cfg, seed=rank, device=dev)
     T, H, I, E, k = cfg.T, cfg.H, cfg.I, cfg.E, cfg.k
     ws = torch.empty(moe.moe_workspace_size(T, H, I, E, k), dtype=torch.uint8, device=dev)
     out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
     counts = work_counts(cfg, inp["topk_ids"])
+    plan = moe.moe_fp8_fused_plan(T, H, I, E, k)
 
     def step():
         moe.moe_fp8_fused(inp["x"], inp["topk_ids"], inp["topk_w"], inp["w13"], inp["w13_scale"],
@@ -405,20 +422,25 @@ def run_ours(args, cfg):
         value = world * counts["flops"] / (ms_step * 1e-3) / 1e12
         e2e_value = world * counts["flops"] / (e2e_ms / args.steps * 1e-3) / 1e12
         hbm, bf16, bf16_sus, src = load_peaks()
-        g1_ms = float(stage_ms[2])
-        g1_tflops = counts["g1_flops"] / (g1_ms * 1e-3) / 1e12
-        g1_gbs = counts["g1_bytes"] / (g1_ms * 1e-3) / 1e9
+        # the dominant kernel: GEMM1, or the fused-expert launch (both GEMMs)
+        fused = plan["fused"]
+        g1_ms = float(stage_ms[2] + stage_ms[3]) if fused else float(stage_ms[2])
+        k_flops = counts["flops"] if fused else counts["g1_flops"]
+        k_bytes = counts["fx_bytes"] if fused else counts["g1_bytes"]
+        g1_tflops = k_flops / (g1_ms * 1e-3) / 1e12
+        g1_gbs = k_bytes / (g1_ms * 1e-3) / 1e9
         fp8_peak = bf16 * FP8_OVER_BF16
-        t_tensor = counts["g1_flops"] / (fp8_peak * 1e12)
-        t_hbm = counts["g1_bytes"] / (hbm * 1e9)
+        t_tensor = k_flops / (fp8_peak * 1e12)
+        t_hbm = k_bytes / (hbm * 1e9)
         if t_tensor >= t_hbm:
             roof = {"bound": "tensor", "achieved": g1_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
                     "frac": g1_tflops / fp8_peak}
         else:
             roof = {"bound": "hbm", "achieved": g1_gbs, "peak": hbm, "unit": "GB/s",
                     "frac": g1_gbs / hbm}
-        roof.update({"traffic": measured_traffic(cfg.name),
-                     "kernel": "grouped GEMM1 (gate/up + SwiGLU + FP8 requant)",
+        roof.update({"traffic": None if fused else measured_traffic(cfg.name),
+                     "kernel": "fused expert (gate/up + SwiGLU + FP8 requant on chip + down)"
+                     if fused else "grouped GEMM1 (gate/up + SwiGLU + FP8 requant)",
                      "peak_source": f"{src} (FP8 = bf16 burst x {FP8_OVER_BF16:g})"
                      if roof["bound"] == "tensor" else f"{src} copy bandwidth"})
         layer_gbs = counts["bytes"] / (ms_step * 1e-3) / 1e9
@@ -437,12 +459,12 @@ def run_ours(args, cfg):
                       "roofline_frac": layer_frac, "rows": counts["R"],
                       "experts_touched": counts["touched"], "alg_bytes": counts["bytes"],
                       "alg_flops": counts["flops"]},
-            "stages_us": {n: float(v) * 1e3 for n, v in
-                          zip(["route", "quant", "gemm1", "gemm2", "finish"], stage_ms)},
+            "stages_us": stage_dict(stage_ms, fused),
+            "plan": plan,
             "roofline": roof,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": T * H * 2 + T * k * 8, "d2h_bytes_per_step": T * H * 2},
-            "gpu_launches": kernels_per_layer(T, k) * args.steps,
+            "gpu_launches": kernels_per_layer(T, k, fused) * args.steps,
             "clocks": clocks.summary(),
         }
         if dec is not None:
@@ -865,6 +887,9 @@ def main():
     ap.add_argument("--op", default="moe", choices=["moe", "swiglu_mxfp8", "mxfp8_gemm", "mxfp8_moe",
                                                      "nvfp4_gemm", "nvfp4_moe", "router"],
                     help="any other than moe: time that op instead")
+    ap.add_argument("--fusion", default="auto", choices=sorted(FUSION_MODES),
+                    help="FP8 layer: fused-expert launch automatic, forced on (where it fits) "
+                         "or off")
     ap.add_argument("--swiglu-shape", default="",
                     help="with --op swiglu_mxfp8: only this MxK shape (e.g. 8192x7168)")
     args = ap.parse_args()

@@ -9,7 +9,7 @@ Functions keep the C names:
   moe_route_permute, moe_fp8_fused, moe_fp8_fused_debug,
   fp8_groupwise_moe_gemm, swiglu_mxfp8_quant, moe_select_tile_m,
   moe_workspace_size, moe_route_workspace_size, moe_get_device_status,
-  moe_set_wait_timeout_ns, moe_status_string.
+  moe_set_wait_timeout_ns, moe_set_expert_fusion, moe_status_string.
 Tensor arguments may be torch tensors (their data_ptr is passed) or raw
 integer device addresses.
 """
@@ -29,6 +29,8 @@ __all__ = [
     "nvfp4_quantize", "moe_tactic_tune_gemm", "moe_tactic_lookup", "moe_tactic_store",
     "moe_tactic_clear", "moe_ep_workspace_size", "moe_ep_plan", "moe_ep_pack",
     "moe_fp8_expert_rows_workspace_size", "moe_fp8_expert_rows", "moe_combine", "moe_router_route",
+    "moe_set_expert_fusion", "moe_fp8_fused_plan",
+    "MOE_FUSION_AUTO", "MOE_FUSION_ON", "MOE_FUSION_OFF",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -42,6 +44,10 @@ MOE_ERR_NO_TILE_CONFIG = 4
 MOE_ERR_DEVICE_TIMEOUT = 5
 MOE_ERR_BAD_EXPERT_ID = 6
 
+MOE_FUSION_AUTO = 0
+MOE_FUSION_ON = 1
+MOE_FUSION_OFF = 2
+
 # Every symbol declared in include/moefp8.h.
 EXPORTS = (
     "moe_status_string", "moe_route_workspace_size", "moe_route_permute", "moe_workspace_size",
@@ -52,7 +58,8 @@ EXPORTS = (
     "nvfp4_tile_scales", "moe_nvfp4_fused", "moe_nvfp4_fused_debug", "nvfp4_quantize",
     "moe_tactic_tune_gemm", "moe_tactic_lookup", "moe_tactic_store", "moe_tactic_clear",
     "moe_ep_workspace_size", "moe_ep_plan", "moe_ep_pack", "moe_fp8_expert_rows_workspace_size",
-    "moe_fp8_expert_rows", "moe_combine", "moe_router_route",
+    "moe_fp8_expert_rows", "moe_combine", "moe_router_route", "moe_set_expert_fusion",
+    "moe_fp8_fused_plan",
 )
 
 _lib = None
@@ -130,6 +137,10 @@ def lib():
     L.moe_get_device_status.argtypes = [P, P]
     L.moe_set_wait_timeout_ns.restype = None
     L.moe_set_wait_timeout_ns.argtypes = [U64]
+    L.moe_set_expert_fusion.restype = I
+    L.moe_set_expert_fusion.argtypes = [I]
+    L.moe_fp8_fused_plan.restype = I
+    L.moe_fp8_fused_plan.argtypes = [I] * 5 + [P] * 3
     L.moe_route_permute_noalloc.restype = I
     L.moe_route_permute_noalloc.argtypes = [P, I, I, I, P, P, P, P]
     L.moe_set_stage_events.restype = I
@@ -181,6 +192,20 @@ def moe_status_string(status: int) -> str:
 
 def moe_set_wait_timeout_ns(ns: int) -> None:
     lib().moe_set_wait_timeout_ns(int(ns))
+
+
+def moe_set_expert_fusion(mode: int) -> None:
+    """MOE_FUSION_AUTO, MOE_FUSION_ON or MOE_FUSION_OFF (process-wide)."""
+    _check(lib().moe_set_expert_fusion(int(mode)), "moe_set_expert_fusion", True)
+
+
+def moe_fp8_fused_plan(T: int, H: int, I: int, E: int, k: int) -> dict:
+    """Launch plan of moe_fp8_fused on the current device:
+    {"tile_m1", "tile_m2", "fused"}."""
+    a, b, c = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib().moe_fp8_fused_plan(T, H, I, E, k, ctypes.byref(a), ctypes.byref(b),
+                                    ctypes.byref(c)), "moe_fp8_fused_plan", True)
+    return {"tile_m1": a.value, "tile_m2": b.value, "fused": bool(c.value)}
 
 
 def moe_workspace_size(T: int, H: int, I: int, E: int, k: int) -> int:

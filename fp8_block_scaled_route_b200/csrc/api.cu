@@ -25,6 +25,7 @@ namespace {
 __device__ int g_lib_status[kStatusInts];
 
 std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
+std::atomic<int> g_fusion{MOE_FUSION_AUTO};
 
 constexpr int kStageEvents = 6;
 cudaEvent_t g_stage_events[kStageEvents];
@@ -182,6 +183,32 @@ int fit_tile_to_k(int tm, int K) {
     return tm;
 }
 
+// The fused-expert launch runs one expert group per SM, streaming that
+// expert's weights through one SM's share of the memory system; it pays when
+// the active experts fill most SMs (the split GEMMs spread each expert's
+// weights over many SMs, and keep all of them busy for any E).
+bool fuse_pays(int R, int E, int num_sms) {
+    const int active = R < E ? R : E;
+    return 4 * active >= 3 * num_sms;
+}
+
+// Launch plan of the FP8 fused layer: GEMM1 / GEMM2 token tiles and whether
+// both GEMMs run as one fused-expert launch.
+struct LayerPlan {
+    int tm1, tm2;
+    bool fuse;
+};
+
+LayerPlan plan_layer(int R, int H, int I, int E, int num_sms) {
+    LayerPlan pl;
+    pl.tm1 = fit_tile_to_k(choose_tile_m(R, 2 * I, H, E, 1, num_sms), H);
+    pl.tm2 = fit_tile_to_k(choose_tile_m(R, H, I, E, 0, num_sms), I);
+    const int fmode = g_fusion.load();
+    pl.fuse = fmode != MOE_FUSION_OFF && fused_expert_fits(H, I) &&
+              (fmode == MOE_FUSION_ON || (pl.tm1 < 128 && fuse_pays(R, E, num_sms)));
+    return pl;
+}
+
 int check_device(const DevInfo* d) {
     if (!d) return MOE_ERR_CUDA;
     if (d->major != 10 || d->minor != 0) return MOE_ERR_UNSUPPORTED;
@@ -206,6 +233,27 @@ const char* moe_status_string(int status) {
 }
 
 void moe_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns > 0 ? ns : 1); }
+
+int moe_fp8_fused_plan(int T, int H, int I, int E, int k, int* tile_m1, int* tile_m2,
+                       int* fused) {
+    if (T < 0 || H <= 0 || I <= 0 || H % 128 || I % 128 || k < 1 || E < 1 || k > E)
+        return MOE_ERR_INVALID_ARG;
+    if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+    const DevInfo* d = dev_info();
+    if (int st = check_device(d)) return st;
+    const LayerPlan pl = plan_layer(T * k, H, I, E, d->sms);
+    if (tile_m1) *tile_m1 = pl.tm1;
+    if (tile_m2) *tile_m2 = pl.tm2;
+    if (fused) *fused = pl.fuse ? 1 : 0;
+    return MOE_OK;
+}
+
+int moe_set_expert_fusion(int mode) {
+    if (mode != MOE_FUSION_AUTO && mode != MOE_FUSION_ON && mode != MOE_FUSION_OFF)
+        return MOE_ERR_INVALID_ARG;
+    g_fusion.store(mode);
+    return MOE_OK;
+}
 
 int moe_set_stage_events(void* const* events, int n) {
     if (events == nullptr) {
@@ -295,21 +343,40 @@ static int fused_impl(const void* x, const int32_t* topk_ids, const float* topk_
     if (st) return st;
     stage_mark(1, s);
     if (T > 0) {
-        int tm1 = choose_tile_m(R, 2 * I, H, E, 1, d->sms);
-        int tm2 = choose_tile_m(R, H, I, E, 0, d->sms);
-        tm1 = fit_tile_to_k(tm1, H);
-        tm2 = fit_tile_to_k(tm2, I);
+        const LayerPlan pl = plan_layer(R, H, I, E, d->sms);
+        const int tm1 = pl.tm1, tm2 = pl.tm2;
         // Swapped (small-group) GEMM1 tiles gather each grouped row's token
         // row through perm (TMA gather4), so x is quantised once per token
         // ([T, H], scales [H/128, T]).  128-token tiles load their rows as
         // two tiled boxes per K block, which gathered rows cannot match, so
         // there the quantiser writes the k grouped copies ([R, H], [H/128, R]).
+        // The fused-expert launch reads token rows through perm as well.
         const bool gather = tm1 < 128;
-        st = gather ? launch_quant_scatter(x, T, H, 1, T, nullptr, xq, xs, nullptr, s)
-                    : launch_quant_scatter(x, T, H, k, R, inv_perm, xq, xs, nullptr, s);
+        const bool fuse = pl.fuse;
+        const bool per_token = gather || fuse;
+        st = per_token ? launch_quant_scatter(x, T, H, 1, T, nullptr, xq, xs, nullptr, s)
+                       : launch_quant_scatter(x, T, H, k, R, inv_perm, xq, xs, nullptr, s);
         if (st) return st;
         stage_mark(2, s);
         const unsigned long long tmo = g_timeout_ns.load();
+        float* y = out_acc;
+        if (fuse) {
+            FusedExpertArgs f{};
+            f.xq = xq; f.xs = xs; f.perm = perm; f.T = T; f.topk = k; f.R = R; f.H = H; f.I = I;
+            f.E = E; f.w13 = w13; f.w13_scale = w13_scale; f.w2 = w2; f.w2_scale = w2_scale;
+            f.m_indptr = m_indptr; f.y = y;
+            // the intermediate leaves the chip only for the debug outputs
+            f.hq = dbg_hq ? hq : nullptr;
+            f.hs = dbg_hs ? hs : nullptr;
+            f.status = status; f.timeout_ns = tmo; f.num_sms = d->sms;
+            st = launch_fused_expert(f, s);
+            if (st) return st;
+            stage_mark(3, s);
+            stage_mark(4, s);
+            st = launch_combine(y, inv_perm, topk_w, T, k, H, out, s);
+            if (st) return st;
+            stage_mark(5, s);
+        } else {
         GemmArgs g1{};
         g1.a = xq; g1.b = w13; g1.R = R; g1.N = 2 * I; g1.K = H; g1.E = E;
         g1.a_scale = xs; g1.as_row = 1; g1.as_kb = gather ? T : R; g1.b_scale = w13_scale;
@@ -321,7 +388,6 @@ static int fused_impl(const void* x, const int32_t* topk_ids, const float* topk_
         stage_mark(3, s);
         // GEMM2 writes each pair's row y once, in grouped order; the combine
         // then sums each token's k rows in ascending slot order
-        float* y = out_acc;
         GemmArgs g2{};
         g2.a = hq; g2.b = w2; g2.R = R; g2.N = H; g2.K = I; g2.E = E;
         g2.a_scale = hs; g2.as_row = 1; g2.as_kb = R; g2.b_scale = w2_scale;
@@ -334,6 +400,7 @@ static int fused_impl(const void* x, const int32_t* topk_ids, const float* topk_
         st = launch_combine(y, inv_perm, topk_w, T, k, H, out, s);
         if (st) return st;
         stage_mark(5, s);
+        }
     }
     if (dbg_m_indptr &&
         cudaMemcpyAsync(dbg_m_indptr, m_indptr, sizeof(int32_t) * (E + 1), cudaMemcpyDeviceToDevice, s))

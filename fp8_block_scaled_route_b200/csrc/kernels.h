@@ -50,6 +50,34 @@ int launch_grouped_gemm(const GemmArgs& g, cudaStream_t stream);
 // Largest K the swapped (tile_m < 128) kernels accept for a token tile.
 int swap_max_k(int tile_m);
 
+// Both expert GEMMs in one launch with the FP8 intermediate in shared memory
+// (fused_expert.cu).  Token rows come from xq [T, H] (one copy per token) with
+// scales xs [H/128, T]; grouped row r reads token perm[r] / topk.  Writes the
+// fp32 rows y [R, H] in grouped order, and the intermediate to hq [R, I] /
+// hs [I/128, R] when those are set.
+struct FusedExpertArgs {
+    const void* xq;
+    const float* xs;
+    const int32_t* perm;
+    int T, topk, R, H, I, E;
+    const void* w13;          // [E, 2I, H]
+    const float* w13_scale;   // [E, 2I/128, H/128]
+    const void* w2;           // [E, H, I]
+    const float* w2_scale;    // [E, H/128, I/128]
+    const int32_t* m_indptr;  // [E+1]
+    float* y;
+    uint8_t* hq;
+    float* hs;
+    int* status;
+    uint64_t timeout_ns;
+    int num_sms;
+};
+
+// Whether the fused expert kernel can hold the intermediate of a 64-token
+// tile for this H, I (and enough pipeline stages) in shared memory.
+bool fused_expert_fits(int H, int I);
+int launch_fused_expert(const FusedExpertArgs& g, cudaStream_t stream);
+
 struct RouteArgs {
     const int32_t* topk_ids;
     int T, k, E;

@@ -534,6 +534,34 @@ MOE_API int moe_get_device_status(const void* ws, moe_stream_t stream);
  * events = NULL switches it off.  Process-wide setting. */
 MOE_API int moe_set_stage_events(void* const* events, int n);
 
+/* How moe_fp8_fused and moe_fp8_fused_debug run the two expert GEMMs.
+ *   MOE_FUSION_AUTO (default): one fused-expert launch when the FP8
+ *     intermediate of a 64-token group (I bytes per token) fits in shared
+ *     memory beside the weight pipeline, the groups are small (the tile
+ *     model picks weight-stationary GEMM1 tiles) and enough experts are
+ *     active to occupy the SMs; otherwise GEMM1 and GEMM2 as two launches.
+ *   MOE_FUSION_ON: the fused launch whenever the intermediate fits.
+ *   MOE_FUSION_OFF: always two launches.
+ * The fused launch keeps each group's intermediate on chip: it is written
+ * to the workspace only for moe_fp8_fused_debug's outputs.  Both paths give
+ * the same quantised intermediate and sum each K block's partial products
+ * in the same order.  With fusion, stage event 3 and 4 are recorded
+ * back to back after the fused launch.  Process-wide; returns
+ * MOE_ERR_INVALID_ARG for an unknown mode. */
+/* The launch plan moe_fp8_fused would use on the calling thread's current
+ * device for these sizes and the current fusion mode: the GEMM1 and GEMM2
+ * token tiles (16, 32, 64: weight-stationary; 128: token-stationary) and
+ * whether both GEMMs run as one fused-expert launch (*fused = 1).  Any
+ * output pointer may be NULL.  Returns MOE_ERR_INVALID_ARG for sizes
+ * moe_fp8_fused rejects, MOE_ERR_UNSUPPORTED off sm_100. */
+MOE_API int moe_fp8_fused_plan(int T, int H, int I, int E, int k, int* tile_m1, int* tile_m2,
+                               int* fused);
+
+#define MOE_FUSION_AUTO 0
+#define MOE_FUSION_ON 1
+#define MOE_FUSION_OFF 2
+MOE_API int moe_set_expert_fusion(int mode);
+
 /* Upper bound, in nanoseconds of %globaltimer, on every spin-wait inside the
  * kernels launched by later calls from this process (default 2e9).  A wait
  * that runs out sets MOE_ERR_DEVICE_TIMEOUT and the kernel returns early. */

@@ -15,7 +15,15 @@ Tolerances (one place, used by every GPU test):
     ulps.  The largest difference over every GPU test is 6.8e-7 (0.71 of
     the bound).
   * final bf16 output: relative L2 error <= 1e-2 and max abs error
-    <= 2e-2 * rms(reference).
+    <= 2e-2 * rms(reference).  The max bound applies to the output rows of
+    tokens whose k intermediate rows carry exactly the oracle's codes.  A
+    token with one of the allowed adjacent codes is checked, with both
+    bounds, against the oracle's down GEMM and combine run on the GPU's own
+    intermediate: one E4M3 step of an element near its block's maximum is
+    1/16-1/8 of that element, which moves an output element by a few
+    percent of the rms on its own (seen: 2.3e-2 with a single differing
+    code out of 102400), so no element bound can hold across an allowed
+    code difference.  The relative L2 bound applies end to end.
 """
 from __future__ import annotations
 
@@ -32,7 +40,8 @@ OUT_MAX_ABS_RMS = 2e-2
 # Worst values seen by the comparisons of this test session (written out by
 # tests/conftest.py when MOE_PARITY_STATS names a file).
 STATS = {"scale_rel_max": 0.0, "code_match_min": 1.0, "out_rel_l2_max": 0.0,
-         "out_max_abs_rms_max": 0.0, "calls": 0}
+         "out_max_abs_rms_max": 0.0, "calls": 0, "rows_with_code_diff": 0,
+         "out_max_abs_rms_e2e_code_diff_rows": 0.0}
 
 # Guard bytes after every output buffer the helpers hand to the library: any
 # write past the end of a buffer changes them.
@@ -119,6 +128,20 @@ def compare_scales(gpu: np.ndarray, ref: np.ndarray, what: str, rtol: float = SC
     assert float(rel.max(initial=0.0)) <= rtol, f"{what}: scale rel diff {rel.max():.3e}"
 
 
+def compare_out_l2(gpu_bits: np.ndarray, ref_bits: np.ndarray, what: str):
+    g = bits_to_f64(gpu_bits)
+    r = bits_to_f64(ref_bits)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite output"
+    if not r.size or not np.any(r):
+        assert np.array_equal(g, r), what
+        return 0.0
+    rel_l2 = float(np.linalg.norm(g - r) / np.linalg.norm(r))
+    STATS["out_rel_l2_max"] = max(STATS["out_rel_l2_max"], rel_l2)
+    STATS["calls"] += 1
+    assert rel_l2 <= OUT_REL_L2, f"{what}: relative L2 {rel_l2:.3e}"
+    return rel_l2
+
+
 def compare_out(gpu_bits: np.ndarray, ref_bits: np.ndarray, what: str):
     g = bits_to_f64(gpu_bits)
     r = bits_to_f64(ref_bits)
@@ -135,6 +158,89 @@ def compare_out(gpu_bits: np.ndarray, ref_bits: np.ndarray, what: str):
     assert rel_l2 <= OUT_REL_L2, f"{what}: relative L2 {rel_l2:.3e}"
     assert max_abs <= OUT_MAX_ABS_RMS, f"{what}: max abs {max_abs:.3e} x rms"
     return rel_l2, max_abs
+
+
+def _max_abs_rms(gpu_bits, ref_bits, rms):
+    g = bits_to_f64(gpu_bits)
+    r = bits_to_f64(ref_bits)
+    assert np.all(np.isfinite(g)), "non-finite output"
+    return float(np.abs(g - r).max(initial=0.0) / rms) if rms > 0 else \
+        (0.0 if np.array_equal(g, r) else np.inf)
+
+
+def own_h_rows(tok_rows, hq, hs, w2, w2_scale, experts, topk_w):
+    """The oracle's down GEMM and combine on given intermediate rows:
+    tok_rows[i] = the k grouped rows of one token (-1: dropped pair),
+    experts[i] = their experts.  Returns bf16 bits [n, H]."""
+    import oracle as O
+    n, k = tok_rows.shape
+    H = w2.shape[1]
+    y = np.zeros((n * k, H), np.float32)
+    inv = np.full(n * k, -1, np.int32)
+    for i in range(n):
+        for j in range(k):
+            r = int(tok_rows[i, j])
+            if r < 0:
+                continue
+            e = int(experts[i, j])
+            y[i * k + j] = O.grouped_gemm(hq[r:r + 1], hs[r:r + 1], w2[e:e + 1], w2_scale[e:e + 1],
+                                          np.array([0, 1], np.int32))[0]
+            inv[i * k + j] = i * k + j
+    return O.combine(y, inv, topk_w)
+
+
+def compare_layer_rows(out_gpu, out_ref, hq_gpu_tok, hq_ref_tok, own_h, what):
+    """Output check of a fused layer on n tokens: out_* [n, H] bf16 bits,
+    hq_*_tok [n, k*I] the tokens' intermediate codes (pairs in slot order),
+    own_h(idx) -> bf16 bits of the oracle's down GEMM + combine on the GPU's
+    intermediate for the tokens idx.  Bounds as in the module docstring."""
+    g = bits_to_f64(out_gpu)
+    r = bits_to_f64(out_ref)
+    rms = float(np.sqrt(np.mean(r * r))) if r.size else 0.0
+    compare_out_l2(out_gpu, out_ref, what)
+    diff = np.any(np.asarray(hq_gpu_tok) != np.asarray(hq_ref_tok), axis=1)
+    same = ~diff
+    m = _max_abs_rms(out_gpu[same], out_ref[same], rms)
+    STATS["out_max_abs_rms_max"] = max(STATS["out_max_abs_rms_max"], m)
+    assert m <= OUT_MAX_ABS_RMS, f"{what}: max abs {m:.3e} x rms"
+    if diff.any():
+        idx = np.nonzero(diff)[0]
+        STATS["rows_with_code_diff"] += int(idx.size)
+        STATS["out_max_abs_rms_e2e_code_diff_rows"] = max(
+            STATS["out_max_abs_rms_e2e_code_diff_rows"], _max_abs_rms(out_gpu[idx], out_ref[idx], rms))
+        own = own_h(idx)
+        go = bits_to_f64(out_gpu[idx])
+        ro = bits_to_f64(own)
+        rel = float(np.linalg.norm(go - ro) / max(np.linalg.norm(ro), 1e-300))
+        assert rel <= OUT_REL_L2, f"{what}: rows with a differing code: relative L2 {rel:.3e}"
+        mo = _max_abs_rms(out_gpu[idx], own, rms)
+        assert mo <= OUT_MAX_ABS_RMS, f"{what}: rows with a differing code: max abs {mo:.3e} x rms"
+
+
+def compare_layer(res: dict, ref: dict, inp: dict, what: str):
+    """compare_layer_rows over a whole layer: res from run_fused(debug=True),
+    ref from the oracle's moe_fused on the same inputs (routing tables
+    already checked equal)."""
+    ids = i32(inp["topk_ids"])
+    T, k = ids.shape
+    perm = ref["perm"]
+    inv = np.full(T * k, -1, np.int64)
+    inv[perm] = np.arange(len(perm))
+    I = res["hq"].shape[1] if res["hq"].ndim == 2 else 0
+    rows = inv.reshape(T, k)
+
+    def tok_codes(hq):
+        z = np.zeros((T, k, I), np.uint8)
+        ok = rows >= 0
+        z[ok] = hq[rows[ok]]
+        return z.reshape(T, k * I)
+
+    def own_h(idx):
+        return own_h_rows(rows[idx], res["hq"], res["hs"], u8(inp["w2"]), f32(inp["w2_scale"]),
+                           ids[idx], f32(inp["topk_w"])[idx])
+
+    compare_layer_rows(res["out"], ref["out"], tok_codes(res["hq"]), tok_codes(ref["hq"]), own_h,
+                       what)
 
 
 def oracle_args(inp: dict):

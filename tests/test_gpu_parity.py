@@ -205,7 +205,7 @@ def _check_fused_full(inp, what):
     assert np.array_equal(res["perm"], ref["perm"]), what
     G.compare_codes(res["hq"], ref["hq"], what + " intermediate codes")
     G.compare_scales(res["hs"], ref["hs"], what + " intermediate scales")
-    G.compare_out(res["out"], ref["out"], what + " output")
+    G.compare_layer(res, ref, inp, what + " output")
 
 
 def test_fused_tiny():
@@ -246,7 +246,8 @@ def test_fused_bad_expert_ids():
     ref = O.moe_fused(*G.oracle_args(inp))
     assert ref["n_bad"] == 2
     assert np.array_equal(res["m_indptr"], ref["m_indptr"])
-    G.compare_out(res["out"], ref["out"], "bad ids")
+    assert np.array_equal(res["perm"], ref["perm"])
+    G.compare_layer(res, ref, inp, "bad ids")
 
 
 def _check_sampled(inp, tokens, what):
@@ -263,10 +264,19 @@ def _check_sampled(inp, tokens, what):
                                      sub["w13_scale"], sub["w2"], sub["w2_scale"],
                                      np.arange(len(tokens), dtype=np.int32), want_h=True)
     k = inp["topk_ids"].shape[1]
+    n = len(tokens)
     rows = np.array([[i_o[t * k + j] for j in range(k)] for t in tokens])
-    G.compare_codes(res["hq"][rows.ravel()], hq_o.reshape(len(tokens) * k, -1), what + " codes")
-    G.compare_scales(res["hs"][rows.ravel()], hs_o.reshape(len(tokens) * k, -1), what + " scales")
-    G.compare_out(res["out"][tokens], out_o, what + " output")
+    G.compare_codes(res["hq"][rows.ravel()], hq_o.reshape(n * k, -1), what + " codes")
+    G.compare_scales(res["hs"][rows.ravel()], hs_o.reshape(n * k, -1), what + " scales")
+    ids = G.i32(inp["topk_ids"])[tokens]
+    tw = G.f32(inp["topk_w"])[tokens]
+    w2, w2s = G.u8(inp["w2"]), G.f32(inp["w2_scale"])
+
+    def own_h(idx):
+        return G.own_h_rows(rows[idx], res["hq"], res["hs"], w2, w2s, ids[idx], tw[idx])
+
+    G.compare_layer_rows(res["out"][tokens], out_o, res["hq"][rows.ravel()].reshape(n, -1),
+                         hq_o.reshape(n, -1), own_h, what + " output")
 
 
 def test_fused_mid_sampled():

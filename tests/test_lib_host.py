@@ -63,6 +63,16 @@ def test_status_strings(L):
         assert moe.moe_status_string(code) == name
 
 
+def test_expert_fusion_mode_setter(L):
+    assert L.moe_set_expert_fusion(moe.MOE_FUSION_OFF) == moe.MOE_OK
+    assert L.moe_set_expert_fusion(moe.MOE_FUSION_ON) == moe.MOE_OK
+    assert L.moe_set_expert_fusion(7) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_set_expert_fusion(-1) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_set_expert_fusion(moe.MOE_FUSION_AUTO) == moe.MOE_OK
+    with pytest.raises(moe.MoEError):
+        moe.moe_set_expert_fusion(3)
+
+
 def test_tile_selector_matches_oracle(L, oracle):
     rng = np.random.default_rng(0)
     for _ in range(3000):
