@@ -136,8 +136,8 @@ def work_counts(cfg: synth.MoEConfig, topk_ids: torch.Tensor):
     # scales, and writes the FP8 intermediate with its scales
     g1_bytes = touched * w13_b + R * H + 4 * R * (H // 128) + R * I + 4 * R * (I // 128)
     # the fused-expert launch reads the touched weights of both GEMMs and the
-    # FP8 activations once per token, and writes the fp32 pair rows
-    fx_bytes = touched * (w13_b + w2_b) + cfg.T * H + 4 * cfg.T * (H // 128) + 4 * R * H
+    # grouped FP8 activation rows with their scales, and writes the fp32 pair rows
+    fx_bytes = touched * (w13_b + w2_b) + R * H + 4 * R * (H // 128) + 4 * R * H
     return dict(R=R, touched=touched, flops=flops, bytes=layer_bytes, g1_flops=g1_flops,
                 g1_bytes=g1_bytes, fx_bytes=fx_bytes)
 

@@ -183,13 +183,20 @@ int fit_tile_to_k(int tm, int K) {
     return tm;
 }
 
-// The fused-expert launch runs one expert group per SM, streaming that
-// expert's weights through one SM's share of the memory system; it pays when
-// the active experts fill most SMs (the split GEMMs spread each expert's
-// weights over many SMs, and keep all of them busy for any E).
-bool fuse_pays(int R, int E, int num_sms) {
-    const int active = R < E ? R : E;
-    return 4 * active >= 3 * num_sms;
+// The fused-expert launch runs each (expert, 64-token group) on one SM,
+// streaming that expert's weights through one SM's share of the memory
+// system; the split GEMMs spread every expert's weights over many SMs.
+// Measured on B200 (whole layer, µs, fused / split, top-8): T=512 H=2048
+// I=768 E=128: 166 / 212; T=1024 H=1024 I=512 E=160: 141 / 154.  A second
+// round of items (T=64 E=256: 267 / 215), half the SMs idle (E=64, top-4:
+// 305 / 263) or 12.6 MB experts (H=4096 I=1024: 317 / 297) lose.  So: about
+// one round of items filling at least half the SMs, experts of at most 6 MB.
+bool fuse_pays(int R, int H, int I, int E, int num_sms) {
+    const long long per = (static_cast<long long>(R) + E - 1) / E;   // rows per expert, balanced
+    const long long active = R < E ? R : E;
+    const long long items = active * ((per + 63) / 64);
+    return items <= num_sms + num_sms / 8 && 2 * items >= num_sms &&
+           3LL * H * I <= 6000000LL;
 }
 
 // Launch plan of the FP8 fused layer: GEMM1 / GEMM2 token tiles and whether
@@ -204,8 +211,8 @@ LayerPlan plan_layer(int R, int H, int I, int E, int num_sms) {
     pl.tm1 = fit_tile_to_k(choose_tile_m(R, 2 * I, H, E, 1, num_sms), H);
     pl.tm2 = fit_tile_to_k(choose_tile_m(R, H, I, E, 0, num_sms), I);
     const int fmode = g_fusion.load();
-    pl.fuse = fmode != MOE_FUSION_OFF && fused_expert_fits(H, I) &&
-              (fmode == MOE_FUSION_ON || (pl.tm1 < 128 && fuse_pays(R, E, num_sms)));
+    pl.fuse = fmode != MOE_FUSION_OFF && fused_expert_fits(H, I, E) &&
+              (fmode == MOE_FUSION_ON || (pl.tm1 < 128 && fuse_pays(R, H, I, E, num_sms)));
     return pl;
 }
 
@@ -350,10 +357,11 @@ static int fused_impl(const void* x, const int32_t* topk_ids, const float* topk_
         // ([T, H], scales [H/128, T]).  128-token tiles load their rows as
         // two tiled boxes per K block, which gathered rows cannot match, so
         // there the quantiser writes the k grouped copies ([R, H], [H/128, R]).
-        // The fused-expert launch reads token rows through perm as well.
-        const bool gather = tm1 < 128;
+        // The fused-expert launch reads the grouped copies too (one tiled box
+        // of 64 rows per K block).
         const bool fuse = pl.fuse;
-        const bool per_token = gather || fuse;
+        const bool gather = tm1 < 128 && !fuse;
+        const bool per_token = gather;
         st = per_token ? launch_quant_scatter(x, T, H, 1, T, nullptr, xq, xs, nullptr, s)
                        : launch_quant_scatter(x, T, H, k, R, inv_perm, xq, xs, nullptr, s);
         if (st) return st;
@@ -362,7 +370,7 @@ static int fused_impl(const void* x, const int32_t* topk_ids, const float* topk_
         float* y = out_acc;
         if (fuse) {
             FusedExpertArgs f{};
-            f.xq = xq; f.xs = xs; f.perm = perm; f.T = T; f.topk = k; f.R = R; f.H = H; f.I = I;
+            f.xq = xq; f.xs = xs; f.R = R; f.H = H; f.I = I;
             f.E = E; f.w13 = w13; f.w13_scale = w13_scale; f.w2 = w2; f.w2_scale = w2_scale;
             f.m_indptr = m_indptr; f.y = y;
             // the intermediate leaves the chip only for the debug outputs

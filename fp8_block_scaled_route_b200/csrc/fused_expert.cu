@@ -14,15 +14,19 @@
 // (expert, 64-token tile); an item streams its expert's gate/up weights once
 // (phase 1, K = H) and its down weights once (phase 2, K = I).
 //
-//  * warp 0 - producer: phase 1 stages the tile's token rows (TMA gather4
-//    through the grouping, four rows per instruction) and two 128-row gate /
-//    up weight blocks per K block; phase 2 stages two 128-row down-weight
-//    blocks per K block (the tokens are already on chip).
+//  * warp 0 - producer: phase 1 stages the tile's 64 grouped token rows (one
+//    tiled TMA box) and two 128-row gate / up weight blocks per K block;
+//    phase 2 stages two 128-row down-weight blocks per K block (the tokens
+//    are already on chip).
 //  * warp 1 - MMA issue (one elected lane): per K block two M=128, N=64
 //    tcgen05.mma groups (one per weight block) into a TMEM slot; phase 2
 //    reads its N operand (the intermediate codes) from shared memory, once
 //    the epilogue has written all of them for the item.
-//  * warps 4-7 - epilogue, thread = one weight row of each block: promotes
+//  * warp 3 - scale loader: stages every item's activation scales and its
+//    expert's gate/up and down weight-block scales in shared memory (two
+//    buffers, one item ahead), so no promotion waits on a global load.
+//  * warps 4-11 - epilogue, thread = one weight row of each block and one
+//    half of the 64 tokens (two warps per TMEM lane quadrant): promotes
 //    every K block (acc += partial * a_scale * b_scale); after phase 1's K
 //    loop of a 128-column block: h = silu(gate) * up, per-token amax over the
 //    block's 128 columns (warp transposing max + shared memory), scale =
@@ -47,7 +51,8 @@ bool make_tma_map_fp8(CUtensorMap* out, const void* ptr, long long rows, long lo
 namespace fx {
 
 constexpr int BT = 64;                        // tokens per work item (MMA N)
-constexpr int EPI_WARPS = 4;
+constexpr int EPI_WARPS = 8;                  // two per TMEM lane quadrant
+constexpr int HT = BT / 2;                    // tokens per epilogue warp
 constexpr int THREADS = 128 + 32 * EPI_WARPS;
 constexpr int A_BYTES = BT * 128;             // token rows of one K block
 constexpr int B_BYTES = 256 * 128;            // two 128-row weight blocks
@@ -56,29 +61,34 @@ constexpr int A_OFF = B_BYTES;                // weights first: both 1024-aligne
 constexpr int TSLOTS = 512 / (2 * BT);        // 4 TMEM slots of 2 x 64 columns
 constexpr int kSmemLimit = 232448;
 constexpr int kMaxE = 1024;
-constexpr int kTableBytes = ((2 * (kMaxE + 1) * 4) + 15) / 16 * 16;
-constexpr int XCH_BYTES = (EPI_WARPS + 2) * BT * 4;
+constexpr int XCH_BYTES = 6 * BT * 4;
 constexpr int BAR_BYTES = 512;
 constexpr int MAX_STAGES = 6;
 constexpr int MIN_STAGES = 3;
 
-// Shared memory: 1024 (alignment) + stages + intermediate codes
-// [I/128][64 rows x 128 B] + phase-1 activation scales [H/128][64] +
-// intermediate scales [I/128][64] + exchange + tables + barriers.
-__host__ __device__ inline int fixed_bytes(int H, int I) {
-    return 1024 + I * BT + (H / 128) * BT * 4 + (I / 128) * BT * 4 + XCH_BYTES + kTableBytes +
-           BAR_BYTES;
+// One item's scales: activations [H/128][BT], gate/up weight blocks
+// [2I/128][H/128], down weight blocks [H/128][I/128]; 16-byte multiple.
+__host__ __device__ inline int scale_buf_floats(int H, int I) {
+    return ((H / 128) * BT + 3 * (I / 128) * (H / 128) + 3) / 4 * 4;
 }
-__host__ __device__ inline int stages_for(int H, int I) {
-    const int n = (kSmemLimit - fixed_bytes(H, I)) / STAGE_BYTES;
+__host__ __device__ inline int table_bytes(int E) { return (2 * (E + 1) * 4 + 15) / 16 * 16; }
+
+// Shared memory: 1024 (alignment) + stages + intermediate codes
+// [I/128][64 rows x 128 B] + two scale buffers + intermediate scales
+// [I/128][64] + exchange + item tables + barriers.
+__host__ __device__ inline int fixed_bytes(int H, int I, int E) {
+    return 1024 + I * BT + 2 * scale_buf_floats(H, I) * 4 + (I / 128) * BT * 4 + XCH_BYTES +
+           table_bytes(E) + BAR_BYTES;
+}
+__host__ __device__ inline int stages_for(int H, int I, int E) {
+    const int n = (kSmemLimit - fixed_bytes(H, I, E)) / STAGE_BYTES;
     return n > MAX_STAGES ? MAX_STAGES : n;
 }
 
 struct Params {
-    int R, H, I, E, T, topk;
+    int R, H, I, E;
     int nstages;
-    const float* xs;          // [H/128, T] activation scales (per token)
-    const int32_t* perm;      // grouped row -> pair id
+    const float* xs;          // [H/128, R] activation scales of the grouped rows
     const float* w13_scale;   // [E, 2I/128, H/128]
     const float* w2_scale;    // [E, H/128, I/128]
     const int32_t* m_indptr;  // [E+1]
@@ -92,7 +102,7 @@ struct Params {
 struct Smem {
     uint8_t* stages;
     uint8_t* hq;      // [I/128][BT x 128 B], swizzled
-    float* as1;       // [H/128][BT]
+    float* sc;        // two scale buffers of scale_buf_floats
     float* hs;        // [I/128][BT]
     float* xch;
     int* tstart;
@@ -101,6 +111,8 @@ struct Smem {
     uint64_t* empty;
     uint64_t* tfull;
     uint64_t* tempty;
+    uint64_t* sfull;
+    uint64_t* sempty;
     uint64_t* hready;
     uint64_t* drain;
     uint64_t* epi;
@@ -115,21 +127,23 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const Params& p) {
     q += p.nstages * STAGE_BYTES;
     s.hq = q;
     q += p.I * BT;
-    s.as1 = reinterpret_cast<float*>(q);
-    q += (p.H / 128) * BT * 4;
+    s.sc = reinterpret_cast<float*>(q);
+    q += 2 * scale_buf_floats(p.H, p.I) * 4;
     s.hs = reinterpret_cast<float*>(q);
     q += (p.I / 128) * BT * 4;
     s.xch = reinterpret_cast<float*>(q);
     q += XCH_BYTES;
     s.tstart = reinterpret_cast<int*>(q);
-    s.mind = s.tstart + (kMaxE + 1);
-    q += kTableBytes;
+    s.mind = s.tstart + (p.E + 1);
+    q += table_bytes(p.E);
     uint64_t* bars = reinterpret_cast<uint64_t*>(q);
     s.full = bars;
     s.empty = bars + MAX_STAGES;
     s.tfull = bars + 2 * MAX_STAGES;
-    s.tempty = bars + 2 * MAX_STAGES + TSLOTS;
-    s.hready = bars + 2 * MAX_STAGES + 2 * TSLOTS;
+    s.tempty = s.tfull + TSLOTS;
+    s.sfull = s.tempty + TSLOTS;
+    s.sempty = s.sfull + 2;
+    s.hready = s.sempty + 2;
     s.drain = s.hready + 1;
     s.epi = s.hready + 2;
     s.tmem = reinterpret_cast<uint32_t*>(s.hready + 3);
@@ -156,35 +170,22 @@ __device__ __forceinline__ Item decode(int t, const Smem& s, const Params& p) {
     return it;
 }
 
-// Token (row of x) that grouped row r reads.
-__device__ __forceinline__ int token_of(const Params& p, int r) {
-    const int rr = min(max(r, 0), p.R - 1);
-    const int tok = __ldg(p.perm + rr) / p.topk;
-    return min(max(tok, 0), p.T - 1);
-}
-
-// Phase-2 column tiles (256 weight rows each) and their second block.
+// Phase-2 column tiles (256 weight rows each).
 __device__ __forceinline__ int ntiles2(const Params& p) { return (p.H + 255) >> 8; }
 
 __device__ void producer(const CUtensorMap* tmA, const CUtensorMap* tmW13, const CUtensorMap* tmW2,
                          const Params& p, const Smem& s, const WaitCtl& wc, int total) {
     const int l = threadIdx.x & 31;
-    const bool g_lane = l < BT / 4;   // one gather4 of four token rows
     const bool b_lane = l < 4;        // one 64-row weight box
+    const bool a_lane = l == 4;       // the 64 token rows
     const int nkb1 = p.H >> 7, nkb2 = p.I >> 7, nt1s = p.I >> 7, nt2s = ntiles2(p);
     uint32_t stage = 0, phase = 0, armed = 0, armed_par = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const Item it = decode(t, s, p);
-        int g0 = 0, g1 = 0, g2 = 0, g3 = 0;
-        if (g_lane) {
-            const int r = it.row0 + 4 * l;
-            g0 = token_of(p, 4 * l + 0 < it.rows ? r + 0 : it.row0);
-            g1 = token_of(p, 4 * l + 1 < it.rows ? r + 1 : it.row0);
-            g2 = token_of(p, 4 * l + 2 < it.rows ? r + 2 : it.row0);
-            g3 = token_of(p, 4 * l + 3 < it.rows ? r + 3 : it.row0);
-        }
-        // phase 1: gate block nt, up block nt (rows e*2I + nt*128 and e*2I + I + nt*128)
+        // phase 1: gate block nt, up block nt (rows e*2I + nt*128 and e*2I + I + nt*128);
+        // token rows past the item's own (the next expert's, or past R:
+        // zero-filled) are loaded but carry a zero scale
         for (int nt = 0; nt < nt1s && ok; ++nt) {
             const int wrow = it.e * 2 * p.I + (l >> 1) * p.I + nt * 128 + (l & 1) * 64;
             for (int kb = 0; kb < nkb1; ++kb) {
@@ -192,10 +193,8 @@ __device__ void producer(const CUtensorMap* tmA, const CUtensorMap* tmW13, const
                 uint8_t* st = s.stages + stage * STAGE_BYTES;
                 if (l == 0) mbar_arrive_expect_tx(&s.full[stage], STAGE_BYTES);
                 __syncwarp();
-                if (g_lane)
-                    tma_gather4_2d(st + A_OFF + l * 4 * 128, tmA, &s.full[stage], kb * 128, g0, g1, g2,
-                                   g3);
                 if (b_lane) tma_load_2d(st + l * 64 * 128, tmW13, &s.full[stage], kb * 128, wrow);
+                if (a_lane) tma_load_2d(st + A_OFF, tmA, &s.full[stage], kb * 128, it.row0);
                 __syncwarp();
                 armed |= 1u << stage;
                 armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
@@ -270,6 +269,32 @@ __device__ void mma(const Params& p, const Smem& s, const WaitCtl& wc, uint32_t 
     __syncwarp();
 }
 
+// Scale loader: item n of this CTA goes to buffer n % 2; every lane arrives
+// on the buffer's full barrier after its own plain stores.
+__device__ void scale_loader(const Params& p, const Smem& s, const WaitCtl& wc, int total) {
+    const int lane = threadIdx.x & 31;
+    const int nkb1 = p.H >> 7, nkb2 = p.I >> 7, nt1s = p.I >> 7, nblk2 = p.H >> 7;
+    const int nbuf = scale_buf_floats(p.H, p.I);
+    uint32_t n = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++n) {
+        const uint32_t b = n & 1u, par = (n >> 1) & 1u;
+        if (!warp_wait(&s.sempty[b], par ^ 1u, wc, 8)) return;
+        const Item it = decode(t, s, p);
+        float* as = s.sc + b * nbuf;
+        float* w13s = as + nkb1 * BT;
+        float* w2s = w13s + 2 * nt1s * nkb1;
+        for (int idx = lane; idx < nkb1 * BT; idx += 32) {
+            const int kb = idx / BT, j = idx - kb * BT;
+            as[idx] = j < it.rows ? __ldg(p.xs + static_cast<long long>(kb) * p.R + it.row0 + j) : 0.0f;
+        }
+        const float* g13 = p.w13_scale + static_cast<long long>(it.e) * 2 * nt1s * nkb1;
+        for (int idx = lane; idx < 2 * nt1s * nkb1; idx += 32) w13s[idx] = __ldg(g13 + idx);
+        const float* g2 = p.w2_scale + static_cast<long long>(it.e) * nblk2 * nkb2;
+        for (int idx = lane; idx < nblk2 * nkb2; idx += 32) w2s[idx] = __ldg(g2 + idx);
+        mbar_arrive(&s.sfull[b]);
+    }
+}
+
 __device__ __forceinline__ bool epi_sync(const Smem& s, uint32_t& phase, const WaitCtl& wc) {
     mbar_arrive(s.epi);
     const bool ok = warp_wait(s.epi, phase, wc, 7);
@@ -286,62 +311,55 @@ __device__ __forceinline__ int sw128_off(int j, int c) {
 __device__ void epilogue(const Params& p, const Smem& s, const WaitCtl& wc, uint32_t tmem_base,
                          int total) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int q = warp & 3;
-    const int w = q * 32 + lane;          // weight row inside each 128-row block
-    const int et = threadIdx.x - 128;     // epilogue thread 0..127
+    const int q = warp & 3;                       // TMEM lane quadrant
+    const int hb = ((warp - 4) >> 2) * HT;        // first token of this warp's half
+    const int w = q * 32 + lane;                  // weight row inside each 128-row block
+    const int et = threadIdx.x - 128;             // epilogue thread 0..255
     const int nkb1 = p.H >> 7, nkb2 = p.I >> 7, nt1s = p.I >> 7, nt2s = ntiles2(p);
     const int nblk2 = p.H >> 7;
-    uint32_t buf = 0, bphase = 0, ephase = 0;
-    float* red = s.xch;                   // [4 warps][BT] partial amax
-    float* s_sc = s.xch + 4 * BT;         // [BT] scale of each token's block
-    float* s_inv = s.xch + 5 * BT;        // [BT] its reciprocal
-    float acc0[BT], acc1[BT];
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+    const int nbuf = scale_buf_floats(p.H, p.I);
+    uint32_t buf = 0, bphase = 0, ephase = 0, n = 0;
+    float* red = s.xch;                   // [4 quadrants][BT] partial amax
+    float* s_inv = s.xch + 4 * BT;        // [BT] reciprocal of each token's block scale
+    float acc0[HT], acc1[HT];
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++n) {
         const Item it = decode(t, s, p);
-        // this item's phase-1 activation scales, [kb][token]
-        if (!epi_sync(s, ephase, wc)) return;
-        for (int idx = et; idx < nkb1 * BT; idx += 128) {
-            const int kb = idx / BT, j = idx - kb * BT;
-            s.as1[idx] = j < it.rows ? p.xs[static_cast<long long>(kb) * p.T + token_of(p, it.row0 + j)]
-                                     : 0.0f;
-        }
-        if (!epi_sync(s, ephase, wc)) return;
+        const uint32_t sb = n & 1u;
+        if (!warp_wait(&s.sfull[sb], (n >> 1) & 1u, wc, 9)) return;
+        const float* as1 = s.sc + sb * nbuf;
+        const float* w13s = as1 + nkb1 * BT;
+        const float* w2s = w13s + 2 * nt1s * nkb1;
         for (int ph = 0; ph < 2; ++ph) {
             const int ntiles = ph == 0 ? nt1s : nt2s;
             const int nkb = ph == 0 ? nkb1 : nkb2;
-            const float* ascale = ph == 0 ? s.as1 : s.hs;
+            const float* ascale = ph == 0 ? as1 : s.hs;
             for (int nt = 0; nt < ntiles; ++nt) {
                 // weight-block scales of this column tile: gate/up (phase 1) or down blocks 2nt, 2nt+1
                 const bool v1 = ph == 0 || 2 * nt + 1 < nblk2;
-                const float* bs0 = ph == 0
-                    ? p.w13_scale + (static_cast<long long>(it.e) * 2 * nt1s + nt) * nkb1
-                    : p.w2_scale + (static_cast<long long>(it.e) * nblk2 + 2 * nt) * nkb2;
-                const float* bs1 = ph == 0
-                    ? p.w13_scale + (static_cast<long long>(it.e) * 2 * nt1s + nt1s + nt) * nkb1
-                    : (v1 ? bs0 + nkb2 : bs0);
+                const float* bs0 = ph == 0 ? w13s + nt * nkb1 : w2s + 2 * nt * nkb2;
+                const float* bs1 = ph == 0 ? w13s + (nt1s + nt) * nkb1 : (v1 ? bs0 + nkb2 : bs0);
 #pragma unroll
-                for (int j = 0; j < BT; ++j) { acc0[j] = 0.0f; acc1[j] = 0.0f; }
-                float b0n = __ldg(bs0), b1n = __ldg(bs1);
+                for (int j = 0; j < HT; ++j) { acc0[j] = 0.0f; acc1[j] = 0.0f; }
                 for (int kb = 0; kb < nkb; ++kb) {
-                    const float b0 = b0n, b1 = b1n;
-                    if (kb + 1 < nkb) { b0n = __ldg(bs0 + kb + 1); b1n = __ldg(bs1 + kb + 1); }
+                    const float b0 = bs0[kb], b1 = bs1[kb];
                     if (!warp_wait(&s.tfull[buf], bphase, wc, 6)) return;
                     tc_fence_after();
-                    const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * (2 * BT);
-                    const float4* asv = reinterpret_cast<const float4*>(ascale + kb * BT);
-                    float v[BT];
-                    tmem_load_cols<BT>(taddr, v);
+                    const uint32_t taddr =
+                        tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * (2 * BT) + hb;
+                    const float4* asv = reinterpret_cast<const float4*>(ascale + kb * BT + hb);
+                    float v[HT];
+                    tmem_load_cols<HT>(taddr, v);
 #pragma unroll
-                    for (int j4 = 0; j4 < BT / 4; ++j4) {
+                    for (int j4 = 0; j4 < HT / 4; ++j4) {
                         const float4 a4 = asv[j4];
                         acc0[4 * j4 + 0] = fmaf(v[4 * j4 + 0], a4.x * b0, acc0[4 * j4 + 0]);
                         acc0[4 * j4 + 1] = fmaf(v[4 * j4 + 1], a4.y * b0, acc0[4 * j4 + 1]);
                         acc0[4 * j4 + 2] = fmaf(v[4 * j4 + 2], a4.z * b0, acc0[4 * j4 + 2]);
                         acc0[4 * j4 + 3] = fmaf(v[4 * j4 + 3], a4.w * b0, acc0[4 * j4 + 3]);
                     }
-                    tmem_load_cols<BT>(taddr + BT, v);
+                    tmem_load_cols<HT>(taddr + BT, v);
 #pragma unroll
-                    for (int j4 = 0; j4 < BT / 4; ++j4) {
+                    for (int j4 = 0; j4 < HT / 4; ++j4) {
                         const float4 a4 = asv[j4];
                         acc1[4 * j4 + 0] = fmaf(v[4 * j4 + 0], a4.x * b1, acc1[4 * j4 + 0]);
                         acc1[4 * j4 + 1] = fmaf(v[4 * j4 + 1], a4.y * b1, acc1[4 * j4 + 1]);
@@ -355,24 +373,21 @@ __device__ void epilogue(const Params& p, const Smem& s, const WaitCtl& wc, uint
                 }
                 if (ph == 0) {
                     // SwiGLU, per-token amax over the block's 128 columns, FP8 codes of column w
+                    float m[HT];
 #pragma unroll
-                    for (int g0 = 0; g0 < BT; g0 += 32) {
-                        float m[32];
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const float h = silu_fast(acc0[g0 + i]) * acc1[g0 + i];
-                            acc0[g0 + i] = h;
-                            m[i] = fabsf(h);
-                        }
-                        warp_transpose_max<32>(m);
-                        red[q * BT + g0 + lane] = m[0];
+                    for (int i = 0; i < HT; ++i) {
+                        const float h = silu_fast(acc0[i]) * acc1[i];
+                        acc0[i] = h;
+                        m[i] = fabsf(h);
                     }
+                    // afterwards lane L holds this warp's max for token hb + L
+                    warp_transpose_max<HT>(m);
+                    red[q * BT + hb + lane] = m[0];
                     if (!epi_sync(s, ephase, wc)) return;
                     if (et < BT) {
                         const float amax = fmaxf(fmaxf(red[et], red[BT + et]),
                                                  fmaxf(red[2 * BT + et], red[3 * BT + et]));
                         const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-                        s_sc[et] = sc;
                         s_inv[et] = __frcp_rn(sc);
                         s.hs[nt * BT + et] = sc;
                         if (p.hs && et < it.rows)
@@ -381,8 +396,9 @@ __device__ void epilogue(const Params& p, const Smem& s, const WaitCtl& wc, uint
                     if (!epi_sync(s, ephase, wc)) return;
                     uint8_t* tile = s.hq + nt * A_BYTES;
 #pragma unroll
-                    for (int j = 0; j < BT; ++j) {
-                        const uint8_t c = static_cast<uint8_t>(cvt_e4m3x2(acc0[j] * s_inv[j], 0.0f) & 0xFF);
+                    for (int i = 0; i < HT; ++i) {
+                        const int j = hb + i;
+                        const uint8_t c = static_cast<uint8_t>(cvt_e4m3x2(acc0[i] * s_inv[j], 0.0f) & 0xFF);
                         tile[sw128_off(j, w)] = c;
                         if (p.hq && j < it.rows)
                             p.hq[static_cast<long long>(it.row0 + j) * p.I + nt * 128 + w] = c;
@@ -396,16 +412,20 @@ __device__ void epilogue(const Params& p, const Smem& s, const WaitCtl& wc, uint
                 } else {
                     const int colA = nt * 256 + w;
 #pragma unroll
-                    for (int j = 0; j < BT; ++j) {
+                    for (int i = 0; i < HT; ++i) {
+                        const int j = hb + i;
                         if (j < it.rows) {
                             float* rowp = p.y + static_cast<long long>(it.row0 + j) * p.H;
-                            rowp[colA] = acc0[j];
-                            if (v1) rowp[colA + 128] = acc1[j];
+                            rowp[colA] = acc0[i];
+                            if (v1) rowp[colA + 128] = acc1[i];
                         }
                     }
                 }
             }
         }
+        // this item's scale buffer may be refilled
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.sempty[sb]);
     }
 }
 
@@ -426,6 +446,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int i = 0; i < TSLOTS; ++i) {
             mbar_init(&s.tfull[i], 1);
             mbar_init(&s.tempty[i], EPI_WARPS);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s.sfull[i], 32);
+            mbar_init(&s.sempty[i], EPI_WARPS);
         }
         mbar_init(s.hready, EPI_WARPS);
         mbar_init(s.drain, 1);
@@ -477,6 +501,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int total = s.tstart[p.E];
     if (warp == 0) producer(&tmA, &tmW13, &tmW2, p, s, wc, total);
     else if (warp == 1) mma(p, s, wc, tmem_base, total);
+    else if (warp == 3) scale_loader(p, s, wc, total);
     else if (warp >= 4) epilogue(p, s, wc, tmem_base, total);
     tc_fence_before();
     __syncthreads();
@@ -486,24 +511,25 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 }  // namespace fx
 
-bool fused_expert_fits(int H, int I) {
-    return H % 128 == 0 && I % 128 == 0 && fx::stages_for(H, I) >= fx::MIN_STAGES;
+bool fused_expert_fits(int H, int I, int E) {
+    return H % 128 == 0 && I % 128 == 0 && E >= 1 && E <= fx::kMaxE &&
+           fx::stages_for(H, I, E) >= fx::MIN_STAGES;
 }
 
 int launch_fused_expert(const FusedExpertArgs& g, cudaStream_t stream) {
     if (g.R <= 0 || g.E <= 0) return ST_OK;
-    if (!fused_expert_fits(g.H, g.I) || g.E > fx::kMaxE) return ST_UNSUPPORTED;
+    if (!fused_expert_fits(g.H, g.I, g.E)) return ST_UNSUPPORTED;
     CUtensorMap ma, m13, m2;
-    if (!make_tma_map_fp8(&ma, g.xq, g.T, g.H, 1)) return ST_CUDA;
+    if (!make_tma_map_fp8(&ma, g.xq, g.R, g.H, fx::BT)) return ST_CUDA;
     if (!make_tma_map_fp8(&m13, g.w13, static_cast<long long>(g.E) * 2 * g.I, g.H, 64)) return ST_CUDA;
     if (!make_tma_map_fp8(&m2, g.w2, static_cast<long long>(g.E) * g.H, g.I, 64)) return ST_CUDA;
     fx::Params p{};
-    p.R = g.R; p.H = g.H; p.I = g.I; p.E = g.E; p.T = g.T; p.topk = g.topk > 0 ? g.topk : 1;
-    p.nstages = fx::stages_for(g.H, g.I);
-    p.xs = g.xs; p.perm = g.perm; p.w13_scale = g.w13_scale; p.w2_scale = g.w2_scale;
+    p.R = g.R; p.H = g.H; p.I = g.I; p.E = g.E;
+    p.nstages = fx::stages_for(g.H, g.I, g.E);
+    p.xs = g.xs; p.w13_scale = g.w13_scale; p.w2_scale = g.w2_scale;
     p.m_indptr = g.m_indptr; p.y = g.y; p.hq = g.hq; p.hs = g.hs;
     p.status = g.status; p.timeout_ns = g.timeout_ns;
-    const int smem = fx::fixed_bytes(g.H, g.I) + p.nstages * fx::STAGE_BYTES;
+    const int smem = fx::fixed_bytes(g.H, g.I, g.E) + p.nstages * fx::STAGE_BYTES;
     static int configured_dev = -1;  // one-time opt-in to the largest dynamic shared memory
     int dev = 0;
     cudaGetDevice(&dev);

@@ -50,16 +50,15 @@ int launch_grouped_gemm(const GemmArgs& g, cudaStream_t stream);
 // Largest K the swapped (tile_m < 128) kernels accept for a token tile.
 int swap_max_k(int tile_m);
 
-// Both expert GEMMs in one launch with the FP8 intermediate in shared memory
-// (fused_expert.cu).  Token rows come from xq [T, H] (one copy per token) with
-// scales xs [H/128, T]; grouped row r reads token perm[r] / topk.  Writes the
+// Both expert GEMMs in one launch with the FP8 intermediate in shared
+// memory (fused_expert.cu).  Reads the grouped token rows xq [R, H] with
+// their scales xs [H/128, R] (the quantiser's k-copy layout).  Writes the
 // fp32 rows y [R, H] in grouped order, and the intermediate to hq [R, I] /
 // hs [I/128, R] when those are set.
 struct FusedExpertArgs {
     const void* xq;
     const float* xs;
-    const int32_t* perm;
-    int T, topk, R, H, I, E;
+    int R, H, I, E;
     const void* w13;          // [E, 2I, H]
     const float* w13_scale;   // [E, 2I/128, H/128]
     const void* w2;           // [E, H, I]
@@ -74,8 +73,8 @@ struct FusedExpertArgs {
 };
 
 // Whether the fused expert kernel can hold the intermediate of a 64-token
-// tile for this H, I (and enough pipeline stages) in shared memory.
-bool fused_expert_fits(int H, int I);
+// tile for this H, I, E (and enough pipeline stages) in shared memory.
+bool fused_expert_fits(int H, int I, int E);
 int launch_fused_expert(const FusedExpertArgs& g, cudaStream_t stream);
 
 struct RouteArgs {

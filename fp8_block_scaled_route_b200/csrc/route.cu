@@ -138,16 +138,23 @@ __global__ void __launch_bounds__(32) route_scatter(const int32_t* __restrict__ 
     }
 }
 
-// Small inputs (at most kSmallChunks chunks): the same three phases in one
-// CTA of 1024 threads, so routing costs one launch.  Warp c owns chunk c in
-// phases 1 and 3; thread e owns expert e in phase 2.  The per-chunk tables
-// live in shared memory.
+// Small inputs (at most kSmallChunks chunks of 1024 pairs): the same three
+// phases in one CTA of 1024 threads, so routing costs one launch.  The pairs
+// are cut into up to 32 consecutive blocks, one per warp (as many as keep the
+// per-block histograms within 48 KB of shared memory), so the serial ranking
+// steps of phase 3 are spread over the warps; thread e owns expert e in
+// phase 2.
 constexpr int kSmallChunks = 8;
-static_assert(kSmallChunks * kMaxRouteExperts * sizeof(int) <= 48 * 1024,
-              "route_small's histogram table must fit the default shared-memory limit");
+constexpr int kSmallTabInts = 11 * 1024;  // 44 KB: with the static scan table within 48 KB
+
+__host__ __device__ constexpr int small_route_warps(int E) {
+    return E * 32 <= kSmallTabInts ? 32 : kSmallTabInts / E;
+}
+static_assert(small_route_warps(kMaxRouteExperts) >= kSmallChunks,
+              "route_small's pair blocks must stay within kRouteChunk pairs");
 
 // The three phases of route_small for a CTA of 1024 threads; tab is
-// [kSmallChunks][E] ints of shared memory.
+// [small_route_warps(E)][E] ints of shared memory.
 __device__ __forceinline__ void route_small_body(const int32_t* __restrict__ ids, int R, int E,
                                                  int32_t* __restrict__ m_indptr,
                                                  int32_t* __restrict__ perm,
@@ -155,15 +162,18 @@ __device__ __forceinline__ void route_small_body(const int32_t* __restrict__ ids
                                                  int* tab) {
     __shared__ int warp_tot[32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nchunks = (R + kRouteChunk - 1) / kRouteChunk;
+    const int W = small_route_warps(E);
+    // pairs per block: a multiple of 32, at most kRouteChunk (R <= 8 chunks, W >= 8)
+    const int B = ((R + W - 1) / W + 31) & ~31;
+    const int nchunks = B > 0 ? (R + B - 1) / B : 0;
     constexpr int kSteps = kRouteChunk / 32;
     for (int i = threadIdx.x; i < nchunks * E; i += blockDim.x) tab[i] = 0;
     __syncthreads();
-    // phase 1: per-chunk histograms
+    // phase 1: per-block histograms
     int my_ids[kSteps];
-    const int base = warp * kRouteChunk;
+    const int base = warp * B;
     if (warp < nchunks) {
-        const int end = min(R, base + kRouteChunk);
+        const int end = min(R, base + B);
         int bad = 0;
 #pragma unroll
         for (int i = 0; i < kSteps; ++i) {
@@ -221,9 +231,9 @@ __device__ __forceinline__ void route_small_body(const int32_t* __restrict__ ids
     }
     if (e == E - 1) m_indptr[E] = excl + count;
     __syncthreads();
-    // phase 3: stable scatter, 32 pairs at a time per chunk
+    // phase 3: stable scatter, 32 pairs at a time per block
     if (warp < nchunks) {
-        const int end = min(R, base + kRouteChunk);
+        const int end = min(R, base + B);
         int* cursor = tab + warp * E;
 #pragma unroll
         for (int i = 0; i < kSteps; ++i) {
@@ -253,7 +263,7 @@ __global__ void __launch_bounds__(1024) route_small(const int32_t* __restrict__ 
                                                     int32_t* __restrict__ m_indptr,
                                                     int32_t* __restrict__ perm,
                                                     int32_t* __restrict__ inv_perm, int* status) {
-    extern __shared__ int tab[];  // [kSmallChunks][E]: histograms, then first rows
+    extern __shared__ int tab[];  // [blocks][E]: histograms, then first rows
     route_small_body(ids, R, E, m_indptr, perm, inv_perm, status, tab);
 }
 
@@ -351,7 +361,7 @@ int launch_router_route(const float* logits, const RouteArgs& r, float* w, cudaS
     const int nchunks = (R + kRouteChunk - 1) / kRouteChunk;
     if (nchunks <= kSmallChunks) {
         int32_t* ids = const_cast<int32_t*>(r.topk_ids);
-        const size_t smem = static_cast<size_t>(kSmallChunks) * r.E * sizeof(int);
+        const size_t smem = static_cast<size_t>(small_route_warps(r.E)) * r.E * sizeof(int);
         if (r.E <= 256)
             router_route_small<8><<<1, 1024, smem, stream>>>(logits, r.T, r.E, r.k, ids, w,
                                                              r.m_indptr, r.perm, r.inv_perm, r.status);
@@ -370,8 +380,8 @@ int launch_route_permute(const RouteArgs& r, cudaStream_t stream) {
     const int nchunks = (R + kRouteChunk - 1) / kRouteChunk;
     const size_t hist_smem = static_cast<size_t>(r.E) * sizeof(int);
     if (nchunks <= kSmallChunks) {
-        // at most 8 x 1024 ints = 32 KB: within the default dynamic shared-memory limit
-        const size_t smem = static_cast<size_t>(kSmallChunks) * r.E * sizeof(int);
+        // within the default dynamic shared-memory limit (48 KB)
+        const size_t smem = static_cast<size_t>(small_route_warps(r.E)) * r.E * sizeof(int);
         route_small<<<1, 1024, smem, stream>>>(r.topk_ids, R, r.E, r.m_indptr, r.perm, r.inv_perm,
                                                r.status);
         return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;

@@ -103,7 +103,8 @@ def test_fused_expert_bad_ids_and_zero_tokens(fusion_on):
     assert res["status"] == moe.MOE_ERR_BAD_EXPERT_ID
     ref = O.moe_fused(*G.oracle_args(inp))
     assert np.array_equal(res["m_indptr"], ref["m_indptr"])
-    assert np.array_equal(res["perm"], ref["perm"])
+    n = int(ref["m_indptr"][-1])
+    assert np.array_equal(res["perm"][:n], ref["perm"])
     G.compare_layer(res, ref, inp, "fused expert, bad ids")
     empty = synth.make_moe_inputs(synth.MoEConfig("empty", 0, 256, 128, 4, 2), seed=1, device=DEV)
     res = G.run_fused(empty, debug=True)

@@ -246,7 +246,8 @@ def test_fused_bad_expert_ids():
     ref = O.moe_fused(*G.oracle_args(inp))
     assert ref["n_bad"] == 2
     assert np.array_equal(res["m_indptr"], ref["m_indptr"])
-    assert np.array_equal(res["perm"], ref["perm"])
+    n = int(ref["m_indptr"][-1])
+    assert np.array_equal(res["perm"][:n], ref["perm"])
     G.compare_layer(res, ref, inp, "bad ids")
 
 
