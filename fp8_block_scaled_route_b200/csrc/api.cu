@@ -185,18 +185,23 @@ int fit_tile_to_k(int tm, int K) {
 
 // The fused-expert launch runs each (expert, 64-token group) on one SM,
 // streaming that expert's weights through one SM's share of the memory
-// system; the split GEMMs spread every expert's weights over many SMs.
-// Measured on B200 (whole layer, µs, fused / split, top-8): T=512 H=2048
-// I=768 E=128: 166 / 212; T=1024 H=1024 I=512 E=160: 141 / 154.  A second
-// round of items (T=64 E=256: 267 / 215), half the SMs idle (E=64, top-4:
-// 305 / 263) or 12.6 MB experts (H=4096 I=1024: 317 / 297) lose.  So: about
-// one round of items filling at least half the SMs, experts of at most 6 MB.
+// system (the groups of one expert run side by side and share its weights
+// through L2); the split GEMMs spread every expert's weights over many SMs.
+// Measured on B200 (whole layer, µs, fused / split, top-8): H=2048 I=768
+// E=128 at T=512: 160 / 213, at T=2048: 385 / 496; T=1024 H=1024 I=512
+// E=160: 135 / 152; T=16 H=256 I=128 E=4: 31 / 34.  A second round of
+// experts (T=64 E=256: 253 / 213), half the SMs idle (E=64, top-4:
+// 287 / 263) or 12.6 MB experts (H=4096 I=1024: 308 / 296) lose.  So: tiny
+// layers (one launch fewer), else about one round of active experts filling
+// at least half the SMs, at most ~2 rounds of groups, experts of <= 6 MB.
 bool fuse_pays(int R, int H, int I, int E, int num_sms) {
     const long long per = (static_cast<long long>(R) + E - 1) / E;   // rows per expert, balanced
     const long long active = R < E ? R : E;
     const long long items = active * ((per + 63) / 64);
-    return items <= num_sms + num_sms / 8 && 2 * items >= num_sms &&
-           3LL * H * I <= 6000000LL;
+    const long long expert_bytes = 3LL * H * I;
+    if (active * expert_bytes <= (16LL << 20)) return true;
+    return active <= num_sms + num_sms / 8 && 2 * active >= num_sms &&
+           items <= 2 * num_sms + num_sms / 4 && expert_bytes <= 6000000LL;
 }
 
 // Launch plan of the FP8 fused layer: GEMM1 / GEMM2 token tiles and whether
@@ -341,10 +346,13 @@ static int fused_impl(const void* x, const int32_t* topk_ids, const float* topk_
     uint8_t* hq = reinterpret_cast<uint8_t*>(b + L.hq);
     float* hs = reinterpret_cast<float*>(b + L.hs);
     float* out_acc = reinterpret_cast<float*>(b + L.out_acc);
-    if (cudaMemsetAsync(status, 0, sizeof(int) * kStatusInts, s) != cudaSuccess) return MOE_ERR_CUDA;
     const int R = T * k;
+    // the single-launch routing kernel clears the status words itself
+    const bool route_clears = route_single_launch(R);
+    if (!route_clears && cudaMemsetAsync(status, 0, sizeof(int) * kStatusInts, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
     RouteArgs ra{topk_ids, T, k, E, m_indptr, perm, inv_perm,
-                 reinterpret_cast<int32_t*>(b + L.chunk_hist), status};
+                 reinterpret_cast<int32_t*>(b + L.chunk_hist), status, route_clears ? 1 : 0};
     stage_mark(0, s);
     int st = launch_route_permute(ra, s);
     if (st) return st;

@@ -321,7 +321,8 @@ __device__ void epilogue(const Params& p, const Smem& s, const WaitCtl& wc, uint
     uint32_t buf = 0, bphase = 0, ephase = 0, n = 0;
     float* red = s.xch;                   // [4 quadrants][BT] partial amax
     float* s_inv = s.xch + 4 * BT;        // [BT] reciprocal of each token's block scale
-    float acc0[HT], acc1[HT];
+    // accumulators as token pairs: acc0[i] = tokens hb + 2i, hb + 2i + 1 of block 0
+    float2 acc0[HT / 2], acc1[HT / 2];
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++n) {
         const Item it = decode(t, s, p);
         const uint32_t sb = n & 1u;
@@ -339,46 +340,58 @@ __device__ void epilogue(const Params& p, const Smem& s, const WaitCtl& wc, uint
                 const float* bs0 = ph == 0 ? w13s + nt * nkb1 : w2s + 2 * nt * nkb2;
                 const float* bs1 = ph == 0 ? w13s + (nt1s + nt) * nkb1 : (v1 ? bs0 + nkb2 : bs0);
 #pragma unroll
-                for (int j = 0; j < HT; ++j) { acc0[j] = 0.0f; acc1[j] = 0.0f; }
+                for (int i = 0; i < HT / 2; ++i) {
+                    acc0[i] = make_float2(0.0f, 0.0f);
+                    acc1[i] = make_float2(0.0f, 0.0f);
+                }
                 for (int kb = 0; kb < nkb; ++kb) {
-                    const float b0 = bs0[kb], b1 = bs1[kb];
+                    const float2 b0 = make_float2(bs0[kb], bs0[kb]);
+                    const float2 b1 = make_float2(bs1[kb], bs1[kb]);
                     if (!warp_wait(&s.tfull[buf], bphase, wc, 6)) return;
                     tc_fence_after();
                     const uint32_t taddr =
                         tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * (2 * BT) + hb;
-                    const float4* asv = reinterpret_cast<const float4*>(ascale + kb * BT + hb);
-                    float v[HT];
-                    tmem_load_cols<HT>(taddr, v);
-#pragma unroll
-                    for (int j4 = 0; j4 < HT / 4; ++j4) {
-                        const float4 a4 = asv[j4];
-                        acc0[4 * j4 + 0] = fmaf(v[4 * j4 + 0], a4.x * b0, acc0[4 * j4 + 0]);
-                        acc0[4 * j4 + 1] = fmaf(v[4 * j4 + 1], a4.y * b0, acc0[4 * j4 + 1]);
-                        acc0[4 * j4 + 2] = fmaf(v[4 * j4 + 2], a4.z * b0, acc0[4 * j4 + 2]);
-                        acc0[4 * j4 + 3] = fmaf(v[4 * j4 + 3], a4.w * b0, acc0[4 * j4 + 3]);
-                    }
-                    tmem_load_cols<HT>(taddr + BT, v);
-#pragma unroll
-                    for (int j4 = 0; j4 < HT / 4; ++j4) {
-                        const float4 a4 = asv[j4];
-                        acc1[4 * j4 + 0] = fmaf(v[4 * j4 + 0], a4.x * b1, acc1[4 * j4 + 0]);
-                        acc1[4 * j4 + 1] = fmaf(v[4 * j4 + 1], a4.y * b1, acc1[4 * j4 + 1]);
-                        acc1[4 * j4 + 2] = fmaf(v[4 * j4 + 2], a4.z * b1, acc1[4 * j4 + 2]);
-                        acc1[4 * j4 + 3] = fmaf(v[4 * j4 + 3], a4.w * b1, acc1[4 * j4 + 3]);
-                    }
+                    // both blocks' partials in flight before one wait
+                    uint32_t u0[HT], u1[HT];
+                    tmem_ld32_async(taddr, u0);
+                    tmem_ld32_async(taddr + BT, u1);
+                    tmem_wait_ld(u0);
+                    tmem_wait_ld(u1);
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&s.tempty[buf]);
                     if (++buf == TSLOTS) { buf = 0; bphase ^= 1; }
+                    // acc += partial * (a_scale * b_scale), two tokens per instruction
+                    const float4* asv = reinterpret_cast<const float4*>(ascale + kb * BT + hb);
+#pragma unroll
+                    for (int j4 = 0; j4 < HT / 4; ++j4) {
+                        const float4 a4 = asv[j4];
+                        const float2 alo = make_float2(a4.x, a4.y), ahi = make_float2(a4.z, a4.w);
+                        const float2 p0lo = __fmul2_rn(alo, b0), p0hi = __fmul2_rn(ahi, b0);
+                        const float2 p1lo = __fmul2_rn(alo, b1), p1hi = __fmul2_rn(ahi, b1);
+                        acc0[2 * j4] = __ffma2_rn(
+                            make_float2(__uint_as_float(u0[4 * j4]), __uint_as_float(u0[4 * j4 + 1])), p0lo,
+                            acc0[2 * j4]);
+                        acc0[2 * j4 + 1] = __ffma2_rn(
+                            make_float2(__uint_as_float(u0[4 * j4 + 2]), __uint_as_float(u0[4 * j4 + 3])),
+                            p0hi, acc0[2 * j4 + 1]);
+                        acc1[2 * j4] = __ffma2_rn(
+                            make_float2(__uint_as_float(u1[4 * j4]), __uint_as_float(u1[4 * j4 + 1])), p1lo,
+                            acc1[2 * j4]);
+                        acc1[2 * j4 + 1] = __ffma2_rn(
+                            make_float2(__uint_as_float(u1[4 * j4 + 2]), __uint_as_float(u1[4 * j4 + 3])),
+                            p1hi, acc1[2 * j4 + 1]);
+                    }
                 }
                 if (ph == 0) {
                     // SwiGLU, per-token amax over the block's 128 columns, FP8 codes of column w
-                    float m[HT];
+                    float m[HT], h[HT];
 #pragma unroll
                     for (int i = 0; i < HT; ++i) {
-                        const float h = silu_fast(acc0[i]) * acc1[i];
-                        acc0[i] = h;
-                        m[i] = fabsf(h);
+                        const float g = (i & 1) ? acc0[i >> 1].y : acc0[i >> 1].x;
+                        const float u = (i & 1) ? acc1[i >> 1].y : acc1[i >> 1].x;
+                        h[i] = silu_fast(g) * u;
+                        m[i] = fabsf(h[i]);
                     }
                     // afterwards lane L holds this warp's max for token hb + L
                     warp_transpose_max<HT>(m);
@@ -398,7 +411,7 @@ __device__ void epilogue(const Params& p, const Smem& s, const WaitCtl& wc, uint
 #pragma unroll
                     for (int i = 0; i < HT; ++i) {
                         const int j = hb + i;
-                        const uint8_t c = static_cast<uint8_t>(cvt_e4m3x2(acc0[i] * s_inv[j], 0.0f) & 0xFF);
+                        const uint8_t c = static_cast<uint8_t>(cvt_e4m3x2(h[i] * s_inv[j], 0.0f) & 0xFF);
                         tile[sw128_off(j, w)] = c;
                         if (p.hq && j < it.rows)
                             p.hq[static_cast<long long>(it.row0 + j) * p.I + nt * 128 + w] = c;
@@ -416,8 +429,8 @@ __device__ void epilogue(const Params& p, const Smem& s, const WaitCtl& wc, uint
                         const int j = hb + i;
                         if (j < it.rows) {
                             float* rowp = p.y + static_cast<long long>(it.row0 + j) * p.H;
-                            rowp[colA] = acc0[i];
-                            if (v1) rowp[colA + 128] = acc1[i];
+                            rowp[colA] = (i & 1) ? acc0[i >> 1].y : acc0[i >> 1].x;
+                            if (v1) rowp[colA + 128] = (i & 1) ? acc1[i >> 1].y : acc1[i >> 1].x;
                         }
                     }
                 }

@@ -65,6 +65,57 @@ __device__ __forceinline__ void tmem_load_cols(uint32_t taddr, float (&v)[BT]) {
     }
 }
 
+// Two TMEM column groups of BT (16 or 32) columns each, both loads in flight
+// before one wait.
+template <int BT>
+__device__ __forceinline__ void tmem_load_pair(uint32_t ta, uint32_t tb, float (&v0)[BT],
+                                               float (&v1)[BT]) {
+    uint32_t* r0 = reinterpret_cast<uint32_t*>(v0);
+    uint32_t* r1 = reinterpret_cast<uint32_t*>(v1);
+    if constexpr (BT == 16) {
+        tmem_ld16_async(ta, *reinterpret_cast<uint32_t(*)[16]>(r0));
+        tmem_ld16_async(tb, *reinterpret_cast<uint32_t(*)[16]>(r1));
+        tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(r0));
+        tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(r1));
+    } else {
+        static_assert(BT == 32, "tmem_load_pair: 16 or 32 columns");
+        tmem_ld32_async(ta, *reinterpret_cast<uint32_t(*)[32]>(r0));
+        tmem_ld32_async(tb, *reinterpret_cast<uint32_t(*)[32]>(r1));
+        tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(r0));
+        tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(r1));
+    }
+}
+
+// acc0[j] += v0[j] * (a[j] * b0), acc1[j] += v1[j] * (a[j] * b1) for BT
+// tokens, two per packed instruction (each product and sum rounded as the
+// scalar fmul / fmaf would round it).
+template <int BT>
+__device__ __forceinline__ void promote2(float (&acc0)[BT], float (&acc1)[BT], const float (&v0)[BT],
+                                         const float (&v1)[BT], const float4* asv, float b0f,
+                                         float b1f) {
+    const float2 b0 = make_float2(b0f, b0f), b1 = make_float2(b1f, b1f);
+#pragma unroll
+    for (int j4 = 0; j4 < BT / 4; ++j4) {
+        const float4 a4 = asv[j4];
+        const float2 alo = make_float2(a4.x, a4.y), ahi = make_float2(a4.z, a4.w);
+        const float2 p0lo = __fmul2_rn(alo, b0), p0hi = __fmul2_rn(ahi, b0);
+        const float2 p1lo = __fmul2_rn(alo, b1), p1hi = __fmul2_rn(ahi, b1);
+        float2 r;
+        r = __ffma2_rn(make_float2(v0[4 * j4], v0[4 * j4 + 1]), p0lo,
+                       make_float2(acc0[4 * j4], acc0[4 * j4 + 1]));
+        acc0[4 * j4] = r.x; acc0[4 * j4 + 1] = r.y;
+        r = __ffma2_rn(make_float2(v0[4 * j4 + 2], v0[4 * j4 + 3]), p0hi,
+                       make_float2(acc0[4 * j4 + 2], acc0[4 * j4 + 3]));
+        acc0[4 * j4 + 2] = r.x; acc0[4 * j4 + 3] = r.y;
+        r = __ffma2_rn(make_float2(v1[4 * j4], v1[4 * j4 + 1]), p1lo,
+                       make_float2(acc1[4 * j4], acc1[4 * j4 + 1]));
+        acc1[4 * j4] = r.x; acc1[4 * j4 + 1] = r.y;
+        r = __ffma2_rn(make_float2(v1[4 * j4 + 2], v1[4 * j4 + 3]), p1hi,
+                       make_float2(acc1[4 * j4 + 2], acc1[4 * j4 + 3]));
+        acc1[4 * j4 + 2] = r.x; acc1[4 * j4 + 3] = r.y;
+    }
+}
+
 __device__ __forceinline__ void ffma_chunk(float2* acc, const uint32_t (&v)[32], float f) {
     const float2 f2 = make_float2(f, f);
 #pragma unroll

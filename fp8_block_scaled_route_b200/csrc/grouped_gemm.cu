@@ -649,28 +649,39 @@ __device__ void epilogue_swap(const KParams& p, const Smem& s, const WaitCtl& wc
             tc_fence_after();
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * (2 * BT);
             const float4* asv = reinterpret_cast<const float4*>(s.as_tile + kb * BT);
-            float v[BT];
-            tmem_load_cols<BT>(taddr, v);
+            if constexpr (BT <= 32) {
+                // both blocks' partials in flight before one wait; the slot is
+                // free again before the promotion arithmetic
+                float v0[BT], v1[BT];
+                tmem_load_pair<BT>(taddr, taddr + BT, v0, v1);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s.tempty[buf]);
+                promote2<BT>(acc0, acc1, v0, v1, asv, b0, b1);
+            } else {
+                float v[BT];
+                tmem_load_cols<BT>(taddr, v);
 #pragma unroll
-            for (int j4 = 0; j4 < BT / 4; ++j4) {
-                const float4 a4 = asv[j4];
-                acc0[4 * j4 + 0] = fmaf(v[4 * j4 + 0], a4.x * b0, acc0[4 * j4 + 0]);
-                acc0[4 * j4 + 1] = fmaf(v[4 * j4 + 1], a4.y * b0, acc0[4 * j4 + 1]);
-                acc0[4 * j4 + 2] = fmaf(v[4 * j4 + 2], a4.z * b0, acc0[4 * j4 + 2]);
-                acc0[4 * j4 + 3] = fmaf(v[4 * j4 + 3], a4.w * b0, acc0[4 * j4 + 3]);
-            }
-            tmem_load_cols<BT>(taddr + BT, v);
+                for (int j4 = 0; j4 < BT / 4; ++j4) {
+                    const float4 a4 = asv[j4];
+                    acc0[4 * j4 + 0] = fmaf(v[4 * j4 + 0], a4.x * b0, acc0[4 * j4 + 0]);
+                    acc0[4 * j4 + 1] = fmaf(v[4 * j4 + 1], a4.y * b0, acc0[4 * j4 + 1]);
+                    acc0[4 * j4 + 2] = fmaf(v[4 * j4 + 2], a4.z * b0, acc0[4 * j4 + 2]);
+                    acc0[4 * j4 + 3] = fmaf(v[4 * j4 + 3], a4.w * b0, acc0[4 * j4 + 3]);
+                }
+                tmem_load_cols<BT>(taddr + BT, v);
 #pragma unroll
-            for (int j4 = 0; j4 < BT / 4; ++j4) {
-                const float4 a4 = asv[j4];
-                acc1[4 * j4 + 0] = fmaf(v[4 * j4 + 0], a4.x * b1, acc1[4 * j4 + 0]);
-                acc1[4 * j4 + 1] = fmaf(v[4 * j4 + 1], a4.y * b1, acc1[4 * j4 + 1]);
-                acc1[4 * j4 + 2] = fmaf(v[4 * j4 + 2], a4.z * b1, acc1[4 * j4 + 2]);
-                acc1[4 * j4 + 3] = fmaf(v[4 * j4 + 3], a4.w * b1, acc1[4 * j4 + 3]);
+                for (int j4 = 0; j4 < BT / 4; ++j4) {
+                    const float4 a4 = asv[j4];
+                    acc1[4 * j4 + 0] = fmaf(v[4 * j4 + 0], a4.x * b1, acc1[4 * j4 + 0]);
+                    acc1[4 * j4 + 1] = fmaf(v[4 * j4 + 1], a4.y * b1, acc1[4 * j4 + 1]);
+                    acc1[4 * j4 + 2] = fmaf(v[4 * j4 + 2], a4.z * b1, acc1[4 * j4 + 2]);
+                    acc1[4 * j4 + 3] = fmaf(v[4 * j4 + 3], a4.w * b1, acc1[4 * j4 + 3]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s.tempty[buf]);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s.tempty[buf]);
             if (++buf == C::TSLOTS) { buf = 0; bphase ^= 1; }
         }
 

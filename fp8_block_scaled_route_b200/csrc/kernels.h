@@ -85,8 +85,13 @@ struct RouteArgs {
     int32_t* inv_perm;
     int32_t* chunk_hist;  // [nchunks, E]
     int* status;
+    // single-launch routing only: the kernel zeroes status[0, kStatusInts)
+    // before it reports anything (the caller then needs no clearing memset)
+    int clear_status;
 };
 constexpr int kRouteChunk = 1024;
+// Whether routing R pairs takes the single-launch (one CTA) path.
+bool route_single_launch(int R);
 // Largest expert count the routing kernels accept (MOE_MAX_EXPERTS of the C ABI).
 constexpr int kMaxRouteExperts = 1024;
 int launch_route_permute(const RouteArgs& r, cudaStream_t stream);

@@ -141,33 +141,40 @@ __global__ void __launch_bounds__(32) route_scatter(const int32_t* __restrict__ 
 // Small inputs (at most kSmallChunks chunks of 1024 pairs): the same three
 // phases in one CTA of 1024 threads, so routing costs one launch.  The pairs
 // are cut into up to 32 consecutive blocks, one per warp (as many as keep the
-// per-block histograms within 48 KB of shared memory), so the serial ranking
-// steps of phase 3 are spread over the warps; thread e owns expert e in
-// phase 2.
+// per-block histograms within the default shared-memory limit), so the
+// serial ranking steps of phase 3 are spread over the warps.  Phase 2 scans
+// each expert's column of block counts with one warp (lane = block; rows of
+// the table padded to E + 1 ints so a column read is conflict-free), then
+// the experts' totals with one thread per expert.
 constexpr int kSmallChunks = 8;
-constexpr int kSmallTabInts = 11 * 1024;  // 44 KB: with the static scan table within 48 KB
+// 43 KB of table; with the static per-expert totals (4 KB) within 48 KB
+constexpr int kSmallTabInts = 11008;
 
 __host__ __device__ constexpr int small_route_warps(int E) {
-    return E * 32 <= kSmallTabInts ? 32 : kSmallTabInts / E;
+    return (E + 1) * 32 <= kSmallTabInts ? 32 : kSmallTabInts / (E + 1);
 }
 static_assert(small_route_warps(kMaxRouteExperts) >= kSmallChunks,
               "route_small's pair blocks must stay within kRouteChunk pairs");
 
 // The three phases of route_small for a CTA of 1024 threads; tab is
-// [small_route_warps(E)][E] ints of shared memory.
+// [small_route_warps(E)][E + 1] ints of shared memory.
 __device__ __forceinline__ void route_small_body(const int32_t* __restrict__ ids, int R, int E,
                                                  int32_t* __restrict__ m_indptr,
                                                  int32_t* __restrict__ perm,
                                                  int32_t* __restrict__ inv_perm, int* status,
-                                                 int* tab) {
+                                                 int* tab, bool clear_status) {
     __shared__ int warp_tot[32];
+    __shared__ int cnt_s[kMaxRouteExperts];   // per-expert totals, then first rows
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int W = small_route_warps(E);
+    const int Ep = E + 1;
     // pairs per block: a multiple of 32, at most kRouteChunk (R <= 8 chunks, W >= 8)
     const int B = ((R + W - 1) / W + 31) & ~31;
     const int nchunks = B > 0 ? (R + B - 1) / B : 0;
     constexpr int kSteps = kRouteChunk / 32;
-    for (int i = threadIdx.x; i < nchunks * E; i += blockDim.x) tab[i] = 0;
+    // the caller's status words start clean before any error is reported
+    if (clear_status && threadIdx.x < kStatusInts) status[threadIdx.x] = 0;
+    for (int i = threadIdx.x; i < nchunks * Ep; i += blockDim.x) tab[i] = 0;
     __syncthreads();
     // phase 1: per-block histograms
     int my_ids[kSteps];
@@ -185,7 +192,7 @@ __device__ __forceinline__ void route_small_body(const int32_t* __restrict__ ids
             const int p = base + i * 32 + lane;
             if (p < end) {
                 const int e = my_ids[i];
-                if (e >= 0 && e < E) atomicAdd(&tab[warp * E + e], 1);
+                if (e >= 0 && e < E) atomicAdd(&tab[warp * Ep + e], 1);
                 else ++bad;
             }
         }
@@ -195,16 +202,22 @@ __device__ __forceinline__ void route_small_body(const int32_t* __restrict__ ids
         }
     }
     __syncthreads();
-    // phase 2: scan over chunks and experts
-    const int e = threadIdx.x;
-    int count = 0;
-    if (e < E) {
-        for (int c = 0; c < nchunks; ++c) {
-            const int h = tab[c * E + e];
-            tab[c * E + e] = count;
-            count += h;
+    // phase 2a: per expert, exclusive scan over the blocks (warp per expert, lane = block)
+    for (int ex = warp; ex < E; ex += 32) {
+        const int h = lane < nchunks ? tab[lane * Ep + ex] : 0;
+        int run = h;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, run, o);
+            if (lane >= o) run += v;
         }
+        if (lane < nchunks) tab[lane * Ep + ex] = run - h;
+        if (lane == 31) cnt_s[ex] = run;
     }
+    __syncthreads();
+    // phase 2b: exclusive scan over the experts' totals (thread e)
+    const int e = threadIdx.x;
+    const int count = e < E ? cnt_s[e] : 0;
     int incl = count;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -227,14 +240,18 @@ __device__ __forceinline__ void route_small_body(const int32_t* __restrict__ ids
     const int excl = warp_tot[warp] + incl - count;
     if (e < E) {
         m_indptr[e] = excl;
-        for (int c = 0; c < nchunks; ++c) tab[c * E + e] += excl;
+        cnt_s[e] = excl;   // only thread e read cnt_s[e] above
     }
     if (e == E - 1) m_indptr[E] = excl + count;
+    __syncthreads();
+    // phase 2c: first output row of every (block, expert)
+    for (int ex = warp; ex < E; ex += 32)
+        if (lane < nchunks) tab[lane * Ep + ex] += cnt_s[ex];
     __syncthreads();
     // phase 3: stable scatter, 32 pairs at a time per block
     if (warp < nchunks) {
         const int end = min(R, base + B);
-        int* cursor = tab + warp * E;
+        int* cursor = tab + warp * Ep;
 #pragma unroll
         for (int i = 0; i < kSteps; ++i) {
             const int p = base + i * 32 + lane;
@@ -262,9 +279,10 @@ __device__ __forceinline__ void route_small_body(const int32_t* __restrict__ ids
 __global__ void __launch_bounds__(1024) route_small(const int32_t* __restrict__ ids, int R, int E,
                                                     int32_t* __restrict__ m_indptr,
                                                     int32_t* __restrict__ perm,
-                                                    int32_t* __restrict__ inv_perm, int* status) {
-    extern __shared__ int tab[];  // [blocks][E]: histograms, then first rows
-    route_small_body(ids, R, E, m_indptr, perm, inv_perm, status, tab);
+                                                    int32_t* __restrict__ inv_perm, int* status,
+                                                    int clear_status) {
+    extern __shared__ int tab[];  // [blocks][E + 1]: histograms, then first rows
+    route_small_body(ids, R, E, m_indptr, perm, inv_perm, status, tab, clear_status != 0);
 }
 
 // Router (the step before the expert computation): one warp per token.
@@ -341,7 +359,7 @@ __global__ void __launch_bounds__(1024) router_route_small(const float* __restri
     extern __shared__ int tab[];
     for (int t = threadIdx.x >> 5; t < T; t += 32) router_token<PER>(logits, t, E, k, ids, w);
     __syncthreads();
-    route_small_body(ids, T * k, E, m_indptr, perm, inv_perm, status, tab);
+    route_small_body(ids, T * k, E, m_indptr, perm, inv_perm, status, tab, false);
 }
 
 int launch_router_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
@@ -361,7 +379,7 @@ int launch_router_route(const float* logits, const RouteArgs& r, float* w, cudaS
     const int nchunks = (R + kRouteChunk - 1) / kRouteChunk;
     if (nchunks <= kSmallChunks) {
         int32_t* ids = const_cast<int32_t*>(r.topk_ids);
-        const size_t smem = static_cast<size_t>(small_route_warps(r.E)) * r.E * sizeof(int);
+        const size_t smem = static_cast<size_t>(small_route_warps(r.E)) * (r.E + 1) * sizeof(int);
         if (r.E <= 256)
             router_route_small<8><<<1, 1024, smem, stream>>>(logits, r.T, r.E, r.k, ids, w,
                                                              r.m_indptr, r.perm, r.inv_perm, r.status);
@@ -375,15 +393,17 @@ int launch_router_route(const float* logits, const RouteArgs& r, float* w, cudaS
     return launch_route_permute(r, stream);
 }
 
+bool route_single_launch(int R) { return (R + kRouteChunk - 1) / kRouteChunk <= kSmallChunks; }
+
 int launch_route_permute(const RouteArgs& r, cudaStream_t stream) {
     const int R = r.T * r.k;
     const int nchunks = (R + kRouteChunk - 1) / kRouteChunk;
     const size_t hist_smem = static_cast<size_t>(r.E) * sizeof(int);
     if (nchunks <= kSmallChunks) {
         // within the default dynamic shared-memory limit (48 KB)
-        const size_t smem = static_cast<size_t>(small_route_warps(r.E)) * r.E * sizeof(int);
+        const size_t smem = static_cast<size_t>(small_route_warps(r.E)) * (r.E + 1) * sizeof(int);
         route_small<<<1, 1024, smem, stream>>>(r.topk_ids, R, r.E, r.m_indptr, r.perm, r.inv_perm,
-                                               r.status);
+                                               r.status, r.clear_status);
         return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
     }
     {

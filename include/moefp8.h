@@ -538,9 +538,11 @@ MOE_API int moe_set_stage_events(void* const* events, int n);
  *   MOE_FUSION_AUTO (default): one fused-expert launch when the FP8
  *     intermediate of a 64-token group (I bytes per token) fits in shared
  *     memory beside the weight pipeline, the groups are small (the tile
- *     model picks weight-stationary GEMM1 tiles), the 64-token groups of a
- *     balanced routing make about one round over the SMs and fill at least
- *     half of them, and an expert holds at most 6 MB of weights (3·H·I
+ *     model picks weight-stationary GEMM1 tiles), and either the layer is
+ *     tiny (at most 16 MB of touched weights: one launch fewer) or, for a
+ *     balanced routing, the active experts make about one round over the
+ *     SMs and fill at least half of them, their 64-token groups at most
+ *     about two rounds, and an expert holds at most 6 MB of weights (3·H·I
  *     bytes); otherwise GEMM1 and GEMM2 as two launches.
  *   MOE_FUSION_ON: the fused launch whenever the intermediate fits.
  *   MOE_FUSION_OFF: always two launches.

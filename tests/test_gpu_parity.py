@@ -208,9 +208,19 @@ def _check_fused_full(inp, what):
     G.compare_layer(res, ref, inp, what + " output")
 
 
-def test_fused_tiny():
+# "off": the two-launch path (GEMM1 then GEMM2); "auto": whatever the plan
+# picks for the shape (the fused-expert launch for tiny layers).
+@pytest.fixture(params=["off", "auto"])
+def fusion(request):
+    mode = {"off": moe.MOE_FUSION_OFF, "auto": moe.MOE_FUSION_AUTO}[request.param]
+    moe.moe_set_expert_fusion(mode)
+    yield request.param
+    moe.moe_set_expert_fusion(moe.MOE_FUSION_AUTO)
+
+
+def test_fused_tiny(fusion):
     inp = synth.make_moe_inputs(synth.CONFIGS["tiny"], seed=0, device=DEV)
-    _check_fused_full(inp, "tiny")
+    _check_fused_full(inp, f"tiny ({fusion})")
 
 
 @pytest.mark.parametrize("T,H,I,E,k,routing", [
@@ -223,10 +233,10 @@ def test_fused_tiny():
     (700, 512, 256, 4, 2, "normal"),      # ~350 rows/expert: 128-row tiles with a ragged tail
     (1500, 256, 256, 3, 1, "zipf"),       # ~500 rows/expert, skewed: several tiles each
 ])
-def test_fused_small_shapes(T, H, I, E, k, routing):
+def test_fused_small_shapes(fusion, T, H, I, E, k, routing):
     cfg = synth.MoEConfig("case", T, H, I, E, k, routing)
     inp = synth.make_moe_inputs(cfg, seed=T + E, device=DEV)
-    _check_fused_full(inp, f"T={T} H={H} I={I} E={E} k={k}")
+    _check_fused_full(inp, f"T={T} H={H} I={I} E={E} k={k} ({fusion})")
 
 
 def test_fused_zero_tokens():
@@ -236,7 +246,7 @@ def test_fused_zero_tokens():
     assert res["status"] == moe.MOE_OK and np.all(res["m_indptr"] == 0)
 
 
-def test_fused_bad_expert_ids():
+def test_fused_bad_expert_ids(fusion):
     cfg = synth.MoEConfig("bad", 32, 256, 128, 8, 2)
     inp = synth.make_moe_inputs(cfg, seed=4, device=DEV)
     inp["topk_ids"][3, 1] = -1
@@ -280,10 +290,10 @@ def _check_sampled(inp, tokens, what):
                          hq_o.reshape(n, -1), own_h, what + " output")
 
 
-def test_fused_mid_sampled():
+def test_fused_mid_sampled(fusion):
     inp = synth.make_moe_inputs(synth.CONFIGS["mid"], seed=0, device=DEV)
     tokens = list(range(0, 512, 16)) + [511]
-    _check_sampled(inp, tokens, "mid")
+    _check_sampled(inp, tokens, f"mid ({fusion})")
 
 
 def test_fused_decode_full_size_sampled():
