@@ -500,10 +500,11 @@ def swiglu_mxfp8_quant(inp, out, scale, *, dims=None, stream=None, check=True) -
 
 def moe_set_stage_events(events) -> int:
     """events: six torch.cuda.Event (timing enabled, already created on the
-    device) or None to switch stage timing off."""
+    device; None entries are not recorded) or None to switch stage timing off."""
     if events is None:
         return _check(lib().moe_set_stage_events(None, 0), "moe_set_stage_events", True)
-    handles = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    handles = (ctypes.c_void_p * len(events))(
+        *[ctypes.c_void_p(e.cuda_event if e is not None else None) for e in events])
     return _check(lib().moe_set_stage_events(handles, len(events)), "moe_set_stage_events", True)
 
 

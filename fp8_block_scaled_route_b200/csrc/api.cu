@@ -32,7 +32,8 @@ cudaEvent_t g_stage_events[kStageEvents];
 std::atomic<bool> g_stage_events_on{false};
 
 inline void stage_mark(int i, cudaStream_t s) {
-    if (g_stage_events_on.load(std::memory_order_relaxed)) cudaEventRecord(g_stage_events[i], s);
+    if (g_stage_events_on.load(std::memory_order_relaxed) && g_stage_events[i])
+        cudaEventRecord(g_stage_events[i], s);
 }
 
 struct DevInfo {
@@ -273,10 +274,10 @@ int moe_set_stage_events(void* const* events, int n) {
         return MOE_OK;
     }
     if (n != kStageEvents) return MOE_ERR_INVALID_ARG;
-    for (int i = 0; i < kStageEvents; ++i) {
-        if (!events[i]) return MOE_ERR_INVALID_ARG;
-        g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
-    }
+    bool any = false;
+    for (int i = 0; i < kStageEvents; ++i) any = any || events[i] != nullptr;
+    if (!any) return MOE_ERR_INVALID_ARG;
+    for (int i = 0; i < kStageEvents; ++i) g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
     g_stage_events_on.store(true);
     return MOE_OK;
 }

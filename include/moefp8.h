@@ -531,6 +531,8 @@ MOE_API int moe_get_device_status(const void* ws, moe_stream_t stream);
  * caller) on the call's stream: 0 before routing, 1 after routing, 2 after
  * activation quantisation, 3 after GEMM1 (gate/up + SwiGLU + requant), 4
  * after GEMM2 (down projection), 5 after the combine and bf16 output.  n must be 6;
+ * a NULL entry is not recorded (at least one must be set: each record costs
+ * 2-3 µs of GPU time, so a caller timing one stage passes only its two);
  * events = NULL switches it off.  Process-wide setting. */
 MOE_API int moe_set_stage_events(void* const* events, int n);
 

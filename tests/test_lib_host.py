@@ -63,6 +63,14 @@ def test_status_strings(L):
         assert moe.moe_status_string(code) == name
 
 
+def test_stage_event_setter_validation(L):
+    import ctypes
+    six_null = (ctypes.c_void_p * 6)()
+    assert L.moe_set_stage_events(six_null, 6) == moe.MOE_ERR_INVALID_ARG   # nothing to record
+    assert L.moe_set_stage_events(six_null, 5) == moe.MOE_ERR_INVALID_ARG   # wrong count
+    assert L.moe_set_stage_events(None, 0) == moe.MOE_OK                    # timing off
+
+
 def test_expert_fusion_mode_setter(L):
     assert L.moe_set_expert_fusion(moe.MOE_FUSION_OFF) == moe.MOE_OK
     assert L.moe_set_expert_fusion(moe.MOE_FUSION_ON) == moe.MOE_OK
