@@ -15,12 +15,34 @@
 //                    output row of every (chunk, expert)
 //  3. route_scatter: one warp per chunk walks its pairs in order, 32 at a
 //                    time; lanes with the same expert are ranked with
-//                    __match_any_sync, so each pair lands at
+//                    one warp ballot per expert-id bit, so each pair lands at
 //                    chunk_base[e] + (earlier pairs of e in the chunk).
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 
 namespace moe {
+
+// Lanes of the warp whose value equals this lane's, among the lanes with
+// ok set, for values in [0, 2^nbits): one ballot per value bit (nbits
+// uniform across the warp).  Used in place of the match instruction, whose
+// cost grows with the number of distinct values in the warp.
+__device__ __forceinline__ unsigned same_value_lanes(int v, bool ok, int nbits) {
+    unsigned m = __ballot_sync(0xffffffffu, ok);
+    for (int b = 0; b < nbits; ++b) {
+        const bool bit = (v >> b) & 1;
+        const unsigned bb = __ballot_sync(0xffffffffu, bit);
+        m &= bit ? bb : ~bb;
+    }
+    return m;
+}
+
+__host__ __device__ inline int value_bits(int E) {
+    int n = 0;
+    while ((1 << n) < E) ++n;
+    return n;
+}
 
 __global__ void __launch_bounds__(256) route_hist(const int32_t* __restrict__ ids, int R, int E,
                                                   int32_t* __restrict__ chunk_hist, int* status) {
@@ -122,7 +144,7 @@ __global__ void __launch_bounds__(32) route_scatter(const int32_t* __restrict__ 
         const bool live = p < end;
         const int e = my_ids[i];
         const bool ok = live && e >= 0 && e < E;
-        const unsigned peers = __match_any_sync(0xffffffffu, ok ? e : -1);
+        const unsigned peers = same_value_lanes(e, ok, value_bits(E));
         const int rank = __popc(peers & ((1u << lane) - 1u));
         const int first = cursor[ok ? e : 0];
         __syncwarp();
@@ -156,8 +178,17 @@ __host__ __device__ constexpr int small_route_warps(int E) {
 static_assert(small_route_warps(kMaxRouteExperts) >= kSmallChunks,
               "route_small's pair blocks must stay within kRouteChunk pairs");
 
+// Dynamic shared memory of route_small: the table, then the R entries of
+// perm, which phase 3 writes in shared memory (scattered) and the CTA then
+// copies out in order: scattered 4-byte global stores from one SM go out at
+// about one sector per clock (4096 of them cost ~4 µs).
+__host__ __device__ inline size_t small_route_smem(int R, int E) {
+    return (static_cast<size_t>(small_route_warps(E)) * (E + 1) + R) * sizeof(int);
+}
+constexpr size_t kSmallRouteSmemMax = (kSmallTabInts + kSmallChunks * kRouteChunk) * sizeof(int);
+
 // The three phases of route_small for a CTA of 1024 threads; tab is
-// [small_route_warps(E)][E + 1] ints of shared memory.
+// [small_route_warps(E)][E + 1] ints of shared memory followed by R ints.
 __device__ __forceinline__ void route_small_body(const int32_t* __restrict__ ids, int R, int E,
                                                  int32_t* __restrict__ m_indptr,
                                                  int32_t* __restrict__ perm,
@@ -165,9 +196,11 @@ __device__ __forceinline__ void route_small_body(const int32_t* __restrict__ ids
                                                  int* tab, bool clear_status) {
     __shared__ int warp_tot[32];
     __shared__ int cnt_s[kMaxRouteExperts];   // per-expert totals, then first rows
+    __shared__ int valid_s;                   // pairs with a valid expert id
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int W = small_route_warps(E);
     const int Ep = E + 1;
+    int* perm_s = tab + W * Ep;               // [R]: perm, staged
     // pairs per block: a multiple of 32, at most kRouteChunk (R <= 8 chunks, W >= 8)
     const int B = ((R + W - 1) / W + 31) & ~31;
     const int nchunks = B > 0 ? (R + B - 1) / B : 0;
@@ -242,13 +275,17 @@ __device__ __forceinline__ void route_small_body(const int32_t* __restrict__ ids
         m_indptr[e] = excl;
         cnt_s[e] = excl;   // only thread e read cnt_s[e] above
     }
-    if (e == E - 1) m_indptr[E] = excl + count;
+    if (e == E - 1) {
+        m_indptr[E] = excl + count;
+        valid_s = excl + count;
+    }
     __syncthreads();
     // phase 2c: first output row of every (block, expert)
     for (int ex = warp; ex < E; ex += 32)
         if (lane < nchunks) tab[lane * Ep + ex] += cnt_s[ex];
     __syncthreads();
     // phase 3: stable scatter, 32 pairs at a time per block
+    const int nbits = value_bits(E);
     if (warp < nchunks) {
         const int end = min(R, base + B);
         int* cursor = tab + warp * Ep;
@@ -259,13 +296,13 @@ __device__ __forceinline__ void route_small_body(const int32_t* __restrict__ ids
             const bool live = p < end;
             const int ex = my_ids[i];
             const bool ok = live && ex >= 0 && ex < E;
-            const unsigned peers = __match_any_sync(0xffffffffu, ok ? ex : -1);
+            const unsigned peers = same_value_lanes(ex, ok, nbits);
             const int rank = __popc(peers & ((1u << lane) - 1u));
             const int first = cursor[ok ? ex : 0];
             __syncwarp();
             if (ok) {
                 const int row = first + rank;
-                perm[row] = p;
+                perm_s[row] = p;
                 if (inv_perm) inv_perm[p] = row;
                 if (rank == 0) cursor[ex] = first + __popc(peers);
             } else if (live && inv_perm) {
@@ -274,6 +311,10 @@ __device__ __forceinline__ void route_small_body(const int32_t* __restrict__ ids
             __syncwarp();
         }
     }
+    __syncthreads();
+    // perm out in order (rows of dropped pairs do not exist: only [0, valid) is written)
+    const int valid = valid_s;
+    for (int i = threadIdx.x; i < valid; i += blockDim.x) perm[i] = perm_s[i];
 }
 
 __global__ void __launch_bounds__(1024) route_small(const int32_t* __restrict__ ids, int R, int E,
@@ -373,13 +414,32 @@ int launch_router_topk(const float* logits, int T, int E, int k, int32_t* ids, f
     return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
 }
 
+// Opt-in of the single-CTA routing kernels to kSmallRouteSmemMax bytes of
+// dynamic shared memory, once per device.
+bool small_route_smem_ready() {
+    static std::atomic<int> ready_dev{-1};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    if (ready_dev.load() == dev) return true;
+    const int n = static_cast<int>(kSmallRouteSmemMax);
+    if (cudaFuncSetAttribute(route_small, cudaFuncAttributeMaxDynamicSharedMemorySize, n) != cudaSuccess ||
+        cudaFuncSetAttribute(router_route_small<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, n) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(router_route_small<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, n) !=
+            cudaSuccess)
+        return false;
+    ready_dev.store(dev);
+    return true;
+}
+
 int launch_router_route(const float* logits, const RouteArgs& r, float* w, cudaStream_t stream) {
     const int R = r.T * r.k;
     if (R == 0) return launch_route_permute(r, stream);
     const int nchunks = (R + kRouteChunk - 1) / kRouteChunk;
     if (nchunks <= kSmallChunks) {
         int32_t* ids = const_cast<int32_t*>(r.topk_ids);
-        const size_t smem = static_cast<size_t>(small_route_warps(r.E)) * (r.E + 1) * sizeof(int);
+        const size_t smem = small_route_smem(R, r.E);
+        if (!small_route_smem_ready()) return ST_CUDA;
         if (r.E <= 256)
             router_route_small<8><<<1, 1024, smem, stream>>>(logits, r.T, r.E, r.k, ids, w,
                                                              r.m_indptr, r.perm, r.inv_perm, r.status);
@@ -400,8 +460,8 @@ int launch_route_permute(const RouteArgs& r, cudaStream_t stream) {
     const int nchunks = (R + kRouteChunk - 1) / kRouteChunk;
     const size_t hist_smem = static_cast<size_t>(r.E) * sizeof(int);
     if (nchunks <= kSmallChunks) {
-        // within the default dynamic shared-memory limit (48 KB)
-        const size_t smem = static_cast<size_t>(small_route_warps(r.E)) * (r.E + 1) * sizeof(int);
+        const size_t smem = small_route_smem(R, r.E);
+        if (!small_route_smem_ready()) return ST_CUDA;
         route_small<<<1, 1024, smem, stream>>>(r.topk_ids, R, r.E, r.m_indptr, r.perm, r.inv_perm,
                                                r.status, r.clear_status);
         return cudaGetLastError() == cudaSuccess ? ST_OK : ST_CUDA;
