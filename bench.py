@@ -485,6 +485,9 @@ def run_ours(args, cfg):
                       "experts_touched": counts["touched"], "alg_bytes": counts["bytes"],
                       "alg_flops": counts["flops"]},
             "stages_us": stage_dict(stage_ms, fused),
+            "stages_note": "per-stage device times from a second pass of the same steps after "
+                           "the timed region, with all six stage events; the roofline kernel is "
+                           "timed inside the timed region",
             "ms_per_step_with_stage_events": staged_ms,
             "plan": plan,
             "roofline": roof,
