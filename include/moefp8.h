@@ -161,7 +161,11 @@ MOE_API size_t moe_workspace_size(int T, int H, int I, int E, int k);
  * down projection: each pair's fp32 down-projection row is written once and
  * the combine sums a token's k weighted rows in ascending slot order (fp32,
  * each product rounded, then bf16), so the output does not depend on the
- * order in which the GEMM's tiles run.  T = 0 is a no-op.  Returns MOE_ERR_INVALID_ARG for
+ * order in which the GEMM's tiles run.  The two expert GEMMs run as two
+ * grouped-GEMM launches, or as one fused-expert launch that keeps each token
+ * group's FP8 intermediate in shared memory (moe_fp8_fused_plan tells which;
+ * moe_set_expert_fusion chooses); both give the same intermediate and
+ * output.  T = 0 is a no-op.  Returns MOE_ERR_INVALID_ARG for
  * sizes that are not multiples of 128, k > E, null pointers, misaligned
  * pointers or a small workspace; MOE_ERR_UNSUPPORTED for E > 1024. */
 MOE_API int moe_fp8_fused(const void* x, const int32_t* topk_ids, const float* topk_w,
