@@ -296,6 +296,14 @@ def test_fused_mid_sampled(fusion):
     _check_sampled(inp, tokens, f"mid ({fusion})")
 
 
+def test_fused_two_groups_per_expert_sampled(fusion):
+    """~128 rows per expert: two 64-token work items per expert in the
+    fused-expert launch (the plan fuses this shape), 128-row tiles otherwise."""
+    cfg = synth.MoEConfig("mid2k", 2048, 2048, 768, 128, 8)
+    inp = synth.make_moe_inputs(cfg, seed=5, device=DEV)
+    _check_sampled(inp, [0, 1, 777, 1500, 2047], f"T=2048 mid shape ({fusion})")
+
+
 def test_fused_decode_full_size_sampled():
     inp = synth.make_moe_inputs(synth.CONFIGS["decode"], seed=0, device=DEV)
     _check_sampled(inp, [0, 17, 42, 63], "decode")
