@@ -36,6 +36,8 @@
 //    token by the combine kernel.
 // Every wait is bounded by %globaltimer; on expiry the CTA records
 // ST_DEVICE_TIMEOUT, drains its copies and MMAs, frees TMEM and returns.
+#include <atomic>
+
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
@@ -543,14 +545,14 @@ int launch_fused_expert(const FusedExpertArgs& g, cudaStream_t stream) {
     p.m_indptr = g.m_indptr; p.y = g.y; p.hq = g.hq; p.hs = g.hs;
     p.status = g.status; p.timeout_ns = g.timeout_ns;
     const int smem = fx::fixed_bytes(g.H, g.I, g.E) + p.nstages * fx::STAGE_BYTES;
-    static int configured_dev = -1;  // one-time opt-in to the largest dynamic shared memory
+    static std::atomic<int> configured_dev{-1};  // opt-in to the largest dynamic shared memory
     int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured_dev != dev) {
+    if (cudaGetDevice(&dev) != cudaSuccess) return ST_CUDA;
+    if (configured_dev.load() != dev) {
         if (cudaFuncSetAttribute(fx::fused_expert_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  fx::kSmemLimit) != cudaSuccess)
             return ST_CUDA;
-        configured_dev = dev;
+        configured_dev.store(dev);
     }
     // at most one work item per 64 grouped rows plus one partial tile per expert
     const long long items = (static_cast<long long>(g.R) + fx::BT - 1) / fx::BT + g.E;
