@@ -42,7 +42,7 @@ __global__ void __launch_bounds__(256) quant_scatter_kernel(
     const int nkb = H >> 7;
     const int kb = c0 >> 7;
     const long long off = static_cast<long long>(t) * H + c0;
-    float f[16];
+    float f[16] = {};
     float amax = 0.0f;
     if (live) {
         const uint4* src = reinterpret_cast<const uint4*>(x + off);
@@ -60,7 +60,8 @@ __global__ void __launch_bounds__(256) quant_scatter_kernel(
     }
 #pragma unroll
     for (int o = 4; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    if (!live) return;
+    // every lane stays to the end (the row broadcast below is warp-wide);
+    // lanes past H only skip their stores
     const float s = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
     uint4 codes;
     uint32_t* cw = reinterpret_cast<uint32_t*>(&codes);
@@ -69,9 +70,13 @@ __global__ void __launch_bounds__(256) quant_scatter_kernel(
         cw[i] = cvt_e4m3x4(__fdiv_rn(f[4 * i], s), __fdiv_rn(f[4 * i + 1], s),
                            __fdiv_rn(f[4 * i + 2], s), __fdiv_rn(f[4 * i + 3], s));
     const bool lead = (lane & 7) == 0;
+    // the token's first 32 destination rows, loaded at once (lane j holds
+    // slot j's) and broadcast per slot, so the loop carries no load latency
+    const int my_row = lane < k ? (inv_perm ? inv_perm[t * k + lane] : t * k + lane) : -1;
     for (int j = 0; j < k; ++j) {
-        const int row = inv_perm ? inv_perm[t * k + j] : t * k + j;
-        if (row < 0) continue;
+        const int row = j < 32 ? __shfl_sync(0xffffffffu, my_row, j)
+                               : (inv_perm ? inv_perm[t * k + j] : t * k + j);
+        if (row < 0 || !live) continue;
         *reinterpret_cast<uint4*>(xq + static_cast<long long>(row) * H + c0) = codes;
         if (lead) {
             if (xs_kmajor) xs[static_cast<long long>(row) * nkb + kb] = s;
@@ -82,7 +87,7 @@ __global__ void __launch_bounds__(256) quant_scatter_kernel(
             }
         }
     }
-    if (out_acc) {
+    if (out_acc && live) {
         float4* z = reinterpret_cast<float4*>(out_acc + off);
         z[0] = z[1] = z[2] = z[3] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
