@@ -63,6 +63,8 @@ def _check(inp, what, debug=True):
     (300, 640, 640, 12, 3, "normal"),     # 5 intermediate blocks, H = 5 x 128
     (130, 1024, 768, 3, 2, "normal"),     # long K loops, ragged last item per expert
     (64, 2048, 768, 128, 8, "normal"),    # the mid workload's expert shape
+    (600, 256, 128, 1024, 8, "zipf"),     # the largest expert count (item table of 1024)
+    (48, 7168, 128, 16, 2, "normal"),     # the pages' H with a small I: 56 K blocks in phase 1
 ])
 def test_fused_expert_parity(fusion_on, T, H, I, E, k, routing):
     cfg = synth.MoEConfig("case", T, H, I, E, k, routing)
