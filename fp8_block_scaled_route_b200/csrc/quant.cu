@@ -214,25 +214,30 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
     const long long pair0 = static_cast<long long>(t) * k;
-    for (int j0 = 0; j0 < k; j0 += 4) {
-        float4 v[4][2];
-        float w[4];
-        bool ok[4];
+    // eight slots at a time: their rows and weights first, then all sixteen
+    // 16-byte row loads in flight, then the sums in ascending slot order
+    for (int j0 = 0; j0 < k; j0 += 8) {
+        int row[8];
+        float w[8];
+        bool ok[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
             const int j = j0 + u;
-            const int row = j < k ? (inv_perm ? __ldg(inv_perm + pair0 + j)
-                                              : static_cast<int>(pair0 + j))
-                                  : -1;
-            ok[u] = row >= 0;
-            w[u] = ok[u] ? __ldg(topk_w + pair0 + j) : 0.0f;
+            row[u] = j < k ? (inv_perm ? __ldg(inv_perm + pair0 + j) : static_cast<int>(pair0 + j))
+                           : -1;
+            w[u] = j < k ? __ldg(topk_w + pair0 + j) : 0.0f;
+        }
+        float4 v[8][2];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            ok[u] = row[u] >= 0;
             const float4* src = reinterpret_cast<const float4*>(
-                y + static_cast<long long>(ok[u] ? row : 0) * H + c);
+                y + static_cast<long long>(ok[u] ? row[u] : 0) * H + c);
             v[u][0] = ok[u] ? __ldg(src) : make_float4(0.f, 0.f, 0.f, 0.f);
             v[u][1] = ok[u] ? __ldg(src + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
             if (!ok[u]) continue;
             const float e[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w,
                                 v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
