@@ -68,8 +68,8 @@ PROFILE_SLICES = {
 # with.
 GEMM_SOURCES = ("grouped_gemm.cu", "gemm_common.cuh", "ptx.cuh", "common.cuh")  # its code
 MEASURED_TRAFFIC = {  # workload -> (source digest, bytes per GEMM1 launch)
-    "prefill": ("705b532ef98dca09", 5551500000),
-    "decode": ("705b532ef98dca09", 6525300000),
+    "prefill": ("705b532ef98dca09", 6003600000),
+    "decode": ("705b532ef98dca09", 6525600000),
 }
 
 
