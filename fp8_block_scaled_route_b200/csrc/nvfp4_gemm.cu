@@ -611,9 +611,10 @@ __global__ void __launch_bounds__(256) nv_quant_scatter_kernel(
     int R, int sf_mn, float* __restrict__ out_acc) {
     const int nch = (H + 511) >> 9;
     const long long item = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-    if (item >= static_cast<long long>(T) * nch) return;
+    const long long items = static_cast<long long>(T) * nch;
+    if (item >= items) return;
     const int lane = threadIdx.x & 31;
-    const int t = static_cast<int>(item / nch);
+    const int t = items <= 0x7fffffffll ? static_cast<int>(item) / nch : static_cast<int>(item / nch);
     const int col = static_cast<int>(item - static_cast<long long>(t) * nch) * 512 + lane * 16;
     if (col >= H) return;
     const long long off = static_cast<long long>(t) * H + col;

@@ -34,9 +34,12 @@ __global__ void __launch_bounds__(256) quant_scatter_kernel(
     int eid_base_div, int32_t* __restrict__ eid_out) {
     const int ng = (H + 511) >> 9;
     const long long item = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-    if (item >= static_cast<long long>(T) * ng) return;
+    const long long items = static_cast<long long>(T) * ng;
+    if (item >= items) return;
     const int lane = threadIdx.x & 31;
-    const int t = static_cast<int>(item / ng);
+    // a 32-bit division where the item count allows it (a 64-bit one costs
+    // several instructions per quantised element)
+    const int t = items <= 0x7fffffffll ? static_cast<int>(item) / ng : static_cast<int>(item / ng);
     const int c0 = static_cast<int>(item - static_cast<long long>(t) * ng) * 512 + lane * 16;
     const bool live = c0 < H;   // H % 128 == 0: a block's eight lanes are all live or none
     const int nkb = H >> 7;
@@ -127,9 +130,10 @@ __global__ void __launch_bounds__(256) mx_quant_scatter_kernel(
     float* __restrict__ out_acc) {
     const int nkb = H >> 7;
     const long long item = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-    if (item >= static_cast<long long>(T) * nkb) return;
+    const long long items = static_cast<long long>(T) * nkb;
+    if (item >= items) return;
     const int lane = threadIdx.x & 31;
-    const int t = static_cast<int>(item / nkb);
+    const int t = items <= 0x7fffffffll ? static_cast<int>(item) / nkb : static_cast<int>(item / nkb);
     const int kb = static_cast<int>(item - static_cast<long long>(t) * nkb);
     const long long off = static_cast<long long>(t) * H + kb * 128 + lane * 4;
     uint2 raw = *reinterpret_cast<const uint2*>(x + off);
@@ -296,16 +300,27 @@ __global__ void __launch_bounds__(256) swiglu_mxfp8_kernel(const __nv_bfloat16* 
     if (status && blockIdx.x == 0 && threadIdx.x < kStatusInts) status[threadIdx.x] = 0;
     const int kg = K / 16;
     const long long groups = static_cast<long long>(M) * kg;
-    for (long long gi = blockIdx.x * 256ll + threadIdx.x; gi - (threadIdx.x & 31) < groups;
-         gi += static_cast<long long>(gridDim.x) * 256) {
+    // group gi = (row m, column group cg); the stride's row / column steps are
+    // divided out once, so the loop does no 64-bit division
+    const long long stride = static_cast<long long>(gridDim.x) * 256;
+    const long long dm = stride / kg;
+    const int dcg = static_cast<int>(stride - dm * kg);
+    long long gi = blockIdx.x * 256ll + threadIdx.x;
+    long long m_it = gi / kg;
+    int cg_it = static_cast<int>(gi - m_it * kg);
+    for (; gi - (threadIdx.x & 31) < groups; gi += stride) {
         const bool live = gi < groups;
         float v[16];
         float amax = 0.0f;
-        long long m = 0;
-        int c0 = 0;
+        const long long m = m_it;
+        const int c0 = cg_it * 16;
+        m_it += dm;
+        cg_it += dcg;
+        if (cg_it >= kg) {
+            cg_it -= kg;
+            ++m_it;
+        }
         if (live) {
-            m = gi / kg;
-            c0 = static_cast<int>(gi - m * kg) * 16;
             const uint4* g4 = reinterpret_cast<const uint4*>(in + m * 2 * K + c0);
             const uint4* u4 = reinterpret_cast<const uint4*>(in + m * 2 * K + K + c0);
             const uint4 gr[2] = {g4[0], g4[1]};
