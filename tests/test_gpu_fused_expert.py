@@ -134,3 +134,20 @@ def test_fused_expert_timeout_is_reported_and_context_survives(fusion_on):
     torch.cuda.synchronize()
     _check(inp, "fused expert after timeout", debug=False)
 
+
+
+def test_plan_reports_the_path_taken():
+    """moe_fp8_fused_plan: fusion where the rule picks it, never where the
+    intermediate does not fit, always off when switched off."""
+    try:
+        moe.moe_set_expert_fusion(moe.MOE_FUSION_AUTO)
+        assert moe.moe_fp8_fused_plan(512, 2048, 768, 128, 8)["fused"]       # the mid workload
+        assert not moe.moe_fp8_fused_plan(64, 7168, 2048, 256, 8)["fused"]   # decode: does not fit
+        assert not moe.moe_fp8_fused_plan(8192, 7168, 2048, 256, 8)["fused"]
+        moe.moe_set_expert_fusion(moe.MOE_FUSION_ON)
+        assert moe.moe_fp8_fused_plan(64, 7168, 896, 256, 8)["fused"]        # fits: forced on
+        assert not moe.moe_fp8_fused_plan(64, 7168, 2048, 256, 8)["fused"]
+        moe.moe_set_expert_fusion(moe.MOE_FUSION_OFF)
+        assert not moe.moe_fp8_fused_plan(512, 2048, 768, 128, 8)["fused"]
+    finally:
+        moe.moe_set_expert_fusion(moe.MOE_FUSION_AUTO)
